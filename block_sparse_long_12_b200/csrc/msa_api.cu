@@ -1,0 +1,415 @@
+// Host side of the MSA C ABI: argument checks, workspace layout, launches.
+// Every check runs before anything is enqueued; the library never allocates,
+// frees or synchronises (except msa_get_device_status, which reads back one
+// word on request).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "msa_internal.h"
+
+namespace msa {
+namespace {
+
+thread_local std::string g_err;
+thread_local cudaEvent_t g_stage_ev[4];
+thread_local int g_n_stage_ev = 0;
+
+msa_status_t fail(msa_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+msa_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(MSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int elem_size(int dtype) { return dtype == MSA_F32 ? 4 : 2; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct DevCache {
+    int checked = 0, ok = 0, sms = 0;
+};
+DevCache g_dev[64];
+
+msa_status_t check_device(int *n_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64) return fail(MSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    DevCache &c = g_dev[dev];
+    if (!c.checked) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        c.ok = (major == 10 && minor == 0);
+        c.sms = sms;
+        c.checked = 1;
+        if (!c.ok) return fail(MSA_ERR_UNSUPPORTED, "compute capability %d.%d: this library runs on sm_100 only",
+                               major, minor);
+    }
+    if (!c.ok) return fail(MSA_ERR_UNSUPPORTED, "this library runs on sm_100 (B200) only");
+    *n_sm = c.sms;
+    return MSA_OK;
+}
+
+enum Mode { DECODE_ONLY, PREFILL_ONLY, ANY_ROWS };
+
+msa_status_t check_params(const msa_params_t *p, Mode mode) {
+    if (p == nullptr) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->dtype != MSA_F32 && p->dtype != MSA_BF16) return fail(MSA_ERR_INVALID_ARG, "dtype %d unknown", p->dtype);
+    if (p->batch < 1) return fail(MSA_ERR_INVALID_ARG, "batch %d < 1", p->batch);
+    if (p->batch > kMaxBatch) return fail(MSA_ERR_UNSUPPORTED, "batch %d > %d", p->batch, kMaxBatch);
+    if (p->n_kv_heads < 1 || p->n_q_heads < 1 || p->n_q_heads % p->n_kv_heads != 0)
+        return fail(MSA_ERR_INVALID_ARG, "n_q_heads %d must be a positive multiple of n_kv_heads %d", p->n_q_heads,
+                    p->n_kv_heads);
+    if (p->n_q_heads / p->n_kv_heads > 16)
+        return fail(MSA_ERR_UNSUPPORTED, "group size %d > 16", p->n_q_heads / p->n_kv_heads);
+    if (p->n_idx_k_heads != 1 && p->n_idx_k_heads != p->n_kv_heads)
+        return fail(MSA_ERR_INVALID_ARG, "n_idx_k_heads %d must be 1 or n_kv_heads %d", p->n_idx_k_heads,
+                    p->n_kv_heads);
+    const int gps = p->n_kv_heads / p->n_idx_k_heads;
+    if (gps > kMaxGroupsPerSeg || !pow2(gps))
+        return fail(MSA_ERR_UNSUPPORTED, "%d groups sharing one index-K head (supported: 1, 2, 4, 8)", gps);
+    if (p->head_dim != 64 && p->head_dim != 128) return fail(MSA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", p->head_dim);
+    const int row = p->idx_dim * elem_size(p->dtype);
+    if (p->idx_dim < 1 || (row != 64 && row != 128 && row != 256))
+        return fail(MSA_ERR_UNSUPPORTED, "idx_dim %d: an index-key row must be 64, 128 or 256 bytes", p->idx_dim);
+    if (!pow2(p->block_size) || p->block_size < 16 || p->block_size > 256)
+        return fail(MSA_ERR_UNSUPPORTED, "block_size %d (a power of two in [16, 256])", p->block_size);
+    if (p->top_k < 1) return fail(MSA_ERR_INVALID_ARG, "top_k %d < 1", p->top_k);
+    if (p->top_k > kMaxTopK) return fail(MSA_ERR_UNSUPPORTED, "top_k %d > %d", p->top_k, kMaxTopK);
+    if (p->max_seq_len < 1) return fail(MSA_ERR_INVALID_ARG, "max_seq_len %d < 1", p->max_seq_len);
+    if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale))
+        return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+    if (p->flags & ~(MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_DENSE))
+        return fail(MSA_ERR_INVALID_ARG, "unknown flags 0x%x", p->flags);
+    if (p->q_len < 1) return fail(MSA_ERR_INVALID_ARG, "q_len %d < 1", p->q_len);
+    if (mode == DECODE_ONLY && p->q_len != 1) return fail(MSA_ERR_INVALID_ARG, "decode entries take q_len = 1");
+    if (mode == PREFILL_ONLY || (mode == ANY_ROWS && p->q_len > 1)) {
+        if (p->q_start < 0 || (long long)p->q_start + p->q_len > p->max_seq_len)
+            return fail(MSA_ERR_INVALID_ARG, "prefill rows [%d, %d) outside max_seq_len %d", p->q_start,
+                        p->q_start + p->q_len, p->max_seq_len);
+    }
+    if (mode == DECODE_ONLY || (mode == ANY_ROWS && p->q_len == 1)) {
+        if (p->seq_lens == nullptr) return fail(MSA_ERR_INVALID_ARG, "seq_lens is NULL");
+    }
+    return MSA_OK;
+}
+
+msa_status_t check_ptr(const void *ptr, const char *name, bool nullable = false) {
+    if (ptr == nullptr) {
+        if (nullable) return MSA_OK;
+        return fail(MSA_ERR_INVALID_ARG, "%s is NULL", name);
+    }
+    if (!aligned16(ptr)) return fail(MSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return MSA_OK;
+}
+
+#define MSA_TRY(x)                          \
+    do {                                    \
+        msa_status_t st_ = (x);             \
+        if (st_ != MSA_OK) return st_;      \
+    } while (0)
+
+int nb_max_of(const msa_params_t &p) { return (p.max_seq_len + p.block_size - 1) / p.block_size; }
+
+}  // namespace
+
+int num_sms() {
+    int n = 0;
+    return check_device(&n) == MSA_OK ? n : 0;
+}
+
+DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm) {
+    DecodeWs L{};
+    L.n_cta = n_sm < 256 ? n_sm : 256;
+    if (L.n_cta < 1) L.n_cta = 1;
+    const int n_seg = p.batch * p.n_idx_k_heads, gps = p.n_kv_heads / p.n_idx_k_heads;
+    const int r = p.n_q_heads / p.n_kv_heads;
+    size_t off = kStatusBytes;
+    if (scan) {
+        L.seg_info = off;
+        off += round256((size_t)n_seg * sizeof(SegInfo));
+        const size_t cand = (size_t)n_seg * L.n_cta * gps * p.top_k * 4;
+        L.cand_s = off;
+        off += round256(cand);
+        L.cand_i = off;
+        off += round256(cand);
+    }
+    if (attend) {
+        if (p.flags & MSA_DENSE) {
+            const int nb = nb_max_of(p);
+            const long long want = 2LL * n_sm;
+            long long S = (want + (long long)p.batch * p.n_kv_heads - 1) / ((long long)p.batch * p.n_kv_heads);
+            if (S < 1) S = 1;
+            if (S > nb) S = nb;
+            L.blocks_per_split = (int)((nb + S - 1) / S);
+            L.S = (nb + L.blocks_per_split - 1) / L.blocks_per_split;
+        } else {
+            L.S = p.top_k;
+            L.blocks_per_split = 1;
+        }
+        const size_t parts = (size_t)p.batch * p.n_kv_heads * L.S * r;
+        L.part_o = off;
+        off += round256(parts * p.head_dim * 4);
+        L.part_lse = off;
+        off += round256(parts * 4);
+    }
+    L.total = off;
+    return L;
+}
+
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+const char *msa_last_error_string(void) { return g_err.c_str(); }
+
+const char *msa_status_string(msa_status_t s) {
+    switch (s) {
+        case MSA_OK: return "MSA_OK";
+        case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+        case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+        case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE";
+        case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+        case MSA_ERR_TIMEOUT: return "MSA_ERR_TIMEOUT";
+    }
+    return "unknown status";
+}
+
+size_t msa_workspace_size(const msa_params_t *p, int entry) {
+    int n_sm = 0;
+    switch (entry) {
+        case MSA_ENTRY_INDEX_SCORE:
+        case MSA_ENTRY_MAXPOOL_TOPK:
+            if (check_params(p, ANY_ROWS) != MSA_OK) return (size_t)-1;
+            return kStatusBytes;
+        case MSA_ENTRY_ATTN_DECODE:
+            if (check_params(p, DECODE_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
+            return decode_ws_layout(*p, false, true, n_sm).total;
+        case MSA_ENTRY_DECODE_FUSED:
+            if (check_params(p, DECODE_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
+            return decode_ws_layout(*p, true, true, n_sm).total;
+        case MSA_ENTRY_ATTN_PREFILL:
+        case MSA_ENTRY_PREFILL_INDEX_TOPK:
+            if (check_params(p, PREFILL_ONLY) != MSA_OK) return (size_t)-1;
+            return kStatusBytes;
+        default:
+            fail(MSA_ERR_INVALID_ARG, "unknown entry %d", entry);
+            return (size_t)-1;
+    }
+}
+
+msa_status_t msa_set_stage_events(void *const *events, int n_events) {
+    if (n_events == 0) {
+        g_n_stage_ev = 0;
+        return MSA_OK;
+    }
+    if (n_events != 4 || events == nullptr) return fail(MSA_ERR_INVALID_ARG, "n_events must be 0 or 4");
+    for (int i = 0; i < 4; ++i) {
+        if (events[i] == nullptr) return fail(MSA_ERR_INVALID_ARG, "event %d is NULL", i);
+        g_stage_ev[i] = (cudaEvent_t)events[i];
+    }
+    g_n_stage_ev = 4;
+    return MSA_OK;
+}
+
+static cudaError_t stage_mark(int i, cudaStream_t s) {
+    return g_n_stage_ev == 4 ? cudaEventRecord(g_stage_ev[i], s) : cudaSuccess;
+}
+
+msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t stream) {
+    if (ws == nullptr || status == nullptr) return fail(MSA_ERR_INVALID_ARG, "ws or status is NULL");
+    cudaError_t e = cudaMemcpyAsync(status, ws, sizeof(int), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    return MSA_OK;
+}
+
+msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream) {
+    if (ws == nullptr) return fail(MSA_ERR_INVALID_ARG, "ws is NULL");
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    return MSA_OK;
+}
+
+msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const void *k_idx, float *scores_out,
+                             void *ws, size_t ws_bytes, msa_stream_t stream) {
+    MSA_TRY(check_params(p, ANY_ROWS));
+    const int mode = p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX);
+    if (mode != MSA_SCORES_TOKEN && mode != MSA_SCORES_BLOCKMAX)
+        return fail(MSA_ERR_INVALID_ARG, "exactly one of MSA_SCORES_TOKEN / MSA_SCORES_BLOCKMAX must be set");
+    if (p->flags & MSA_DENSE) return fail(MSA_ERR_INVALID_ARG, "MSA_DENSE does not apply to index scores");
+    MSA_TRY(check_ptr(q_idx, "q_idx"));
+    MSA_TRY(check_ptr(k_idx, "k_idx"));
+    MSA_TRY(check_ptr(scores_out, "scores_out"));
+    MSA_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    if (p->q_len != 1)
+        return fail(MSA_ERR_UNSUPPORTED, "stored prefill index scores are not available; use msa_prefill_index_topk");
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int nb_max = nb_max_of(*p);
+    const long long n_out = (long long)p->batch * p->n_kv_heads * (mode == MSA_SCORES_TOKEN ? p->max_seq_len : nb_max);
+    cudaError_t e = launch_fill_neg_inf(scores_out, n_out, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fill");
+    ScanArgs a{};
+    a.q_idx = q_idx; a.k_idx = k_idx; a.seq_lens = p->seq_lens;
+    a.B = p->batch; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.di = p->idx_dim; a.Bk = p->block_size;
+    a.k = p->top_k; a.L_max = p->max_seq_len; a.nb_max = nb_max;
+    a.n_cta = decode_ws_layout(*p, true, false, n_sm).n_cta;
+    a.token_scores = mode == MSA_SCORES_TOKEN ? scores_out : nullptr;
+    a.block_scores = mode == MSA_SCORES_BLOCKMAX ? scores_out : nullptr;
+    a.status = reinterpret_cast<int *>(ws);
+    const int lpt = p->idx_dim * elem_size(p->dtype) / 16;
+    e = launch_decode_scan(a, p->dtype, lpt, p->n_kv_heads / p->n_idx_k_heads, s, false);
+    if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
+    return MSA_OK;
+}
+
+msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_in, int32_t *ids_out,
+                                    float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
+    MSA_TRY(check_params(p, ANY_ROWS));
+    if (p->flags & (MSA_SCORES_TOKEN | MSA_DENSE))
+        return fail(MSA_ERR_INVALID_ARG, "only MSA_SCORES_BLOCKMAX may be set for msa_block_maxpool_topk");
+    MSA_TRY(check_ptr(scores_in, "scores_in"));
+    MSA_TRY(check_ptr(ids_out, "ids_out"));
+    MSA_TRY(check_ptr(top_scores_out, "top_scores_out", true));
+    MSA_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    PoolTopkArgs a{};
+    a.scores = scores_in; a.seq_lens = p->seq_lens; a.ids_out = ids_out; a.top_scores_out = top_scores_out;
+    a.B = p->batch; a.q_len = p->q_len; a.q_start = p->q_start; a.G = p->n_kv_heads; a.Bk = p->block_size;
+    a.k = p->top_k; a.L_max = p->max_seq_len; a.nb_max = nb_max_of(*p);
+    a.is_block = (p->flags & MSA_SCORES_BLOCKMAX) != 0;
+    a.prefill = p->q_len > 1;
+    cudaError_t e = launch_pool_topk(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "pool/topk launch");
+    return MSA_OK;
+}
+
+static msa_status_t attend_decode(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
+                                  const int32_t *ids_in, bool from_scan, const DecodeWs &L, unsigned char *wsb,
+                                  void *o, int32_t *ids_out, float *lse, cudaStream_t s) {
+    AttnArgs a{};
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.seq_lens = p->seq_lens;
+    a.ids_in = ids_in;
+    if (from_scan) {
+        a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
+        a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
+        a.seg_info = reinterpret_cast<const SegInfo *>(wsb + L.seg_info);
+    }
+    a.n_cta = L.n_cta;
+    a.ids_out = ids_out;
+    a.part_o = reinterpret_cast<float *>(wsb + L.part_o);
+    a.part_lse = reinterpret_cast<float *>(wsb + L.part_lse);
+    a.B = p->batch; a.Hq = p->n_q_heads; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.D = p->head_dim;
+    a.Bk = p->block_size; a.k = p->top_k; a.L_max = p->max_seq_len; a.r = p->n_q_heads / p->n_kv_heads;
+    a.S = L.S; a.blocks_per_split = L.blocks_per_split; a.dense = (p->flags & MSA_DENSE) != 0;
+    a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+    a.status = reinterpret_cast<int *>(wsb);
+    cudaError_t e = launch_decode_attn(a, p->dtype, s, from_scan);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    if (from_scan && (e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    CombineArgs c{};
+    c.part_o = a.part_o; c.part_lse = a.part_lse; c.o = o; c.lse = lse;
+    c.B = p->batch; c.Hq = p->n_q_heads; c.G = p->n_kv_heads; c.D = p->head_dim; c.r = a.r; c.S = L.S;
+    e = launch_decode_combine(c, p->dtype, s, true);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    if (from_scan && (e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    return MSA_OK;
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
+                                    const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
+                                    msa_stream_t stream) {
+    MSA_TRY(check_params(p, DECODE_ONLY));
+    if (p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX))
+        return fail(MSA_ERR_INVALID_ARG, "score flags do not apply to attention");
+    const bool dense = (p->flags & MSA_DENSE) != 0;
+    MSA_TRY(check_ptr(q, "q"));
+    MSA_TRY(check_ptr(k_cache, "k_cache"));
+    MSA_TRY(check_ptr(v_cache, "v_cache"));
+    MSA_TRY(check_ptr(ids, "ids", dense));
+    MSA_TRY(check_ptr(o, "o"));
+    MSA_TRY(check_ptr(lse, "lse", true));
+    MSA_TRY(check_ptr(ws, "ws"));
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    const DecodeWs L = decode_ws_layout(*p, false, true, n_sm);
+    if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+    return attend_decode(p, q, k_cache, v_cache, dense ? nullptr : ids, false, L,
+                         reinterpret_cast<unsigned char *>(ws), o, nullptr, lse, (cudaStream_t)stream);
+}
+
+msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *q_idx, const void *k_cache,
+                              const void *v_cache, const void *k_idx, void *o, int32_t *ids_out, float *lse, void *ws,
+                              size_t ws_bytes, msa_stream_t stream) {
+    MSA_TRY(check_params(p, DECODE_ONLY));
+    if (p->flags != 0)
+        return fail(MSA_ERR_INVALID_ARG, "msa_decode_fused takes no flags (dense decode: msa_sparse_attn_decode + MSA_DENSE)");
+    MSA_TRY(check_ptr(q, "q"));
+    MSA_TRY(check_ptr(q_idx, "q_idx"));
+    MSA_TRY(check_ptr(k_cache, "k_cache"));
+    MSA_TRY(check_ptr(v_cache, "v_cache"));
+    MSA_TRY(check_ptr(k_idx, "k_idx"));
+    MSA_TRY(check_ptr(o, "o"));
+    MSA_TRY(check_ptr(ids_out, "ids_out", true));
+    MSA_TRY(check_ptr(lse, "lse", true));
+    MSA_TRY(check_ptr(ws, "ws"));
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    const DecodeWs L = decode_ws_layout(*p, true, true, n_sm);
+    if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+    unsigned char *wsb = reinterpret_cast<unsigned char *>(ws);
+    const cudaStream_t s = (cudaStream_t)stream;
+    ScanArgs a{};
+    a.q_idx = q_idx; a.k_idx = k_idx; a.seq_lens = p->seq_lens;
+    a.B = p->batch; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.di = p->idx_dim; a.Bk = p->block_size;
+    a.k = p->top_k; a.L_max = p->max_seq_len; a.nb_max = nb_max_of(*p);
+    a.n_cta = L.n_cta;
+    a.cand_s = reinterpret_cast<float *>(wsb + L.cand_s);
+    a.cand_i = reinterpret_cast<int *>(wsb + L.cand_i);
+    a.seg_info = reinterpret_cast<SegInfo *>(wsb + L.seg_info);
+    a.status = reinterpret_cast<int *>(wsb);
+    const int lpt = p->idx_dim * elem_size(p->dtype) / 16;
+    cudaError_t e = stage_mark(0, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    e = launch_decode_scan(a, p->dtype, lpt, p->n_kv_heads / p->n_idx_k_heads, s, false);
+    if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
+    if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    return attend_decode(p, q, k_cache, v_cache, nullptr, true, L, wsb, o, ids_out, lse, s);
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
+                                     const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
+                                     msa_stream_t stream) {
+    MSA_TRY(check_params(p, PREFILL_ONLY));
+    (void)q; (void)k_cache; (void)v_cache; (void)ids; (void)o; (void)lse; (void)ws; (void)ws_bytes; (void)stream;
+    return fail(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_prefill is not built yet");
+}
+
+msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, const void *k_idx, int32_t *ids_out,
+                                    float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
+    MSA_TRY(check_params(p, PREFILL_ONLY));
+    (void)q_idx; (void)k_idx; (void)ids_out; (void)top_scores_out; (void)ws; (void)ws_bytes; (void)stream;
+    return fail(MSA_ERR_UNSUPPORTED, "msa_prefill_index_topk is not built yet");
+}
+
+}  // extern "C"

@@ -1,0 +1,185 @@
+// Device-side building blocks shared by the MSA kernels (sm_100a only).
+//
+//  - bf16 <-> fp32 unpacking of 16-byte vectors,
+//  - mbarrier + cp.async.bulk (TMA bulk copy) helpers with bounded waits,
+//  - programmatic dependent launch (PDL) controls,
+//  - the selection order of TopK (higher score first, ties to the lower
+//    block id) and warp-cooperative sorted top-k lists.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msa_internal.h"
+
+namespace msa {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---------------------------------------------------------------- elements
+// A 16-byte vector of stored elements widened to fp32.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ static inline void unpack(const uint4 &u, float (&f)[4]) {
+        f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+        f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    // a bf16 is the high half of an IEEE fp32: widening is a shift / mask
+    __device__ static inline void unpack(const uint4 &u, float (&f)[8]) {
+        f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+        f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+        f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
+        f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+    }
+};
+
+__device__ inline float load_elem(const float *p) { return *p; }
+__device__ inline float load_elem(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ inline void store_elem(float *p, float v) { *p = v; }
+__device__ inline void store_elem(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+
+// ---------------------------------------------------------------- smem / mbarrier / bulk copy
+__device__ inline uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ inline void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ inline void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ inline bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ inline uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+// Wait for phase `parity` of an mbarrier for at most kWaitLimitNs.  On
+// timeout the workspace status word is set to MSA_ERR_TIMEOUT and false is
+// returned; the caller then stops issuing work and drains what it issued.
+__device__ inline bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (status) atomicExch(status, (int)MSA_ERR_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// L2 policy for data read exactly once per call (streamed caches).
+__device__ inline uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// TMA bulk copy global -> shared (contiguous bytes, 16-byte aligned, size a
+// multiple of 16), completion counted on `bar`.
+__device__ inline void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar,
+                                uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+// ---------------------------------------------------------------- PDL
+__device__ inline void pdl_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ inline void pdl_allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ inline void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------- selection order
+// TopK keeps the best blocks in the order: higher score first, then lower id.
+// Empty slots hold (-inf, -1) and lose to every finite score.
+__device__ inline bool better(float s1, int i1, float s2, int i2) {
+    return s1 > s2 || (s1 == s2 && (unsigned)i1 < (unsigned)i2);
+}
+
+// Warp-distributed sorted list of the k best (score, id) pairs, k <= 32:
+// lane i holds the i-th best.  (thr_s, thr_i) mirror slot k-1 in every lane
+// so that a losing candidate costs one comparison.
+struct WarpTopK {
+    float s; int id; float thr_s; int thr_i;
+    __device__ inline void reset() { s = -INFINITY; id = -1; thr_s = -INFINITY; thr_i = -1; }
+    // cs/ci must be warp-uniform.
+    __device__ inline void insert(float cs, int ci, int k, int lane) {
+        if (!better(cs, ci, thr_s, thr_i)) return;
+        const unsigned m = __ballot_sync(FULL, lane < k && better(cs, ci, s, id));
+        const int p = __ffs(m) - 1;
+        const float us = __shfl_up_sync(FULL, s, 1);
+        const int ui = __shfl_up_sync(FULL, id, 1);
+        if (lane == p) { s = cs; id = ci; }
+        else if (lane > p && lane < k) { s = us; id = ui; }
+        thr_s = __shfl_sync(FULL, s, k - 1);
+        thr_i = __shfl_sync(FULL, id, k - 1);
+    }
+};
+
+// Warp argmax of (s, i) under `better`; every lane receives the winner.
+__device__ inline void warp_best(float &s, int &i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float os = __shfl_xor_sync(FULL, s, off);
+        const int oi = __shfl_xor_sync(FULL, i, off);
+        if (better(os, oi, s, i)) { s = os; i = oi; }
+    }
+}
+
+// Merge of n_lists sorted lists (each `len` long, padded with (-inf, -1))
+// into the k best, by one warp: lane l owns lists l, l+32, ... (at most
+// kMaxOwnedLists each).  Lists live at ls[list * stride + j] / li[...].
+// Writes out_s/out_i[0..k) (padded with (-inf, -1)).  Ids must be unique.
+template <int kMaxOwned>
+__device__ inline void warp_merge_sorted_lists(const float *ls, const int *li, int n_lists, int len, int stride,
+                                               int k, float *out_s, int *out_i, int lane) {
+    int head[kMaxOwned];
+#pragma unroll
+    for (int o = 0; o < kMaxOwned; ++o) head[o] = 0;
+    for (int r = 0; r < k; ++r) {
+        float bs = -INFINITY; int bi = -1; int bo = -1;
+#pragma unroll
+        for (int o = 0; o < kMaxOwned; ++o) {
+            const int l = lane + 32 * o;
+            if (l < n_lists && head[o] < len) {
+                const float s = ls[(size_t)l * stride + head[o]];
+                const int i = li[(size_t)l * stride + head[o]];
+                if (i >= 0 && better(s, i, bs, bi)) { bs = s; bi = i; bo = o; }
+            }
+        }
+        float ws = bs; int wi = bi;
+        warp_best(ws, wi);
+        if (wi >= 0 && wi == bi) {
+#pragma unroll
+            for (int o = 0; o < kMaxOwned; ++o) if (o == bo) head[o] += 1;
+        }
+        if (lane == 0) { out_s[r] = ws; out_i[r] = wi; }
+    }
+}
+
+}  // namespace msa

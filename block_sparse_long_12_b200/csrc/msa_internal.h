@@ -1,0 +1,108 @@
+// Internal declarations shared by the MSA translation units (host + device).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+// Bounded device-side waits give up after this long and report MSA_ERR_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+constexpr int kMaxBatch = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxGroupsPerSeg = 8;   // n_kv_heads / n_idx_k_heads handled by one index-K stream
+constexpr int kMaxPiecesPerSeg = 256; // lists merged per (segment, group) by one warp (8 per lane)
+constexpr size_t kStatusBytes = 256;  // workspace head: device status word + padding
+
+// ---- decode index scan (Step 1 for decode): persistent, 1 CTA per SM
+constexpr int kScanWarps = 8;
+constexpr int kScanStages = 3;          // per-warp ring depth
+constexpr int kScanChunkBytes = 8192;   // bytes of index keys per bulk copy
+
+// ---- decode sparse attention (Step 2 for decode)
+constexpr int kAttnThreads = 256;
+
+// A segment is the index-K stream of one (sequence b, index-K head): blocks
+// 0..nb_b-1 of k_idx[b, hik].  The scan splits the concatenation of all
+// segments evenly over its CTAs; a CTA's share of one segment is a piece.
+struct SegInfo {
+    int first_cta;  // CTA holding the segment's first block (-1: empty segment)
+    int n_pieces;   // CTAs that touched it
+};
+
+struct ScanArgs {
+    const void *q_idx;
+    const void *k_idx;
+    const int *seq_lens;
+    int B, G, Hik, di, Bk, k, L_max, nb_max;
+    int n_cta;
+    float *cand_s;  // [n_seg, n_cta, G/Hik, k] per-piece sorted top-k (nullable)
+    int *cand_i;
+    SegInfo *seg_info;     // [n_seg] (written by CTA 0 when cand_s != nullptr)
+    float *token_scores;   // [B, 1, G, L_max] (nullable)
+    float *block_scores;   // [B, 1, G, nb_max] (nullable)
+    int *status;
+};
+
+struct AttnArgs {
+    const void *q;
+    const void *k_cache;
+    const void *v_cache;
+    const int *seq_lens;
+    const int *ids_in;         // [B, 1, G, k] given selection (nullable)
+    const float *cand_s;       // candidates of the scan when ids_in == nullptr
+    const int *cand_i;
+    const SegInfo *seg_info;
+    int n_cta;                 // scan grid size (candidate stride)
+    int *ids_out;              // nullable
+    float *top_scores_out;     // nullable
+    float *part_o;             // [B, G, S, r, D] fp32, normalised per split
+    float *part_lse;           // [B, G, S, r] log2-domain normaliser
+    int B, Hq, G, Hik, D, Bk, k, L_max, r;
+    int S, blocks_per_split, dense;
+    float scale_log2;          // softmax_scale * log2(e)
+    int *status;
+};
+
+struct CombineArgs {
+    const float *part_o;
+    const float *part_lse;
+    void *o;
+    float *lse;                // nullable, natural log
+    int B, Hq, G, D, r, S;
+};
+
+struct PoolTopkArgs {
+    const float *scores;       // token [rows, L_max] or block [rows, nb_max]
+    const int *seq_lens;
+    int32_t *ids_out;
+    float *top_scores_out;
+    int B, q_len, q_start, G, Bk, k, L_max, nb_max, is_block, prefill;
+};
+
+struct FillArgs {
+    float *scores;
+    long long n;
+};
+
+// Workspace layout of the decode entries (offsets in bytes from ws).
+struct DecodeWs {
+    size_t seg_info, cand_s, cand_i, part_o, part_lse, total;
+    int n_cta, S, blocks_per_split;
+};
+DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);
+
+// launchers (return cudaError_t of the launch)
+cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);
+cudaError_t launch_decode_scan(const ScanArgs &a, int dtype, int lpt, int gps, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_combine(const CombineArgs &a, int dtype, cudaStream_t s, bool pdl);
+cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace msa

@@ -1,0 +1,208 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) MiniMax Sparse Attention hot path.
+ *
+ * The method (page "MiniMax wird duenn: M3-Attention anhand eines einzigen
+ * Diagramms entschluesselt", atlascloud.ai, section 1 and Figure 1) is a GQA
+ * attention block in two steps:
+ *   Step 1, index branch: each KV group g has one small index query q_idx;
+ *     every cached token j carries an index key k_idx[j]; token scores
+ *     s_j = q_idx . k_idx[j] are reduced per fixed block of block_size tokens
+ *     by their maximum ("Block Max Pool"), and TopK keeps the top_k blocks of
+ *     the group.
+ *   Step 2, sparse branch: every query head of the group (contiguous heads:
+ *     head h belongs to group h / (n_q_heads / n_kv_heads)) runs exact softmax
+ *     attention over only the selected blocks of the real, uncompressed K/V.
+ *
+ * Readings taken where the page is silent (its formulas were lost):
+ *   - index score: raw dot product, no scale, no activation, fp32 accumulate;
+ *   - causality: a query at position pos sees tokens 0..pos; a block is
+ *     eligible if it holds any visible token, its score is the max over its
+ *     visible tokens only, and attention masks keys after pos;
+ *   - decode: pos = seq_lens[b] - 1 (the new token's K/V and index key are
+ *     already in the cache); prefill chunk: pos = q_start + t;
+ *   - top-k order: higher score first, ties to the lower block id; with fewer
+ *     than top_k valid blocks all are taken and ids are padded with -1;
+ *   - index-K head of group g: g mod n_idx_k_heads (1 shared head, or one per
+ *     KV group);
+ *   - softmax: z = softmax_scale * q . k, no bias, sink or soft-cap.
+ *
+ * Layouts (all contiguous, row-major, element type = params.dtype):
+ *   q      [B, q_len, n_q_heads, head_dim]
+ *   q_idx  [B, q_len, G, idx_dim]                       G = n_kv_heads
+ *   k, v   [B, n_kv_heads, max_seq_len, head_dim]       (caches)
+ *   k_idx  [B, n_idx_k_heads, max_seq_len, idx_dim]     (index-key cache)
+ *   ids    int32 [B, q_len, G, top_k]
+ *   o      [B, q_len, n_q_heads, head_dim]               (params.dtype)
+ *   lse    fp32 [B, q_len, n_q_heads]   natural-log softmax normaliser
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are caller-owned device memory, 16-byte aligned.
+ *     The library never allocates, frees or synchronises: work is enqueued on
+ *     `stream` and returns immediately.
+ *   - Scratch memory comes from the caller: `ws` of at least
+ *     msa_workspace_size(params, entry) bytes (256-byte aligned).  Each call
+ *     overwrites the workspace; calls that share a workspace must not overlap.
+ *   - Arguments are checked before anything is enqueued; on error nothing is
+ *     launched and the call returns the status (text: msa_last_error_string).
+ *   - A CUDA launch error returns MSA_ERR_CUDA.  Devices other than
+ *     compute capability 10.0 return MSA_ERR_UNSUPPORTED.
+ *   - seq_lens is a device pointer; values outside [1, max_seq_len] are out of
+ *     contract: kernels clamp them and never read outside the caches.
+ *   - Non-finite inputs are out of contract (results undefined, no fault).
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+typedef struct CUstream_st *msa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misalignment        */
+    MSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (dims, dtype, GPU)  */
+    MSA_ERR_WORKSPACE = 3,   /* ws_bytes < msa_workspace_size(...)           */
+    MSA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed          */
+    MSA_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out            */
+} msa_status_t;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype_t;
+
+/* params.flags */
+enum {
+    MSA_SCORES_TOKEN = 1,    /* token scores s_j  [B, q_len, G, max_seq_len]  */
+    MSA_SCORES_BLOCKMAX = 2, /* block scores S_n  [B, q_len, G, nb_max]       */
+    MSA_DENSE = 8            /* attend every visible block (plain GQA), ids unused */
+};
+
+/* entry ids for msa_workspace_size */
+enum {
+    MSA_ENTRY_INDEX_SCORE = 0,
+    MSA_ENTRY_MAXPOOL_TOPK = 1,
+    MSA_ENTRY_ATTN_DECODE = 2,
+    MSA_ENTRY_ATTN_PREFILL = 3,
+    MSA_ENTRY_DECODE_FUSED = 4,
+    MSA_ENTRY_PREFILL_INDEX_TOPK = 5
+};
+
+typedef struct {
+    int batch;            /* B >= 1                                            */
+    int n_q_heads;        /* multiple of n_kv_heads                            */
+    int n_kv_heads;       /* G, the number of GQA groups                      */
+    int n_idx_k_heads;    /* 1 or n_kv_heads                                   */
+    int head_dim;         /* D: 64 or 128                                      */
+    int idx_dim;          /* di: idx_dim * sizeof(elem) in {64, 128, 256} bytes */
+    int block_size;       /* Bk: 16..256, power of two                         */
+    int top_k;            /* 1..32                                             */
+    int q_len;            /* decode entries: 1; prefill: chunk length          */
+    int q_start;          /* prefill: absolute position of query row 0         */
+    int max_seq_len;      /* Lmax, the caches' token stride                    */
+    const int32_t *seq_lens; /* device int32[B]: cached length incl. current token(s) */
+    float softmax_scale;  /* > 0; 1/sqrt(head_dim) in the usual attention      */
+    int dtype;            /* msa_dtype_t; prefill entries take MSA_BF16 only   */
+    int flags;            /* MSA_SCORES_* / MSA_DENSE                          */
+} msa_params_t;
+
+/*
+ * Step 1a (+1b): index scores.  Exactly one of MSA_SCORES_TOKEN or
+ * MSA_SCORES_BLOCKMAX must be set in params->flags.
+ *   TOKEN:    scores_out [B, q_len, G, max_seq_len] fp32, s_j for j <= pos,
+ *             -inf for j > pos.
+ *   BLOCKMAX: scores_out [B, q_len, G, nb_max] fp32 with
+ *             nb_max = ceil(max_seq_len / block_size); S_n for visible blocks,
+ *             -inf for blocks after pos.
+ * Decode (q_len == 1) streams k_idx once per index-K head.
+ */
+MSA_API msa_status_t msa_index_score(const msa_params_t *params, const void *q_idx, const void *k_idx,
+                             float *scores_out, void *ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Step 1b + 1c: block max pool and TopK from stored scores.  scores_in holds
+ * token scores ([B, q_len, G, max_seq_len], default) or, with
+ * MSA_SCORES_BLOCKMAX, block scores ([B, q_len, G, nb_max]); only entries of
+ * visible tokens/blocks are read.  ids_out [B, q_len, G, top_k] int32 in
+ * selection order; top_scores_out (nullable) the matching fp32 scores
+ * (-inf for padding).
+ */
+MSA_API msa_status_t msa_block_maxpool_topk(const msa_params_t *params, const float *scores_in,
+                                    int32_t *ids_out, float *top_scores_out, void *ws,
+                                    size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Step 2 for decode (q_len == 1): o = softmax attention of each query head
+ * over the keys j <= pos of its group's listed blocks (ids entries of -1 are
+ * skipped; with MSA_DENSE every visible block, ids may be NULL).
+ * lse (nullable) receives the log normaliser.
+ */
+MSA_API msa_status_t msa_sparse_attn_decode(const msa_params_t *params, const void *q, const void *k_cache,
+                                    const void *v_cache, const int32_t *ids, void *o, float *lse,
+                                    void *ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * Step 2 for a causal prefill chunk: query rows t = 0..q_len-1 at positions
+ * q_start + t, each with its own list ids[b, t, g, :].  bf16 only.
+ */
+MSA_API msa_status_t msa_sparse_attn_prefill(const msa_params_t *params, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *ids, void *o, float *lse,
+                                     void *ws, size_t ws_bytes, msa_stream_t stream);
+
+/*
+ * One decode step, Steps 1 and 2 fused into back-to-back kernels on `stream`
+ * (the block list never leaves the device).  ids_out and lse are nullable.
+ */
+MSA_API msa_status_t msa_decode_fused(const msa_params_t *params, const void *q, const void *q_idx,
+                              const void *k_cache, const void *v_cache, const void *k_idx, void *o,
+                              int32_t *ids_out, float *lse, void *ws, size_t ws_bytes,
+                              msa_stream_t stream);
+
+/*
+ * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,
+ * block max pool and TopK in the epilogue; scores are never stored.
+ * ids_out [B, q_len, G, top_k]; top_scores_out nullable.  bf16 only.
+ */
+MSA_API msa_status_t msa_prefill_index_topk(const msa_params_t *params, const void *q_idx, const void *k_idx,
+                                    int32_t *ids_out, float *top_scores_out, void *ws, size_t ws_bytes,
+                                    msa_stream_t stream);
+
+/*
+ * Measurement hook (not part of the method): while set, msa_decode_fused
+ * records events[0] before its first kernel and events[i] after its i-th
+ * kernel (1 = index scan, 2 = sparse attention, 3 = split combine) on the
+ * call's stream, so a caller can time each kernel with cudaEventElapsedTime.
+ * events are cudaEvent_t handles owned by the caller; n_events must be 0
+ * (unset) or 4.  Per calling thread.  Recording between the kernels removes
+ * their launch overlap, so time whole steps without it.
+ */
+MSA_API msa_status_t msa_set_stage_events(void *const *events, int n_events);
+
+/* Scratch bytes an entry needs for these params (0 if none); queries the
+ * current device.  Returns (size_t)-1 for invalid params. */
+MSA_API size_t msa_workspace_size(const msa_params_t *params, int entry);
+
+/* Text of the last error on the calling thread ("" if none). */
+MSA_API const char *msa_last_error_string(void);
+
+/* Fixed text of a status code. */
+MSA_API const char *msa_status_string(msa_status_t status);
+
+/* Device status word kept in a workspace (first 4 bytes): MSA_OK, or
+ * MSA_ERR_TIMEOUT after a bounded wait ran out.  Copies it to *status after
+ * synchronising `stream`; msa_clear_device_status resets it asynchronously. */
+MSA_API msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t stream);
+MSA_API msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H */

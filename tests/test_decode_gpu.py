@@ -1,0 +1,221 @@
+"""GPU parity of the decode path (C ABI -> CUDA kernels) against the fp64 oracle.
+
+Step 1 (index score, block max pool, TopK) and Step 2 (sparse attention of
+every head of the group over the group's selected blocks), page "MiniMax wird
+duenn" (atlascloud.ai), section 1.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_12_b200.inputs import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+from parity import compare_decode, oracle_params, to_np  # noqa: E402
+
+
+def _api():
+    from block_sparse_long_12_b200 import api
+    return api
+
+
+def run_fused(inp, w):
+    api = _api()
+    o, ids, lse = api.decode(inp["q"], inp["q_idx"], inp["k"], inp["v"], inp["k_idx"], inp["seq_lens"],
+                             block_size=w.block_size, top_k=w.top_k)
+    torch.cuda.synchronize()
+    return o, ids, lse
+
+
+def small(name="decode_b8_ctx128k_ragged", **kw):
+    base = dict(batch=3, max_seq_len=5000, min_seq_len=1, n_q_heads=16, n_kv_heads=4, n_idx_k_heads=4, head_dim=128,
+                idx_dim=64, block_size=64, top_k=8, hot_blocks=6, seed=11)
+    base.update(kw)
+    return WORKLOADS[name].scaled(**base)
+
+
+def test_tiny_fp32_decode_full():
+    """4096-token fp32 decode, 4 query heads on 1 KV head, k = 8 of 64 blocks."""
+    w = WORKLOADS["decode_fp32_ctx4k"]
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    res = compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+    assert res["err_o"] <= 1e-4
+
+
+@pytest.mark.parametrize("case", [
+    dict(),                                                           # ragged, partial last blocks
+    dict(dtype="f32", idx_dim=32, head_dim=64),                        # fp32, D 64
+    dict(n_idx_k_heads=1, hot_blocks=0),                               # one index-K head shared by all groups
+    dict(n_kv_heads=8, n_q_heads=8, n_idx_k_heads=1, hot_blocks=0),    # 8 groups on one index-K stream, r = 1
+    dict(block_size=16, top_k=32, max_seq_len=3000),                   # small blocks, largest k
+    dict(block_size=256, top_k=1, max_seq_len=9000),                   # big blocks, k = 1
+    dict(block_size=128, top_k=20, max_seq_len=1500, min_seq_len=1),  # fewer valid blocks than k: -1 padding
+    dict(n_q_heads=24, n_kv_heads=4, n_idx_k_heads=4),                 # group size 6 (padded to 8)
+    dict(n_q_heads=64, n_kv_heads=4, n_idx_k_heads=4, head_dim=64),    # group size 16
+    dict(idx_dim=128, dtype="bf16"),                                   # 256-byte index rows
+    dict(idx_dim=32, dtype="bf16"),                                    # 64-byte index rows
+    dict(batch=9, max_seq_len=700, min_seq_len=1, seed=5),             # many short sequences
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()) or "base")
+def test_decode_fused_variants(case):
+    w = small(**case)
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+
+
+def test_decode_exact_lengths_edges():
+    """Lengths 1, Bk-1, Bk, Bk+1 and Lmax in one batch."""
+    w = small(batch=5, max_seq_len=1000, block_size=64, top_k=4, hot_blocks=0)
+    inp = make_inputs(w, device="cuda")
+    inp["seq_lens"].copy_(torch.tensor([1, 63, 64, 65, 1000], dtype=torch.int32))
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=64, top_k=4), o, ids, lse)
+    idn = ids.cpu().numpy()
+    assert idn[0, 0, :, 0].tolist() == [0] * 4 and (idn[0, 0, :, 1:] == -1).all()
+
+
+def test_index_scores_and_pool_topk():
+    """Stored token / block scores, then the stand-alone pool + TopK entry."""
+    api = _api()
+    w = small(dtype="bf16", hot_blocks=4)
+    inp = make_inputs(w, device="cuda")
+    x = to_np(inp)
+    p = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
+    tok = api.index_scores(inp["q_idx"], inp["k_idx"], inp["seq_lens"], n_kv_heads=w.n_kv_heads,
+                           block_size=w.block_size, mode="token")
+    blk = api.index_scores(inp["q_idx"], inp["k_idx"], inp["seq_lens"], n_kv_heads=w.n_kv_heads,
+                           block_size=w.block_size, mode="block")
+    torch.cuda.synchronize()
+    tok_n, blk_n = tok.cpu().numpy(), blk.cpu().numpy()
+    for b in range(w.batch):
+        L = int(x["seq_lens"][b])
+        for g in range(w.n_kv_heads):
+            s = oracle.token_scores(p, x["q_idx"], x["k_idx"], b, 0, g, L - 1)
+            S = oracle.block_scores(p, s, L - 1)
+            scale = np.abs(s).max() + 1.0
+            assert np.abs(tok_n[b, 0, g, :L] - s).max() <= 1e-5 * scale
+            assert np.isneginf(tok_n[b, 0, g, L:]).all()
+            assert np.abs(blk_n[b, 0, g, :len(S)] - S).max() <= 1e-5 * scale
+            assert np.isneginf(blk_n[b, 0, g, len(S):]).all()
+    # pool + TopK from the stored fp32 scores: the oracle on the same fp32 values must agree exactly
+    for is_block, sc in ((False, tok), (True, blk)):
+        ids, ts = api.pool_topk(sc, inp["seq_lens"], block_size=w.block_size, top_k=w.top_k,
+                                max_seq_len=w.max_seq_len, is_block=is_block)
+        torch.cuda.synchronize()
+        ids_n, ts_n = ids.cpu().numpy(), ts.cpu().numpy()
+        for b in range(w.batch):
+            L = int(x["seq_lens"][b])
+            for g in range(w.n_kv_heads):
+                S = oracle.block_scores(p, tok_n[b, 0, g, :L].astype(np.float64), L - 1)
+                ref_ids, ref_sc, _, _ = oracle.topk(p, S)
+                assert ids_n[b, 0, g].tolist() == ref_ids.tolist()
+                np.testing.assert_array_equal(ts_n[b, 0, g][ref_ids >= 0], ref_sc[ref_ids >= 0].astype(np.float32))
+
+
+def test_pool_topk_prefill_rows():
+    """The stand-alone TopK entry on prefill rows (pos = q_start + t) from stored token scores."""
+    api = _api()
+    B, T, G, L, bk, k = 1, 40, 2, 300, 16, 5
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    sc = torch.randn(B, T, G, L, device="cuda", generator=gen).round(decimals=1)  # many exact ties
+    ids, ts = api.pool_topk(sc, None, block_size=bk, top_k=k, max_seq_len=L, is_block=False, q_start=200)
+    torch.cuda.synchronize()
+    p = oracle.Params(B, G, G, G, 64, 32, bk, k, T, 200, L, "f32", 0.125, prefill=True)
+    scn, idn = sc.cpu().numpy(), ids.cpu().numpy()
+    for t in range(T):
+        pos = 200 + t
+        for g in range(G):
+            S = oracle.block_scores(p, scn[0, t, g, :pos + 1].astype(np.float64), pos)
+            assert idn[0, t, g].tolist() == oracle.topk(p, S)[0].tolist()
+
+
+def test_attend_decode_given_ids_and_dense():
+    api = _api()
+    w = small(batch=4, max_seq_len=3000, top_k=6, hot_blocks=0)
+    inp = make_inputs(w, device="cuda")
+    x = to_np(inp)
+    gen = np.random.default_rng(5)
+    ids = np.full((w.batch, 1, w.n_kv_heads, w.top_k), -1, np.int32)
+    for b in range(w.batch):
+        nb = -(-int(x["seq_lens"][b]) // w.block_size)
+        for g in range(w.n_kv_heads):
+            m = min(nb, int(gen.integers(1, w.top_k + 1)))
+            ids[b, 0, g, :m] = gen.choice(nb, m, replace=False)
+            gen.shuffle(ids[b, 0, g])  # -1 entries anywhere in the list
+    o, lse = api.attend_decode(inp["q"], inp["k"], inp["v"], torch.from_numpy(ids).cuda(), inp["seq_lens"],
+                               block_size=w.block_size, top_k=w.top_k)
+    torch.cuda.synchronize()
+    p = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
+    rows = [(b, 0) for b in range(w.batch)]
+    ref = oracle.msa_rows(p, x["seq_lens"], x["q"], x["q_idx"], x["k"], x["v"], x["k_idx"], rows,
+                          ids_in=ids[:, 0])
+    assert np.abs(o.float().cpu().numpy()[:, 0] - ref["o"]).max() <= 2e-2
+    assert np.abs(lse.cpu().numpy()[:, 0] - ref["lse"]).max() <= 1e-3
+    od, lsed = api.attend_decode(inp["q"], inp["k"], inp["v"], None, inp["seq_lens"], block_size=w.block_size,
+                                 top_k=w.top_k, dense=True)
+    torch.cuda.synchronize()
+    pd = oracle_params(x, block_size=w.block_size, top_k=w.top_k, dense=True)
+    refd = oracle.msa_rows(pd, x["seq_lens"], x["q"], x["q_idx"], x["k"], x["v"], x["k_idx"], rows)
+    assert np.abs(od.float().cpu().numpy()[:, 0] - refd["o"]).max() <= 2e-2
+    assert np.abs(lsed.cpu().numpy()[:, 0] - refd["lse"]).max() <= 1e-3
+
+
+def test_dense_equals_sparse_when_k_covers_all():
+    """With k >= number of blocks, MSA decode equals the dense GQA decode (both GPU paths)."""
+    api = _api()
+    w = small(batch=2, max_seq_len=1024, block_size=64, top_k=16, hot_blocks=0)
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w)
+    od, lsed = api.attend_decode(inp["q"], inp["k"], inp["v"], None, inp["seq_lens"], block_size=64, top_k=16,
+                                 dense=True)
+    torch.cuda.synchronize()
+    assert (o.float() - od.float()).abs().max().item() <= 2e-2
+    assert (lse - lsed).abs().max().item() <= 1e-4
+
+
+def test_repeat_calls_same_workspace():
+    """The workspace is rewritten by each call: two calls give identical results."""
+    api = _api()
+    w = small()
+    inp = make_inputs(w, device="cuda")
+    p = api.params_from(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], block_size=w.block_size, top_k=w.top_k,
+                        seq_lens=inp["seq_lens"])
+    ws = api.workspace(p, api.MSA_ENTRY_DECODE_FUSED, "cuda")
+    a = api.decode(inp["q"], inp["q_idx"], inp["k"], inp["v"], inp["k_idx"], inp["seq_lens"],
+                   block_size=w.block_size, top_k=w.top_k, ws=ws)
+    a = [t.clone() for t in a]
+    b = api.decode(inp["q"], inp["q_idx"], inp["k"], inp["v"], inp["k_idx"], inp["seq_lens"],
+                   block_size=w.block_size, top_k=w.top_k, ws=ws)
+    torch.cuda.synchronize()
+    for t1, t2 in zip(a, b):
+        assert torch.equal(t1, t2)
+    from block_sparse_long_12_b200 import _lib
+    assert _lib.msa_get_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m"])
+def test_full_size_decode(name):
+    """The benchmark workloads at full size, checked against the oracle on every (sequence, group)."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    hot = inp["hot"].cpu().numpy()
+    del inp
+    torch.cuda.empty_cache()
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+    # planted data: every selected block is hot
+    idn = ids.cpu().numpy()
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            assert set(idn[b, 0, g].tolist()) <= set(hot[b, g % w.n_idx_k_heads].tolist())
