@@ -5,16 +5,20 @@
 // Q4/Q5/Q6 -> I2) and attends over only those blocks of the full, real K/V
 // cache, so one group loads one set of KV blocks for all its heads.
 //
-// Grid (split s, group g, sequence b).  A CTA first obtains the group's list
-// -- merging the scan's per-piece candidate lists (fused decode) or reading
-// a given ids tensor -- then streams the K/V tiles of its share of the
-// blocks through a two-stage TMA bulk-copy ring and keeps an online softmax
-// for all r heads of the group: scores with one warp per key (lanes split
-// the head dimension, a reduce-scatter butterfly finishes the r dot
-// products), then per-head max/exp2/sum, then P.V with each thread owning a
-// few output elements.  Splits write normalised partial outputs and their
-// log2 normalisers; the combine kernel merges them (log-sum-exp).  With
-// MSA_DENSE the splits cover every visible block: plain GQA decode.
+// decode_select_kernel finishes Step 1: one CTA per (sequence, group) stages
+// the scan's per-piece sorted candidate lists in shared memory and merges
+// them into the group's final TopK list.
+//
+// decode_attn_kernel, grid (split s, group g, sequence b): a CTA reads the
+// group's list, streams the K/V tiles of its share of the blocks through a
+// two-stage TMA bulk-copy ring and keeps an online softmax for all r heads
+// of the group: scores with one warp per key (lanes split the head
+// dimension, a reduce-scatter butterfly finishes the r dot products), then
+// per-head max/exp2/sum, then P.V with each thread owning a few output
+// elements.  Each split writes a normalised partial output and its log2
+// normaliser; the last split of a group to finish (atomic arrival count)
+// merges them by log-sum-exp into the output.  With MSA_DENSE the splits
+// cover every visible block: plain GQA decode.
 #include "msa_device.cuh"
 
 namespace msa {
@@ -136,27 +140,9 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const int pos = L - 1;
     const int nb = (L + a.Bk - 1) / a.Bk;
 
-    pdl_wait_prior_grid();  // the scan's candidates are complete from here on
+    pdl_wait_prior_grid();  // the selection is complete from here on
     pdl_allow_next_grid();
-
-    if (!a.dense) {
-        if (a.ids_in != nullptr) {
-            if (tid < a.k) sel_i[tid] = a.ids_in[((size_t)b * a.G + g) * a.k + tid];
-        } else if (w == 0) {
-            const int gps = a.G / a.Hik;
-            const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
-            const SegInfo si = a.seg_info[seg];
-            const size_t base = ((size_t)seg * a.n_cta * gps + gl) * a.k;
-            warp_merge_sorted_lists<kMaxPiecesPerSeg / 32>(a.cand_s + base, a.cand_i + base, si.n_pieces, a.k,
-                                                           gps * a.k, a.k, sel_s, sel_i, lane);
-            __syncwarp();
-            if (s == 0) {
-                if (a.ids_out != nullptr && lane < a.k) a.ids_out[((size_t)b * a.G + g) * a.k + lane] = sel_i[lane];
-                if (a.top_scores_out != nullptr && lane < a.k)
-                    a.top_scores_out[((size_t)b * a.G + g) * a.k + lane] = sel_s[lane];
-            }
-        }
-    }
+    if (!a.dense && tid < a.k) sel_i[tid] = a.ids_in[((size_t)b * a.G + g) * a.k + tid];
     __syncthreads();
 
     // this split's blocks: list positions [j0, j1)
@@ -297,7 +283,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     }
 
     // normalised partial output and log2 normaliser of this split
-    const size_t split = ((size_t)b * a.G + g) * a.S + s;
+    const size_t bg = (size_t)b * a.G + g;
+    const size_t split = bg * a.S + s;
     if (c_live) {
         const float l = l_s[ch];
         const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -309,41 +296,86 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
         const float l = l_s[tid];
         a.part_lse[split * r + tid] = l > 0.f ? m_s[tid] + log2f(l) : -INFINITY;
     }
+
+    // the last split of (b, g) to arrive merges all splits
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) sel_s[0] = (atomicAdd(&a.counters[bg], 1) == a.S - 1) ? 1.f : 0.f;
+    __syncthreads();
+    if (sel_s[0] == 0.f) return;
+    __threadfence();
+    float *wgt = p_s;  // [S][r] merge weights (S <= max(k, kMaxSplits))
+    for (int i = tid; i < a.S * r; i += kAttnThreads) wgt[i] = __ldcg(a.part_lse + bg * a.S * r + i);
+    __syncthreads();
+    if (tid < r) {
+        float M = -INFINITY;
+        for (int j = 0; j < a.S; ++j) M = fmaxf(M, wgt[j * r + tid]);
+        float den = 0.f;
+        for (int j = 0; j < a.S; ++j) {
+            const float e = M > -INFINITY ? exp2f(wgt[j * r + tid] - M) : 0.f;
+            wgt[j * r + tid] = e;
+            den += e;
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int j = 0; j < a.S; ++j) wgt[j * r + tid] *= inv;
+        if (a.lse != nullptr)
+            a.lse[(size_t)b * a.Hq + (size_t)g * r + tid] =
+                den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+    T *o = reinterpret_cast<T *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
+    const float *po = a.part_o + bg * a.S * r * D;
+    for (int f = tid; f < r * D; f += kAttnThreads) {
+        const int h = f / D;
+        float num = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < a.S; ++j) num = fmaf(wgt[j * r + h], __ldcg(po + ((size_t)j * r) * D + f), num);
+        store_elem(o + f, num);
+    }
+    if (tid == 0) a.counters[bg] = 0;  // ready for the next call
 }
 
-template <typename T>
-__global__ void __launch_bounds__(256) decode_combine_kernel(const CombineArgs a) {
-    const int g = blockIdx.x, b = blockIdx.y;
+// Final TopK of a group from the scan's per-piece sorted lists (staged in
+// shared memory), written to the selection buffer and the optional outputs.
+__global__ void __launch_bounds__(256) decode_select_kernel(const SelectArgs a) {
+    extern __shared__ __align__(16) unsigned char sm_raw[];
+    float *ls = reinterpret_cast<float *>(sm_raw);
+    int *li = reinterpret_cast<int *>(ls + (size_t)a.n_cta * a.k);
+    float *out_s = reinterpret_cast<float *>(li + (size_t)a.n_cta * a.k);
+    int *out_i = reinterpret_cast<int *>(out_s + 32);
+    const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
     pdl_wait_prior_grid();
-    const size_t base = ((size_t)b * a.G + g) * a.S;
-    for (int f = threadIdx.x; f < a.r * a.D; f += blockDim.x) {
-        const int h = f / a.D, d = f % a.D;
-        float M = -INFINITY;
-        for (int s = 0; s < a.S; ++s) M = fmaxf(M, a.part_lse[(base + s) * a.r + h]);
-        float num = 0.f, den = 0.f;
-        if (M > -INFINITY) {
-            for (int s = 0; s < a.S; ++s) {
-                const float ls = a.part_lse[(base + s) * a.r + h];
-                if (ls == -INFINITY) continue;
-                const float wgt = exp2f(ls - M);
-                den += wgt;
-                num = fmaf(wgt, a.part_o[((base + s) * a.r + h) * a.D + d], num);
-            }
-        }
-        const int hq = g * a.r + h;
-        T *o = reinterpret_cast<T *>(a.o) + ((size_t)b * a.Hq + hq) * a.D + d;
-        store_elem(o, den > 0.f ? num / den : 0.f);
-        if (a.lse != nullptr && d == 0)
-            a.lse[(size_t)b * a.Hq + hq] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+    pdl_allow_next_grid();
+    const int gps = a.G / a.Hik;
+    const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
+    const SegInfo si = a.seg_info[seg];
+    const int n = si.n_pieces * a.k;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const size_t src = (((size_t)seg * a.n_cta + i / a.k) * gps + gl) * a.k + i % a.k;
+        ls[i] = a.cand_s[src];
+        li[i] = a.cand_i[src];
     }
+    __syncthreads();
+    if (tid < 32) {
+        warp_merge_sorted_lists<kMaxPiecesPerSeg / 32>(ls, li, si.n_pieces, a.k, a.k, a.k, out_s, out_i, tid);
+        __syncwarp();
+        if (tid < a.k) {
+            const size_t o = ((size_t)b * a.G + g) * a.k + tid;
+            a.sel_ids[o] = out_i[tid];
+            if (a.ids_out != nullptr) a.ids_out[o] = out_i[tid];
+            if (a.top_scores_out != nullptr) a.top_scores_out[o] = out_s[tid];
+        }
+    }
+    if (tid == 0) a.counters[(size_t)b * a.G + g] = 0;
 }
 
 template <typename T, int D, int R>
 cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s, bool pdl) {
     using Cfg = AttnCfg<T, D, R>;
     const int KT = a.Bk < Cfg::KT_MAX ? a.Bk : Cfg::KT_MAX;
+    // p_s doubles as the [S][r] merge weights of the last split: R * max(KT, kMaxSplits) floats
     const size_t smem = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
-                        (size_t)R * KT * 4 + 16;
+                        (size_t)R * (KT > kMaxSplits ? KT : kMaxSplits) * 4 + 16;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -385,18 +417,25 @@ cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, boo
     return dtype == MSA_F32 ? launch_attn_d<float>(a, s, pdl) : launch_attn_d<__nv_bfloat16>(a, s, pdl);
 }
 
-cudaError_t launch_decode_combine(const CombineArgs &a, int dtype, cudaStream_t s, bool pdl) {
+cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.G, a.B);
     cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = (size_t)a.n_cta * a.k * 8 + 256;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return dtype == MSA_F32 ? cudaLaunchKernelEx(&cfg, decode_combine_kernel<float>, a)
-                            : cudaLaunchKernelEx(&cfg, decode_combine_kernel<__nv_bfloat16>, a);
+    cfg.numAttrs = 1;
+    static size_t attr_bytes = 48 * 1024;
+    if (cfg.dynamicSmemBytes > attr_bytes) {
+        cudaError_t e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)cfg.dynamicSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_bytes = cfg.dynamicSmemBytes;
+    }
+    return cudaLaunchKernelEx(&cfg, decode_select_kernel, a);
 }
 
 }  // namespace msa

@@ -7,8 +7,9 @@
 // kernel is a stream of k_idx from HBM: each byte is read once.
 //
 // Work split: the index-K streams of all (sequence b, index-K head) pairs are
-// concatenated (block granularity) and cut into n_cta equal ranges, one per
-// persistent CTA (one CTA per SM), so ragged lengths stay balanced.  Inside a
+// concatenated (block granularity) and cut into n_cta ranges of equal length
+// (the last one shorter), one per persistent CTA (one CTA per SM), so ragged
+// lengths stay balanced.  Inside a
 // CTA every warp owns a private ring of kScanStages 8 KB shared-memory stages
 // filled by TMA bulk copies (cp.async.bulk, L2 evict-first) and consumes the
 // blocks w, w+8, ... of the CTA's range.  For one 16-byte vector of a key row
@@ -29,15 +30,14 @@ struct Piece {
     long long seg_start;
 };
 
-// CTA whose range [T*i/C, T*(i+1)/C) holds global block x.
-__device__ inline int cta_of(long long x, long long T, int C) {
-    return (int)(((x + 1) * C + T - 1) / T) - 1;
-}
+// CTA i owns the global blocks [i*per, (i+1)*per) (clipped to the total), so
+// every CTA below ceil(total/per) has a non-empty range and the CTAs that
+// touch a segment are consecutive and all write a piece.
+__device__ inline int cta_of(long long x, long long per) { return (int)(x / per); }
 
 // Enumerates the pieces of the range [x, x1) in order.
 struct PieceWalker {
-    long long x, x1, T;
-    int C;
+    long long x, x1;
     __device__ inline bool next(const long long *off, const int *nbs, int B, int Hik, Piece &p) {
         if (x >= x1) return false;
         int lo = 0, hi = B - 1;  // largest b with off[b] <= x (never an empty sequence since x < off[B])
@@ -142,7 +142,10 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
     }
     __syncthreads();
     const long long total = off[B];
-    const long long x0 = total * blockIdx.x / C, x1 = total * (blockIdx.x + 1) / C;
+    const long long per = total > 0 ? (total + C - 1) / C : 1;  // blocks per CTA
+    long long x0 = per * blockIdx.x, x1 = x0 + per;
+    x0 = x0 < total ? x0 : total;
+    x1 = x1 < total ? x1 : total;
 
     if (blockIdx.x == 0 && a.seg_info != nullptr) {
         for (int s = tid; s < B * Hik; s += blockDim.x) {
@@ -150,8 +153,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
             SegInfo si{-1, 0};
             if (nbs[b] > 0) {
                 const long long st = off[b] + (long long)h * nbs[b];
-                si.first_cta = cta_of(st, total, C);
-                si.n_pieces = cta_of(st + nbs[b] - 1, total, C) - si.first_cta + 1;
+                si.first_cta = cta_of(st, per);
+                si.n_pieces = cta_of(st + nbs[b] - 1, per) - si.first_cta + 1;
             }
             a.seg_info[s] = si;
         }
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
 
     // producer cursor (lane 0 issues, every lane tracks it to stay uniform)
     ChunkCursor prod;
-    prod.pw = PieceWalker{x0, x1, total, C};
+    prod.pw = PieceWalker{x0, x1};
     prod.w = w; prod.Bk = Bk; prod.row_bytes = ROW; prod.ct = CT;
     prod.start(off, nbs, lens, B, Hik);
     bool failed = false;
@@ -194,7 +197,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
     float qv[GPS][EPV];
     int q_b = -1, q_h = -1;
     WarpTopK lst[GPS];
-    PieceWalker pw{x0, x1, total, C};
+    PieceWalker pw{x0, x1};
     Piece p;
     while (pw.next(off, nbs, B, Hik, p)) {
         if (p.b != q_b || p.hik != q_h) {
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
             if (w < GPS) {
                 const int gl = w;
                 const int seg = p.b * Hik + p.hik;
-                const int piece = blockIdx.x - cta_of(p.seg_start, total, C);
+                const int piece = blockIdx.x - cta_of(p.seg_start, per);
                 const size_t o = (((size_t)seg * C + piece) * GPS + gl) * a.k;
                 warp_merge_sorted_lists<1>(lists_s + gl * 32, lists_i + gl * 32, kScanWarps, a.k, GPS * 32, a.k,
                                            a.cand_s + o, a.cand_i + o, lane);

@@ -147,12 +147,17 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
         L.cand_i = off;
         off += round256(cand);
     }
+    if (scan) {
+        L.sel_ids = off;
+        off += round256((size_t)p.batch * p.n_kv_heads * p.top_k * 4);
+    }
     if (attend) {
         if (p.flags & MSA_DENSE) {
             const int nb = nb_max_of(p);
             const long long want = 2LL * n_sm;
             long long S = (want + (long long)p.batch * p.n_kv_heads - 1) / ((long long)p.batch * p.n_kv_heads);
             if (S < 1) S = 1;
+            if (S > kMaxSplits) S = kMaxSplits;
             if (S > nb) S = nb;
             L.blocks_per_split = (int)((nb + S - 1) / S);
             L.S = (nb + L.blocks_per_split - 1) / L.blocks_per_split;
@@ -160,6 +165,8 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
             L.S = p.top_k;
             L.blocks_per_split = 1;
         }
+        L.counters = off;
+        off += round256((size_t)p.batch * p.n_kv_heads * 4);
         const size_t parts = (size_t)p.batch * p.n_kv_heads * L.S * r;
         L.part_o = off;
         off += round256(parts * p.head_dim * 4);
@@ -305,34 +312,28 @@ msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_i
 }
 
 static msa_status_t attend_decode(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
-                                  const int32_t *ids_in, bool from_scan, const DecodeWs &L, unsigned char *wsb,
-                                  void *o, int32_t *ids_out, float *lse, cudaStream_t s) {
+                                  const int32_t *ids, bool after_select, const DecodeWs &L, unsigned char *wsb,
+                                  void *o, float *lse, cudaStream_t s) {
     AttnArgs a{};
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.seq_lens = p->seq_lens;
-    a.ids_in = ids_in;
-    if (from_scan) {
-        a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
-        a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
-        a.seg_info = reinterpret_cast<const SegInfo *>(wsb + L.seg_info);
-    }
-    a.n_cta = L.n_cta;
-    a.ids_out = ids_out;
+    a.ids_in = ids;
     a.part_o = reinterpret_cast<float *>(wsb + L.part_o);
     a.part_lse = reinterpret_cast<float *>(wsb + L.part_lse);
+    a.counters = reinterpret_cast<int *>(wsb + L.counters);
+    a.o = o; a.lse = lse;
     a.B = p->batch; a.Hq = p->n_q_heads; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.D = p->head_dim;
     a.Bk = p->block_size; a.k = p->top_k; a.L_max = p->max_seq_len; a.r = p->n_q_heads / p->n_kv_heads;
     a.S = L.S; a.blocks_per_split = L.blocks_per_split; a.dense = (p->flags & MSA_DENSE) != 0;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(wsb);
-    cudaError_t e = launch_decode_attn(a, p->dtype, s, from_scan);
+    cudaError_t e;
+    if (!after_select) {  // the select kernel zeroes the counters in the fused path
+        e = cudaMemsetAsync(a.counters, 0, (size_t)p->batch * p->n_kv_heads * 4, s);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the split counters");
+    }
+    e = launch_decode_attn(a, p->dtype, s, after_select);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    if (from_scan && (e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    CombineArgs c{};
-    c.part_o = a.part_o; c.part_lse = a.part_lse; c.o = o; c.lse = lse;
-    c.B = p->batch; c.Hq = p->n_q_heads; c.G = p->n_kv_heads; c.D = p->head_dim; c.r = a.r; c.S = L.S;
-    e = launch_decode_combine(c, p->dtype, s, true);
-    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-    if (from_scan && (e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if (after_select && (e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return MSA_OK;
 }
 
@@ -355,7 +356,7 @@ msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const 
     const DecodeWs L = decode_ws_layout(*p, false, true, n_sm);
     if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     return attend_decode(p, q, k_cache, v_cache, dense ? nullptr : ids, false, L,
-                         reinterpret_cast<unsigned char *>(ws), o, nullptr, lse, (cudaStream_t)stream);
+                         reinterpret_cast<unsigned char *>(ws), o, lse, (cudaStream_t)stream);
 }
 
 msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *q_idx, const void *k_cache,
@@ -394,7 +395,16 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     e = launch_decode_scan(a, p->dtype, lpt, p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    return attend_decode(p, q, k_cache, v_cache, nullptr, true, L, wsb, o, ids_out, lse, s);
+    SelectArgs sa{};
+    sa.cand_s = a.cand_s; sa.cand_i = a.cand_i; sa.seg_info = a.seg_info;
+    sa.n_cta = L.n_cta; sa.B = p->batch; sa.G = p->n_kv_heads; sa.Hik = p->n_idx_k_heads; sa.k = p->top_k;
+    sa.sel_ids = reinterpret_cast<int *>(wsb + L.sel_ids);
+    sa.ids_out = ids_out;
+    sa.counters = reinterpret_cast<int *>(wsb + L.counters);
+    e = launch_decode_select(sa, s);
+    if (e != cudaSuccess) return cuda_fail(e, "select launch");
+    if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    return attend_decode(p, q, k_cache, v_cache, sa.sel_ids, true, L, wsb, o, lse, s);
 }
 
 msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
@@ -408,8 +418,28 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
 msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, const void *k_idx, int32_t *ids_out,
                                     float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
     MSA_TRY(check_params(p, PREFILL_ONLY));
-    (void)q_idx; (void)k_idx; (void)ids_out; (void)top_scores_out; (void)ws; (void)ws_bytes; (void)stream;
-    return fail(MSA_ERR_UNSUPPORTED, "msa_prefill_index_topk is not built yet");
+    if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes no flags");
+    if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
+    if (p->idx_dim != 64) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes idx_dim 64");
+    if (p->block_size < 32) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes block_size >= 32");
+    MSA_TRY(check_ptr(q_idx, "q_idx"));
+    MSA_TRY(check_ptr(k_idx, "k_idx"));
+    MSA_TRY(check_ptr(ids_out, "ids_out"));
+    MSA_TRY(check_ptr(top_scores_out, "top_scores_out", true));
+    MSA_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    PrefillIdxArgs a{};
+    a.B = p->batch; a.T = p->q_len; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.Bk = p->block_size;
+    a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len;
+    a.n_mt = (p->q_len + 255) / 256;
+    a.ids_out = ids_out; a.top_scores_out = top_scores_out;
+    a.status = reinterpret_cast<int *>(ws);
+    const char *why = "";
+    cudaError_t e = launch_prefill_index(a, q_idx, k_idx, n_sm, (cudaStream_t)stream, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return MSA_OK;
 }
 
 }  // extern "C"

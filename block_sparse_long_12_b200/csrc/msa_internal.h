@@ -25,6 +25,7 @@ constexpr int kScanChunkBytes = 8192;   // bytes of index keys per bulk copy
 
 // ---- decode sparse attention (Step 2 for decode)
 constexpr int kAttnThreads = 256;
+constexpr int kMaxSplits = 64;           // dense decode: splits per (sequence, group)
 
 // A segment is the index-K stream of one (sequence b, index-K head): blocks
 // 0..nb_b-1 of k_idx[b, hik].  The scan splits the concatenation of all
@@ -48,32 +49,32 @@ struct ScanArgs {
     int *status;
 };
 
+struct SelectArgs {
+    const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]
+    const int *cand_i;
+    const SegInfo *seg_info;
+    int n_cta, B, G, Hik, k;
+    int *sel_ids;              // [B, G, k] final list (workspace)
+    int *ids_out;              // nullable
+    float *top_scores_out;     // nullable
+    int *counters;             // [B, G] attention arrival counters, zeroed here
+};
+
 struct AttnArgs {
     const void *q;
     const void *k_cache;
     const void *v_cache;
     const int *seq_lens;
-    const int *ids_in;         // [B, 1, G, k] given selection (nullable)
-    const float *cand_s;       // candidates of the scan when ids_in == nullptr
-    const int *cand_i;
-    const SegInfo *seg_info;
-    int n_cta;                 // scan grid size (candidate stride)
-    int *ids_out;              // nullable
-    float *top_scores_out;     // nullable
+    const int *ids_in;         // [B, 1, G, k] selection (unused with dense)
     float *part_o;             // [B, G, S, r, D] fp32, normalised per split
     float *part_lse;           // [B, G, S, r] log2-domain normaliser
+    int *counters;             // [B, G] arrival counts, zero on entry; reset by the last split
+    void *o;                   // [B, 1, Hq, D]
+    float *lse;                // nullable, natural log
     int B, Hq, G, Hik, D, Bk, k, L_max, r;
     int S, blocks_per_split, dense;
     float scale_log2;          // softmax_scale * log2(e)
     int *status;
-};
-
-struct CombineArgs {
-    const float *part_o;
-    const float *part_lse;
-    void *o;
-    float *lse;                // nullable, natural log
-    int B, Hq, G, D, r, S;
 };
 
 struct PoolTopkArgs {
@@ -84,6 +85,14 @@ struct PoolTopkArgs {
     int B, q_len, q_start, G, Bk, k, L_max, nb_max, is_block, prefill;
 };
 
+struct PrefillIdxArgs {
+    int B, T, G, Hik, Bk, k, q_start, L_max;
+    int n_mt;                  // 256-row query tiles per (b, g)
+    int32_t *ids_out;          // [B, T, G, k]
+    float *top_scores_out;     // nullable
+    int *status;
+};
+
 struct FillArgs {
     float *scores;
     long long n;
@@ -91,7 +100,7 @@ struct FillArgs {
 
 // Workspace layout of the decode entries (offsets in bytes from ws).
 struct DecodeWs {
-    size_t seg_info, cand_s, cand_i, part_o, part_lse, total;
+    size_t seg_info, cand_s, cand_i, sel_ids, counters, part_o, part_lse, total;
     int n_cta, S, blocks_per_split;
 };
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);
@@ -100,8 +109,10 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
 cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);
 cudaError_t launch_decode_scan(const ScanArgs &a, int dtype, int lpt, int gps, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
-cudaError_t launch_decode_combine(const CombineArgs &a, int dtype, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
+                                 cudaStream_t s, const char **why);
 
 int num_sms();
 

@@ -1,0 +1,345 @@
+// Step 1 of MSA for a causal prefill chunk on the tensor cores: index scores,
+// block max pool and TopK, fused (scores never leave the SM).
+//
+// Page "MiniMax wird duenn" (atlascloud.ai), section 1, Step 1: the group's
+// index query scores every visible token (Q_idx . K_idx^T), the scores are
+// max-pooled per fixed block and TopK keeps the best blocks of the group.
+// In prefill every query row has its own index query, so Step 1 is a causal
+// GEMM with a reduction epilogue; section 3 of the page notes that this scan
+// of the full input remains in prefill.
+//
+// One persistent CTA per SM takes work units (sequence b, group g, 256 query
+// rows), heaviest first.  Warp roles:
+//   warp 0      TMA producer: the unit's two 128-row index-query tiles, then
+//               the index-key tiles (128 keys x 64 dims, 128-byte swizzle)
+//               through a kStages ring;
+//   warp 1      owns 512 TMEM columns and issues tcgen05.mma (M=128, N=128,
+//               K=16, bf16 in, fp32 accumulate) for both row tiles into a
+//               double-buffered pair of accumulators;
+//   warps 4-11  epilogue, one TMEM lane (= query row) per thread: tcgen05.ld
+//               of the scores, causal mask on diagonal tiles, 3-input max per
+//               32 columns, block max, and a register-resident sorted top-k.
+// The next tile's MMAs overlap the epilogue of the current one.
+#include <cudaTypedefs.h>
+
+#include "tcgen05.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr int kRows = 128;              // rows per accumulator (one TMEM lane each)
+constexpr int kAccs = 2;                // row tiles per unit
+constexpr int kUnitRows = kRows * kAccs;
+constexpr int kKeys = 128;              // keys per tile (N)
+constexpr int kStages = 6;
+constexpr int kThreads = 384;
+constexpr int kEpiWarp0 = 4;
+constexpr int kTileBytes = kKeys * 128; // 128 rows of 64 bf16
+constexpr int kABytes = kRows * 128;
+constexpr uint32_t kTmemCols = 512;     // 2 buffers x 2 accumulators x 128 columns
+
+struct Smem {
+    // 1024-byte aligned operand tiles come first (set up by hand in the kernel)
+    uint64_t full[kStages], empty[kStages];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t a_full, a_empty, mma_done;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+__device__ inline void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Row-wise sorted top-K (score desc, id asc) in registers.
+template <int K>
+struct RowTopK {
+    float s[K];
+    int id[K];
+    __device__ inline void reset() {
+#pragma unroll
+        for (int i = 0; i < K; ++i) { s[i] = -INFINITY; id[i] = 0x7fffffff; }
+    }
+    __device__ inline void insert(float cs, int ci) {
+        if (!better(cs, ci, s[K - 1], id[K - 1])) return;
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            const bool take = better(cs, ci, s[i], id[i]);
+            const float ts = s[i];
+            const int ti = id[i];
+            s[i] = take ? cs : ts;
+            id[i] = take ? ci : ti;
+            cs = take ? ts : cs;
+            ci = take ? ti : ci;
+        }
+    }
+};
+
+// Max over the 32 keys j0..j0+31 of one row, counting only keys j <= pos.
+__device__ inline float chunk_max_masked(const uint32_t (&r)[32], int j0, int pos) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m = (j0 + i <= pos) ? fmaxf(m, __uint_as_float(r[i])) : m;
+    return m;
+}
+
+template <int K>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_index_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                         const PrefillIdxArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    unsigned char *base = smem_raw + ((1024 - (raw & 1023)) & 1023);
+    unsigned char *smA = base;                               // [kAccs][128 rows][128 B]
+    unsigned char *smB = base + kAccs * kABytes;             // [kStages][128 keys][128 B]
+    Smem &S = *reinterpret_cast<Smem *>(smB + kStages * kTileBytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int BG = a.B * a.G;
+    const int n_units = a.n_mt * BG;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&S.acc_full[i], 1); mbar_init(&S.acc_empty[i], 8); }
+        mbar_init(&S.a_full, 1);
+        mbar_init(&S.a_empty, 1);
+        mbar_init(&S.mma_done, 1);
+        S.abort_flag = 0;
+        fence_mbar_init();
+        tc::prefetch_tmap(&qmap);
+        tc::prefetch_tmap(&kmap);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(&S.tmem_base, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = S.tmem_base;
+    volatile int *abort_flag = &S.abort_flag;
+
+    auto unit_of = [&](int u, int &b, int &g, int &m0, int &ntiles) {
+        const int mt = a.n_mt - 1 - u / BG;  // heaviest (latest rows) first
+        const int bg = u % BG;
+        b = bg / a.G;
+        g = bg % a.G;
+        m0 = mt * kUnitRows;
+        int last = m0 + kUnitRows - 1;
+        if (last > a.T - 1) last = a.T - 1;
+        const int pos_max = a.q_start + last;
+        const int nb_last = pos_max / a.Bk;
+        ntiles = ((nb_last + 1) * a.Bk + kKeys - 1) / kKeys;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int it = 0, ui = 0;
+            for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
+                int b, g, m0, ntiles;
+                unit_of(u, b, g, m0, ntiles);
+                if (!tc::wait_or_abort(&S.a_empty, (ui & 1) ^ 1, abort_flag, a.status)) break;
+                mbar_arrive_expect_tx(&S.a_full, kAccs * kABytes);
+                for (int acc = 0; acc < kAccs; ++acc)
+                    tc::tma_load_3d(smA + acc * kABytes, &qmap, 0, g, b * a.T + m0 + acc * kRows, &S.a_full);
+                const int hik = g % a.Hik;
+                const int row0 = (b * a.Hik + hik) * a.L_max;
+                bool ok = true;
+                for (int n = 0; n < ntiles; ++n, ++it) {
+                    const int st = it % kStages;
+                    if (!tc::wait_or_abort(&S.empty[st], ((it / kStages) & 1) ^ 1, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&S.full[st], kTileBytes);
+                    tc::tma_load_2d(smB + st * kTileBytes, &kmap, 0, row0 + n * kKeys, &S.full[st]);
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16_f32(kRows, kKeys);
+            int it = 0, ti = 0, ui = 0;
+            for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++ui) {
+                int b, g, m0, ntiles;
+                unit_of(u, b, g, m0, ntiles);
+                if (!tc::wait_or_abort(&S.a_full, ui & 1, abort_flag, a.status)) break;
+                tc::fence_after_sync();
+                bool ok = true;
+                for (int n = 0; n < ntiles; ++n, ++it, ++ti) {
+                    const int st = it % kStages;
+                    const int buf = ti & 1;
+                    if (!tc::wait_or_abort(&S.full[st], (it / kStages) & 1, abort_flag, a.status) ||
+                        !tc::wait_or_abort(&S.acc_empty[buf], ((ti >> 1) & 1) ^ 1, abort_flag, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t b_addr = smem_u32(smB + st * kTileBytes);
+#pragma unroll
+                    for (int acc = 0; acc < kAccs; ++acc) {
+                        const uint32_t a_addr = smem_u32(smA + acc * kABytes);
+                        const uint32_t d = tmem + (uint32_t)((buf * kAccs + acc) * kKeys);
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            tc::mma_bf16_ss(d, tc::sw128_kmajor_desc(a_addr + ks * 32),
+                                            tc::sw128_kmajor_desc(b_addr + ks * 32), idesc, ks > 0);
+                    }
+                    tc::mma_commit(&S.empty[st]);
+                    tc::mma_commit(&S.acc_full[buf]);
+                }
+                if (!ok) break;
+                tc::mma_commit(&S.a_empty);
+            }
+            // every MMA issued by this thread has completed before TMEM is released
+            tc::mma_commit(&S.mma_done);
+            mbar_wait(&S.mma_done, 0, a.status);
+        }
+    } else if (warp >= kEpiWarp0) {
+        // ------------------------------------------------ epilogue: one query row per thread
+        const int q4 = warp & 3, acc = (warp - kEpiWarp0) >> 2;
+        const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        int ti = 0;
+        RowTopK<K> top;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+            int b, g, m0, ntiles;
+            unit_of(u, b, g, m0, ntiles);
+            const int t = m0 + acc * kRows + q4 * 32 + lane;
+            const int pos = a.q_start + t;
+            const int pos_min = a.q_start + m0;  // smallest position of the unit
+            top.reset();
+            float bm = -INFINITY;
+            bool ok = true;
+            for (int n = 0; n < ntiles; ++n, ++ti) {
+                const int buf = ti & 1;
+                if (!tc::wait_or_abort(&S.acc_full[buf], (ti >> 1) & 1, abort_flag, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t col = tmem + lane_addr + (uint32_t)((buf * kAccs + acc) * kKeys);
+                const int kb = n * kKeys;
+                const bool diag = kb + kKeys - 1 > pos_min;
+                float cm[4];
+                {
+                    uint32_t r0[32], r1[32];
+                    tc::tmem_ld32(col, r0);
+                    tc::tmem_ld32(col + 32, r1);
+                    tc::tmem_ld_wait();
+                    cm[0] = diag ? chunk_max_masked(r0, kb, pos) : tc::max32(r0);
+                    cm[1] = diag ? chunk_max_masked(r1, kb + 32, pos) : tc::max32(r1);
+                    tc::tmem_ld32(col + 64, r0);
+                    tc::tmem_ld32(col + 96, r1);
+                    tc::tmem_ld_wait();
+                    cm[2] = diag ? chunk_max_masked(r0, kb + 64, pos) : tc::max32(r0);
+                    cm[3] = diag ? chunk_max_masked(r1, kb + 96, pos) : tc::max32(r1);
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int j0 = kb + 32 * c;
+                    bm = fmaxf(bm, cm[c]);
+                    if (((j0 + 32) & (a.Bk - 1)) == 0) {  // last chunk of block j0 / Bk
+                        const int blk = j0 / a.Bk;
+                        if (blk * a.Bk <= pos) top.insert(bm, blk);
+                        bm = -INFINITY;
+                    }
+                }
+            }
+            if (!ok) break;
+            if (t < a.T) {
+                const size_t o = (((size_t)b * a.T + t) * a.G + g) * a.k;
+#pragma unroll
+                for (int i = 0; i < K; ++i) {
+                    if (i < a.k) {
+                        const bool live = top.s[i] > -INFINITY;
+                        a.ids_out[o + i] = live ? top.id[i] : -1;
+                        if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = top.s[i];
+                    }
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+template <int K>
+cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid,
+                     cudaStream_t s) {
+    const size_t smem = 1024 + kAccs * kABytes + kStages * kTileBytes + sizeof(Smem) + 64;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e =
+            cudaFuncSetAttribute(prefill_index_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    prefill_index_kernel<K><<<grid, kThreads, smem, s>>>(qm, km, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
+                                 cudaStream_t s, const char **why) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (enc == nullptr) {
+        *why = "cuTensorMapEncodeTiled is not available from the driver";
+        return cudaErrorNotSupported;
+    }
+    CUtensorMap qm, km;
+    // q_idx [B*T, G, 64] bf16: box of 64 dims x 1 group x 128 rows
+    const cuuint64_t qdim[3] = {64, (cuuint64_t)a.G, (cuuint64_t)a.B * a.T};
+    const cuuint64_t qstr[2] = {64 * 2, (cuuint64_t)a.G * 64 * 2};
+    const cuuint32_t qbox[3] = {64, 1, kRows};
+    const cuuint32_t ones[3] = {1, 1, 1};
+    CUresult r = enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q_idx), qdim, qstr, qbox, ones,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *why = "encoding the index-query tensor map failed";
+        return cudaErrorInvalidValue;
+    }
+    // k_idx [B*Hik*Lmax, 64] bf16: box of 64 dims x 128 keys
+    const cuuint64_t kdim[2] = {64, (cuuint64_t)a.B * a.Hik * a.L_max};
+    const cuuint64_t kstr[1] = {64 * 2};
+    const cuuint32_t kbox[2] = {64, kKeys};
+    r = enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(k_idx), kdim, kstr, kbox, ones,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        *why = "encoding the index-key tensor map failed";
+        return cudaErrorInvalidValue;
+    }
+    const int units = a.n_mt * a.B * a.G;
+    const int grid = units < n_sm ? units : n_sm;
+    *why = "prefill index kernel launch";
+    if (a.k <= 8) return launch_k<8>(a, qm, km, grid, s);
+    if (a.k <= 16) return launch_k<16>(a, qm, km, grid, s);
+    return launch_k<32>(a, qm, km, grid, s);
+}
+
+}  // namespace msa

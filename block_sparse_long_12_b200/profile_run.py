@@ -1,0 +1,64 @@
+"""Small, self-contained runs of the MSA kernels for profilers (ncu).
+
+  python -m block_sparse_long_12_b200.profile_run decode --context 262144 --steps 3
+  python -m block_sparse_long_12_b200.profile_run prefill_index --context 65536 --chunk 8192 --steps 1
+
+Inputs are the seeded synthetic workloads of ``inputs`` at the requested
+size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
+64, block 128, top-k 16), kept small enough for a profiler's replay passes.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import _lib, api
+from .inputs import WORKLOADS, make_inputs
+
+
+def run_decode(args):
+    w = WORKLOADS["decode_ctx1m"].scaled(max_seq_len=args.context, batch=args.batch)
+    inp = make_inputs(w, device="cuda")
+    q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
+    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
+    ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, "cuda")
+    o = torch.empty_like(q)
+    ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device="cuda")
+    for _ in range(args.steps):
+        _lib.msa_decode_fused(p, q, q_idx, k, v, k_idx, o, ids, None, ws)
+    torch.cuda.synchronize()
+    print("decode done", ids[0, 0, 0].tolist())
+
+
+def run_prefill_index(args):
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=args.context)
+    inp = make_inputs(w, device="cuda")
+    q_idx, k_idx = inp["q_idx"], inp["k_idx"]
+    T = args.chunk
+    for step in range(args.steps):
+        q_start = args.context - T
+        qi = q_idx[:, q_start:q_start + T].contiguous()
+        p = api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
+                            head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=w.block_size, top_k=w.top_k,
+                            max_seq_len=w.max_seq_len, dtype=_lib.MSA_BF16, q_len=T, q_start=q_start)
+        ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device="cuda")
+        ws = api.workspace(p, _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, "cuda")
+        _lib.msa_prefill_index_topk(p, qi, k_idx, ids, None, ws)
+    torch.cuda.synchronize()
+    print("prefill index done")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("what", choices=["decode", "prefill_index"])
+    ap.add_argument("--context", type=int, default=262144)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--chunk", type=int, default=8192)
+    ap.add_argument("--steps", type=int, default=3)
+    args = ap.parse_args()
+    {"decode": run_decode, "prefill_index": run_prefill_index}[args.what](args)
+
+
+if __name__ == "__main__":
+    main()

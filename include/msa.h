@@ -178,8 +178,9 @@ MSA_API msa_status_t msa_prefill_index_topk(const msa_params_t *params, const vo
 /*
  * Measurement hook (not part of the method): while set, msa_decode_fused
  * records events[0] before its first kernel and events[i] after its i-th
- * kernel (1 = index scan, 2 = sparse attention, 3 = split combine) on the
- * call's stream, so a caller can time each kernel with cudaEventElapsedTime.
+ * kernel (1 = index scan, 2 = TopK merge, 3 = sparse attention with the split
+ * merge) on the call's stream, so a caller can time each kernel with
+ * cudaEventElapsedTime.
  * events are cudaEvent_t handles owned by the caller; n_events must be 0
  * (unset) or 4.  Per calling thread.  Recording between the kernels removes
  * their launch overlap, so time whole steps without it.

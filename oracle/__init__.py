@@ -92,7 +92,7 @@ def _load():
         lib.oracle_topk.argtypes = [P, dp, ip, vp, dp, dp, dp]
         lib.oracle_attention_row.argtypes = [P, vp, vp, vp, ip, ip, ip, ip, vp, ip, dp, dp, dp]
         lib.oracle_attention_row.restype = ctypes.c_int
-        lib.oracle_msa_rows.argtypes = [P, vp, vp, vp, vp, vp, vp, ip, vp, vp, vp, dp, dp, dp, dp, dp]
+        lib.oracle_msa_rows.argtypes = [P, vp, vp, vp, vp, vp, vp, ip, vp, vp, vp, dp, dp, dp, dp, dp, ip]
         _lib = lib
     return _lib
 
@@ -147,13 +147,14 @@ def attention_row(p: Params, q, k, v, b: int, t: int, h: int, pos: int, ids):
     return o, float(lse[0]), w, n
 
 
-def msa_rows(p: Params, seq_lens, q, q_idx, k, v, k_idx, rows, ids_in=None) -> dict:
+def msa_rows(p: Params, seq_lens, q, q_idx, k, v, k_idx, rows, ids_in=None, attention: bool = True) -> dict:
     """Steps 1 and 2 for the (b, t) query rows listed in ``rows`` (shape [n, 2]).
 
     Returns a dict with ``ids`` int32[n, G, k], ``top_scores`` f64[n, G, k],
     ``kth``/``kth_next`` f64[n, G] (k-th and (k+1)-th block scores of the full
     ranking, NaN where absent), ``o`` f64[n, Hq, D] and ``lse`` f64[n, Hq].
-    With ``ids_in`` the given selection drives Step 2 instead.
+    With ``ids_in`` the given selection drives Step 2 instead; with
+    ``attention=False`` only Step 1 runs (``o``/``lse`` stay NaN).
     """
     q, q_idx, k, v, k_idx = (_raw(x, p) for x in (q, q_idx, k, v, k_idx))
     rows = np.ascontiguousarray(np.asarray(rows, np.int32).reshape(-1, 2))
@@ -164,12 +165,12 @@ def msa_rows(p: Params, seq_lens, q, q_idx, k, v, k_idx, rows, ids_in=None) -> d
     ts = np.full((n, G, K), -np.inf)
     kth = np.empty((n, G), np.float64)
     kn = np.empty((n, G), np.float64)
-    o = np.empty((n, p.n_q_heads, p.head_dim), np.float64)
-    lse = np.empty((n, p.n_q_heads), np.float64)
+    o = np.full((n, p.n_q_heads, p.head_dim), np.nan)
+    lse = np.full((n, p.n_q_heads), np.nan)
     idin = None if ids_in is None else np.ascontiguousarray(np.asarray(ids_in, np.int32).reshape(n, G, K))
     _load().oracle_msa_rows(ctypes.byref(p.c()), _ptr(sl), _ptr(q), _ptr(q_idx), _ptr(k), _ptr(v),
                             _ptr(k_idx), n, _ptr(rows), None if idin is None else _ptr(idin),
-                            _ptr(ids), _ptr(ts), _ptr(kth), _ptr(kn), _ptr(o), _ptr(lse))
+                            _ptr(ids), _ptr(ts), _ptr(kth), _ptr(kn), _ptr(o), _ptr(lse), int(attention))
     return {"ids": ids, "top_scores": ts, "kth": kth, "kth_next": kn, "o": o, "lse": lse}
 
 

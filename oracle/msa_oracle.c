@@ -195,12 +195,13 @@ static int query_pos(const oracle_params *p, const int *seq_lens, int b, int t)
  * query head: o [n_rows, Hq, D], lse [n_rows, Hq].
  * If ids_in is non-NULL the selection is not computed: the given ids
  * ([n_rows, G, k]) drive Step 2 (used to re-run a near-tie row with another
- * implementation's choice). */
+ * implementation's choice).  With with_attention == 0 only Step 1 runs and
+ * o / lse are left untouched. */
 void oracle_msa_rows(const oracle_params *p, const int *seq_lens,
                      const void *q, const void *q_idx, const void *k, const void *v,
                      const void *k_idx, int n_rows, const int *rows, const int *ids_in,
                      int *ids_out, double *top_scores_out, double *kth_out,
-                     double *kth_next_out, double *o_out, double *lse_out)
+                     double *kth_next_out, double *o_out, double *lse_out, int with_attention)
 {
     const int G = n_groups(p), K = p->top_k, r = p->n_q_heads / p->n_kv_heads;
     const int D = p->head_dim;
@@ -226,6 +227,7 @@ void oracle_msa_rows(const oracle_params *p, const int *seq_lens,
             free(s);
             free(S);
         }
+        if (!with_attention) continue;
         int *attend = ids;
         int n_attend = K;
         int *all = NULL;

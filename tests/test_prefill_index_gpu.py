@@ -1,0 +1,118 @@
+"""GPU parity of the fused prefill index branch (tensor-core index scores, block
+max pool, TopK) against the fp64 oracle.  Page "MiniMax wird duenn"
+(atlascloud.ai), section 1, Step 1, and section 3 (in prefill the index
+branch still scans the whole visible input)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_12_b200.inputs import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+from parity import check_ids_row, to_np  # noqa: E402
+
+
+def prefill_ids(inp, w, q_start, T, top_k=None, block_size=None, scores=False):
+    from block_sparse_long_12_b200 import _lib, api
+    k = top_k or w.top_k
+    bk = block_size or w.block_size
+    B = inp["q_idx"].shape[0]
+    qi = inp["q_idx"][:, q_start:q_start + T].contiguous()
+    p = api.make_params(batch=B, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
+                        head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=bk, top_k=k, max_seq_len=w.max_seq_len,
+                        dtype=_lib.MSA_BF16, q_len=T, q_start=q_start)
+    ids = torch.full((B, T, w.n_kv_heads, k), -7, dtype=torch.int32, device="cuda")
+    ts = torch.empty(B, T, w.n_kv_heads, k, dtype=torch.float32, device="cuda") if scores else None
+    ws = api.workspace(p, _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, "cuda")
+    _lib.msa_prefill_index_topk(p, qi, inp["k_idx"], ids, ts, ws)
+    torch.cuda.synchronize()
+    assert _lib.msa_get_device_status(ws) == 0
+    return ids, ts
+
+
+def check_rows(inp, w, q_start, T, ids, rows, top_k=None, block_size=None):
+    """Compare GPU ids with the oracle on the given chunk rows (t relative to the chunk)."""
+    x = to_np(inp)
+    k = top_k or w.top_k
+    bk = block_size or w.block_size
+    B = x["q_idx"].shape[0]
+    xq = {n: np.ascontiguousarray(x[n][:, q_start:q_start + T]) for n in ("q", "q_idx")}
+    p = oracle.Params(B, w.n_q_heads, w.n_kv_heads, w.n_idx_k_heads, w.head_dim, w.idx_dim, bk, k, T, q_start,
+                      w.max_seq_len, "bf16", w.softmax_scale, prefill=True)
+    ref = oracle.msa_rows(p, None, xq["q"], xq["q_idx"], x["k"], x["v"], x["k_idx"], rows, attention=False)
+    idn = ids.cpu().numpy()
+    xo = {"q_idx": xq["q_idx"], "k_idx": x["k_idx"]}
+    ties = 0
+    for i, (b, t) in enumerate(rows):
+        for g in range(w.n_kv_heads):
+            exact = check_ids_row(p, xo, b, t, g, q_start + t, idn[b, t, g], ref["ids"][i, g], ref["kth"][i, g],
+                                  ref["kth_next"][i, g], where=f"b={b} t={t} g={g}")
+            ties += not exact
+    return ties
+
+
+def test_prefill_16k_all_rows():
+    """16K causal prefill, 16 heads / 2 groups, block 64, k 16: every row checked."""
+    w = WORKLOADS["prefill_causal_16k"]
+    inp = make_inputs(w, device="cuda")
+    ids, _ = prefill_ids(inp, w, 0, w.max_seq_len)
+    rows = [(0, t) for t in range(w.max_seq_len)]
+    check_rows(inp, w, 0, w.max_seq_len, ids, rows)
+
+
+@pytest.mark.parametrize("case", [
+    dict(block_size=128, top_k=16),
+    dict(block_size=64, top_k=8),
+    dict(block_size=32, top_k=32),
+    dict(block_size=256, top_k=4),
+    dict(block_size=128, top_k=1),
+    dict(block_size=128, top_k=16, n_idx_k_heads=1),
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()))
+def test_prefill_index_chunk_variants(case):
+    """A ragged chunk (1000 rows starting at 1500) of a 3000-token batch-2 sequence."""
+    hik = case.pop("n_idx_k_heads", 8)
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=3000, batch=2, n_idx_k_heads=hik, hot_blocks=5, seed=21)
+    inp = make_inputs(w, device="cuda")
+    q_start, T = 1500, 1000
+    ids, ts = prefill_ids(inp, w, q_start, T, top_k=case["top_k"], block_size=case["block_size"], scores=True)
+    rows = [(b, t) for b in range(2) for t in range(T)]
+    check_rows(inp, w, q_start, T, ids, rows, top_k=case["top_k"], block_size=case["block_size"])
+    # scores come out sorted (desc) and are -inf exactly where ids are -1
+    tsn, idn = ts.cpu().numpy(), ids.cpu().numpy()
+    assert (np.diff(tsn, axis=-1) <= 0).all()
+    assert ((idn == -1) == np.isneginf(tsn)).all()
+
+
+def test_prefill_index_first_rows_and_padding():
+    """The first rows of a sequence see fewer blocks than k: the lists are padded with -1."""
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=2048, batch=1, hot_blocks=0, seed=4)
+    inp = make_inputs(w, device="cuda")
+    ids, _ = prefill_ids(inp, w, 0, 600)
+    idn = ids.cpu().numpy()
+    for t in (0, 1, 127, 128, 599):
+        nvalid = t // w.block_size + 1
+        for g in range(w.n_kv_heads):
+            assert sorted(idn[0, t, g, :nvalid].tolist()) == list(range(nvalid))
+            assert (idn[0, t, g, nvalid:] == -1).all()
+    check_rows(inp, w, 0, 600, ids, [(0, t) for t in range(600)])
+
+
+def test_prefill_1m_sampled_rows():
+    """The 1M-token workload chunk by chunk (8192 rows each): the first chunk fully and
+    rows sampled across the whole sequence are checked against the oracle."""
+    w = WORKLOADS["prefill_causal_1m"]
+    inp = make_inputs(w, device="cuda")
+    T = w.chunk
+    rng = np.random.default_rng(1005)
+    chunks = sorted(set([0] + rng.choice(w.max_seq_len // T, 6, replace=False).tolist()))
+    for c in chunks:
+        ids, _ = prefill_ids(inp, w, c * T, T)
+        if c == 0:
+            rows = [(0, t) for t in range(T)]
+        else:
+            rows = [(0, int(t)) for t in rng.choice(T, 16, replace=False)]
+        check_rows(inp, w, c * T, T, ids, rows)
