@@ -6,8 +6,8 @@
 // cache, so one group loads one set of KV blocks for all its heads.
 //
 // decode_select_kernel finishes Step 1: one CTA per (sequence, group) stages
-// the scan's per-piece sorted candidate lists in shared memory and merges
-// them into the group's final TopK list.
+// the scan's per-piece sorted candidate lists in shared memory and selects
+// the group's final TopK list from them.
 //
 // decode_attn_kernel, grid (split s, group g, sequence b): a CTA reads the
 // group's list, streams the K/V tiles of its share of the blocks through a
@@ -335,15 +335,24 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     if (tid == 0) a.counters[bg] = 0;  // ready for the next call
 }
 
-// Final TopK of a group from the scan's per-piece sorted lists (staged in
-// shared memory), written to the selection buffer and the optional outputs.
+// Final TopK of a group from the scan's per-piece sorted lists.  All
+// candidates are staged in shared memory; any candidate worse than the k-th
+// entry of some full list cannot be in the final k (that list alone already
+// has k better ones), so only the survivors are ranked, each by counting the
+// survivors that beat it.
 __global__ void __launch_bounds__(256) decode_select_kernel(const SelectArgs a) {
     extern __shared__ __align__(16) unsigned char sm_raw[];
+    const int cap = a.n_cta * a.k;
     float *ls = reinterpret_cast<float *>(sm_raw);
-    int *li = reinterpret_cast<int *>(ls + (size_t)a.n_cta * a.k);
-    float *out_s = reinterpret_cast<float *>(li + (size_t)a.n_cta * a.k);
+    int *li = reinterpret_cast<int *>(ls + cap);
+    float *ss = reinterpret_cast<float *>(li + cap);   // survivors
+    int *si_ = reinterpret_cast<int *>(ss + cap);
+    float *out_s = reinterpret_cast<float *>(si_ + cap);
     int *out_i = reinterpret_cast<int *>(out_s + 32);
-    const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+    __shared__ float thr_s[8];
+    __shared__ int thr_i[8];
+    __shared__ int n_surv;
+    const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait_prior_grid();
     pdl_allow_next_grid();
     const int gps = a.G / a.Hik;
@@ -355,16 +364,46 @@ __global__ void __launch_bounds__(256) decode_select_kernel(const SelectArgs a) 
         ls[i] = a.cand_s[src];
         li[i] = a.cand_i[src];
     }
+    if (tid < 32) { out_s[tid] = -INFINITY; out_i[tid] = -1; }
+    if (tid == 0) n_surv = 0;
     __syncthreads();
-    if (tid < 32) {
-        warp_merge_sorted_lists<kMaxPiecesPerSeg / 32>(ls, li, si.n_pieces, a.k, a.k, a.k, out_s, out_i, tid);
-        __syncwarp();
-        if (tid < a.k) {
-            const size_t o = ((size_t)b * a.G + g) * a.k + tid;
-            a.sel_ids[o] = out_i[tid];
-            if (a.ids_out != nullptr) a.ids_out[o] = out_i[tid];
-            if (a.top_scores_out != nullptr) a.top_scores_out[o] = out_s[tid];
+    // threshold: the best k-th entry over all lists
+    float ts = -INFINITY;
+    int ti = -1;
+    for (int l = tid; l < si.n_pieces; l += blockDim.x) {
+        const float s = ls[l * a.k + a.k - 1];
+        const int i = li[l * a.k + a.k - 1];
+        if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
+    }
+    warp_best(ts, ti);
+    if (lane == 0) { thr_s[warp] = ts; thr_i[warp] = ti; }
+    __syncthreads();
+    ts = thr_s[0];
+    ti = thr_i[0];
+    for (int w2 = 1; w2 < 8; ++w2)
+        if (better(thr_s[w2], thr_i[w2], ts, ti)) { ts = thr_s[w2]; ti = thr_i[w2]; }
+    for (int i = tid; i < n; i += blockDim.x) {
+        if (li[i] >= 0 && !better(ts, ti, ls[i], li[i])) {
+            const int at = atomicAdd(&n_surv, 1);
+            ss[at] = ls[i];
+            si_[at] = li[i];
         }
+    }
+    __syncthreads();
+    const int m = n_surv;
+    for (int i = tid; i < m; i += blockDim.x) {
+        const float s = ss[i];
+        const int id = si_[i];
+        int rank = 0;
+        for (int j = 0; j < m; ++j) rank += better(ss[j], si_[j], s, id) ? 1 : 0;
+        if (rank < a.k) { out_s[rank] = s; out_i[rank] = id; }
+    }
+    __syncthreads();
+    if (tid < a.k) {
+        const size_t o = ((size_t)b * a.G + g) * a.k + tid;
+        a.sel_ids[o] = out_i[tid];
+        if (a.ids_out != nullptr) a.ids_out[o] = out_i[tid];
+        if (a.top_scores_out != nullptr) a.top_scores_out[o] = out_s[tid];
     }
     if (tid == 0) a.counters[(size_t)b * a.G + g] = 0;
 }
@@ -421,7 +460,7 @@ cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.G, a.B);
     cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = (size_t)a.n_cta * a.k * 8 + 256;
+    cfg.dynamicSmemBytes = (size_t)a.n_cta * a.k * 16 + 256;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -9,17 +9,17 @@
 // Work split: the index-K streams of all (sequence b, index-K head) pairs are
 // concatenated (block granularity) and cut into n_cta ranges of equal length
 // (the last one shorter), one per persistent CTA (one CTA per SM), so ragged
-// lengths stay balanced.  Inside a
-// CTA every warp owns a private ring of kScanStages 8 KB shared-memory stages
-// filled by TMA bulk copies (cp.async.bulk, L2 evict-first) and consumes the
-// blocks w, w+8, ... of the CTA's range.  For one 16-byte vector of a key row
-// a lane does the fp32 dot-product part against its slice of the index query
-// (held in registers); a butterfly over the lanes of the row completes the
-// token score, a running max gives the block score, and a warp-distributed
-// sorted list keeps the warp's best blocks.  At the end of each piece the
-// eight warp lists are merged into one sorted candidate list per group; the
-// attention kernel merges the pieces of a segment into the final TopK.
-#include "msa_device.cuh"
+// lengths stay balanced.  Inside a CTA every warp owns a private two-stage
+// ring of 8 KB shared-memory tiles filled by TMA tensor copies
+// (cp.async.bulk.tensor, 128-byte swizzle) and consumes the blocks w, w+W, ...
+// of the CTA's range.  One lane owns one index-key row: the swizzle makes the
+// 32 lanes' 16-byte reads of the same vector position hit distinct banks, so
+// the fp32 dot product against the index query (registers) needs no
+// cross-lane reduction; a warp max per block gives the block score and a
+// warp-distributed sorted list keeps the warp's best blocks.  At the end of
+// each piece the warp lists are merged into one sorted candidate list per
+// group; decode_select_kernel merges the pieces of a segment.
+#include "tcgen05.cuh"
 
 namespace msa {
 
@@ -64,7 +64,7 @@ struct ChunkCursor {
     PieceWalker pw;
     Piece p;
     int n, c, nch, valid;
-    int w, Bk, row_bytes, ct;  // ct = tokens per chunk
+    int w, W, Bk, ct;  // warp, warps per CTA, block size, tokens per chunk
     __device__ inline int block_tokens(const int *lens) const {
         const int L = lens[p.b];
         const int t = L - n * Bk;
@@ -86,7 +86,7 @@ struct ChunkCursor {
     }
     __device__ inline void advance(const long long *off, const int *nbs, const int *lens, int B, int Hik) {
         if (++c < nch) return;
-        n += kScanWarps;
+        n += W;
         if (n < p.n1) {
             c = 0;
             nch = (block_tokens(lens) + ct - 1) / ct;
@@ -96,21 +96,34 @@ struct ChunkCursor {
     }
 };
 
-template <typename T, int GPS, int LPT>
-__global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const ScanArgs a) {
-    constexpr int EPV = Vec16<T>::N;          // elements per 16-byte vector
-    constexpr int ROW = LPT * 16;             // bytes per index-key row
-    constexpr int CT = kScanChunkBytes / ROW; // tokens per chunk
-    constexpr int TPI = 32 / LPT;             // tokens per warp step
+// Warps per CTA and stages per warp ring: one index-K head per stream (GPS 1)
+// keeps the index query in registers and affords 12 warps; several groups
+// on one stream (GPS > 1) read it from shared memory and use 8 warps.
+template <int GPS> struct ScanShape {
+    static constexpr int W = GPS == 1 ? 12 : 8;
+    static constexpr int S = 2;
+};
 
-    extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *ring = smem;                                             // [W][S][chunk]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + (size_t)kScanWarps * kScanStages * kScanChunkBytes);
-    float *lists_s = reinterpret_cast<float *>(bars + kScanWarps * kScanStages); // [W][GPS][32]
-    int *lists_i = reinterpret_cast<int *>(lists_s + kScanWarps * GPS * 32);
-    long long *off = reinterpret_cast<long long *>(lists_i + kScanWarps * GPS * 32); // [B+1]
-    int *nbs = reinterpret_cast<int *>(off + a.B + 1);                   // [B]
-    int *lens = nbs + a.B;                                               // [B] clamped lengths
+template <typename T, int GPS, int ROWB>
+__global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
+    decode_scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
+    constexpr int W = ScanShape<GPS>::W, S = ScanShape<GPS>::S;
+    constexpr int ES = (int)sizeof(T);
+    constexpr int EPV = Vec16<T>::N;      // elements per 16-byte vector
+    constexpr int NCH = ROWB / 16;        // 16-byte vectors per index-key row
+    constexpr int DI = ROWB / ES;         // index dim
+    constexpr bool QREG = GPS == 1 && DI <= 64;
+    const int CT = a.chunk_tokens;        // tokens per chunk (<= block size, 8 KB at most)
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);  // [W][S][8 KB]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + (size_t)W * S * kScanChunkBytes);
+    float *lists_s = reinterpret_cast<float *>(bars + W * S);                 // [W][GPS][32]
+    int *lists_i = reinterpret_cast<int *>(lists_s + W * GPS * 32);
+    float *q_s = reinterpret_cast<float *>(lists_i + W * GPS * 32);           // [GPS][DI] (QREG: unused)
+    long long *off = reinterpret_cast<long long *>(q_s + GPS * DI);           // [B+1]
+    int *nbs = reinterpret_cast<int *>(off + a.B + 1);                        // [B]
+    int *lens = nbs + a.B;                                                    // [B] clamped lengths
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int B = a.B, Hik = a.Hik, Bk = a.Bk, C = a.n_cta;
@@ -122,7 +135,8 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
         lens[b] = L;
         nbs[b] = (L + Bk - 1) / Bk;
     }
-    if (tid < kScanWarps * kScanStages) mbar_init(&bars[tid], 1);
+    if (tid < W * S) mbar_init(&bars[tid], 1);
+    if (tid == 0) tc::prefetch_tmap(&kmap);
     fence_mbar_init();
     __syncthreads();
     if (w == 0) {
@@ -159,42 +173,37 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
             a.seg_info[s] = si;
         }
     }
-    // the attention grid may start its prologue while this grid runs
+    // the next grid may start its prologue while this grid runs
     pdl_allow_next_grid();
 
     const T *qg = reinterpret_cast<const T *>(a.q_idx);
-    const unsigned char *kg = reinterpret_cast<const unsigned char *>(a.k_idx);
-    const uint64_t pol = l2_evict_first_policy();
-    unsigned char *my_ring = ring + (size_t)w * kScanStages * kScanChunkBytes;
-    uint64_t *my_bars = bars + w * kScanStages;
+    unsigned char *my_ring = ring + (size_t)w * S * kScanChunkBytes;
+    uint64_t *my_bars = bars + w * S;
     const bool want_cand = a.cand_s != nullptr;
+    const uint32_t chunk_bytes = (uint32_t)CT * ROWB;
 
     // producer cursor (lane 0 issues, every lane tracks it to stay uniform)
     ChunkCursor prod;
     prod.pw = PieceWalker{x0, x1};
-    prod.w = w; prod.Bk = Bk; prod.row_bytes = ROW; prod.ct = CT;
+    prod.w = w; prod.W = W; prod.Bk = Bk; prod.ct = CT;
     prod.start(off, nbs, lens, B, Hik);
     bool failed = false;
     int issued = 0;
     auto issue = [&](int slot) {
-        const int tok0 = prod.n * Bk + prod.c * CT;
-        int nt = lens[prod.p.b] - tok0;
-        nt = nt < CT ? nt : CT;
-        if (nt > Bk - prod.c * CT) nt = Bk - prod.c * CT;
-        const uint32_t bytes = (uint32_t)nt * ROW;
         if (lane == 0) {
-            const unsigned char *src =
-                kg + (((size_t)prod.p.b * Hik + prod.p.hik) * (size_t)a.L_max + (size_t)tok0) * ROW;
-            mbar_arrive_expect_tx(&my_bars[slot], bytes);
-            bulk_g2s(my_ring + (size_t)slot * kScanChunkBytes, src, bytes, &my_bars[slot], pol);
+            const int row = (prod.p.b * Hik + prod.p.hik) * a.L_max + prod.n * Bk + prod.c * CT;
+            unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
+            mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
+            tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
+            if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
         }
         ++issued;
         prod.advance(off, nbs, lens, B, Hik);
     };
-    for (int s = 0; s < kScanStages && prod.valid; ++s) issue(s);
+    for (int st = 0; st < S && prod.valid; ++st) issue(st);
 
     int consumed = 0;
-    float qv[GPS][EPV];
+    float qv[QREG ? DI : 1];
     int q_b = -1, q_h = -1;
     WarpTopK lst[GPS];
     PieceWalker pw{x0, x1};
@@ -202,18 +211,23 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
     while (pw.next(off, nbs, B, Hik, p)) {
         if (p.b != q_b || p.hik != q_h) {
             q_b = p.b; q_h = p.hik;
+            if constexpr (QREG) {
+                const T *src = qg + ((size_t)p.b * a.G + p.hik) * DI;
 #pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) {
-                const int g = p.hik + Hik * gl;
-                const T *src = qg + ((size_t)p.b * a.G + g) * a.di + (lane % LPT) * EPV;
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) qv[gl][e] = load_elem(src + e);
+                for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
+            } else {
+                __syncthreads();  // every warp is done with the previous segment's query
+                for (int i = tid; i < GPS * DI; i += blockDim.x) {
+                    const int g = p.hik + Hik * (i / DI);
+                    q_s[i] = load_elem(qg + ((size_t)p.b * a.G + g) * DI + i % DI);
+                }
+                __syncthreads();
             }
         }
 #pragma unroll
         for (int gl = 0; gl < GPS; ++gl) lst[gl].reset();
         const int L = lens[p.b];
-        for (int n = p.n0 + w; n < p.n1; n += kScanWarps) {
+        for (int n = p.n0 + w; n < p.n1; n += W) {
             int bt = L - n * Bk;
             bt = bt < Bk ? bt : Bk;
             const int nch = (bt + CT - 1) / CT;
@@ -221,44 +235,55 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
 #pragma unroll
             for (int gl = 0; gl < GPS; ++gl) m[gl] = -INFINITY;
             for (int c = 0; c < nch; ++c) {
-                const int slot = consumed % kScanStages;
-                const uint32_t parity = (consumed / kScanStages) & 1;
+                const int slot = consumed % S;
+                const uint32_t parity = (consumed / S) & 1;
                 if (!failed && !mbar_wait(&my_bars[slot], parity, a.status)) {
                     // give up: wait (bounded) for this warp's copies still in flight, then
                     // run the loop to its end without waiting or issuing again
                     failed = true;
-                    for (int q2 = consumed + 1; q2 < issued; ++q2)
-                        mbar_wait(&my_bars[q2 % kScanStages], (q2 / kScanStages) & 1, nullptr);
+                    for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;
                 const unsigned char *base = my_ring + (size_t)slot * kScanChunkBytes;
                 const int tok_base = n * Bk + c * CT;
-#pragma unroll 4
-                for (int it = 0; it < CT / TPI; ++it) {
-                    const int tok = it * TPI + lane / LPT;
+                for (int t0 = 0; t0 < nt; t0 += 32) {
+                    const int tok = t0 + lane;  // one index-key row per lane
                     const bool live = tok < nt && !failed;
                     float dot[GPS];
 #pragma unroll
                     for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
                     if (live) {
-                        const uint4 u = *reinterpret_cast<const uint4 *>(base + tok * ROW + (lane % LPT) * 16);
-                        float f[EPV];
-                        Vec16<T>::unpack(u, f);
 #pragma unroll
-                        for (int gl = 0; gl < GPS; ++gl)
+                        for (int c16 = 0; c16 < NCH; ++c16) {
+                            // position of 16-byte vector c16 of row `tok` in the swizzled tile
+                            int o;
+                            if constexpr (ROWB == 64) {
+                                o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
+                            } else {
+                                o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
+                            }
+                            const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
+                            float f[EPV];
+                            Vec16<T>::unpack(u, f);
+                            if constexpr (QREG) {
 #pragma unroll
-                            for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qv[gl][e], f[e], dot[gl]);
+                                for (int e = 0; e < EPV; ++e) dot[0] = fmaf(qv[c16 * EPV + e], f[e], dot[0]);
+                            } else {
+#pragma unroll
+                                for (int gl = 0; gl < GPS; ++gl) {
+                                    const float *qq = q_s + gl * DI + c16 * EPV;
+#pragma unroll
+                                    for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qq[e], f[e], dot[gl]);
+                                }
+                            }
+                        }
                     }
-#pragma unroll
-                    for (int o = LPT / 2; o > 0; o >>= 1)
-#pragma unroll
-                        for (int gl = 0; gl < GPS; ++gl) dot[gl] += __shfl_xor_sync(FULL, dot[gl], o);
 #pragma unroll
                     for (int gl = 0; gl < GPS; ++gl) {
                         const float sc = live ? dot[gl] : -INFINITY;
                         m[gl] = fmaxf(m[gl], sc);
-                        if (a.token_scores != nullptr && live && (lane % LPT) == 0) {
+                        if (a.token_scores != nullptr && live) {
                             const int g = p.hik + Hik * gl;
                             a.token_scores[((size_t)p.b * a.G + g) * a.L_max + tok_base + tok] = sc;
                         }
@@ -269,7 +294,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
                 if (prod.valid && !failed) issue(slot);
             }
 #pragma unroll
-            for (int o = LPT; o < 32; o <<= 1)
+            for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
                 for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], __shfl_xor_sync(FULL, m[gl], o));
 #pragma unroll
@@ -294,7 +319,7 @@ __global__ void __launch_bounds__(kScanWarps * 32, 1) decode_scan_kernel(const S
                 const int seg = p.b * Hik + p.hik;
                 const int piece = blockIdx.x - cta_of(p.seg_start, per);
                 const size_t o = (((size_t)seg * C + piece) * GPS + gl) * a.k;
-                warp_merge_sorted_lists<1>(lists_s + gl * 32, lists_i + gl * 32, kScanWarps, a.k, GPS * 32, a.k,
+                warp_merge_sorted_lists<1>(lists_s + gl * 32, lists_i + gl * 32, W, a.k, GPS * 32, a.k,
                                            a.cand_s + o, a.cand_i + o, lane);
             }
             __syncthreads();
@@ -307,20 +332,21 @@ __global__ void fill_neg_inf_kernel(const FillArgs a) {
         a.scores[i] = -INFINITY;
 }
 
-template <typename T, int GPS, int LPT>
-cudaError_t launch_scan_t(const ScanArgs &a, cudaStream_t s, bool pdl) {
-    const size_t smem = (size_t)kScanWarps * kScanStages * kScanChunkBytes + kScanWarps * kScanStages * 8 +
-                        (size_t)kScanWarps * GPS * 32 * 8 + (size_t)(a.B + 1) * 8 + (size_t)a.B * 8;
+template <typename T, int GPS, int ROWB>
+cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
+    constexpr int W = ScanShape<GPS>::W, S = ScanShape<GPS>::S;
+    const size_t smem = 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 +
+                        (size_t)GPS * (ROWB / sizeof(T)) * 4 + (size_t)(a.B + 1) * 8 + (size_t)a.B * 8;
     static size_t attr_bytes = 0;  // opt-in raised on demand (smem grows with the batch)
     if (smem > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, LPT>,
+        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_bytes = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.n_cta);
-    cfg.blockDim = dim3(kScanWarps * 32);
+    cfg.blockDim = dim3(W * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -328,35 +354,47 @@ cudaError_t launch_scan_t(const ScanArgs &a, cudaStream_t s, bool pdl) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, LPT>, a);
+    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, ROWB>, km, a);
 }
 
-template <typename T, int LPT>
-cudaError_t launch_scan_g(const ScanArgs &a, int gps, cudaStream_t s, bool pdl) {
+template <typename T, int ROWB>
+cudaError_t launch_scan_g(const ScanArgs &a, const CUtensorMap &km, int gps, cudaStream_t s, bool pdl) {
     switch (gps) {
-        case 1: return launch_scan_t<T, 1, LPT>(a, s, pdl);
-        case 2: return launch_scan_t<T, 2, LPT>(a, s, pdl);
-        case 4: return launch_scan_t<T, 4, LPT>(a, s, pdl);
-        case 8: return launch_scan_t<T, 8, LPT>(a, s, pdl);
+        case 1: return launch_scan_t<T, 1, ROWB>(a, km, s, pdl);
+        case 2: return launch_scan_t<T, 2, ROWB>(a, km, s, pdl);
+        case 4: return launch_scan_t<T, 4, ROWB>(a, km, s, pdl);
+        case 8: return launch_scan_t<T, 8, ROWB>(a, km, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
 
 template <typename T>
-cudaError_t launch_scan_l(const ScanArgs &a, int lpt, int gps, cudaStream_t s, bool pdl) {
-    switch (lpt) {
-        case 4: return launch_scan_g<T, 4>(a, gps, s, pdl);
-        case 8: return launch_scan_g<T, 8>(a, gps, s, pdl);
-        case 16: return launch_scan_g<T, 16>(a, gps, s, pdl);
+cudaError_t launch_scan_r(const ScanArgs &a, const CUtensorMap &km, int rowb, int gps, cudaStream_t s, bool pdl) {
+    switch (rowb) {
+        case 64: return launch_scan_g<T, 64>(a, km, gps, s, pdl);
+        case 128: return launch_scan_g<T, 128>(a, km, gps, s, pdl);
+        case 256: return launch_scan_g<T, 256>(a, km, gps, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_decode_scan(const ScanArgs &a, int dtype, int lpt, int gps, cudaStream_t s, bool pdl) {
-    return dtype == MSA_F32 ? launch_scan_l<float>(a, lpt, gps, s, pdl)
-                            : launch_scan_l<__nv_bfloat16>(a, lpt, gps, s, pdl);
+cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cudaStream_t s, bool pdl) {
+    const int es = dtype == MSA_F32 ? 4 : 2;
+    int ct = kScanChunkBytes / row_bytes;
+    if (ct > a.Bk) ct = a.Bk;
+    a.chunk_tokens = ct;
+    // index keys as a 2D tensor [B * Hik * Lmax rows, di]; one box = ct rows x 128 bytes
+    // (64 for 64-byte rows), swizzled so that one lane per row reads without bank conflicts
+    const int box_x = (row_bytes >= 128 ? 128 : 64) / es;
+    CUtensorMap km;
+    if (!encode_2d(&km, dtype == MSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   const_cast<void *>(a.k_idx), row_bytes / es, (unsigned long long)a.B * a.Hik * a.L_max, row_bytes,
+                   box_x, ct, row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    return dtype == MSA_F32 ? launch_scan_r<float>(a, km, row_bytes, gps, s, pdl)
+                            : launch_scan_r<__nv_bfloat16>(a, km, row_bytes, gps, s, pdl);
 }
 
 cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s) {

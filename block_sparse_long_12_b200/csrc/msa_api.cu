@@ -90,6 +90,8 @@ msa_status_t check_params(const msa_params_t *p, Mode mode) {
     if (p->top_k < 1) return fail(MSA_ERR_INVALID_ARG, "top_k %d < 1", p->top_k);
     if (p->top_k > kMaxTopK) return fail(MSA_ERR_UNSUPPORTED, "top_k %d > %d", p->top_k, kMaxTopK);
     if (p->max_seq_len < 1) return fail(MSA_ERR_INVALID_ARG, "max_seq_len %d < 1", p->max_seq_len);
+    if ((long long)p->batch * p->n_kv_heads * p->max_seq_len >= (1LL << 31))
+        return fail(MSA_ERR_UNSUPPORTED, "batch * n_kv_heads * max_seq_len must stay below 2^31 cache rows");
     if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale))
         return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
     if (p->flags & ~(MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_DENSE))
@@ -282,8 +284,7 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
     a.token_scores = mode == MSA_SCORES_TOKEN ? scores_out : nullptr;
     a.block_scores = mode == MSA_SCORES_BLOCKMAX ? scores_out : nullptr;
     a.status = reinterpret_cast<int *>(ws);
-    const int lpt = p->idx_dim * elem_size(p->dtype) / 16;
-    e = launch_decode_scan(a, p->dtype, lpt, p->n_kv_heads / p->n_idx_k_heads, s, false);
+    e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     return MSA_OK;
 }
@@ -389,10 +390,9 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.cand_i = reinterpret_cast<int *>(wsb + L.cand_i);
     a.seg_info = reinterpret_cast<SegInfo *>(wsb + L.seg_info);
     a.status = reinterpret_cast<int *>(wsb);
-    const int lpt = p->idx_dim * elem_size(p->dtype) / 16;
     cudaError_t e = stage_mark(0, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    e = launch_decode_scan(a, p->dtype, lpt, p->n_kv_heads / p->n_idx_k_heads, s, false);
+    e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     SelectArgs sa{};

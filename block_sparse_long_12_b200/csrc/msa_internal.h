@@ -1,6 +1,7 @@
 // Internal declarations shared by the MSA translation units (host + device).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -19,9 +20,7 @@ constexpr int kMaxPiecesPerSeg = 256; // lists merged per (segment, group) by on
 constexpr size_t kStatusBytes = 256;  // workspace head: device status word + padding
 
 // ---- decode index scan (Step 1 for decode): persistent, 1 CTA per SM
-constexpr int kScanWarps = 8;
-constexpr int kScanStages = 3;          // per-warp ring depth
-constexpr int kScanChunkBytes = 8192;   // bytes of index keys per bulk copy
+constexpr int kScanChunkBytes = 8192;   // ring stage: bytes of index keys per TMA copy
 
 // ---- decode sparse attention (Step 2 for decode)
 constexpr int kAttnThreads = 256;
@@ -41,6 +40,7 @@ struct ScanArgs {
     const int *seq_lens;
     int B, G, Hik, di, Bk, k, L_max, nb_max;
     int n_cta;
+    int chunk_tokens;      // tokens per bulk copy (set by the launcher)
     float *cand_s;  // [n_seg, n_cta, G/Hik, k] per-piece sorted top-k (nullable)
     int *cand_i;
     SegInfo *seg_info;     // [n_seg] (written by CTA 0 when cand_s != nullptr)
@@ -107,7 +107,7 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
 
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);
-cudaError_t launch_decode_scan(const ScanArgs &a, int dtype, int lpt, int gps, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
@@ -115,5 +115,12 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
                                  cudaStream_t s, const char **why);
 
 int num_sms();
+
+// TMA tensor maps (host); false if the driver cannot encode the map
+bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, void *base, unsigned long long inner,
+               unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_x, unsigned box_y,
+               CUtensorMapSwizzle swizzle);
+bool encode_3d(CUtensorMap *map, CUtensorMapDataType dt, void *base, const unsigned long long dims[3],
+               const unsigned long long strides_bytes[2], const unsigned box[3], CUtensorMapSwizzle swizzle);
 
 }  // namespace msa

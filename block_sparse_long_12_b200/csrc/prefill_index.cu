@@ -20,8 +20,6 @@
 //               of the scores, causal mask on diagonal tiles, 3-input max per
 //               32 columns, block max, and a register-resident sorted top-k.
 // The next tile's MMAs overlap the epilogue of the current one.
-#include <cudaTypedefs.h>
-
 #include "tcgen05.cuh"
 
 namespace msa {
@@ -274,18 +272,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 template <int K>
 cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid,
                      cudaStream_t s) {
@@ -305,32 +291,19 @@ cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUten
 
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
                                  cudaStream_t s, const char **why) {
-    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
-    if (enc == nullptr) {
-        *why = "cuTensorMapEncodeTiled is not available from the driver";
-        return cudaErrorNotSupported;
-    }
     CUtensorMap qm, km;
     // q_idx [B*T, G, 64] bf16: box of 64 dims x 1 group x 128 rows
-    const cuuint64_t qdim[3] = {64, (cuuint64_t)a.G, (cuuint64_t)a.B * a.T};
-    const cuuint64_t qstr[2] = {64 * 2, (cuuint64_t)a.G * 64 * 2};
-    const cuuint32_t qbox[3] = {64, 1, kRows};
-    const cuuint32_t ones[3] = {1, 1, 1};
-    CUresult r = enc(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q_idx), qdim, qstr, qbox, ones,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
+    const unsigned long long qdim[3] = {64, (unsigned long long)a.G, (unsigned long long)a.B * a.T};
+    const unsigned long long qstr[2] = {64 * 2, (unsigned long long)a.G * 64 * 2};
+    const unsigned qbox[3] = {64, 1, kRows};
+    if (!encode_3d(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(q_idx), qdim, qstr, qbox,
+                   CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "encoding the index-query tensor map failed";
         return cudaErrorInvalidValue;
     }
     // k_idx [B*Hik*Lmax, 64] bf16: box of 64 dims x 128 keys
-    const cuuint64_t kdim[2] = {64, (cuuint64_t)a.B * a.Hik * a.L_max};
-    const cuuint64_t kstr[1] = {64 * 2};
-    const cuuint32_t kbox[2] = {64, kKeys};
-    r = enc(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(k_idx), kdim, kstr, kbox, ones,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
+    if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(k_idx), 64,
+                   (unsigned long long)a.B * a.Hik * a.L_max, 128, 64, kKeys, CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "encoding the index-key tensor map failed";
         return cudaErrorInvalidValue;
     }

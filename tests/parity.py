@@ -40,11 +40,29 @@ def oracle_block_score(p: oracle.Params, x: dict, b: int, t: int, g: int, pos: i
     return float(oracle.block_scores(p, s, pos)[n])
 
 
-def check_ids_row(p, x, b, t, g, pos, gpu_ids, ref_ids, kth, kth_next, where=""):
-    """Returns True if the row is exact, False if it passed under the near-tie rule (raises otherwise)."""
+def _close(a, b):
+    return abs(a - b) <= TIE_REL * max(abs(a), abs(b))
+
+
+def check_ids_row(p, x, b, t, g, pos, gpu_ids, ref_ids, kth, kth_next, where="", ref_scores=None):
+    """Returns True if the row is exact, False if it passed under the near-tie rule (raises otherwise).
+
+    The same set in another order is exact when every position that differs
+    holds two blocks whose oracle scores are within the tie tolerance (the
+    list is ordered by score, which fp32 and fp64 may order differently)."""
     gpu_ids = [int(i) for i in gpu_ids]
     ref_ids = [int(i) for i in ref_ids]
     if gpu_ids == ref_ids:
+        return True
+    if sorted(gpu_ids) == sorted(ref_ids):
+        def score(i):
+            if ref_scores is not None:
+                return float(ref_scores[ref_ids.index(i)])
+            return oracle_block_score(p, x, b, t, g, pos, i)
+        for a_, r_ in zip(gpu_ids, ref_ids):
+            if a_ != r_:
+                assert a_ >= 0 and r_ >= 0 and _close(score(a_), score(r_)), \
+                    f"{where}: order differs beyond ties: gpu {gpu_ids} oracle {ref_ids}"
         return True
     tie = (not math.isnan(kth) and not math.isnan(kth_next)
            and abs(kth - kth_next) <= TIE_REL * max(abs(kth), abs(kth_next)))
@@ -83,7 +101,7 @@ def compare_decode(x: dict, p: oracle.Params, o_gpu, ids_gpu, lse_gpu, batches=N
         if ids is not None and not p.dense:
             for g in range(G):
                 exact = check_ids_row(p, x, b, 0, g, pos, ids[b, 0, g], ref["ids"][i, g], ref["kth"][i, g],
-                                      ref["kth_next"][i, g], where=f"b={b} g={g}")
+                                      ref["kth_next"][i, g], where=f"b={b} g={g}", ref_scores=ref["top_scores"][i, g])
                 if not exact:
                     tie_rows.append((i, b, g))
     o_ref = ref["o"].copy()

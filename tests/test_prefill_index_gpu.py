@@ -50,7 +50,8 @@ def check_rows(inp, w, q_start, T, ids, rows, top_k=None, block_size=None):
     for i, (b, t) in enumerate(rows):
         for g in range(w.n_kv_heads):
             exact = check_ids_row(p, xo, b, t, g, q_start + t, idn[b, t, g], ref["ids"][i, g], ref["kth"][i, g],
-                                  ref["kth_next"][i, g], where=f"b={b} t={t} g={g}")
+                                  ref["kth_next"][i, g], where=f"b={b} t={t} g={g}",
+                                  ref_scores=ref["top_scores"][i, g])
             ties += not exact
     return ties
 
