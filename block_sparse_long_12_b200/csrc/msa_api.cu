@@ -411,8 +411,36 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
                                      const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
                                      msa_stream_t stream) {
     MSA_TRY(check_params(p, PREFILL_ONLY));
-    (void)q; (void)k_cache; (void)v_cache; (void)ids; (void)o; (void)lse; (void)ws; (void)ws_bytes; (void)stream;
-    return fail(MSA_ERR_UNSUPPORTED, "msa_sparse_attn_prefill is not built yet");
+    if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_sparse_attn_prefill takes no flags");
+    if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
+    if (p->block_size != 64 && p->block_size != 128)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes block_size 64 or 128");
+    const int r = p->n_q_heads / p->n_kv_heads;
+    if (128 % r != 0) return fail(MSA_ERR_UNSUPPORTED, "prefill attention needs a group size dividing 128");
+    if ((128 / r) * p->top_k > 512)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill attention: (128 / group size) * top_k must not exceed 512");
+    if ((((long long)p->max_seq_len + p->block_size - 1) / p->block_size + 31) / 32 > 2048)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill attention: at most 65536 blocks per sequence");
+    MSA_TRY(check_ptr(q, "q"));
+    MSA_TRY(check_ptr(k_cache, "k_cache"));
+    MSA_TRY(check_ptr(v_cache, "v_cache"));
+    MSA_TRY(check_ptr(ids, "ids"));
+    MSA_TRY(check_ptr(o, "o"));
+    MSA_TRY(check_ptr(lse, "lse", true));
+    MSA_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    PrefillAttnArgs a{};
+    a.ids = ids; a.o = o; a.lse = lse;
+    a.B = p->batch; a.T = p->q_len; a.Hq = p->n_q_heads; a.G = p->n_kv_heads; a.D = p->head_dim;
+    a.Bk = p->block_size; a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len; a.r = r;
+    a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
+    a.status = reinterpret_cast<int *>(ws);
+    const char *why = "";
+    cudaError_t e = launch_prefill_attn(a, q, k_cache, v_cache, n_sm, (cudaStream_t)stream, &why);
+    if (e != cudaSuccess) return cuda_fail(e, why);
+    return MSA_OK;
 }
 
 msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, const void *k_idx, int32_t *ids_out,

@@ -93,6 +93,16 @@ struct PrefillIdxArgs {
     int *status;
 };
 
+struct PrefillAttnArgs {
+    const int *ids;            // [B, T, G, k]
+    void *o;                   // [B, T, Hq, D] bf16
+    float *lse;                // [B, T, Hq] nullable
+    int B, T, Hq, G, D, Bk, k, q_start, L_max, r;
+    float scale_log2;
+    int max_union, mask_words, bitmap_words;  // set by the launcher
+    int *status;
+};
+
 struct FillArgs {
     float *scores;
     long long n;
@@ -111,6 +121,8 @@ cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cu
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
+cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_cache, const void *v_cache, int n_sm,
+                                cudaStream_t s, const char **why);
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
                                  cudaStream_t s, const char **why);
 
