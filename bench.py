@@ -258,24 +258,23 @@ def run_ours(args, world, rank, local):
     assert _lib.msa_get_device_status(ws) == 0, "device status word reports a timeout"
 
     # per-kernel durations inside the same step (stage events; separate pass)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     for e in evs:
         e.record(stream)
     torch.cuda.synchronize()
     _lib.msa_set_stage_events(evs)
-    stage = [[], [], []]  # index scan, TopK merge, sparse attention (+ split merge)
+    stage = [[], []]  # index scan; TopK merge + sparse attention + split merge
     try:
         for _ in range(args.steps):
             flush()
             step()
             torch.cuda.synchronize()
-            for i in range(3):
+            for i in range(2):
                 stage[i].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
     finally:
         _lib.msa_set_stage_events(None)
     scan_us = max_over_ranks(statistics.mean(stage[0]), world)
-    sel_us = max_over_ranks(statistics.mean(stage[1]), world)
-    attn_us = max_over_ranks(statistics.mean(stage[2]), world)
+    attn_us = max_over_ranks(statistics.mean(stage[1]), world)
 
     # dense GQA decode over the same cache (the sparse-vs-dense ratio)
     pd = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens,
@@ -363,13 +362,12 @@ def run_ours(args, world, rank, local):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "peak_kind": peak_kind, "algorithmic_bytes": scan_bytes, "kernel_us": round(scan_us, 2),
                      "traffic": traffic},
-        "stages_us": {"index_scan": round(scan_us, 2), "topk_merge": round(sel_us, 2),
-                      "sparse_attention": round(attn_us, 2)},
+        "stages_us": {"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)},
         "step_roofline_frac": round((scan_bytes + w.batch * w.n_kv_heads * w.top_k * w.block_size * w.head_dim * es * 2)
                                     / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
         "dense_gqa_us": round(dense_us, 2), "sparse_vs_dense_speedup": round(dense_us / step_us, 2),
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -153,9 +153,9 @@ def msa_clear_device_status(ws, stream=None):
 
 
 def msa_set_stage_events(events):
-    """events: a list of 4 torch.cuda.Event (created, not yet recorded) or None to unset."""
+    """events: a list of 3 recorded-once torch.cuda.Event, or None to unset."""
     if not events:
         _check(lib().msa_set_stage_events(None, 0))
         return
-    arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
-    _check(lib().msa_set_stage_events(arr, 4))
+    arr = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
+    _check(lib().msa_set_stage_events(arr, 3))

@@ -5,21 +5,21 @@
 // Q4/Q5/Q6 -> I2) and attends over only those blocks of the full, real K/V
 // cache, so one group loads one set of KV blocks for all its heads.
 //
-// decode_select_kernel finishes Step 1: one CTA per (sequence, group) stages
-// the scan's per-piece sorted candidate lists in shared memory and selects
-// the group's final TopK list from them.
+// Grid (split s, group g, sequence b); split s owns list positions
+// [s * blocks_per_split, ...).  In the fused decode step a CTA first finishes
+// Step 1 for its group (select_group_topk: the scan's per-piece sorted
+// candidate lists are staged in shared memory and the k best kept).  Then it
+// streams its blocks' K/V tiles through a TMA ring and keeps an online
+// softmax for all r heads of the group.  Each split writes a normalised
+// partial output and its log2 normaliser; the last split of a group to
+// finish (atomic arrival count) merges them by log-sum-exp.  With MSA_DENSE
+// the splits cover every visible block: plain GQA decode.
 //
-// decode_attn_kernel, grid (split s, group g, sequence b): a CTA reads the
-// group's list, streams the K/V tiles of its share of the blocks through a
-// two-stage TMA bulk-copy ring and keeps an online softmax for all r heads
-// of the group: scores with one warp per key (lanes split the head
-// dimension, a reduce-scatter butterfly finishes the r dot products), then
-// per-head max/exp2/sum, then P.V with each thread owning a few output
-// elements.  Each split writes a normalised partial output and its log2
-// normaliser; the last split of a group to finish (atomic arrival count)
-// merges them by log-sum-exp into the output.  With MSA_DENSE the splits
-// cover every visible block: plain GQA decode.
-#include "msa_device.cuh"
+// bf16: decode_attn_mma_kernel runs both products on mma.sync tensor-core
+// fragments (the r <= 16 heads padded to 16 rows), K/V tiles in the 128-byte
+// swizzle layout written by TMA tensor copies.  fp32: decode_attn_kernel on
+// CUDA cores (exact fp32 products).
+#include "tcgen05.cuh"
 
 namespace msa {
 
@@ -87,6 +87,130 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
     return x[0];
 }
 
+
+// Final TopK of group g of sequence b from the scan's per-piece sorted lists
+// (the fused decode step).  The candidates are staged in `scratch` (at least
+// 16 * n_cta * k bytes); a candidate worse than the k-th entry of some full
+// list cannot be among the final k (that list alone has k better ones), so
+// only the survivors are ranked, each by counting the survivors that beat
+// it.  Leaves the list in sel_s / sel_i[0..32), padded with (-inf, -1).
+// Called by every thread of the CTA.
+__device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i,
+                                  float *red_s, int *red_i, int *n_surv) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int cap = a.n_cta * a.k;
+    float *ls = reinterpret_cast<float *>(scratch);
+    int *li = reinterpret_cast<int *>(ls + cap);
+    float *ss = reinterpret_cast<float *>(li + cap);
+    int *si = reinterpret_cast<int *>(ss + cap);
+    const int gps = a.G / a.Hik;
+    const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
+    const SegInfo info = a.seg_info[seg];
+    const int n = info.n_pieces * a.k;
+    for (int i = tid; i < n; i += nthr) {
+        const size_t src = (((size_t)seg * a.n_cta + i / a.k) * gps + gl) * a.k + i % a.k;
+        ls[i] = a.cand_s[src];
+        li[i] = a.cand_i[src];
+    }
+    if (tid < 32) { sel_s[tid] = -INFINITY; sel_i[tid] = -1; }
+    if (tid == 0) *n_surv = 0;
+    __syncthreads();
+    float ts = -INFINITY;
+    int ti = -1;
+    for (int l = tid; l < info.n_pieces; l += nthr) {
+        const float s = ls[l * a.k + a.k - 1];
+        const int i = li[l * a.k + a.k - 1];
+        if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
+    }
+    warp_best(ts, ti);
+    if (lane == 0) { red_s[warp] = ts; red_i[warp] = ti; }
+    __syncthreads();
+    ts = red_s[0];
+    ti = red_i[0];
+    for (int w2 = 1; w2 < nwarps; ++w2)
+        if (better(red_s[w2], red_i[w2], ts, ti)) { ts = red_s[w2]; ti = red_i[w2]; }
+    for (int i = tid; i < n; i += nthr) {
+        if (li[i] >= 0 && !better(ts, ti, ls[i], li[i])) {
+            const int at = atomicAdd(n_surv, 1);
+            ss[at] = ls[i];
+            si[at] = li[i];
+        }
+    }
+    __syncthreads();
+    const int m = *n_surv;
+    for (int i = tid; i < m; i += nthr) {
+        const float s = ss[i];
+        const int id = si[i];
+        int rank = 0;
+        for (int j = 0; j < m; ++j) rank += better(ss[j], si[j], s, id) ? 1 : 0;
+        if (rank < a.k) { sel_s[rank] = s; sel_i[rank] = id; }
+    }
+    __syncthreads();
+}
+
+// The last split CTA of (b, g) merges the normalised partial outputs of all
+// splits by log-sum-exp (weights staged in `wgt`, S * r floats).
+template <typename T>
+__device__ void merge_splits(const AttnArgs &a, int b, int g, float *wgt) {
+    const int tid = threadIdx.x, nthr = blockDim.x, r = a.r, D = a.D;
+    const size_t bg = (size_t)b * a.G + g;
+    __threadfence();
+    for (int i = tid; i < a.S * r; i += nthr) wgt[i] = __ldcg(a.part_lse + bg * a.S * r + i);
+    __syncthreads();
+    if (tid < r) {
+        float M = -INFINITY;
+        for (int j = 0; j < a.S; ++j) M = fmaxf(M, wgt[j * r + tid]);
+        float den = 0.f;
+        for (int j = 0; j < a.S; ++j) {
+            const float e = M > -INFINITY ? exp2f(wgt[j * r + tid] - M) : 0.f;
+            wgt[j * r + tid] = e;
+            den += e;
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        for (int j = 0; j < a.S; ++j) wgt[j * r + tid] *= inv;
+        if (a.lse != nullptr)
+            a.lse[(size_t)b * a.Hq + (size_t)g * r + tid] =
+                den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+    T *o = reinterpret_cast<T *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
+    const float *po = a.part_o + bg * a.S * r * D;
+    for (int f = tid; f < r * D; f += nthr) {
+        const int h = f / D;
+        float num = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < a.S; ++j) num = fmaf(wgt[j * r + h], __ldcg(po + ((size_t)j * r) * D + f), num);
+        store_elem(o + f, num);
+    }
+    if (tid == 0) a.counters[bg] = 0;  // ready for the next call
+}
+
+// True in every thread of the CTA that finished last among the S splits of (b, g).
+__device__ inline bool last_split(const AttnArgs &a, int b, int g, int *flag) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) *flag = (atomicAdd(&a.counters[(size_t)b * a.G + g], 1) == a.S - 1) ? 1 : 0;
+    __syncthreads();
+    return *flag != 0;
+}
+
+// Obtain the group's list: fused selection from the scan, or a given ids tensor.
+__device__ inline void group_list(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i,
+                                  float *red_s, int *red_i, int *n_surv) {
+    if (a.dense) return;
+    if (a.cand_s != nullptr) {
+        select_group_topk(a, b, g, scratch, sel_s, sel_i, red_s, red_i, n_surv);
+        if (blockIdx.x == 0 && threadIdx.x < a.k) {
+            const size_t o = ((size_t)b * a.G + g) * a.k + threadIdx.x;
+            if (a.ids_out != nullptr) a.ids_out[o] = sel_i[threadIdx.x];
+            if (a.top_scores_out != nullptr) a.top_scores_out[o] = sel_s[threadIdx.x];
+        }
+    } else {
+        if (threadIdx.x < a.k) sel_i[threadIdx.x] = a.ids_in[((size_t)b * a.G + g) * a.k + threadIdx.x];
+        __syncthreads();
+    }
+}
+
 template <typename T, int D, int R>
 struct AttnCfg {
     static constexpr int ES = (int)sizeof(T);
@@ -104,8 +228,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const size_t tile_bytes = (size_t)KT * D * ES;
 
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *ring = smem;                                             // [NST][K tile | V tile]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + NST * 2 * tile_bytes); // [NST]
+    unsigned char *ring = smem;  // [NST][K tile | V tile]; also the selection scratch
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + a.ring_bytes);  // [NST]
     float *sel_s = reinterpret_cast<float *>(bars + NST);                   // [32]
     int *sel_i = reinterpret_cast<int *>(sel_s + 32);                       // [32]
     float *m_s = reinterpret_cast<float *>(sel_i + 32);                     // running max (log2 domain)
@@ -140,10 +264,11 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const int pos = L - 1;
     const int nb = (L + a.Bk - 1) / a.Bk;
 
-    pdl_wait_prior_grid();  // the selection is complete from here on
+    pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
-    if (!a.dense && tid < a.k) sel_i[tid] = a.ids_in[((size_t)b * a.G + g) * a.k + tid];
-    __syncthreads();
+    __shared__ float red_s[32];
+    __shared__ int red_i[32], n_surv, last_flag;
+    group_list(a, b, g, ring, sel_s, sel_i, red_s, red_i, &n_surv);
 
     // this split's blocks: list positions [j0, j1)
     const int bps = a.blocks_per_split;
@@ -297,130 +422,296 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
         a.part_lse[split * r + tid] = l > 0.f ? m_s[tid] + log2f(l) : -INFINITY;
     }
 
-    // the last split of (b, g) to arrive merges all splits
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) sel_s[0] = (atomicAdd(&a.counters[bg], 1) == a.S - 1) ? 1.f : 0.f;
-    __syncthreads();
-    if (sel_s[0] == 0.f) return;
-    __threadfence();
-    float *wgt = p_s;  // [S][r] merge weights (S <= max(k, kMaxSplits))
-    for (int i = tid; i < a.S * r; i += kAttnThreads) wgt[i] = __ldcg(a.part_lse + bg * a.S * r + i);
-    __syncthreads();
-    if (tid < r) {
-        float M = -INFINITY;
-        for (int j = 0; j < a.S; ++j) M = fmaxf(M, wgt[j * r + tid]);
-        float den = 0.f;
-        for (int j = 0; j < a.S; ++j) {
-            const float e = M > -INFINITY ? exp2f(wgt[j * r + tid] - M) : 0.f;
-            wgt[j * r + tid] = e;
-            den += e;
-        }
-        const float inv = den > 0.f ? 1.f / den : 0.f;
-        for (int j = 0; j < a.S; ++j) wgt[j * r + tid] *= inv;
-        if (a.lse != nullptr)
-            a.lse[(size_t)b * a.Hq + (size_t)g * r + tid] =
-                den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
-    }
-    __syncthreads();
-    T *o = reinterpret_cast<T *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
-    const float *po = a.part_o + bg * a.S * r * D;
-    for (int f = tid; f < r * D; f += kAttnThreads) {
-        const int h = f / D;
-        float num = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < a.S; ++j) num = fmaf(wgt[j * r + h], __ldcg(po + ((size_t)j * r) * D + f), num);
-        store_elem(o + f, num);
-    }
-    if (tid == 0) a.counters[bg] = 0;  // ready for the next call
+    if (!last_split(a, b, g, &last_flag)) return;
+    merge_splits<T>(a, b, g, p_s);  // p_s holds R * max(KT, kMaxSplits) floats
 }
 
-// Final TopK of a group from the scan's per-piece sorted lists.  All
-// candidates are staged in shared memory; any candidate worse than the k-th
-// entry of some full list cannot be in the final k (that list alone already
-// has k better ones), so only the survivors are ranked, each by counting the
-// survivors that beat it.
-__global__ void __launch_bounds__(256) decode_select_kernel(const SelectArgs a) {
-    extern __shared__ __align__(16) unsigned char sm_raw[];
-    const int cap = a.n_cta * a.k;
-    float *ls = reinterpret_cast<float *>(sm_raw);
-    int *li = reinterpret_cast<int *>(ls + cap);
-    float *ss = reinterpret_cast<float *>(li + cap);   // survivors
-    int *si_ = reinterpret_cast<int *>(ss + cap);
-    float *out_s = reinterpret_cast<float *>(si_ + cap);
-    int *out_i = reinterpret_cast<int *>(out_s + 32);
-    __shared__ float thr_s[8];
-    __shared__ int thr_i[8];
-    __shared__ int n_surv;
-    const int g = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_wait_prior_grid();
-    pdl_allow_next_grid();
-    const int gps = a.G / a.Hik;
-    const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
-    const SegInfo si = a.seg_info[seg];
-    const int n = si.n_pieces * a.k;
-    for (int i = tid; i < n; i += blockDim.x) {
-        const size_t src = (((size_t)seg * a.n_cta + i / a.k) * gps + gl) * a.k + i % a.k;
-        ls[i] = a.cand_s[src];
-        li[i] = a.cand_i[src];
+
+// ---------------------------------------------------------------- bf16: mma.sync tensor-core fragments
+__device__ inline void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ inline void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// byte offset of 16-byte vector c (0..7) of row `row` in a 128-byte-swizzled tile of 128-byte rows
+__device__ inline uint32_t sw128(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
+
+constexpr int kMmaThreads = 128;  // 4 warps
+constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
+
+template <int D>
+__global__ void __launch_bounds__(kMmaThreads) decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                                      const __grid_constant__ CUtensorMap vmap,
+                                                                      const AttnArgs a) {
+    constexpr int NH = D / 64;     // 64-dim halves of a K/V row
+    constexpr int KS = D / 16;     // k-steps of Q.K^T
+    constexpr int DT = D / 8 / 4;  // 8-dim output tiles per warp
+    const int KT = a.Bk < 128 ? a.Bk : 128;  // keys per tile
+    const int KVH = KT * 128;                // bytes of one 64-dim half tile
+    const int STAGE = 2 * NH * KVH;
+    const int PST = KT + 8;                  // P row stride (bf16 elements), padded against bank conflicts
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    __nv_bfloat16 *Ps = reinterpret_cast<__nv_bfloat16 *>(ring + a.ring_bytes);   // [16][PST]
+    float *red_m = reinterpret_cast<float *>(Ps + kMmaRows * PST);                 // [4][16]
+    float *red_l = red_m + 64;                                                     // [4][16]
+    float *sel_s = red_l + 64;                                                     // [32]
+    int *sel_i = reinterpret_cast<int *>(sel_s + 32);                              // [32]
+    float *red_s = reinterpret_cast<float *>(sel_i + 32);                          // [32]
+    int *red_i = reinterpret_cast<int *>(red_s + 32);                              // [32]
+    int *misc = red_i + 32;                                                        // [4]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 4);                       // [2]
+
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, tig = lane & 3;  // fragment row group / thread in group
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int r = a.r;
+    const int nst = a.nst;
+
+    if (tid == 0) {
+        for (int i = 0; i < nst; ++i) mbar_init(&bars[i], 1);
+        fence_mbar_init();
+        tc::prefetch_tmap(&kmap);
+        tc::prefetch_tmap(&vmap);
     }
-    if (tid < 32) { out_s[tid] = -INFINITY; out_i[tid] = -1; }
-    if (tid == 0) n_surv = 0;
-    __syncthreads();
-    // threshold: the best k-th entry over all lists
-    float ts = -INFINITY;
-    int ti = -1;
-    for (int l = tid; l < si.n_pieces; l += blockDim.x) {
-        const float s = ls[l * a.k + a.k - 1];
-        const int i = li[l * a.k + a.k - 1];
-        if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
-    }
-    warp_best(ts, ti);
-    if (lane == 0) { thr_s[warp] = ts; thr_i[warp] = ti; }
-    __syncthreads();
-    ts = thr_s[0];
-    ti = thr_i[0];
-    for (int w2 = 1; w2 < 8; ++w2)
-        if (better(thr_s[w2], thr_i[w2], ts, ti)) { ts = thr_s[w2]; ti = thr_i[w2]; }
-    for (int i = tid; i < n; i += blockDim.x) {
-        if (li[i] >= 0 && !better(ts, ti, ls[i], li[i])) {
-            const int at = atomicAdd(&n_surv, 1);
-            ss[at] = ls[i];
-            si_[at] = li[i];
+    // Q fragments (rows = heads of the group; rows >= r are zero), independent of Step 1
+    uint32_t qa[KS][4];
+    {
+        const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + (size_t)g * r) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int c0 = ks * 16 + tig * 2;
+            qa[ks][0] = grp < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)grp * D + c0) : 0u;
+            qa[ks][1] = grp + 8 < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)(grp + 8) * D + c0) : 0u;
+            qa[ks][2] = grp < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)grp * D + c0 + 8) : 0u;
+            qa[ks][3] = grp + 8 < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)(grp + 8) * D + c0 + 8) : 0u;
         }
     }
-    __syncthreads();
-    const int m = n_surv;
-    for (int i = tid; i < m; i += blockDim.x) {
-        const float s = ss[i];
-        const int id = si_[i];
-        int rank = 0;
-        for (int j = 0; j < m; ++j) rank += better(ss[j], si_[j], s, id) ? 1 : 0;
-        if (rank < a.k) { out_s[rank] = s; out_i[rank] = id; }
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int pos = L - 1;
+    const int nb = (L + a.Bk - 1) / a.Bk;
+
+    pdl_wait_prior_grid();  // the scan's candidates are complete from here on
+    pdl_allow_next_grid();
+    group_list(a, b, g, ring, sel_s, sel_i, red_s, red_i, &misc[0]);
+
+    // this split's blocks: list positions [j0, j1), each cut into tiles of KT keys
+    const int j0 = s * a.blocks_per_split;
+    int j1 = j0 + a.blocks_per_split;
+    const int jmax = a.dense ? nb : a.k;
+    if (j1 > jmax) j1 = jmax;
+    auto block_at = [&](int j) -> int {
+        const int id = a.dense ? j : sel_i[j];
+        return (id >= 0 && id < nb) ? id : -1;
+    };
+    auto tiles_of = [&](int id) -> int {
+        if (id < 0) return 0;
+        int keys = pos + 1 - id * a.Bk;
+        keys = keys < a.Bk ? keys : a.Bk;
+        return (keys + KT - 1) / KT;
+    };
+    int pj = j0, pt = 0, issued = 0;
+    while (pj < j1 && tiles_of(block_at(pj)) == 0) ++pj;
+    const int row0 = (b * a.G + g) * a.L_max;
+    auto issue = [&]() {
+        const int id = block_at(pj);
+        const int slot = issued % nst;
+        if (tid == 0) {
+            unsigned char *dst = ring + slot * STAGE;
+            mbar_arrive_expect_tx(&bars[slot], STAGE);
+            const int row = row0 + id * a.Bk + pt * KT;
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                tc::tma_load_2d(dst + h * KVH, &kmap, h * 64, row, &bars[slot]);
+                tc::tma_load_2d(dst + (NH + h) * KVH, &vmap, h * 64, row, &bars[slot]);
+            }
+        }
+        ++issued;
+        if (++pt >= tiles_of(id)) {
+            pt = 0;
+            ++pj;
+            while (pj < j1 && tiles_of(block_at(pj)) == 0) ++pj;
+        }
+    };
+    __syncthreads();  // barrier init and the list visible; the selection scratch is free
+    for (int i = 0; i < nst && pj < j1; ++i) issue();
+
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    float oacc[DT][4];
+#pragma unroll
+    for (int t = 0; t < DT; ++t) oacc[t][0] = oacc[t][1] = oacc[t][2] = oacc[t][3] = 0.f;
+    const uint32_t ps_addr = smem_u32(Ps);
+    int consumed = 0;
+    bool failed = false;
+    for (int j = j0; j < j1; ++j) {
+        const int id = block_at(j);
+        const int ntl = tiles_of(id);
+        for (int t = 0; t < ntl; ++t) {
+            const int key0 = id * a.Bk + t * KT;
+            int nk = pos + 1 - key0;
+            nk = nk < KT ? nk : KT;
+            const int slot = consumed % nst;
+            if (!failed && !mbar_wait(&bars[slot], (consumed / nst) & 1, a.status)) {
+                failed = true;
+                for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&bars[q2 % nst], (q2 / nst) & 1, nullptr);
+            }
+            const uint32_t k_addr = smem_u32(ring + slot * STAGE);
+            const uint32_t v_addr = k_addr + NH * KVH;
+            // S = Q K^T for this warp's 8-key tiles kn = w, w+4, ...
+            float mx[2] = {-INFINITY, -INFINITY};
+            float sv[4][4];
+            const int n_kt = KT / 8;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kn = w + 4 * i;
+                sv[i][0] = sv[i][1] = sv[i][2] = sv[i][3] = 0.f;
+                if (kn < n_kt) {
+#pragma unroll
+                    for (int ks = 0; ks < KS; ks += 2) {
+                        const int mi = lane >> 3;
+                        const int key = kn * 8 + (lane & 7);
+                        const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(k_addr + (d0 >> 6) * KVH + sw128(key, (d0 & 63) >> 3), b0, b1, b2, b3);
+                        mma_16816(sv[i], qa[ks], b0, b1);
+                        mma_16816(sv[i], qa[ks + 1], b2, b3);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = kn * 8 + tig * 2 + (e & 1);
+                        sv[i][e] = key < nk ? sv[i][e] * a.scale_log2 : -INFINITY;
+                        mx[e >> 1] = fmaxf(mx[e >> 1], sv[i][e]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(FULL, mx[h], 1));
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(FULL, mx[h], 2));
+            }
+            if (tig == 0) { red_m[w * 16 + grp] = mx[0]; red_m[w * 16 + grp + 8] = mx[1]; }
+            __syncthreads();
+            float alpha[2], m_new[2], ls[2] = {0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = grp + 8 * h;
+                const float mb = fmaxf(fmaxf(red_m[row], red_m[16 + row]), fmaxf(red_m[32 + row], red_m[48 + row]));
+                m_new[h] = fmaxf(m_run[h], mb);
+                alpha[h] = m_run[h] > -INFINITY ? exp2f(m_run[h] - m_new[h]) : 0.f;
+            }
+            // P = exp2(S - m) as bf16 into shared memory
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kn = w + 4 * i;
+                if (kn < n_kt) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float p0 = sv[i][2 * h] > -INFINITY ? exp2f(sv[i][2 * h] - m_new[h]) : 0.f;
+                        const float p1 = sv[i][2 * h + 1] > -INFINITY ? exp2f(sv[i][2 * h + 1] - m_new[h]) : 0.f;
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        ls[h] += __low2float(pb) + __high2float(pb);
+                        *reinterpret_cast<__nv_bfloat162 *>(Ps + (grp + 8 * h) * PST + kn * 8 + tig * 2) = pb;
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                ls[h] += __shfl_xor_sync(FULL, ls[h], 1);
+                ls[h] += __shfl_xor_sync(FULL, ls[h], 2);
+            }
+            if (tig == 0) { red_l[w * 16 + grp] = ls[0]; red_l[w * 16 + grp + 8] = ls[1]; }
+            __syncthreads();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int row = grp + 8 * h;
+                const float lb = red_l[row] + red_l[16 + row] + red_l[32 + row] + red_l[48 + row];
+                l_run[h] = l_run[h] * alpha[h] + lb;
+                m_run[h] = m_new[h];
+            }
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                oacc[dt][0] *= alpha[0]; oacc[dt][1] *= alpha[0];
+                oacc[dt][2] *= alpha[1]; oacc[dt][3] *= alpha[1];
+            }
+            // O += P V: this warp's 8-dim output tiles dn = w, w+4, ...
+            for (int ks = 0; ks < KT / 16; ++ks) {
+                uint32_t pa[4];
+                {
+                    const int mi = lane >> 3;
+                    const int row = (mi & 1) * 8 + (lane & 7);
+                    const int key = ks * 16 + (mi >> 1) * 8;
+                    ldsm_x4(ps_addr + (uint32_t)(row * PST + key) * 2, pa[0], pa[1], pa[2], pa[3]);
+                }
+#pragma unroll
+                for (int dp = 0; dp < DT; dp += 2) {
+                    const int mi = lane >> 3;
+                    const int dn = w + 4 * (dp + (mi >> 1));
+                    const int key = ks * 16 + (mi & 1) * 8 + (lane & 7);
+                    const int d0 = dn * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(v_addr + (d0 >> 6) * KVH + sw128(key, (d0 & 63) >> 3), b0, b1, b2, b3);
+                    mma_16816(oacc[dp], pa, b0, b1);
+                    mma_16816(oacc[dp + 1], pa, b2, b3);
+                }
+            }
+            __syncthreads();  // stage and P free
+            ++consumed;
+            if (pj < j1 && !failed) issue();
+        }
     }
-    __syncthreads();
-    if (tid < a.k) {
-        const size_t o = ((size_t)b * a.G + g) * a.k + tid;
-        a.sel_ids[o] = out_i[tid];
-        if (a.ids_out != nullptr) a.ids_out[o] = out_i[tid];
-        if (a.top_scores_out != nullptr) a.top_scores_out[o] = out_s[tid];
+
+    // normalised partial output and log2 normaliser of this split
+    const size_t split = ((size_t)b * a.G + g) * a.S + s;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int row = grp + 8 * h;
+        if (row < r) {
+            const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+            float *dst = a.part_o + (split * r + row) * D;
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                const int d = (w + 4 * dt) * 8 + tig * 2;
+                *reinterpret_cast<float2 *>(dst + d) = make_float2(oacc[dt][2 * h] * inv, oacc[dt][2 * h + 1] * inv);
+            }
+            if (w == 0 && tig == 0)
+                a.part_lse[split * r + row] = l_run[h] > 0.f ? m_run[h] + log2f(l_run[h]) : -INFINITY;
+        }
     }
-    if (tid == 0) a.counters[(size_t)b * a.G + g] = 0;
+    if (!last_split(a, b, g, &misc[1])) return;
+    merge_splits<__nv_bfloat16>(a, b, g, reinterpret_cast<float *>(ring));
 }
 
 template <typename T, int D, int R>
-cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s, bool pdl) {
+cudaError_t launch_attn_t(AttnArgs a, cudaStream_t s, bool pdl) {
     using Cfg = AttnCfg<T, D, R>;
     const int KT = a.Bk < Cfg::KT_MAX ? a.Bk : Cfg::KT_MAX;
+    const size_t ring = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES;
+    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k : 0;
+    a.ring_bytes = (int)((ring > scratch ? ring : scratch) + 15) / 16 * 16;
     // p_s doubles as the [S][r] merge weights of the last split: R * max(KT, kMaxSplits) floats
-    const size_t smem = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
+    const size_t smem = (size_t)a.ring_bytes + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
                         (size_t)R * (KT > kMaxSplits ? KT : kMaxSplits) * 4 + 16;
-    static bool attr_done = false;
-    if (!attr_done) {
+    static size_t attr_bytes = 0;
+    if (smem > attr_bytes) {
         cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             160 * 1024);
+                                             (int)smem);
         if (e != cudaSuccess) return e;
-        attr_done = true;
+        attr_bytes = smem;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.S, a.G, a.B);
@@ -445,36 +736,52 @@ cudaError_t launch_attn_r(const AttnArgs &a, cudaStream_t s, bool pdl) {
     return launch_attn_t<T, D, 16>(a, s, pdl);
 }
 
-template <typename T>
-cudaError_t launch_attn_d(const AttnArgs &a, cudaStream_t s, bool pdl) {
-    return a.D == 64 ? launch_attn_r<T, 64>(a, s, pdl) : launch_attn_r<T, 128>(a, s, pdl);
-}
-
-}  // namespace
-
-cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl) {
-    return dtype == MSA_F32 ? launch_attn_d<float>(a, s, pdl) : launch_attn_d<__nv_bfloat16>(a, s, pdl);
-}
-
-cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s) {
+template <int D>
+cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
+    const int KT = a.Bk < 128 ? a.Bk : 128;
+    const size_t stage = (size_t)2 * (D / 64) * KT * 128;
+    // one stage when every split is a single tile, two otherwise
+    const bool one_tile = a.blocks_per_split == 1 && a.Bk <= 128;
+    a.nst = one_tile ? 1 : 2;
+    const size_t ring = a.nst * stage;
+    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k : 0;
+    const size_t wgt = (size_t)a.S * a.r * 4;
+    size_t rb = ring > scratch ? ring : scratch;
+    rb = rb > wgt ? rb : wgt;
+    a.ring_bytes = (int)((rb + 1023) / 1024 * 1024);
+    const size_t smem = 1024 + (size_t)a.ring_bytes + (size_t)kMmaRows * (KT + 8) * 2 + (64 + 64 + 32 * 4 + 4) * 4 + 64;
+    static size_t attr_bytes = 0;
+    if (smem > attr_bytes) {
+        cudaError_t e = cudaFuncSetAttribute(decode_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_bytes = smem;
+    }
+    CUtensorMap km, vm;
+    const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
+    if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.k_cache), D, rows, D * 2, 64, KT,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.v_cache), D, rows, D * 2, 64, KT,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.G, a.B);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = (size_t)a.n_cta * a.k * 16 + 256;
+    cfg.gridDim = dim3(a.S, a.G, a.B);
+    cfg.blockDim = dim3(kMmaThreads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    static size_t attr_bytes = 48 * 1024;
-    if (cfg.dynamicSmemBytes > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)cfg.dynamicSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_bytes = cfg.dynamicSmemBytes;
-    }
-    return cudaLaunchKernelEx(&cfg, decode_select_kernel, a);
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_attn_mma_kernel<D>, km, vm, a);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl) {
+    if (dtype == MSA_BF16) return a.D == 64 ? launch_mma<64>(a, s, pdl) : launch_mma<128>(a, s, pdl);
+    return a.D == 64 ? launch_attn_r<float, 64>(a, s, pdl) : launch_attn_r<float, 128>(a, s, pdl);
 }
 
 }  // namespace msa

@@ -161,6 +161,8 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     x0 = x0 < total ? x0 : total;
     x1 = x1 < total ? x1 : total;
 
+    if (blockIdx.x == 0 && a.counters != nullptr)
+        for (int i = tid; i < B * a.G; i += blockDim.x) a.counters[i] = 0;  // the attention's split counters
     if (blockIdx.x == 0 && a.seg_info != nullptr) {
         for (int s = tid; s < B * Hik; s += blockDim.x) {
             const int b = s / Hik, h = s % Hik;

@@ -13,7 +13,7 @@ namespace msa {
 namespace {
 
 thread_local std::string g_err;
-thread_local cudaEvent_t g_stage_ev[4];
+thread_local cudaEvent_t g_stage_ev[3];
 thread_local int g_n_stage_ev = 0;
 
 msa_status_t fail(msa_status_t st, const char *fmt, ...) {
@@ -149,10 +149,6 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
         L.cand_i = off;
         off += round256(cand);
     }
-    if (scan) {
-        L.sel_ids = off;
-        off += round256((size_t)p.batch * p.n_kv_heads * p.top_k * 4);
-    }
     if (attend) {
         if (p.flags & MSA_DENSE) {
             const int nb = nb_max_of(p);
@@ -227,17 +223,17 @@ msa_status_t msa_set_stage_events(void *const *events, int n_events) {
         g_n_stage_ev = 0;
         return MSA_OK;
     }
-    if (n_events != 4 || events == nullptr) return fail(MSA_ERR_INVALID_ARG, "n_events must be 0 or 4");
-    for (int i = 0; i < 4; ++i) {
+    if (n_events != 3 || events == nullptr) return fail(MSA_ERR_INVALID_ARG, "n_events must be 0 or 3");
+    for (int i = 0; i < 3; ++i) {
         if (events[i] == nullptr) return fail(MSA_ERR_INVALID_ARG, "event %d is NULL", i);
         g_stage_ev[i] = (cudaEvent_t)events[i];
     }
-    g_n_stage_ev = 4;
+    g_n_stage_ev = 3;
     return MSA_OK;
 }
 
 static cudaError_t stage_mark(int i, cudaStream_t s) {
-    return g_n_stage_ev == 4 ? cudaEventRecord(g_stage_ev[i], s) : cudaSuccess;
+    return g_n_stage_ev == 3 ? cudaEventRecord(g_stage_ev[i], s) : cudaSuccess;
 }
 
 msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t stream) {
@@ -313,11 +309,18 @@ msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_i
 }
 
 static msa_status_t attend_decode(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
-                                  const int32_t *ids, bool after_select, const DecodeWs &L, unsigned char *wsb,
-                                  void *o, float *lse, cudaStream_t s) {
+                                  const int32_t *ids, bool after_scan, const DecodeWs &L, unsigned char *wsb,
+                                  void *o, int32_t *ids_out, float *lse, cudaStream_t s) {
     AttnArgs a{};
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.seq_lens = p->seq_lens;
     a.ids_in = ids;
+    if (after_scan) {  // select the group's list inside the attention kernel
+        a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
+        a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
+        a.seg_info = reinterpret_cast<const SegInfo *>(wsb + L.seg_info);
+        a.ids_out = ids_out;
+    }
+    a.n_cta = L.n_cta;
     a.part_o = reinterpret_cast<float *>(wsb + L.part_o);
     a.part_lse = reinterpret_cast<float *>(wsb + L.part_lse);
     a.counters = reinterpret_cast<int *>(wsb + L.counters);
@@ -328,13 +331,13 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(wsb);
     cudaError_t e;
-    if (!after_select) {  // the select kernel zeroes the counters in the fused path
+    if (!after_scan) {  // the scan zeroes the counters in the fused path
         e = cudaMemsetAsync(a.counters, 0, (size_t)p->batch * p->n_kv_heads * 4, s);
         if (e != cudaSuccess) return cuda_fail(e, "clearing the split counters");
     }
-    e = launch_decode_attn(a, p->dtype, s, after_select);
+    e = launch_decode_attn(a, p->dtype, s, after_scan);
     if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-    if (after_select && (e = stage_mark(3, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    if (after_scan && (e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return MSA_OK;
 }
 
@@ -357,7 +360,7 @@ msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const 
     const DecodeWs L = decode_ws_layout(*p, false, true, n_sm);
     if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     return attend_decode(p, q, k_cache, v_cache, dense ? nullptr : ids, false, L,
-                         reinterpret_cast<unsigned char *>(ws), o, lse, (cudaStream_t)stream);
+                         reinterpret_cast<unsigned char *>(ws), o, nullptr, lse, (cudaStream_t)stream);
 }
 
 msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *q_idx, const void *k_cache,
@@ -389,22 +392,14 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.cand_s = reinterpret_cast<float *>(wsb + L.cand_s);
     a.cand_i = reinterpret_cast<int *>(wsb + L.cand_i);
     a.seg_info = reinterpret_cast<SegInfo *>(wsb + L.seg_info);
+    a.counters = reinterpret_cast<int *>(wsb + L.counters);
     a.status = reinterpret_cast<int *>(wsb);
     cudaError_t e = stage_mark(0, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    SelectArgs sa{};
-    sa.cand_s = a.cand_s; sa.cand_i = a.cand_i; sa.seg_info = a.seg_info;
-    sa.n_cta = L.n_cta; sa.B = p->batch; sa.G = p->n_kv_heads; sa.Hik = p->n_idx_k_heads; sa.k = p->top_k;
-    sa.sel_ids = reinterpret_cast<int *>(wsb + L.sel_ids);
-    sa.ids_out = ids_out;
-    sa.counters = reinterpret_cast<int *>(wsb + L.counters);
-    e = launch_decode_select(sa, s);
-    if (e != cudaSuccess) return cuda_fail(e, "select launch");
-    if ((e = stage_mark(2, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    return attend_decode(p, q, k_cache, v_cache, sa.sel_ids, true, L, wsb, o, lse, s);
+    return attend_decode(p, q, k_cache, v_cache, nullptr, true, L, wsb, o, ids_out, lse, s);
 }
 
 msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,

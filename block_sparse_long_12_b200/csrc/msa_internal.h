@@ -46,18 +46,8 @@ struct ScanArgs {
     SegInfo *seg_info;     // [n_seg] (written by CTA 0 when cand_s != nullptr)
     float *token_scores;   // [B, 1, G, L_max] (nullable)
     float *block_scores;   // [B, 1, G, nb_max] (nullable)
+    int *counters;         // [B, G] attention arrival counters, zeroed by CTA 0 (nullable)
     int *status;
-};
-
-struct SelectArgs {
-    const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]
-    const int *cand_i;
-    const SegInfo *seg_info;
-    int n_cta, B, G, Hik, k;
-    int *sel_ids;              // [B, G, k] final list (workspace)
-    int *ids_out;              // nullable
-    float *top_scores_out;     // nullable
-    int *counters;             // [B, G] attention arrival counters, zeroed here
 };
 
 struct AttnArgs {
@@ -65,7 +55,13 @@ struct AttnArgs {
     const void *k_cache;
     const void *v_cache;
     const int *seq_lens;
-    const int *ids_in;         // [B, 1, G, k] selection (unused with dense)
+    const int *ids_in;         // [B, 1, G, k] given selection (unused with dense or cand_s)
+    const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]: select in the kernel (fused decode)
+    const int *cand_i;
+    const SegInfo *seg_info;
+    int n_cta;
+    int *ids_out;              // nullable (fused decode)
+    float *top_scores_out;     // nullable (fused decode)
     float *part_o;             // [B, G, S, r, D] fp32, normalised per split
     float *part_lse;           // [B, G, S, r] log2-domain normaliser
     int *counters;             // [B, G] arrival counts, zero on entry; reset by the last split
@@ -74,6 +70,7 @@ struct AttnArgs {
     int B, Hq, G, Hik, D, Bk, k, L_max, r;
     int S, blocks_per_split, dense;
     float scale_log2;          // softmax_scale * log2(e)
+    int ring_bytes, nst;       // set by the launcher
     int *status;
 };
 
@@ -110,7 +107,7 @@ struct FillArgs {
 
 // Workspace layout of the decode entries (offsets in bytes from ws).
 struct DecodeWs {
-    size_t seg_info, cand_s, cand_i, sel_ids, counters, part_o, part_lse, total;
+    size_t seg_info, cand_s, cand_i, counters, part_o, part_lse, total;
     int n_cta, S, blocks_per_split;
 };
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);
@@ -119,7 +116,6 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
 cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);
 cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
-cudaError_t launch_decode_select(const SelectArgs &a, cudaStream_t s);
 cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_cache, const void *v_cache, int n_sm,
                                 cudaStream_t s, const char **why);

@@ -177,13 +177,12 @@ MSA_API msa_status_t msa_prefill_index_topk(const msa_params_t *params, const vo
 
 /*
  * Measurement hook (not part of the method): while set, msa_decode_fused
- * records events[0] before its first kernel and events[i] after its i-th
- * kernel (1 = index scan, 2 = TopK merge, 3 = sparse attention with the split
- * merge) on the call's stream, so a caller can time each kernel with
- * cudaEventElapsedTime.
- * events are cudaEvent_t handles owned by the caller; n_events must be 0
- * (unset) or 4.  Per calling thread.  Recording between the kernels removes
- * their launch overlap, so time whole steps without it.
+ * records events[0] before its first kernel, events[1] after the index scan
+ * and events[2] after the attention kernel (TopK merge, sparse attention and
+ * split merge) on the call's stream, so a caller can time each kernel with
+ * cudaEventElapsedTime.  events are cudaEvent_t handles owned by the caller;
+ * n_events must be 0 (unset) or 3.  Per calling thread.  Recording between
+ * the kernels removes their launch overlap, so time whole steps without it.
  */
 MSA_API msa_status_t msa_set_stage_events(void *const *events, int n_events);
 
