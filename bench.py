@@ -332,11 +332,25 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_qi, new_k, new_v, new_ki))
     d2h = h_o.numel() * h_o.element_size() + h_ids.numel() * h_ids.element_size()
 
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        x = {n: to_numpy_raw(inp[n]) for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens")}
+        sec, threads = oracle_decode_seconds(w, x, repeats=2)
+        cpu = {"value": round(sec * 1e6, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"one full decode step of {w.name} (batch {w.batch}), fp64 C oracle, median of 2"}
+        del x
+
+    lens_host = lens.tolist()
+    prefill = None
+    if not args.no_prefill:
+        del inp, q, q_idx, k, v, k_idx, ws, wsd, o, od, flush_buf
+        torch.cuda.empty_cache()
+        prefill = run_prefill(world, rank, local, stream)
+
     if rank != 0:
         return
     peaks, peak_kind = measured_peaks()
     es = 2 if w.dtype == "bf16" else 4
-    lens_host = lens.tolist()
     scan_bytes = sum(lens_host) * w.n_idx_k_heads * w.idx_dim * es  # every index key read once
     achieved = scan_bytes / (scan_us * 1e-6) / 1e9
     traffic = None
@@ -345,13 +359,6 @@ def run_ours(args, world, rank, local):
         if rec.get("source_sha256") == scan_source_hash() and rec.get("workload") == w.name:
             traffic = rec.get("dram_bytes_per_launch")
     clocks = clk.summary()
-
-    cpu = None
-    if world == 1 and not args.no_cpu_baseline:
-        x = {n: to_numpy_raw(inp[n]) for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens")}
-        sec, threads = oracle_decode_seconds(w, x, repeats=2)
-        cpu = {"value": round(sec * 1e6, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"one full decode step of {w.name} (batch {w.batch}), fp64 C oracle, median of 2"}
 
     line = {
         "metric": METRIC, "value": round(step_us, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -368,10 +375,74 @@ def run_ours(args, world, rank, local):
         "dense_gqa_us": round(dense_us, 2), "sparse_vs_dense_speedup": round(dense_us / step_us, 2),
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
+        "prefill": prefill,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
+
+
+def run_prefill(world, rank, local, stream):
+    """The 1M-token causal prefill in 8192-token chunks: Step 1 (tensor-core index scores, block max
+    pool, TopK) then Step 2 (tensor-core sparse attention) for every chunk.  Returns tok/s and the
+    index kernel's tensor-core roofline fraction (max over ranks)."""
+    from block_sparse_long_12_b200 import _lib, api
+    w = WORKLOADS["prefill_causal_1m"]
+    dev = torch.device("cuda", local)
+    inp = make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
+    T, C = w.max_seq_len, w.chunk
+    n_chunks = T // C
+    ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
+    o = torch.empty_like(inp["q"])
+    chunks = []
+    for c in range(n_chunks):
+        p = api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
+                            head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=w.block_size, top_k=w.top_k,
+                            max_seq_len=T, dtype=_lib.MSA_BF16, q_len=C, q_start=c * C)
+        chunks.append((p, inp["q"][:, c * C:(c + 1) * C], inp["q_idx"][:, c * C:(c + 1) * C],
+                       ids[:, c * C:(c + 1) * C], o[:, c * C:(c + 1) * C]))
+    ws = api.workspace(chunks[0][0], _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, dev)
+
+    def index_pass():
+        for (p, q, qi, idc, oc) in chunks:
+            _lib.msa_prefill_index_topk(p, qi, inp["k_idx"], idc, None, ws, stream)
+
+    def attn_pass():
+        for (p, q, qi, idc, oc) in chunks:
+            _lib.msa_sparse_attn_prefill(p, q, inp["k"], inp["v"], idc, oc, None, ws, stream)
+
+    index_pass()
+    attn_pass()
+    torch.cuda.synchronize()
+    ti, ta = [], []
+    for _ in range(3):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        index_pass()
+        e[1].record(stream)
+        attn_pass()
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        ti.append(e[0].elapsed_time(e[1]) / 1e3)
+        ta.append(e[1].elapsed_time(e[2]) / 1e3)
+    assert _lib.msa_get_device_status(ws) == 0
+    t_idx = max_over_ranks(statistics.median(ti), world)
+    t_att = max_over_ranks(statistics.median(ta), world)
+    peaks, kind = measured_peaks()
+    # algorithmic FLOPs: every visible (row, key) pair of every group scores d_i MACs; attention
+    # touches top_k blocks of block_size keys per (row, head) for Q.K and P.V
+    pairs = T * (T + 1) // 2
+    idx_flops = 2.0 * w.idx_dim * w.n_kv_heads * pairs
+    att_flops = 4.0 * w.head_dim * w.n_q_heads * w.top_k * w.block_size * T
+    total = t_idx + t_att
+    return {"workload": w.name, "tokens": T, "chunk": C, "tok_per_s": round(T * world / total, 1),
+            "seconds": round(total, 4), "index_s": round(t_idx, 4), "attention_s": round(t_att, 4),
+            "index_tflops": round(idx_flops / t_idx / 1e12, 1),
+            "index_frac_of_bf16_peak": round(idx_flops / t_idx / 1e12 / peaks["bf16_tflops_sustained"], 4),
+            "attention_useful_tflops": round(att_flops / t_att / 1e12, 1),
+            "overall_frac_of_bf16_peak": round((idx_flops + att_flops) / total / 1e12 / peaks["bf16_tflops_sustained"], 4),
+            "peak": peaks["bf16_tflops_sustained"], "peak_kind": f"{kind} sustained (long step)",
+            "gpu_launches": 2 * n_chunks * 3}
 
 
 def main():
@@ -383,6 +454,7 @@ def main():
     ap.add_argument("--workload", default="decode_ctx1m", choices=["decode_ctx1m", "decode_b4_ctx1m",
                                                                     "decode_b8_ctx128k_ragged"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -173,14 +173,49 @@ __device__ void merge_splits(const AttnArgs &a, int b, int g, float *wgt) {
                 den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
     }
     __syncthreads();
+    // every thread owns up to 4 float4 groups of outputs and keeps 4 splits x 4 groups of loads in
+    // flight, so the merge costs a few L2 round trips rather than one per split
     T *o = reinterpret_cast<T *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
-    const float *po = a.part_o + bg * a.S * r * D;
-    for (int f = tid; f < r * D; f += nthr) {
-        const int h = f / D;
-        float num = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < a.S; ++j) num = fmaf(wgt[j * r + h], __ldcg(po + ((size_t)j * r) * D + f), num);
-        store_elem(o + f, num);
+    const float4 *po = reinterpret_cast<const float4 *>(a.part_o + bg * a.S * r * D);
+    const int n4 = r * D / 4, split4 = r * D / 4;
+    for (int f0 = tid; f0 < n4; f0 += 4 * nthr) {
+        float4 acc[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j0 = 0; j0 < a.S; j0 += 4) {
+            float4 v[4][4];
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int f = f0 + u * nthr;
+                    v[jj][u] = (j0 + jj < a.S && f < n4) ? __ldcg(po + (size_t)(j0 + jj) * split4 + f)
+                                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int f = f0 + u * nthr;
+                    if (j0 + jj < a.S && f < n4) {
+                        const float wj = wgt[(j0 + jj) * r + (f * 4) / D];
+                        acc[u].x = fmaf(wj, v[jj][u].x, acc[u].x);
+                        acc[u].y = fmaf(wj, v[jj][u].y, acc[u].y);
+                        acc[u].z = fmaf(wj, v[jj][u].z, acc[u].z);
+                        acc[u].w = fmaf(wj, v[jj][u].w, acc[u].w);
+                    }
+                }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int f = f0 + u * nthr;
+            if (f < n4) {
+                store_elem(o + 4 * f, acc[u].x);
+                store_elem(o + 4 * f + 1, acc[u].y);
+                store_elem(o + 4 * f + 2, acc[u].z);
+                store_elem(o + 4 * f + 3, acc[u].w);
+            }
+        }
     }
     if (tid == 0) a.counters[bg] = 0;  // ready for the next call
 }
