@@ -24,7 +24,8 @@ MSA_SCORES_TOKEN, MSA_SCORES_BLOCKMAX, MSA_DENSE = 1, 2, 8
 # every symbol include/msa.h declares
 EXPORTED = ["msa_index_score", "msa_block_maxpool_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
             "msa_decode_fused", "msa_prefill_index_topk", "msa_workspace_size", "msa_last_error_string",
-            "msa_status_string", "msa_get_device_status", "msa_clear_device_status", "msa_set_stage_events"]
+            "msa_status_string", "msa_get_device_status", "msa_clear_device_status", "msa_set_stage_events",
+            "msa_decode_fused_noalloc"]
 
 
 class MsaError(RuntimeError):
@@ -61,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "msa_sparse_attn_decode": [P, vp, vp, vp, vp, vp, vp, vp, sz, st],
             "msa_sparse_attn_prefill": [P, vp, vp, vp, vp, vp, vp, vp, sz, st],
             "msa_decode_fused": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, st],
+            "msa_decode_fused_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp, st],
             "msa_prefill_index_topk": [P, vp, vp, vp, vp, vp, sz, st],
             "msa_get_device_status": [vp, ctypes.POINTER(ctypes.c_int), st],
             "msa_clear_device_status": [vp, st],
@@ -134,6 +136,12 @@ def msa_decode_fused(params, q, q_idx, k_cache, v_cache, k_idx, o, ids_out, lse,
     _check(lib().msa_decode_fused(ctypes.byref(params), _ptr(q), _ptr(q_idx), _ptr(k_cache), _ptr(v_cache),
                                   _ptr(k_idx), _ptr(o), _ptr(ids_out), _ptr(lse), _ptr(ws),
                                   ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def msa_decode_fused_noalloc(params, q, q_idx, k_cache, v_cache, k_idx, o, ids_out, lse, stream=None):
+    """msa_decode_fused without a workspace argument: scratch comes from the library's fixed device array."""
+    _check(lib().msa_decode_fused_noalloc(ctypes.byref(params), _ptr(q), _ptr(q_idx), _ptr(k_cache), _ptr(v_cache),
+                                          _ptr(k_idx), _ptr(o), _ptr(ids_out), _ptr(lse), _stream(stream)))
 
 
 def msa_prefill_index_topk(params, q_idx, k_idx, ids_out, top_scores_out, ws, stream=None):

@@ -133,6 +133,24 @@ int num_sms() {
     return check_device(&n) == MSA_OK ? n : 0;
 }
 
+msa_status_t set_error(msa_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return st;
+}
+
+msa_status_t decode_fused_scratch_bytes(const msa_params_t *p, size_t *bytes) {
+    MSA_TRY(check_params(p, DECODE_ONLY));
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    *bytes = decode_ws_layout(*p, true, true, n_sm).total;
+    return MSA_OK;
+}
+
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm) {
     DecodeWs L{};
     L.n_cta = n_sm < 256 ? n_sm : 256;

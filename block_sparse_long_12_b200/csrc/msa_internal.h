@@ -124,6 +124,11 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
 
 int num_sms();
 
+// set the calling thread's error string and return `st`
+msa_status_t set_error(msa_status_t st, const char *fmt, ...);
+// scratch bytes msa_decode_fused needs for these params (checks params and device first)
+msa_status_t decode_fused_scratch_bytes(const msa_params_t *p, size_t *bytes);
+
 // TMA tensor maps (host); false if the driver cannot encode the map
 bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, void *base, unsigned long long inner,
                unsigned long long rows, unsigned long long row_stride_bytes, unsigned box_x, unsigned box_y,

@@ -167,6 +167,30 @@ MSA_API msa_status_t msa_decode_fused(const msa_params_t *params, const void *q,
                               msa_stream_t stream);
 
 /*
+ * msa_decode_fused for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry; it exists for callers that are
+ * handed only their input and output buffers -- plugin or foreign-function
+ * hosts whose calling convention has no slot for scratch memory, or serving
+ * loops that reserve all device memory at start-up and allocate nothing
+ * afterwards -- and so cannot supply msa_decode_fused's workspace.
+ * Scratch comes from a fixed 8 MiB array that the library keeps in device
+ * memory on every GPU that loads it, for as long as it stays loaded.
+ *   - Shapes whose scratch (msa_workspace_size(params, MSA_ENTRY_DECODE_FUSED))
+ *     exceeds 8 MiB are rejected with MSA_ERR_WORKSPACE before any launch;
+ *     1M-token decode at batch 1 needs well under 1 MiB.
+ *   - The array is shared by every call on a device: calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race on it
+ *     and must be ordered by the caller.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make it before
+ *     capturing any stream.
+ *   - Nothing is allocated or freed; results equal msa_decode_fused's.
+ */
+MSA_API msa_status_t msa_decode_fused_noalloc(const msa_params_t *params, const void *q, const void *q_idx,
+                                              const void *k_cache, const void *v_cache, const void *k_idx, void *o,
+                                              int32_t *ids_out, float *lse, msa_stream_t stream);
+
+/*
  * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,
  * block max pool and TopK in the epilogue; scores are never stored.
  * ids_out [B, q_len, G, top_k]; top_scores_out nullable.  bf16 only.
