@@ -311,17 +311,11 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                 const int sb = sc & 1;
                 if (!tc::wait_or_abort(&S.s_full[sb], (sc >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
                 tc::fence_after_sync();
-                float z[BK];
-                {
-                    uint32_t rr[32];
+                uint32_t zr[BK];
 #pragma unroll
-                    for (int c = 0; c < BK / 32; ++c) {
-                        tc::tmem_ld32(tmem + lane_addr + sb * BK + c * 32, rr);
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) z[c * 32 + i] = __uint_as_float(rr[i]);
-                    }
-                }
+                for (int c = 0; c < BK / 32; ++c)
+                    tc::tmem_ld32(tmem + lane_addr + sb * BK + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&zr[c * 32]));
+                tc::tmem_ld_wait();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive1(&S.s_empty[sb]);
@@ -329,53 +323,63 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                 const bool member = row_live && ((um[j * MW + (tq >> 5)] >> (tq & 31)) & 1u);
                 const int kb = id * a.Bk;
                 float mb = -INFINITY;
+                if (member) {
+                    // only the block holding the query needs the causal mask
+                    const bool diag = kb + BK - 1 > pos;
 #pragma unroll
-                for (int c = 0; c < BK; ++c) {
-                    const bool vis = member && (kb + c <= pos);
-                    z[c] = vis ? z[c] * a.scale_log2 : -INFINITY;
-                    mb = fmaxf(mb, z[c]);
+                    for (int c = 0; c < BK; ++c) {
+                        float v = __uint_as_float(zr[c]) * a.scale_log2;
+                        if (diag && kb + c > pos) v = -INFINITY;
+                        zr[c] = __float_as_uint(v);
+                        mb = fmaxf(mb, v);
+                    }
                 }
                 const float m_new = fmaxf(m, mb);
                 const bool grow = m_new > m + 8.f;  // rescale only when the max grows by more than 2^8
                 const float alpha = grow ? exp2f(m - m_new) : 1.f;
                 if (grow) m = m_new;
-                // P buffer and O are free once the previous block's P.V has completed
+                // P = exp2(z - m) as packed bf16 pairs (rows whose token did not select the block: 0)
+                uint32_t pk[BK / 2];
+                float ps = 0.f;
+                if (member) {
+#pragma unroll
+                    for (int e = 0; e < BK / 2; ++e) {
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(__uint_as_float(zr[2 * e]) - m),
+                                                                        exp2f(__uint_as_float(zr[2 * e + 1]) - m));
+                        ps += __low2float(pb) + __high2float(pb);
+                        pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
+                }
+                // the P buffer and O are free once the previous block's P.V has completed
                 if (j > 0) {
                     if (!tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status)) { ok = false; break; }
                     ++pv_waits;
                     tc::fence_after_sync();
                     if (__any_sync(FULL, grow && alpha != 1.f)) {
-                        uint32_t ov[32];
+                        uint32_t ov[D];
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            tc::tmem_ld32(tmem + lane_addr + O_COL + c * 32, ov);
-                            tc::tmem_ld_wait();
+                        for (int c = 0; c < D / 32; ++c)
+                            tc::tmem_ld32(tmem + lane_addr + O_COL + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[c * 32]));
+                        tc::tmem_ld_wait();
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                            tmem_st32(tmem + lane_addr + O_COL + c * 32, ov);
-                        }
+                        for (int i = 0; i < D; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c)
+                            tmem_st32(tmem + lane_addr + O_COL + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&ov[c * 32]));
                         tmem_st_wait();
                     }
                 }
-                float ps = 0.f;
 #pragma unroll
-                for (int h = 0; h < PH; ++h) {
+                for (int h = 0; h < PH; ++h)
 #pragma unroll
                     for (int c16 = 0; c16 < 8; ++c16) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int c = h * 64 + c16 * 8 + 2 * e;
-                            const float p0 = z[c] > -INFINITY ? exp2f(z[c] - m) : 0.f;
-                            const float p1 = z[c + 1] > -INFINITY ? exp2f(z[c + 1] - m) : 0.f;
-                            const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                            ps += __low2float(pb) + __high2float(pb);
-                            pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                        }
                         unsigned char *dst = smP + h * kHalf + row * 128 + ((c16 ^ (row & 7)) << 4);
-                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        const int e0 = h * 32 + c16 * 4;
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[e0], pk[e0 + 1], pk[e0 + 2], pk[e0 + 3]);
                     }
-                }
                 l = l * alpha + ps;
                 fence_proxy_async_smem();
                 tc::fence_before_sync();
