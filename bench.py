@@ -120,11 +120,18 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The job's time is the slowest rank's (all ranks run the same steps in the same order)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(w, rank: int) -> int:
+    """Weak scaling: every rank decodes its own sequence(s), drawn from a rank-specific seed."""
+    return w.seed + 7919 * rank
 
 
 def barrier(world):
@@ -228,7 +235,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
-    inp = make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
+    inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
     stream = torch.cuda.current_stream()
     p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
@@ -389,7 +396,7 @@ def run_prefill(world, rank, local, stream):
     from block_sparse_long_12_b200 import _lib, api
     w = WORKLOADS["prefill_causal_1m"]
     dev = torch.device("cuda", local)
-    inp = make_inputs(w, device=dev, seed=w.seed + 7919 * rank)
+    inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     T, C = w.max_seq_len, w.chunk
     n_chunks = T // C
     ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
