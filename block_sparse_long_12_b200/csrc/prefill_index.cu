@@ -16,9 +16,12 @@
 //   warp 1      owns 512 TMEM columns and issues tcgen05.mma (M=128, N=128,
 //               K=16, bf16 in, fp32 accumulate) for both row tiles into a
 //               double-buffered pair of accumulators;
-//   warps 4-11  epilogue, one TMEM lane (= query row) per thread: tcgen05.ld
-//               of the scores, causal mask on diagonal tiles, 3-input max per
-//               32 columns, block max, and a register-resident sorted top-k.
+//   warps 4-19  epilogue, one TMEM lane (= query row) per thread, in two
+//               groups of 8 warps that take alternate blocks of tiles:
+//               tcgen05.ld of the scores, causal mask on diagonal tiles,
+//               3-input max per 32 columns, block max, and a sorted top-k per
+//               row in shared memory; the groups' lists are merged per row
+//               when the unit ends.
 // The next tile's MMAs overlap the epilogue of the current one.
 #include "tcgen05.cuh"
 
@@ -30,16 +33,19 @@ constexpr int kRows = 128;              // rows per accumulator (one TMEM lane e
 constexpr int kAccs = 2;                // row tiles per unit
 constexpr int kUnitRows = kRows * kAccs;
 constexpr int kKeys = 128;              // keys per tile (N)
-constexpr int kStages = 6;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;           // 4 control warps + 16 epilogue warps
 constexpr int kEpiWarp0 = 4;
+constexpr int kEpiThreads = 512;
+// ring stages: the per-row lists take K x 512 x 8 bytes of shared memory
+template <int K> struct PiShape { static constexpr int S = K >= 32 ? 4 : 6; };
+constexpr int kMaxStages = 6;
 constexpr int kTileBytes = kKeys * 128; // 128 rows of 64 bf16
 constexpr int kABytes = kRows * 128;
 constexpr uint32_t kTmemCols = 512;     // 2 buffers x 2 accumulators x 128 columns
 
 struct Smem {
     // 1024-byte aligned operand tiles come first (set up by hand in the kernel)
-    uint64_t full[kStages], empty[kStages];
+    uint64_t full[kMaxStages], empty[kMaxStages];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t a_full, a_empty, mma_done;
     uint32_t tmem_base;
@@ -50,27 +56,37 @@ __device__ inline void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Row-wise sorted top-K (score desc, id asc) in registers.
+// Row-wise sorted top-K (score desc, id asc) kept in shared memory, entry i of
+// list j at [i * kEpiThreads + j] (consecutive threads, consecutive words); the
+// K-th entry is mirrored in registers so that a losing block costs one compare.
 template <int K>
-struct RowTopK {
-    float s[K];
-    int id[K];
+struct SmemTopK {
+    float *s;
+    int *id;
+    int j;
+    float thr_s;
+    int thr_i;
     __device__ inline void reset() {
 #pragma unroll
-        for (int i = 0; i < K; ++i) { s[i] = -INFINITY; id[i] = 0x7fffffff; }
+        for (int i = 0; i < K; ++i) { s[i * kEpiThreads + j] = -INFINITY; id[i * kEpiThreads + j] = 0x7fffffff; }
+        thr_s = -INFINITY;
+        thr_i = 0x7fffffff;
     }
     __device__ inline void insert(float cs, int ci) {
-        if (!better(cs, ci, s[K - 1], id[K - 1])) return;
+        if (!better(cs, ci, thr_s, thr_i)) return;
 #pragma unroll
         for (int i = 0; i < K; ++i) {
-            const bool take = better(cs, ci, s[i], id[i]);
-            const float ts = s[i];
-            const int ti = id[i];
-            s[i] = take ? cs : ts;
-            id[i] = take ? ci : ti;
-            cs = take ? ts : cs;
-            ci = take ? ti : ci;
+            const float ts = s[i * kEpiThreads + j];
+            const int ti = id[i * kEpiThreads + j];
+            if (better(cs, ci, ts, ti)) {
+                s[i * kEpiThreads + j] = cs;
+                id[i * kEpiThreads + j] = ci;
+                cs = ts;
+                ci = ti;
+            }
         }
+        thr_s = s[(K - 1) * kEpiThreads + j];
+        thr_i = id[(K - 1) * kEpiThreads + j];
     }
 };
 
@@ -90,8 +106,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char *base = smem_raw + ((1024 - (raw & 1023)) & 1023);
     unsigned char *smA = base;                               // [kAccs][128 rows][128 B]
+    constexpr int kStages = PiShape<K>::S;
     unsigned char *smB = base + kAccs * kABytes;             // [kStages][128 keys][128 B]
-    Smem &S = *reinterpret_cast<Smem *>(smB + kStages * kTileBytes);
+    float *list_s = reinterpret_cast<float *>(smB + kStages * kTileBytes);  // [K][512]
+    int *list_i = reinterpret_cast<int *>(list_s + K * kEpiThreads);        // [K][512]
+    Smem &S = *reinterpret_cast<Smem *>(list_i + K * kEpiThreads);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int BG = a.B * a.G;
@@ -199,10 +218,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------ epilogue: one query row per thread
-        const int q4 = warp & 3, acc = (warp - kEpiWarp0) >> 2;
+        // two groups of 8 warps take alternate blocks of tiles; each keeps its own list per row and
+        // the two lists are merged when the unit ends
+        const int e = warp - kEpiWarp0;
+        const int grp = e >> 3;
+        const int q4 = warp & 3, acc = (e >> 2) & 1;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+        const int tpb = a.Bk > kKeys ? a.Bk / kKeys : 1;  // tiles per block
+        SmemTopK<K> top{list_s, list_i, e * 32 + lane};
         int ti = 0;
-        RowTopK<K> top;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
             int b, g, m0, ntiles;
             unit_of(u, b, g, m0, ntiles);
@@ -213,6 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float bm = -INFINITY;
             bool ok = true;
             for (int n = 0; n < ntiles; ++n, ++ti) {
+                if (((n / tpb) & 1) != grp) continue;  // the other group's tile
                 const int buf = ti & 1;
                 if (!tc::wait_or_abort(&S.acc_full[buf], (ti >> 1) & 1, abort_flag, a.status)) {
                     ok = false;
@@ -250,18 +275,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (!ok) break;
-            if (t < a.T) {
+            // merge the two groups' lists of each row (disjoint block sets) into the output; after
+            // an abort every warp still runs both barriers of every unit (its waits then fail fast)
+            named_barrier(1, kEpiThreads);
+            if (ok && grp == 0 && t < a.T) {
+                const int ja = e * 32 + lane, jb = ja + 8 * 32;
                 const size_t o = (((size_t)b * a.T + t) * a.G + g) * a.k;
-#pragma unroll
-                for (int i = 0; i < K; ++i) {
-                    if (i < a.k) {
-                        const bool live = top.s[i] > -INFINITY;
-                        a.ids_out[o + i] = live ? top.id[i] : -1;
-                        if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = top.s[i];
-                    }
+                int ia = 0, ib = 0;
+                for (int i = 0; i < a.k; ++i) {
+                    const float sa = list_s[ia * kEpiThreads + ja], sb = list_s[ib * kEpiThreads + jb];
+                    const int da = list_i[ia * kEpiThreads + ja], db = list_i[ib * kEpiThreads + jb];
+                    const bool take_a = ib >= K || (ia < K && better(sa, da, sb, db));
+                    const float sv = take_a ? sa : sb;
+                    const int dv = take_a ? da : db;
+                    if (take_a) ++ia; else ++ib;
+                    const bool live = sv > -INFINITY;
+                    a.ids_out[o + i] = live ? dv : -1;
+                    if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = sv;
                 }
             }
+            named_barrier(1, kEpiThreads);
         }
     }
     tc::fence_before_sync();
@@ -275,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int K>
 cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid,
                      cudaStream_t s) {
-    const size_t smem = 1024 + kAccs * kABytes + kStages * kTileBytes + sizeof(Smem) + 64;
+    const size_t smem = 1024 + kAccs * kABytes + PiShape<K>::S * kTileBytes + (size_t)K * kEpiThreads * 8 +
+                        sizeof(Smem) + 64;
     static bool attr = false;
     if (!attr) {
         cudaError_t e =
