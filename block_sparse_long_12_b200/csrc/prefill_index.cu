@@ -224,7 +224,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int grp = e >> 3;
         const int q4 = warp & 3, acc = (e >> 2) & 1;
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        const int tpb = a.Bk > kKeys ? a.Bk / kKeys : 1;  // tiles per block
+        // With blocks of at most one tile, group n & 1 takes tile n, so within a unit each group
+        // consumes the phases of one accumulator buffer in order (the unit-end barriers keep the
+        // groups in step across units).  Blocks spanning two tiles go to group 0 alone: a group
+        // skipping tiles of its own buffer could otherwise wait on a phase two steps ahead.
+        const bool two_groups = a.Bk <= kKeys;
         SmemTopK<K> top{list_s, list_i, e * 32 + lane};
         int ti = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float bm = -INFINITY;
             bool ok = true;
             for (int n = 0; n < ntiles; ++n, ++ti) {
-                if (((n / tpb) & 1) != grp) continue;  // the other group's tile
+                if ((two_groups ? (n & 1) : 0) != grp) continue;  // the other group's tile
                 const int buf = ti & 1;
                 if (!tc::wait_or_abort(&S.acc_full[buf], (ti >> 1) & 1, abort_flag, a.status)) {
                     ok = false;
