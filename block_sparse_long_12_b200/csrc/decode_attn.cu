@@ -484,6 +484,24 @@ __device__ inline void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t
 // byte offset of 16-byte vector c (0..7) of row `row` in a 128-byte-swizzled tile of 128-byte rows
 __device__ inline uint32_t sw128(int row, int c) { return (uint32_t)(row * 128 + ((c ^ (row & 7)) << 4)); }
 
+// thread-block cluster helpers (distributed shared memory)
+__device__ inline void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ inline int cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return (int)r;
+}
+// load a float from the shared memory of CTA `rank` of the cluster, at the same offset as `local`
+__device__ inline float ld_peer(const float *local, int rank) {
+    uint32_t ra;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+    return v;
+}
+
 constexpr int kMmaThreads = 128;  // 4 warps
 constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
 
@@ -710,6 +728,55 @@ __global__ void __launch_bounds__(kMmaThreads) decode_attn_mma_kernel(const __gr
         }
     }
 
+    if (a.cluster > 1) {
+        // the splits of (b, g) form one thread-block cluster: partials stay in shared memory and
+        // every CTA merges a slice of the output reading its peers' partials directly
+        float *po_s = reinterpret_cast<float *>(ring);  // [16][D], the ring is idle now
+        float *pl_s = po_s + kMmaRows * D;               // [16]
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = grp + 8 * h;
+            const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                const int d = (w + 4 * dt) * 8 + tig * 2;
+                *reinterpret_cast<float2 *>(po_s + row * D + d) =
+                    make_float2(oacc[dt][2 * h] * inv, oacc[dt][2 * h + 1] * inv);
+            }
+            if (w == 0 && tig == 0) pl_s[row] = l_run[h] > 0.f ? m_run[h] + log2f(l_run[h]) : -INFINITY;
+        }
+        cluster_sync_all();
+        const int cs = a.cluster, rank = cluster_rank();
+        const int n_out = r * D, per = (n_out + cs - 1) / cs;
+        const int f_end = (rank + 1) * per < n_out ? (rank + 1) * per : n_out;
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
+        for (int f = rank * per + tid; f < f_end; f += kMmaThreads) {
+            const int h = f / D;
+            float ls[8];
+            float M = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                ls[c] = c < cs ? ld_peer(pl_s + h, c) : -INFINITY;
+                M = fmaxf(M, ls[c]);
+            }
+            float num = 0.f, den = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                if (c < cs && ls[c] > -INFINITY) {
+                    const float wgt = exp2f(ls[c] - M);
+                    den += wgt;
+                    num = fmaf(wgt, ld_peer(po_s + h * D + f % D, c), num);
+                }
+            }
+            o[f] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+            if (a.lse != nullptr && f % D == 0)
+                a.lse[(size_t)b * a.Hq + (size_t)g * r + h] =
+                    den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+        }
+        cluster_sync_all();  // peers may still be reading this CTA's partials
+        return;
+    }
+
     // normalised partial output and log2 normaliser of this split
     const size_t split = ((size_t)b * a.G + g) * a.S + s;
 #pragma unroll
@@ -773,6 +840,7 @@ cudaError_t launch_attn_r(const AttnArgs &a, cudaStream_t s, bool pdl) {
 
 template <int D>
 cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
+    a.cluster = (!a.dense && a.S <= 8) ? a.S : 1;
     const int KT = a.Bk < 128 ? a.Bk : 128;
     const size_t stage = (size_t)2 * (D / 64) * KT * 128;
     // one stage when every split is a single tile, two otherwise
@@ -780,7 +848,8 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     a.nst = one_tile ? 1 : 2;
     const size_t ring = a.nst * stage;
     const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k : 0;
-    const size_t wgt = (size_t)a.S * a.r * 4;
+    const size_t wgt = (size_t)a.S * a.r * 4 > (size_t)kMmaRows * D * 4 + 64 ? (size_t)a.S * a.r * 4
+                                                                            : (size_t)kMmaRows * D * 4 + 64;
     size_t rb = ring > scratch ? ring : scratch;
     rb = rb > wgt ? rb : wgt;
     a.ring_bytes = (int)((rb + 1023) / 1024 * 1024);
@@ -804,11 +873,22 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     cfg.blockDim = dim3(kMmaThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (a.cluster > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = a.cluster;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, decode_attn_mma_kernel<D>, km, vm, a);
 }
 

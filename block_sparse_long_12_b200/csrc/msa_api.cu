@@ -178,8 +178,8 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
             L.blocks_per_split = (int)((nb + S - 1) / S);
             L.S = (nb + L.blocks_per_split - 1) / L.blocks_per_split;
         } else {
-            L.S = p.top_k;
-            L.blocks_per_split = 1;
+            L.S = p.top_k < kSparseSplits ? p.top_k : kSparseSplits;
+            L.blocks_per_split = (p.top_k + L.S - 1) / L.S;
         }
         L.counters = off;
         off += round256((size_t)p.batch * p.n_kv_heads * 4);

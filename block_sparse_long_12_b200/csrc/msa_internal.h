@@ -25,6 +25,7 @@ constexpr int kScanChunkBytes = 8192;   // ring stage: bytes of index keys per T
 // ---- decode sparse attention (Step 2 for decode)
 constexpr int kAttnThreads = 256;
 constexpr int kMaxSplits = 64;           // dense decode: splits per (sequence, group)
+constexpr int kSparseSplits = 8;         // sparse decode: splits (= cluster size) per (sequence, group)
 
 // A segment is the index-K stream of one (sequence b, index-K head): blocks
 // 0..nb_b-1 of k_idx[b, hik].  The scan splits the concatenation of all
@@ -71,6 +72,7 @@ struct AttnArgs {
     int S, blocks_per_split, dense;
     float scale_log2;          // softmax_scale * log2(e)
     int ring_bytes, nst;       // set by the launcher
+    int cluster;               // > 1: the S splits of a (b, g) form one cluster and merge in shared memory
     int *status;
 };
 
