@@ -90,14 +90,14 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
 
 // Final TopK of group g of sequence b from the scan's per-piece sorted lists
 // (the fused decode step).  The candidates are staged in `scratch` (at least
-// 16 * n_cta * k bytes); a candidate worse than the k-th entry of some full
-// list cannot be among the final k (that list alone has k better ones), so
-// only the survivors are ranked, each by counting the survivors that beat
+// 16 * n_cta * k bytes) by the whole CTA; then one warp finishes: a candidate
+// worse than the k-th entry of some full list cannot be among the final k
+// (that list alone has k better ones), so only the survivors are kept
+// (ballot compaction) and ranked, each by counting the survivors that beat
 // it.  Leaves the list in sel_s / sel_i[0..32), padded with (-inf, -1).
 // Called by every thread of the CTA.
-__device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i,
-                                  float *red_s, int *red_i, int *n_surv) {
-    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+__device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
     const int cap = a.n_cta * a.k;
     float *ls = reinterpret_cast<float *>(scratch);
     int *li = reinterpret_cast<int *>(ls + cap);
@@ -112,38 +112,38 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
         ls[i] = a.cand_s[src];
         li[i] = a.cand_i[src];
     }
-    if (tid < 32) { sel_s[tid] = -INFINITY; sel_i[tid] = -1; }
-    if (tid == 0) *n_surv = 0;
     __syncthreads();
-    float ts = -INFINITY;
-    int ti = -1;
-    for (int l = tid; l < info.n_pieces; l += nthr) {
-        const float s = ls[l * a.k + a.k - 1];
-        const int i = li[l * a.k + a.k - 1];
-        if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
-    }
-    warp_best(ts, ti);
-    if (lane == 0) { red_s[warp] = ts; red_i[warp] = ti; }
-    __syncthreads();
-    ts = red_s[0];
-    ti = red_i[0];
-    for (int w2 = 1; w2 < nwarps; ++w2)
-        if (better(red_s[w2], red_i[w2], ts, ti)) { ts = red_s[w2]; ti = red_i[w2]; }
-    for (int i = tid; i < n; i += nthr) {
-        if (li[i] >= 0 && !better(ts, ti, ls[i], li[i])) {
-            const int at = atomicAdd(n_surv, 1);
-            ss[at] = ls[i];
-            si[at] = li[i];
+    if (tid < 32) {
+        float ts = -INFINITY;
+        int ti = -1;
+        for (int l = lane; l < info.n_pieces; l += 32) {
+            const float s = ls[l * a.k + a.k - 1];
+            const int i = li[l * a.k + a.k - 1];
+            if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
         }
-    }
-    __syncthreads();
-    const int m = *n_surv;
-    for (int i = tid; i < m; i += nthr) {
-        const float s = ss[i];
-        const int id = si[i];
-        int rank = 0;
-        for (int j = 0; j < m; ++j) rank += better(ss[j], si[j], s, id) ? 1 : 0;
-        if (rank < a.k) { sel_s[rank] = s; sel_i[rank] = id; }
+        warp_best(ts, ti);
+        int m = 0;
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            const int i = i0 + lane;
+            const bool keep = i < n && li[i] >= 0 && !better(ts, ti, ls[i], li[i]);
+            const unsigned msk = __ballot_sync(FULL, keep);
+            if (keep) {
+                const int at = m + __popc(msk & ((1u << lane) - 1u));
+                ss[at] = ls[i];
+                si[at] = li[i];
+            }
+            m += __popc(msk);
+        }
+        sel_s[lane] = -INFINITY;
+        sel_i[lane] = -1;
+        __syncwarp();
+        for (int i = lane; i < m; i += 32) {
+            const float s = ss[i];
+            const int id = si[i];
+            int rank = 0;
+            for (int j = 0; j < m; ++j) rank += better(ss[j], si[j], s, id) ? 1 : 0;
+            if (rank < a.k) { sel_s[rank] = s; sel_i[rank] = id; }
+        }
     }
     __syncthreads();
 }
@@ -230,11 +230,10 @@ __device__ inline bool last_split(const AttnArgs &a, int b, int g, int *flag) {
 }
 
 // Obtain the group's list: fused selection from the scan, or a given ids tensor.
-__device__ inline void group_list(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i,
-                                  float *red_s, int *red_i, int *n_surv) {
+__device__ inline void group_list(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
     if (a.dense) return;
     if (a.cand_s != nullptr) {
-        select_group_topk(a, b, g, scratch, sel_s, sel_i, red_s, red_i, n_surv);
+        select_group_topk(a, b, g, scratch, sel_s, sel_i);
         if (blockIdx.x == 0 && threadIdx.x < a.k) {
             const size_t o = ((size_t)b * a.G + g) * a.k + threadIdx.x;
             if (a.ids_out != nullptr) a.ids_out[o] = sel_i[threadIdx.x];
@@ -301,9 +300,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
 
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
-    __shared__ float red_s[32];
-    __shared__ int red_i[32], n_surv, last_flag;
-    group_list(a, b, g, ring, sel_s, sel_i, red_s, red_i, &n_surv);
+    __shared__ int last_flag;
+    group_list(a, b, g, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1)
     const int bps = a.blocks_per_split;
@@ -561,7 +559,7 @@ __global__ void __launch_bounds__(kMmaThreads) decode_attn_mma_kernel(const __gr
 
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
-    group_list(a, b, g, ring, sel_s, sel_i, red_s, red_i, &misc[0]);
+    group_list(a, b, g, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1), each cut into tiles of KT keys
     const int j0 = s * a.blocks_per_split;

@@ -180,7 +180,8 @@ def test_dense_equals_sparse_when_k_covers_all():
                                  dense=True)
     torch.cuda.synchronize()
     assert (o.float() - od.float()).abs().max().item() <= 2e-2
-    assert (lse - lsed).abs().max().item() <= 1e-4
+    # the two paths merge different numbers of fp32 splits: compare at the LSE tolerance used against the oracle
+    assert (lse - lsed).abs().max().item() <= 1e-3
 
 
 def test_repeat_calls_same_workspace():
