@@ -9,28 +9,33 @@
 // union of the TQ tokens' lists.  Per union block:
 //   S = Q K^T      tcgen05.mma (M=128, N=block, K=16 steps over head_dim),
 //                  fp32 accumulator in TMEM (double-buffered);
-//   softmax        one row per thread: tcgen05.ld of S, mask (block not in
-//                  this token's list, or key after the token), running max
+//   softmax        two warps per TMEM lane quadrant, each on half of the
+//                  block's columns: tcgen05.ld of S, mask (block not in this
+//                  token's list, or key after the token), row max exchanged
+//                  between the two warps through shared memory, running max
 //                  with lazy rescaling (the output is rescaled in TMEM only
-//                  when the max grows by more than 2^8), P = exp2(z - m) as
+//                  when the max grows by more than 2^8), P = 2^(z*c - m) as
 //                  bf16 into shared memory in the 128-byte swizzle layout;
 //   O += P V       tcgen05.mma with V as an MN-major operand, O in TMEM.
-// Warp roles: 0 TMA producer (Q tile, K/V block tiles), 1 MMA issuer and
-// TMEM owner, 2 builds the per-unit block union and per-token membership
-// masks, 4-7 softmax and the final normalisation.
+// K and V tiles have their own stages: a K stage is refilled as soon as its
+// Q K^T has completed, a V stage once its P V has.
+// Warp roles: 0 TMA producer of Q and K, 1 MMA issuer and TMEM owner, 2
+// builds the per-unit block union and per-token membership masks, 3 TMA
+// producer of V, 4-11 softmax and the final normalisation.
 #include "tcgen05.cuh"
 
 namespace msa {
 
 namespace {
 
-constexpr int kPaThreads = 256;
+constexpr int kPaThreads = 384;
 constexpr int kPaRows = 128;
-constexpr int kPaSm0 = 4;   // first softmax warp
+constexpr int kPaSm0 = 4;    // first softmax warp
+constexpr int kPaSmWarps = 8;
 constexpr int kHalf = 16384; // one 128-row x 128-byte operand tile
 
 struct PaBars {
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full, pv_done;
     uint64_t q_full, q_empty;
@@ -39,6 +44,8 @@ struct PaBars {
     uint32_t tmem_base;
     int abort_flag;
     int u_count[2];
+    float red_m[2][2][kPaRows];  // [block parity][column half][row]: raw row max of the half
+    float red_l[2][kPaRows];     // [column half][row]: row sum of the half
 };
 
 __device__ inline void mbar_arrive1(uint64_t *bar) {
@@ -58,6 +65,30 @@ __device__ inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
         : "memory");
 }
 __device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x with the hardware approximation (2^-inf = +0).
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Barrier over the two softmax warps of one lane quadrant (64 threads) that
+// also ANDs a per-thread flag across them, so both warps leave a loop at the
+// same barrier when either has given up a wait.
+__device__ inline bool pair_sync_and(int id, bool ok) {
+    uint32_t r;
+    __syncwarp();
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, 64, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(id)
+        : "memory");
+    return r != 0;
+}
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte swizzle
 // layout: 64-element rows of 128 bytes along N, consecutive K rows 128 bytes
@@ -83,6 +114,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     constexpr int STAGE = 2 * NH * KVH;
     constexpr uint32_t TMEM_COLS = (2 * BK + D) <= 256 ? 256 : 512;
     constexpr uint32_t O_COL = 2 * BK;
+    constexpr int CW = BK / 2;        // S columns of one softmax warp
+    constexpr int DW = D / 2;         // O columns of one softmax warp
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -102,11 +135,13 @@ __global__ void __launch_bounds__(kPaThreads, 1)
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.kv_full[i], 1); mbar_init(&S.kv_empty[i], 1);
-            mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 4);
-            mbar_init(&S.u_full[i], 1); mbar_init(&S.u_empty[i], 6);
+            mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1);
+            mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1);
+            mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], kPaSmWarps);
+            // K producer, V producer, MMA issuer and the softmax warps release a union slot
+            mbar_init(&S.u_full[i], 1); mbar_init(&S.u_empty[i], 3 + kPaSmWarps);
         }
-        mbar_init(&S.p_full, 4);
+        mbar_init(&S.p_full, kPaSmWarps);
         mbar_init(&S.pv_done, 1);
         mbar_init(&S.q_full, 1);
         mbar_init(&S.q_empty, 1);
@@ -201,9 +236,14 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                 mbar_arrive1(&S.u_full[slot]);
             }
         }
-    } else if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    } else if (warp == 0 || warp == 3) {
+        // ------------------------------------------------ TMA producers: warp 0 the Q tile and K tiles, warp 3 V tiles
         if (lane == 0) {
+            const bool is_k = warp == 0;
+            const CUtensorMap *map = is_k ? &kmap : &vmap;
+            uint64_t *full = is_k ? S.k_full : S.v_full;
+            uint64_t *empty = is_k ? S.k_empty : S.v_empty;
+            const int off = is_k ? 0 : NH * KVH;
             int ui = 0, it = 0;
             for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
                 int b, g, t0;
@@ -211,24 +251,24 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                 const int slot = ui & 1;
                 if (!tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status)) break;
                 const int U = S.u_count[slot];
-                if (!tc::wait_or_abort(&S.q_empty, (ui & 1) ^ 1, abort_flag, a.status)) break;
-                mbar_arrive_expect_tx(&S.q_full, NH * kHalf);
-                for (int h = 0; h < NH; ++h) tc::tma_load_3d(smQ + h * kHalf, &qmap, h * 64, g * r, b * a.T + t0, &S.q_full);
+                if (is_k) {
+                    if (!tc::wait_or_abort(&S.q_empty, (ui & 1) ^ 1, abort_flag, a.status)) break;
+                    mbar_arrive_expect_tx(&S.q_full, NH * kHalf);
+                    for (int h = 0; h < NH; ++h)
+                        tc::tma_load_3d(smQ + h * kHalf, &qmap, h * 64, g * r, b * a.T + t0, &S.q_full);
+                }
                 const int *uid = u_ids + slot * a.max_union;
                 bool ok = true;
                 for (int j = 0; j < U; ++j, ++it) {
                     const int st = it & 1;
-                    if (!tc::wait_or_abort(&S.kv_empty[st], ((it >> 1) & 1) ^ 1, abort_flag, a.status)) {
+                    if (!tc::wait_or_abort(&empty[st], ((it >> 1) & 1) ^ 1, abort_flag, a.status)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&S.kv_full[st], STAGE);
+                    mbar_arrive_expect_tx(&full[st], NH * KVH);
                     const int row = (b * a.G + g) * a.L_max + uid[j] * a.Bk;
-                    unsigned char *kd = smKV + st * STAGE;
-                    for (int h = 0; h < NH; ++h) {
-                        tc::tma_load_2d(kd + h * KVH, &kmap, h * 64, row, &S.kv_full[st]);
-                        tc::tma_load_2d(kd + (NH + h) * KVH, &vmap, h * 64, row, &S.kv_full[st]);
-                    }
+                    unsigned char *dst = smKV + st * STAGE + off;
+                    for (int h = 0; h < NH; ++h) tc::tma_load_2d(dst + h * KVH, map, h * 64, row, &full[st]);
                 }
                 mbar_arrive1(&S.u_empty[slot]);
                 if (!ok) break;
@@ -248,11 +288,11 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                 tc::fence_after_sync();
                 const uint32_t q_addr = smem_u32(smQ);
                 bool ok = true;
-                // QK of block j into S buffer (sc + j) & 1
+                // Q K^T of block j into S buffer (sc + j) & 1; its K stage is free once it completes
                 auto qk = [&](int j) -> bool {
                     const int st = (it + j) & 1;
                     const int sb = (sc + j) & 1;
-                    if (!tc::wait_or_abort(&S.kv_full[st], ((it + j) >> 1) & 1, abort_flag, a.status)) return false;
+                    if (!tc::wait_or_abort(&S.k_full[st], ((it + j) >> 1) & 1, abort_flag, a.status)) return false;
                     if (!tc::wait_or_abort(&S.s_empty[sb], (((sc + j) >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
                     tc::fence_after_sync();
                     const uint32_t k_addr = smem_u32(smKV + st * STAGE);
@@ -260,6 +300,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                     for (int ks = 0; ks < D / 16; ++ks)
                         tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (ks >> 2) * kHalf + (ks & 3) * 32),
                                         tc::sw128_kmajor_desc(k_addr + (ks >> 2) * KVH + (ks & 3) * 32), idesc_qk, ks > 0);
+                    tc::mma_commit(&S.k_empty[st]);
                     tc::mma_commit(&S.s_full[sb]);
                     return true;
                 };
@@ -268,15 +309,16 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                     if (j + 1 < U && !qk(j + 1)) { ok = false; break; }
                     if (!tc::wait_or_abort(&S.p_full, pc & 1, abort_flag, a.status)) { ok = false; break; }
                     ++pc;
-                    tc::fence_after_sync();
                     const int st = (it + j) & 1;
+                    if (!tc::wait_or_abort(&S.v_full[st], ((it + j) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+                    tc::fence_after_sync();
                     const uint32_t v_addr = smem_u32(smKV + st * STAGE + NH * KVH);
                     const uint32_t p_addr = smem_u32(smP);
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks)
                         tc::mma_bf16_ss(tmem + O_COL, tc::sw128_kmajor_desc(p_addr + (ks >> 2) * kHalf + (ks & 3) * 32),
                                         sw128_mnmajor_desc(v_addr + ks * 2048, KVH), idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-                    tc::mma_commit(&S.kv_empty[st]);
+                    tc::mma_commit(&S.v_empty[st]);
                     tc::mma_commit(&S.pv_done);
                 }
                 if (!ok) break;
@@ -288,17 +330,27 @@ __global__ void __launch_bounds__(kPaThreads, 1)
             tc::mma_commit(&S.mma_done);
             mbar_wait(&S.mma_done, 0, a.status);
         }
-    } else if (warp >= kPaSm0) {
-        // ------------------------------------------------ softmax / epilogue, one query row per thread
-        const int row = (warp - kPaSm0) * 32 + lane;
+    } else {
+        // ------------------------------------------------ softmax / epilogue
+        // Warps w and w + 4 share TMEM lane quadrant w % 4 (one query row per
+        // lane); warp half hf takes S columns [hf*CW, hf*CW + CW) and O
+        // columns [hf*DW, hf*DW + DW).  Every wait result is made uniform over
+        // the pair through pair_sync_and before either warp acts on it, so the
+        // two always execute the same sequence of pair barriers.
+        const int sw = warp - kPaSm0;
+        const int qd = sw & 3, hf = sw >> 2;
+        const int pair_bar = 1 + qd;
+        const int row = qd * 32 + lane;
         const int tq = row / r, hh = row % r;
-        const uint32_t lane_addr = (uint32_t)((warp - kPaSm0) * 32) << 16;
+        const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         int ui = 0, sc = 0, pv_waits = 0;
+        bool p_zero = false;  // this warp's part of P already holds zeros
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
             int b, g, t0;
             unit_of(u, b, g, t0);
             const int slot = ui & 1;
-            if (!tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status)) break;
+            bool ok = __all_sync(FULL, tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status));
+            if (!pair_sync_and(pair_bar, ok)) break;
             const int U = S.u_count[slot];
             const int *uid = u_ids + slot * a.max_union;
             const uint32_t *um = u_mask + (size_t)slot * a.max_union * MW;
@@ -306,102 +358,132 @@ __global__ void __launch_bounds__(kPaThreads, 1)
             const bool row_live = t < a.T;
             const int pos = a.q_start + t;
             float m = -INFINITY, l = 0.f;
-            bool ok = true;
             for (int j = 0; j < U; ++j, ++sc) {
                 const int sb = sc & 1;
-                if (!tc::wait_or_abort(&S.s_full[sb], (sc >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                tc::fence_after_sync();
-                uint32_t zr[BK];
-#pragma unroll
-                for (int c = 0; c < BK / 32; ++c)
-                    tc::tmem_ld32(tmem + lane_addr + sb * BK + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&zr[c * 32]));
-                tc::tmem_ld_wait();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive1(&S.s_empty[sb]);
+                if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.s_full[sb], (sc >> 1) & 1, abort_flag, a.status));
                 const int id = uid[j];
                 const bool member = row_live && ((um[j * MW + (tq >> 5)] >> (tq & 31)) & 1u);
-                const int kb = id * a.Bk;
+                const bool active = __any_sync(FULL, member);
+                uint32_t zr[CW];
                 float mb = -INFINITY;
-                if (member) {
-                    // only the block holding the query needs the causal mask
-                    const bool diag = kb + BK - 1 > pos;
+                if (ok) {
+                    if (active) {
+                        tc::fence_after_sync();
 #pragma unroll
-                    for (int c = 0; c < BK; ++c) {
-                        float v = __uint_as_float(zr[c]) * a.scale_log2;
-                        if (diag && kb + c > pos) v = -INFINITY;
-                        zr[c] = __float_as_uint(v);
-                        mb = fmaxf(mb, v);
+                        for (int c = 0; c < CW / 32; ++c)
+                            tc::tmem_ld32(tmem + lane_addr + sb * BK + hf * CW + c * 32,
+                                          *reinterpret_cast<uint32_t(*)[32]>(&zr[c * 32]));
+                        tc::tmem_ld_wait();
+                        tc::fence_before_sync();
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive1(&S.s_empty[sb]);
+                    if (active) {
+                        // only the block holding the query needs the causal mask
+                        const int kb = id * a.Bk + hf * CW;
+                        if (member && kb + CW - 1 > pos) {
+#pragma unroll
+                            for (int c = 0; c < CW; ++c)
+                                if (kb + c > pos) zr[c] = __float_as_uint(-INFINITY);
+                        }
+                        float mx[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) mx[i] = -INFINITY;
+#pragma unroll
+                        for (int c = 0; c < CW; c += 8)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                mx[i] = tc::fmax3(mx[i], __uint_as_float(zr[c + 2 * i]), __uint_as_float(zr[c + 2 * i + 1]));
+                        mb = member ? fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) : -INFINITY;
                     }
                 }
-                const float m_new = fmaxf(m, mb);
+                S.red_m[sc & 1][hf][row] = mb;
+                ok = pair_sync_and(pair_bar, ok);
+                if (!ok) break;
+                // row max of the block (raw scores), then the running max in the log2 domain
+                const float mraw = fmaxf(mb, S.red_m[sc & 1][hf ^ 1][row]);
+                const float m_new = fmaxf(m, mraw * a.scale_log2);
                 const bool grow = m_new > m + 8.f;  // rescale only when the max grows by more than 2^8
-                const float alpha = grow ? exp2f(m - m_new) : 1.f;
+                const float alpha = grow ? exp2_approx(m - m_new) : 1.f;
                 if (grow) m = m_new;
-                // P = exp2(z - m) as packed bf16 pairs (rows whose token did not select the block: 0)
-                uint32_t pk[BK / 2];
+                // P = 2^(z*c - m) as packed bf16 pairs; rows whose token did not select the block get 0
+                uint32_t pk[CW / 2];
                 float ps = 0.f;
-                if (member) {
+                if (active) {
+                    const float cz = member ? a.scale_log2 : 0.f;
+                    const float off = member ? -m : -INFINITY;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int e = 0; e < BK / 2; ++e) {
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(exp2f(__uint_as_float(zr[2 * e]) - m),
-                                                                        exp2f(__uint_as_float(zr[2 * e + 1]) - m));
-                        ps += __low2float(pb) + __high2float(pb);
+                    for (int e = 0; e < CW / 2; ++e) {
+                        const float p0 = exp2_approx(fmaf(__uint_as_float(zr[2 * e]), cz, off));
+                        const float p1 = exp2_approx(fmaf(__uint_as_float(zr[2 * e + 1]), cz, off));
+                        acc[e & 3] += p0 + p1;
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
                         pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
                     }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < BK / 2; ++e) pk[e] = 0u;
+                    ps = (acc[0] + acc[1]) + (acc[2] + acc[3]);
                 }
                 // the P buffer and O are free once the previous block's P.V has completed
                 if (j > 0) {
-                    if (!tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status)) { ok = false; break; }
+                    ok = __all_sync(FULL, tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status));
                     ++pv_waits;
+                    if (!ok) continue;  // both warps of the pair leave at the next pair barrier
                     tc::fence_after_sync();
-                    if (__any_sync(FULL, grow && alpha != 1.f)) {
-                        uint32_t ov[D];
+                    if (__any_sync(FULL, alpha != 1.f)) {
+#pragma unroll 1
+                        for (int c = 0; c < DW / 32; ++c) {
+                            uint32_t ov[32];
+                            const uint32_t ta = tmem + lane_addr + O_COL + hf * DW + c * 32;
+                            tc::tmem_ld32(ta, ov);
+                            tc::tmem_ld_wait();
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c)
-                            tc::tmem_ld32(tmem + lane_addr + O_COL + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[c * 32]));
-                        tc::tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < D; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-#pragma unroll
-                        for (int c = 0; c < D / 32; ++c)
-                            tmem_st32(tmem + lane_addr + O_COL + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(&ov[c * 32]));
+                            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                            tmem_st32(ta, ov);
+                        }
                         tmem_st_wait();
                     }
                 }
+                if (active || !p_zero) {
+                    if (!active) {
 #pragma unroll
-                for (int h = 0; h < PH; ++h)
-#pragma unroll
-                    for (int c16 = 0; c16 < 8; ++c16) {
-                        unsigned char *dst = smP + h * kHalf + row * 128 + ((c16 ^ (row & 7)) << 4);
-                        const int e0 = h * 32 + c16 * 4;
-                        *reinterpret_cast<uint4 *>(dst) = make_uint4(pk[e0], pk[e0 + 1], pk[e0 + 2], pk[e0 + 3]);
+                        for (int e = 0; e < CW / 2; ++e) pk[e] = 0u;
                     }
+                    p_zero = !active;
+                    // this warp's CW keys of the row: 16-byte chunks of P half-tile (hf*CW)/64
+#pragma unroll
+                    for (int c16 = 0; c16 < CW / 8; ++c16) {
+                        const int kc = hf * CW + c16 * 8;  // first key of the chunk
+                        unsigned char *dst = smP + (kc >> 6) * kHalf + row * 128 + ((((kc & 63) >> 3) ^ (row & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(dst) =
+                            make_uint4(pk[c16 * 4], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
+                    }
+                    fence_proxy_async_smem();
+                }
                 l = l * alpha + ps;
-                fence_proxy_async_smem();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive1(&S.p_full);
             }
-            if (!ok) break;
             // final normalisation once the last P.V has completed
+            if (ok && U > 0) {
+                ok = __all_sync(FULL, tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status));
+                ++pv_waits;
+            }
+            S.red_l[hf][row] = l;
+            if (!pair_sync_and(pair_bar, ok)) break;
+            const float l_row = l + S.red_l[hf ^ 1][row];
             float o_scale = 0.f;
             if (U > 0) {
-                if (!tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status)) break;
-                ++pv_waits;
                 tc::fence_after_sync();
-                o_scale = l > 0.f ? 1.f / l : 0.f;
+                o_scale = l_row > 0.f ? 1.f / l_row : 0.f;
             }
             const int hq = g * r + hh;
-            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + hq) * D;
+            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + hq) * D + hf * DW;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < DW / 32; ++c) {
                 uint32_t ov[32];
                 if (U > 0) {
-                    tc::tmem_ld32(tmem + lane_addr + O_COL + c * 32, ov);
+                    tc::tmem_ld32(tmem + lane_addr + O_COL + hf * DW + c * 32, ov);
                     tc::tmem_ld_wait();
                 } else {
 #pragma unroll
@@ -421,8 +503,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                     }
                 }
             }
-            if (row_live && a.lse != nullptr)
-                a.lse[((size_t)b * a.T + t) * a.Hq + hq] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            if (hf == 0 && row_live && a.lse != nullptr)
+                a.lse[((size_t)b * a.T + t) * a.Hq + hq] = l_row > 0.f ? (m + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive1(&S.u_empty[slot]);

@@ -2,6 +2,7 @@
 
   python -m block_sparse_long_12_b200.profile_run decode --context 262144 --steps 3
   python -m block_sparse_long_12_b200.profile_run prefill_index --context 65536 --chunk 8192 --steps 1
+  python -m block_sparse_long_12_b200.profile_run prefill_attn --context 65536 --chunk 8192 --steps 1
 
 Inputs are the seeded synthetic workloads of ``inputs`` at the requested
 size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
@@ -49,15 +50,37 @@ def run_prefill_index(args):
     print("prefill index done")
 
 
+def run_prefill_attn(args):
+    """Index branch, then the sparse branch, for the last chunk of the context."""
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=args.context)
+    inp = make_inputs(w, device="cuda")
+    T = args.chunk
+    q_start = args.context - T
+    p = api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
+                        head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=w.block_size, top_k=w.top_k,
+                        max_seq_len=w.max_seq_len, dtype=_lib.MSA_BF16, q_len=T, q_start=q_start)
+    qi = inp["q_idx"][:, q_start:q_start + T].contiguous()
+    q = inp["q"][:, q_start:q_start + T].contiguous()
+    ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device="cuda")
+    o = torch.empty_like(q)
+    ws_i = api.workspace(p, _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, "cuda")
+    ws_a = api.workspace(p, _lib.MSA_ENTRY_ATTN_PREFILL, "cuda")
+    for _ in range(args.steps):
+        _lib.msa_prefill_index_topk(p, qi, inp["k_idx"], ids, None, ws_i)
+        _lib.msa_sparse_attn_prefill(p, q, inp["k"], inp["v"], ids, o, None, ws_a)
+    torch.cuda.synchronize()
+    print("prefill attention done", int(_lib.msa_get_device_status(ws_a)))
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["decode", "prefill_index"])
+    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn"])
     ap.add_argument("--context", type=int, default=262144)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=8192)
     ap.add_argument("--steps", type=int, default=3)
     args = ap.parse_args()
-    {"decode": run_decode, "prefill_index": run_prefill_index}[args.what](args)
+    {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn}[args.what](args)
 
 
 if __name__ == "__main__":
