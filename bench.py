@@ -411,7 +411,7 @@ def run_prefill(world, rank, local, stream):
                             max_seq_len=T, dtype=_lib.MSA_BF16, q_len=C, q_start=c * C)
         chunks.append((p, inp["q"][:, c * C:(c + 1) * C], inp["q_idx"][:, c * C:(c + 1) * C],
                        ids[:, c * C:(c + 1) * C], o[:, c * C:(c + 1) * C]))
-    ws = api.workspace(chunks[0][0], _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, dev)
+    ws = api.workspace([c[0] for c in chunks], _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, dev)
 
     def index_pass():
         for (p, q, qi, idc, oc) in chunks:

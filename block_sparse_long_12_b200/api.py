@@ -42,9 +42,11 @@ def params_from(q, q_idx, k, k_idx, *, block_size, top_k, seq_lens=None, q_start
                        softmax_scale=softmax_scale, flags=flags)
 
 
-def workspace(params: Params, entry: int, device) -> torch.Tensor:
-    """Zeroed scratch for one entry (the first word is the device status)."""
-    n = _lib.msa_workspace_size(params, entry)
+def workspace(params, entry: int, device) -> torch.Tensor:
+    """Zeroed scratch for one entry (the first word is the device status).  `params` may be
+    a list: the scratch then serves every call made with any of them."""
+    plist = params if isinstance(params, (list, tuple)) else [params]
+    n = max(_lib.msa_workspace_size(p, entry) for p in plist)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 

@@ -193,6 +193,41 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
     return L;
 }
 
+PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm) {
+    PrefillIdxPlan L{};
+    L.n_mt = (p.q_len + 255) / 256;
+    L.kt = p.top_k <= 8 ? 8 : p.top_k <= 16 ? 16 : 32;
+    const long long units = (long long)L.n_mt * p.batch * p.n_kv_heads;
+    const int max_tiles = prefill_unit_tiles(0, L.n_mt, p.q_len, p.q_start, p.block_size);
+    const int gran = p.block_size > 128 ? p.block_size / 128 : 1;
+    // segments per unit: the fewest that fill whole waves of CTAs (to within ~2 %), never
+    // shorter than 64 tiles or one block
+    L.n_seg = 1;
+    double best = 0.0;
+    for (int sgm = 1; sgm <= 16; ++sgm) {
+        if (sgm > 1 && (max_tiles / sgm < 64 || max_tiles / sgm < gran)) break;
+        const long long pieces = units * sgm;
+        const long long waves = (pieces + n_sm - 1) / n_sm;
+        const double eff = (double)pieces / ((double)waves * n_sm);
+        if (eff > best + 0.02) {
+            best = eff;
+            L.n_seg = sgm;
+        }
+    }
+    const long long pieces = units * L.n_seg;
+    L.grid = (int)(pieces < n_sm ? pieces : n_sm);
+    size_t off = kStatusBytes;
+    L.counters = off;
+    off += round256((size_t)units * 4);
+    const size_t part = L.n_seg > 1 ? (size_t)units * L.n_seg * L.kt * 256 * 4 : 0;
+    L.part_s = off;
+    off += round256(part);
+    L.part_i = off;
+    off += round256(part);
+    L.total = off;
+    return L;
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -227,9 +262,11 @@ size_t msa_workspace_size(const msa_params_t *p, int entry) {
             if (check_params(p, DECODE_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
             return decode_ws_layout(*p, true, true, n_sm).total;
         case MSA_ENTRY_ATTN_PREFILL:
-        case MSA_ENTRY_PREFILL_INDEX_TOPK:
             if (check_params(p, PREFILL_ONLY) != MSA_OK) return (size_t)-1;
             return kStatusBytes;
+        case MSA_ENTRY_PREFILL_INDEX_TOPK:
+            if (check_params(p, PREFILL_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
+            return prefill_index_plan(*p, n_sm).total;
         default:
             fail(MSA_ERR_INVALID_ARG, "unknown entry %d", entry);
             return (size_t)-1;
@@ -468,17 +505,24 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     MSA_TRY(check_ptr(ids_out, "ids_out"));
     MSA_TRY(check_ptr(top_scores_out, "top_scores_out", true));
     MSA_TRY(check_ptr(ws, "ws"));
-    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
     int n_sm = 0;
     MSA_TRY(check_device(&n_sm));
+    const PrefillIdxPlan L = prefill_index_plan(*p, n_sm);
+    if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     PrefillIdxArgs a{};
     a.B = p->batch; a.T = p->q_len; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.Bk = p->block_size;
     a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len;
-    a.n_mt = (p->q_len + 255) / 256;
+    a.n_mt = L.n_mt;
+    a.n_seg = L.n_seg;
     a.ids_out = ids_out; a.top_scores_out = top_scores_out;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    a.counters = reinterpret_cast<int *>(w + L.counters);
+    a.part_s = reinterpret_cast<float *>(w + L.part_s);
+    a.part_i = reinterpret_cast<int *>(w + L.part_i);
     a.status = reinterpret_cast<int *>(ws);
-    const char *why = "";
-    cudaError_t e = launch_prefill_index(a, q_idx, k_idx, n_sm, (cudaStream_t)stream, &why);
+    const char *why = "clearing the prefill index piece counters";
+    cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)L.n_mt * p->batch * p->n_kv_heads * 4, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = launch_prefill_index(a, q_idx, k_idx, L.grid, (cudaStream_t)stream, &why);
     if (e != cudaSuccess) return cuda_fail(e, why);
     return MSA_OK;
 }

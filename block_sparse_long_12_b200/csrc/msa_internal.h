@@ -87,10 +87,39 @@ struct PoolTopkArgs {
 struct PrefillIdxArgs {
     int B, T, G, Hik, Bk, k, q_start, L_max;
     int n_mt;                  // 256-row query tiles per (b, g)
+    int n_seg;                 // key segments per unit
     int32_t *ids_out;          // [B, T, G, k]
     float *top_scores_out;     // nullable
+    int *counters;             // [units] segments finished (zeroed before the launch)
+    float *part_s;             // [units][n_seg][Kt][256] per-segment row lists of split units
+    int *part_i;
     int *status;
 };
+
+// Key tiles (128 keys) of the i-th prefill index unit in processing order:
+// query rows [m0, m0 + 256) of tile mt = n_mt - 1 - i (latest rows first)
+// see keys up to the end of the block holding their last position.
+__host__ __device__ inline int prefill_unit_tiles(int i, int n_mt, int T, int q_start, int Bk) {
+    const int m0 = (n_mt - 1 - i) * 256;
+    const int last = m0 + 255 < T - 1 ? m0 + 255 : T - 1;
+    const int nb_last = (q_start + last) / Bk;
+    return ((nb_last + 1) * Bk + 127) / 128;
+}
+
+// Key tiles of one segment of a unit with nt tiles cut into n_seg segments
+// (a whole number of blocks of Bk keys).
+__host__ __device__ inline int prefill_seg_tiles(int nt, int n_seg, int Bk) {
+    const int gran = Bk > 128 ? Bk / 128 : 1;
+    const int per = (nt + n_seg - 1) / n_seg;
+    return (per + gran - 1) / gran * gran;
+}
+
+// How a prefill index call splits its work and where its scratch lives.
+struct PrefillIdxPlan {
+    int n_mt, n_seg, grid, kt;
+    size_t counters, part_s, part_i, total;
+};
+PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm);
 
 struct PrefillAttnArgs {
     const int *ids;            // [B, T, G, k]

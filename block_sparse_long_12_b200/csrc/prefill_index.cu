@@ -8,8 +8,15 @@
 // GEMM with a reduction epilogue; section 3 of the page notes that this scan
 // of the full input remains in prefill.
 //
-// One persistent CTA per SM takes work units (sequence b, group g, 256 query
-// rows), heaviest first.  Warp roles:
+// A work unit is (sequence b, group g, 256 query rows) against all the key
+// tiles its rows can see.  When the units alone would leave the last wave of
+// CTAs part-empty, each unit's keys are cut into n_seg segments (whole
+// blocks); the pieces are taken segment by segment, heaviest unit first, so
+// the CTAs running at the same time read the same keys of a group (shared in
+// L2), and the SMs finish together.  A unit cut into segments leaves one
+// per-row list per segment in the workspace; the CTA that finishes its last
+// segment merges them (same order: higher score, then lower block id).
+// Warp roles:
 //   warp 0      TMA producer: the unit's two 128-row index-query tiles, then
 //               the index-key tiles (128 keys x 64 dims, 128-byte swizzle)
 //               through a kStages ring;
@@ -21,7 +28,7 @@
 //               tcgen05.ld of the scores, causal mask on diagonal tiles,
 //               3-input max per 32 columns, block max, and a sorted top-k per
 //               row in shared memory; the groups' lists are merged per row
-//               when the unit ends.
+//               when the piece ends.
 // The next tile's MMAs overlap the epilogue of the current one.
 #include "tcgen05.cuh"
 
@@ -50,6 +57,13 @@ struct Smem {
     uint64_t a_full, a_empty, mma_done;
     uint32_t tmem_base;
     int abort_flag;
+    int merge_here;  // this CTA finished the last segment of a split unit
+};
+
+// One piece of work: segment s of unit u = i * (B*G) + bg, key tiles [n0, n1)
+// of the unit's nt, which has n_parts non-empty segments.
+struct Piece {
+    int u, i, bg, s, n0, n1, nt, n_parts;
 };
 
 __device__ inline void mbar_arrive(uint64_t *bar) {
@@ -114,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int BG = a.B * a.G;
-    const int n_units = a.n_mt * BG;
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
@@ -137,34 +150,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = S.tmem_base;
     volatile int *abort_flag = &S.abort_flag;
 
-    auto unit_of = [&](int u, int &b, int &g, int &m0, int &ntiles) {
-        const int mt = a.n_mt - 1 - u / BG;  // heaviest (latest rows) first
-        const int bg = u % BG;
-        b = bg / a.G;
-        g = bg % a.G;
-        m0 = mt * kUnitRows;
-        int last = m0 + kUnitRows - 1;
-        if (last > a.T - 1) last = a.T - 1;
-        const int pos_max = a.q_start + last;
-        const int nb_last = pos_max / a.Bk;
-        ntiles = ((nb_last + 1) * a.Bk + kKeys - 1) / kKeys;
+    // every role takes the same pieces (segment-major, heaviest unit first) and skips the empty ones
+    const int n_units = a.n_mt * BG;
+    const int n_pieces = n_units * a.n_seg;
+    auto piece_of = [&](int p, Piece &w) -> bool {
+        w.s = p / n_units;
+        w.u = p - w.s * n_units;
+        w.i = w.u / BG;
+        w.bg = w.u - w.i * BG;
+        w.nt = prefill_unit_tiles(w.i, a.n_mt, a.T, a.q_start, a.Bk);
+        const int len = a.n_seg > 1 ? prefill_seg_tiles(w.nt, a.n_seg, a.Bk) : w.nt;
+        w.n0 = w.s * len;
+        w.n1 = w.n0 + len < w.nt ? w.n0 + len : w.nt;
+        w.n_parts = (w.nt + len - 1) / len;
+        return w.n0 < w.nt;
     };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int it = 0, ui = 0;
-            for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-                int b, g, m0, ntiles;
-                unit_of(u, b, g, m0, ntiles);
-                if (!tc::wait_or_abort(&S.a_empty, (ui & 1) ^ 1, abort_flag, a.status)) break;
+            int it = 0, pc = 0;
+            Piece w;
+            for (int p = blockIdx.x; p < n_pieces; p += gridDim.x) {
+                if (!piece_of(p, w)) continue;
+                const int b = w.bg / a.G, g = w.bg % a.G, m0 = (a.n_mt - 1 - w.i) * kUnitRows;
+                if (!tc::wait_or_abort(&S.a_empty, (pc++ & 1) ^ 1, abort_flag, a.status)) break;
                 mbar_arrive_expect_tx(&S.a_full, kAccs * kABytes);
                 for (int acc = 0; acc < kAccs; ++acc)
                     tc::tma_load_3d(smA + acc * kABytes, &qmap, 0, g, b * a.T + m0 + acc * kRows, &S.a_full);
                 const int hik = g % a.Hik;
                 const int row0 = (b * a.Hik + hik) * a.L_max;
                 bool ok = true;
-                for (int n = 0; n < ntiles; ++n, ++it) {
+                for (int n = w.n0; n < w.n1; ++n, ++it) {
                     const int st = it % kStages;
                     if (!tc::wait_or_abort(&S.empty[st], ((it / kStages) & 1) ^ 1, abort_flag, a.status)) {
                         ok = false;
@@ -180,14 +197,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16_f32(kRows, kKeys);
-            int it = 0, ti = 0, ui = 0;
-            for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++ui) {
-                int b, g, m0, ntiles;
-                unit_of(u, b, g, m0, ntiles);
-                if (!tc::wait_or_abort(&S.a_full, ui & 1, abort_flag, a.status)) break;
+            int it = 0, ti = 0, pc = 0;
+            Piece w;
+            for (int p = blockIdx.x; p < n_pieces && !*abort_flag; p += gridDim.x) {
+                if (!piece_of(p, w)) continue;
+                if (!tc::wait_or_abort(&S.a_full, pc++ & 1, abort_flag, a.status)) break;
                 tc::fence_after_sync();
                 bool ok = true;
-                for (int n = 0; n < ntiles; ++n, ++it, ++ti) {
+                for (int n = w.n0; n < w.n1; ++n, ++it, ++ti) {
                     const int st = it % kStages;
                     const int buf = ti & 1;
                     if (!tc::wait_or_abort(&S.full[st], (it / kStages) & 1, abort_flag, a.status) ||
@@ -219,28 +236,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp >= kEpiWarp0) {
         // ------------------------------------------------ epilogue: one query row per thread
         // two groups of 8 warps take alternate blocks of tiles; each keeps its own list per row and
-        // the two lists are merged when the unit ends
+        // the two lists are merged when the piece ends
         const int e = warp - kEpiWarp0;
         const int grp = e >> 3;
         const int q4 = warp & 3, acc = (e >> 2) & 1;
+        const int rl = acc * kRows + q4 * 32 + lane;  // row within the unit
         const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-        // With blocks of at most one tile, group n & 1 takes tile n, so within a unit each group
-        // consumes the phases of one accumulator buffer in order (the unit-end barriers keep the
-        // groups in step across units).  Blocks spanning two tiles go to group 0 alone: a group
+        // With blocks of at most one tile, group n & 1 takes tile n, so within a piece each group
+        // consumes the phases of one accumulator buffer in order (the piece-end barriers keep the
+        // groups in step across pieces).  Blocks spanning two tiles go to group 0 alone: a group
         // skipping tiles of its own buffer could otherwise wait on a phase two steps ahead.
         const bool two_groups = a.Bk <= kKeys;
         SmemTopK<K> top{list_s, list_i, e * 32 + lane};
         int ti = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-            int b, g, m0, ntiles;
-            unit_of(u, b, g, m0, ntiles);
-            const int t = m0 + acc * kRows + q4 * 32 + lane;
+        bool ok = true;
+        Piece w;
+        for (int p = blockIdx.x; p < n_pieces; p += gridDim.x) {
+            if (!piece_of(p, w)) continue;
+            const int b = w.bg / a.G, g = w.bg % a.G, m0 = (a.n_mt - 1 - w.i) * kUnitRows;
+            const int t = m0 + rl;
             const int pos = a.q_start + t;
             const int pos_min = a.q_start + m0;  // smallest position of the unit
             top.reset();
             float bm = -INFINITY;
-            bool ok = true;
-            for (int n = 0; n < ntiles; ++n, ++ti) {
+            for (int n = w.n0; n < w.n1 && ok; ++n, ++ti) {
                 if ((two_groups ? (n & 1) : 0) != grp) continue;  // the other group's tile
                 const int buf = ti & 1;
                 if (!tc::wait_or_abort(&S.acc_full[buf], (ti >> 1) & 1, abort_flag, a.status)) {
@@ -279,23 +298,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // merge the two groups' lists of each row (disjoint block sets) into the output; after
-            // an abort every warp still runs both barriers of every unit (its waits then fail fast)
+            // After an abort every warp still runs every barrier of every piece (its waits fail fast).
+            const bool whole = w.n_parts == 1;
             named_barrier(1, kEpiThreads);
-            if (ok && grp == 0 && t < a.T) {
+            if (grp == 0) {
+                // merge the two groups' lists of each row (disjoint block sets)
                 const int ja = e * 32 + lane, jb = ja + 8 * 32;
                 const size_t o = (((size_t)b * a.T + t) * a.G + g) * a.k;
+                const size_t po = ((size_t)w.u * a.n_seg + w.s) * K * kUnitRows + rl;
                 int ia = 0, ib = 0;
-                for (int i = 0; i < a.k; ++i) {
+                const int n_out = whole ? a.k : K;
+                for (int i = 0; ok && i < n_out; ++i) {
                     const float sa = list_s[ia * kEpiThreads + ja], sb = list_s[ib * kEpiThreads + jb];
                     const int da = list_i[ia * kEpiThreads + ja], db = list_i[ib * kEpiThreads + jb];
                     const bool take_a = ib >= K || (ia < K && better(sa, da, sb, db));
                     const float sv = take_a ? sa : sb;
                     const int dv = take_a ? da : db;
                     if (take_a) ++ia; else ++ib;
-                    const bool live = sv > -INFINITY;
-                    a.ids_out[o + i] = live ? dv : -1;
-                    if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = sv;
+                    if (whole) {
+                        if (t < a.T) {
+                            a.ids_out[o + i] = sv > -INFINITY ? dv : -1;
+                            if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = sv;
+                        }
+                    } else {
+                        a.part_s[po + (size_t)i * kUnitRows] = sv;
+                        a.part_i[po + (size_t)i * kUnitRows] = dv;
+                    }
+                }
+                if (!whole) {
+                    // the CTA that finishes the unit's last segment merges every segment's lists
+                    __threadfence();
+                    named_barrier(2, kEpiThreads / 2);
+                    if (e == 0 && lane == 0) S.merge_here = ok && atomicAdd(&a.counters[w.u], 1) == w.n_parts - 1;
+                    named_barrier(2, kEpiThreads / 2);
+                    if (S.merge_here) {
+                        __threadfence();
+                        top.reset();
+                        for (int sg = 0; sg < w.n_parts; ++sg) {
+                            const size_t q = ((size_t)w.u * a.n_seg + sg) * K * kUnitRows + rl;
+                            for (int i = 0; i < K; ++i) {
+                                const float cs = __ldcg(a.part_s + q + (size_t)i * kUnitRows);
+                                const int ci = __ldcg(a.part_i + q + (size_t)i * kUnitRows);
+                                if (!better(cs, ci, top.thr_s, top.thr_i)) break;  // the rest of this list is worse
+                                top.insert(cs, ci);
+                            }
+                        }
+                        if (t < a.T) {
+                            for (int i = 0; i < a.k; ++i) {
+                                const float sv = list_s[i * kEpiThreads + ja];
+                                a.ids_out[o + i] = sv > -INFINITY ? list_i[i * kEpiThreads + ja] : -1;
+                                if (a.top_scores_out != nullptr) a.top_scores_out[o + i] = sv;
+                            }
+                        }
+                    }
                 }
             }
             named_barrier(1, kEpiThreads);
@@ -345,8 +400,7 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
         *why = "encoding the index-key tensor map failed";
         return cudaErrorInvalidValue;
     }
-    const int units = a.n_mt * a.B * a.G;
-    const int grid = units < n_sm ? units : n_sm;
+    const int grid = n_sm;  // the plan's CTA count (at most one per SM)
     *why = "prefill index kernel launch";
     if (a.k <= 8) return launch_k<8>(a, qm, km, grid, s);
     if (a.k <= 16) return launch_k<16>(a, qm, km, grid, s);

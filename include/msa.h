@@ -194,6 +194,10 @@ MSA_API msa_status_t msa_decode_fused_noalloc(const msa_params_t *params, const 
  * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,
  * block max pool and TopK in the epilogue; scores are never stored.
  * ids_out [B, q_len, G, top_k]; top_scores_out nullable.  bf16 only.
+ * The work (every query row against every key it can see) is cut into equal
+ * ranges, one per SM; ws holds the per-row lists of rows whose keys were
+ * split between ranges until they are merged (msa_workspace_size(params,
+ * MSA_ENTRY_PREFILL_INDEX_TOPK) bytes, contents need no initialisation).
  */
 MSA_API msa_status_t msa_prefill_index_topk(const msa_params_t *params, const void *q_idx, const void *k_idx,
                                     int32_t *ids_out, float *top_scores_out, void *ws, size_t ws_bytes,

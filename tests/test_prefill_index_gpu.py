@@ -4,6 +4,8 @@ max pool, TopK) against the fp64 oracle.  Page "MiniMax wird duenn"
 branch still scans the whole visible input)."""
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -118,3 +120,33 @@ def test_prefill_1m_sampled_rows():
         else:
             rows = [(0, int(t)) for t in rng.choice(T, 16, replace=False)]
         check_rows(inp, w, c * T, T, ids, rows)
+
+
+@pytest.mark.parametrize("case", [
+    dict(block_size=128, top_k=16),
+    dict(block_size=256, top_k=8),
+    dict(block_size=32, top_k=32),
+    dict(block_size=64, top_k=16, n_idx_k_heads=1),
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()))
+def test_prefill_index_key_segments(case):
+    """Few query rows against a long context: the kernel cuts every unit's keys into
+    segments, keeps one list per segment and merges them; sampled rows (including the
+    ragged last row tile) against the oracle."""
+    from block_sparse_long_12_b200 import _lib, api
+    hik = case.pop("n_idx_k_heads", 8)
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=40000, batch=1, n_idx_k_heads=hik, hot_blocks=6, seed=77)
+    inp = make_inputs(w, device="cuda")
+    q_start, T = 39000, 1000
+    p = api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=hik,
+                        head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=case["block_size"], top_k=case["top_k"],
+                        max_seq_len=w.max_seq_len, dtype=_lib.MSA_BF16, q_len=T, q_start=q_start)
+    units = (T + 255) // 256 * w.n_kv_heads
+    # the workspace holds per-segment lists only when units are split
+    assert _lib.lib().msa_workspace_size(ctypes.byref(p), _lib.MSA_ENTRY_PREFILL_INDEX_TOPK) > 256 + (units * 4 + 255) // 256 * 256
+    ids, ts = prefill_ids(inp, w, q_start, T, top_k=case["top_k"], block_size=case["block_size"], scores=True)
+    rng = np.random.default_rng(5)
+    rows = [(0, int(t)) for t in sorted(set(rng.choice(T, 160, replace=False).tolist()) | {0, 255, 256, 767, 768, T - 1})]
+    check_rows(inp, w, q_start, T, ids, rows, top_k=case["top_k"], block_size=case["block_size"])
+    tsn, idn = ts.cpu().numpy(), ids.cpu().numpy()
+    assert ((idn == -1) == np.isneginf(tsn)).all()
+    assert (idn >= -1).all() and (idn <= (q_start + T - 1) // case["block_size"]).all()
