@@ -90,59 +90,80 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
 
 // Final TopK of group g of sequence b from the scan's per-piece sorted lists
 // (the fused decode step).  The candidates are staged in `scratch` (at least
-// 16 * n_cta * k bytes) by the whole CTA; then one warp finishes: a candidate
-// worse than the k-th entry of some full list cannot be among the final k
-// (that list alone has k better ones), so only the survivors are kept
-// (ballot compaction) and ranked, each by counting the survivors that beat
-// it.  Leaves the list in sel_s / sel_i[0..32), padded with (-inf, -1).
-// Called by every thread of the CTA.
+// 16 * n_cta * k + 16 bytes) by the whole CTA.  A threshold that the final k
+// all reach is the k-th best of a subset (the heads of the pieces' lists);
+// only candidates at least that good are kept, and each is ranked by
+// counting the survivors that beat it.  Leaves the list in sel_s /
+// sel_i[0..32), padded with (-inf, -1).  Called by every thread of the CTA.
 __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
-    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
+    const int tid = threadIdx.x, nthr = blockDim.x;
     const int cap = a.n_cta * a.k;
     float *ls = reinterpret_cast<float *>(scratch);
     int *li = reinterpret_cast<int *>(ls + cap);
     float *ss = reinterpret_cast<float *>(li + cap);
     int *si = reinterpret_cast<int *>(ss + cap);
+    int *st = si + cap;  // [0] survivors, [1] threshold id, [2] threshold score (bits)
     const int gps = a.G / a.Hik;
     const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
     const SegInfo info = a.seg_info[seg];
-    const int n = info.n_pieces * a.k;
+    const int k = a.k, np = info.n_pieces, n = np * k;
     for (int i = tid; i < n; i += nthr) {
-        const size_t src = (((size_t)seg * a.n_cta + i / a.k) * gps + gl) * a.k + i % a.k;
+        const size_t src = (((size_t)seg * a.n_cta + i / k) * gps + gl) * k + i % k;
         ls[i] = a.cand_s[src];
         li[i] = a.cand_i[src];
     }
-    __syncthreads();
+    if (tid == 0) {
+        st[0] = 0;
+        st[1] = -1;
+        st[2] = __float_as_int(-INFINITY);
+    }
     if (tid < 32) {
-        float ts = -INFINITY;
-        int ti = -1;
-        for (int l = lane; l < info.n_pieces; l += 32) {
-            const float s = ls[l * a.k + a.k - 1];
-            const int i = li[l * a.k + a.k - 1];
-            if (i >= 0 && better(s, i, ts, ti)) { ts = s; ti = i; }
-        }
-        warp_best(ts, ti);
-        int m = 0;
-        for (int i0 = 0; i0 < n; i0 += 32) {
-            const int i = i0 + lane;
-            const bool keep = i < n && li[i] >= 0 && !better(ts, ti, ls[i], li[i]);
-            const unsigned msk = __ballot_sync(FULL, keep);
-            if (keep) {
-                const int at = m + __popc(msk & ((1u << lane) - 1u));
-                ss[at] = ls[i];
-                si[at] = li[i];
+        sel_s[tid] = -INFINITY;
+        sel_i[tid] = -1;
+    }
+    __syncthreads();
+    // Threshold: the k-th best among the first J entries of every piece.  The k-th best of any
+    // subset is no better than the k-th best of all candidates, so the whole top-k passes it;
+    // taking each piece's head makes it tight, and few candidates survive.
+    const int J = np > 0 ? min(k, 2 * ((k + np - 1) / np)) : 0;
+    for (int t = tid; t < np * J; t += nthr) {
+        const int e = (t / J) * k + t % J;
+        const float s = ls[e];
+        const int id = li[e];
+        if (id < 0) continue;
+        int rank = 0;
+        for (int pc = 0; pc < np; ++pc)
+            for (int j = 0; j < J; ++j) {
+                const int f = pc * k + j;
+                rank += (li[f] >= 0 && better(ls[f], li[f], s, id)) ? 1 : 0;
             }
-            m += __popc(msk);
+        if (rank == k - 1) {
+            st[1] = id;
+            st[2] = __float_as_int(s);
         }
-        sel_s[lane] = -INFINITY;
-        sel_i[lane] = -1;
-        __syncwarp();
-        for (int i = lane; i < m; i += 32) {
-            const float s = ss[i];
-            const int id = si[i];
-            int rank = 0;
-            for (int j = 0; j < m; ++j) rank += better(ss[j], si[j], s, id) ? 1 : 0;
-            if (rank < a.k) { sel_s[rank] = s; sel_i[rank] = id; }
+    }
+    __syncthreads();
+    // survivors: candidates at least as good as the threshold (all valid ones when the subset
+    // holds fewer than k), then their exact ranks (ids are unique, so ranks are distinct)
+    const float ts = __int_as_float(st[2]);
+    const int ti = st[1];
+    for (int i = tid; i < n; i += nthr) {
+        if (li[i] >= 0 && !better(ts, ti, ls[i], li[i])) {
+            const int at = atomicAdd(&st[0], 1);
+            ss[at] = ls[i];
+            si[at] = li[i];
+        }
+    }
+    __syncthreads();
+    const int m = st[0];
+    for (int i = tid; i < m; i += nthr) {
+        const float s = ss[i];
+        const int id = si[i];
+        int rank = 0;
+        for (int j = 0; j < m; ++j) rank += better(ss[j], si[j], s, id) ? 1 : 0;
+        if (rank < k) {
+            sel_s[rank] = s;
+            sel_i[rank] = id;
         }
     }
     __syncthreads();
@@ -801,7 +822,7 @@ cudaError_t launch_attn_t(AttnArgs a, cudaStream_t s, bool pdl) {
     using Cfg = AttnCfg<T, D, R>;
     const int KT = a.Bk < Cfg::KT_MAX ? a.Bk : Cfg::KT_MAX;
     const size_t ring = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES;
-    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k : 0;
+    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k + 16 : 0;
     a.ring_bytes = (int)((ring > scratch ? ring : scratch) + 15) / 16 * 16;
     // p_s doubles as the [S][r] merge weights of the last split: R * max(KT, kMaxSplits) floats
     const size_t smem = (size_t)a.ring_bytes + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
@@ -845,7 +866,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     const bool one_tile = a.blocks_per_split == 1 && a.Bk <= 128;
     a.nst = one_tile ? 1 : 2;
     const size_t ring = a.nst * stage;
-    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k : 0;
+    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k + 16 : 0;
     const size_t wgt = (size_t)a.S * a.r * 4 > (size_t)kMmaRows * D * 4 + 64 ? (size_t)a.S * a.r * 4
                                                                             : (size_t)kMmaRows * D * 4 + 64;
     size_t rb = ring > scratch ? ring : scratch;
