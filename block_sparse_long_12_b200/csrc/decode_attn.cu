@@ -167,6 +167,53 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
         }
     }
     __syncthreads();
+    if (a.tail_scores == nullptr) return;
+    // The tail of the stream (blocks [nb - nt, nb)) left block scores only: every warp keeps
+    // the k best of its share of those that beat the k-th entry so far (the others cost one
+    // comparison), and one warp merges these lists with the ranges' k best.
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int nb = (L + a.Bk - 1) / a.Bk, nt = scan_tail_blocks(nb);
+    const int nb_max = (a.L_max + a.Bk - 1) / a.Bk;
+    const float *tsc = a.tail_scores + ((size_t)b * a.G + g) * nb_max;
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    WarpTopK t;
+    t.reset();
+    // floor: a tail block must beat the k-th entry of the ranges' list (while the warp's own
+    // list is not full its threshold is below that)
+    const float fl_s = sel_s[k - 1];
+    const int fl_i = sel_i[k - 1];
+    constexpr int kBatch = 16;  // loads in flight per lane
+    for (int base = nb - nt + warp * 32 * kBatch; base < nb; base += nwarps * 32 * kBatch) {
+        float v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = base + u * 32 + lane;
+            v[u] = n < nb ? tsc[n] : -INFINITY;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n0 = base + u * 32;
+            unsigned msk = __ballot_sync(FULL, n0 + lane < nb && better(v[u], n0 + lane, fl_s, fl_i) &&
+                                                   better(v[u], n0 + lane, t.thr_s, t.thr_i));
+            while (msk) {
+                const int l = __ffs(msk) - 1;
+                msk &= msk - 1;
+                t.insert(__shfl_sync(FULL, v[u], l), n0 + l, k, lane);
+            }
+        }
+    }
+    float *tl_s = ls;  // [1 + nwarps][32] lists (the staging area is free now)
+    int *tl_i = li;
+    tl_s[(1 + warp) * 32 + lane] = t.s;
+    tl_i[(1 + warp) * 32 + lane] = t.id;
+    if (warp == 0) {
+        tl_s[lane] = sel_s[lane];
+        tl_i[lane] = sel_i[lane];
+    }
+    __syncthreads();
+    if (warp == 0) warp_merge_sorted_lists<1>(tl_s, tl_i, 1 + nwarps, k, 32, k, sel_s, sel_i, lane);
+    __syncthreads();
 }
 
 // The last split CTA of (b, g) merges the normalised partial outputs of all
@@ -822,7 +869,7 @@ cudaError_t launch_attn_t(AttnArgs a, cudaStream_t s, bool pdl) {
     using Cfg = AttnCfg<T, D, R>;
     const int KT = a.Bk < Cfg::KT_MAX ? a.Bk : Cfg::KT_MAX;
     const size_t ring = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES;
-    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k + 16 : 0;
+    const size_t scratch = a.cand_s != nullptr ? max((size_t)16 * a.n_cta * a.k + 16, (size_t)2 * 9 * 32 * 4) : 0;
     a.ring_bytes = (int)((ring > scratch ? ring : scratch) + 15) / 16 * 16;
     // p_s doubles as the [S][r] merge weights of the last split: R * max(KT, kMaxSplits) floats
     const size_t smem = (size_t)a.ring_bytes + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
@@ -866,7 +913,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     const bool one_tile = a.blocks_per_split == 1 && a.Bk <= 128;
     a.nst = one_tile ? 1 : 2;
     const size_t ring = a.nst * stage;
-    const size_t scratch = a.cand_s != nullptr ? (size_t)16 * a.n_cta * a.k + 16 : 0;
+    const size_t scratch = a.cand_s != nullptr ? max((size_t)16 * a.n_cta * a.k + 16, (size_t)2 * 9 * 32 * 4) : 0;
     const size_t wgt = (size_t)a.S * a.r * 4 > (size_t)kMmaRows * D * 4 + 64 ? (size_t)a.S * a.r * 4
                                                                             : (size_t)kMmaRows * D * 4 + 64;
     size_t rb = ring > scratch ? ring : scratch;

@@ -6,10 +6,15 @@
 // group.  For decode this is a single query against the whole cache, so the
 // kernel is a stream of k_idx from HBM: each byte is read once.
 //
-// Work split: the index-K streams of all (sequence b, index-K head) pairs are
-// concatenated (block granularity) and cut into n_cta ranges of equal length
-// (the last one shorter), one per persistent CTA (one CTA per SM), so ragged
-// lengths stay balanced.  Inside a CTA every warp owns a private two-stage
+// Work split: the first three quarters of the index-K streams of all
+// (sequence b, index-K head) pairs are concatenated (block granularity) and
+// cut into n_cta ranges of equal length (the last one shorter), one per
+// persistent CTA (one CTA per SM), so ragged lengths stay balanced.  SMs do
+// not stream equally fast, so the last quarter of every stream is a shared
+// tail: each warp that is done with its range takes tail blocks one at a
+// time from a few interleaved counters in the workspace, and the faster SMs
+// take more of them.  Tail blocks leave only their block scores; the
+// attention kernel's select merges them with the ranges' candidate lists.  Inside a CTA every warp owns a private two-stage
 // ring of 8 KB shared-memory tiles filled by TMA tensor copies
 // (cp.async.bulk.tensor, 128-byte swizzle) and consumes the blocks w, w+W, ...
 // of the CTA's range.  One lane owns one index-key row: the swizzle makes the
@@ -121,9 +126,14 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     float *lists_s = reinterpret_cast<float *>(bars + W * S);                 // [W][GPS][32]
     int *lists_i = reinterpret_cast<int *>(lists_s + W * GPS * 32);
     float *q_s = reinterpret_cast<float *>(lists_i + W * GPS * 32);           // [GPS][DI] (QREG: unused)
-    long long *off = reinterpret_cast<long long *>(q_s + GPS * DI);           // [B+1]
-    int *nbs = reinterpret_cast<int *>(off + a.B + 1);                        // [B]
+    int4 *trec = reinterpret_cast<int4 *>(q_s + GPS * DI);                    // [W][4] tail blocks in flight
+    float *q_w = reinterpret_cast<float *>(trec + W * 4);                     // [W][GPS][DI] (QREG: unused)
+    long long *off = reinterpret_cast<long long *>(q_w + (QREG ? 0 : W * GPS * DI));  // [B+1] ranges' prefix
+    long long *offt = off + a.B + 1;                                          // [B+1] tail pool prefix
+    int *nbs = reinterpret_cast<int *>(offt + a.B + 1);                       // [B] blocks
     int *lens = nbs + a.B;                                                    // [B] clamped lengths
+    int *nba = lens + a.B;                                                    // [B] blocks before the tail
+    int *exh = nba + a.B;                                                     // [kTailPools] pool is empty
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int B = a.B, Hik = a.Hik, Bk = a.Bk, C = a.n_cta;
@@ -134,25 +144,29 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
         L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
         lens[b] = L;
         nbs[b] = (L + Bk - 1) / Bk;
+        nba[b] = nbs[b] - scan_tail_blocks(nbs[b]);
     }
+    if (tid < kTailPools) exh[tid] = 0;
     if (tid < W * S) mbar_init(&bars[tid], 1);
     if (tid == 0) tc::prefetch_tmap(&kmap);
     fence_mbar_init();
     __syncthreads();
-    if (w == 0) {
+    if (w < 2) {
+        // warp 0: prefix of the ranges' blocks (nba), warp 1: of the tails' blocks
+        long long *dst = w == 0 ? off : offt;
         long long carry = 0;
         for (int b0 = 0; b0 < B; b0 += 32) {
             const int b = b0 + lane;
-            long long v = b < B ? (long long)nbs[b] * Hik : 0;
+            long long v = b < B ? (long long)(w == 0 ? nba[b] : nbs[b] - nba[b]) * Hik : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const long long u = __shfl_up_sync(FULL, v, o);
                 if (lane >= o) v += u;
             }
-            if (b < B) off[b + 1] = carry + v;
+            if (b < B) dst[b + 1] = carry + v;
             carry += __shfl_sync(FULL, v, 31);
         }
-        if (lane == 0) off[0] = 0;
+        if (lane == 0) dst[0] = 0;
     }
     __syncthreads();
     const long long total = off[B];
@@ -167,10 +181,10 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
         for (int s = tid; s < B * Hik; s += blockDim.x) {
             const int b = s / Hik, h = s % Hik;
             SegInfo si{-1, 0};
-            if (nbs[b] > 0) {
-                const long long st = off[b] + (long long)h * nbs[b];
+            if (nba[b] > 0) {
+                const long long st = off[b] + (long long)h * nba[b];
                 si.first_cta = cta_of(st, per);
-                si.n_pieces = cta_of(st + nbs[b] - 1, per) - si.first_cta + 1;
+                si.n_pieces = cta_of(st + nba[b] - 1, per) - si.first_cta + 1;
             }
             a.seg_info[s] = si;
         }
@@ -188,7 +202,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     ChunkCursor prod;
     prod.pw = PieceWalker{x0, x1};
     prod.w = w; prod.W = W; prod.Bk = Bk; prod.ct = CT;
-    prod.start(off, nbs, lens, B, Hik);
+    prod.start(off, nba, lens, B, Hik);
     bool failed = false;
     int issued = 0;
     auto issue = [&](int slot) {
@@ -200,9 +214,57 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
             if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
         }
         ++issued;
-        prod.advance(off, nbs, lens, B, Hik);
+        prod.advance(off, nba, lens, B, Hik);
     };
     for (int st = 0; st < S && prod.valid; ++st) issue(st);
+
+    // one chunk of nt index-key rows of segment (b, hik) starting at token tok_base: fp32 dot
+    // products with the index query (qv in registers, or qsrc in shared memory), running max m
+    auto scan_chunk = [&](const unsigned char *base, int nt, int b, int hik, int tok_base, const float *qv_,
+                          const float *qsrc, float *m) {
+        for (int t0 = 0; t0 < nt; t0 += 32) {
+            const int tok = t0 + lane;  // one index-key row per lane
+            const bool live = tok < nt && !failed;
+            float dot[GPS];
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
+            if (live) {
+#pragma unroll
+                for (int c16 = 0; c16 < NCH; ++c16) {
+                    // position of 16-byte vector c16 of row `tok` in the swizzled tile
+                    int o;
+                    if constexpr (ROWB == 64) {
+                        o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
+                    } else {
+                        o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
+                    }
+                    const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
+                    float f[EPV];
+                    Vec16<T>::unpack(u, f);
+                    if constexpr (QREG) {
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) dot[0] = fmaf(qv_[c16 * EPV + e], f[e], dot[0]);
+                    } else {
+#pragma unroll
+                        for (int gl = 0; gl < GPS; ++gl) {
+                            const float *qq = qsrc + gl * DI + c16 * EPV;
+#pragma unroll
+                            for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qq[e], f[e], dot[gl]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) {
+                const float sc = live ? dot[gl] : -INFINITY;
+                m[gl] = fmaxf(m[gl], sc);
+                if (a.token_scores != nullptr && live) {
+                    const int g = hik + Hik * gl;
+                    a.token_scores[((size_t)b * a.G + g) * a.L_max + tok_base + tok] = sc;
+                }
+            }
+        }
+    };
 
     int consumed = 0;
     float qv[QREG ? DI : 1];
@@ -210,7 +272,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     WarpTopK lst[GPS];
     PieceWalker pw{x0, x1};
     Piece p;
-    while (pw.next(off, nbs, B, Hik, p)) {
+    while (pw.next(off, nba, B, Hik, p)) {
         if (p.b != q_b || p.hik != q_h) {
             q_b = p.b; q_h = p.hik;
             if constexpr (QREG) {
@@ -247,50 +309,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;
-                const unsigned char *base = my_ring + (size_t)slot * kScanChunkBytes;
-                const int tok_base = n * Bk + c * CT;
-                for (int t0 = 0; t0 < nt; t0 += 32) {
-                    const int tok = t0 + lane;  // one index-key row per lane
-                    const bool live = tok < nt && !failed;
-                    float dot[GPS];
-#pragma unroll
-                    for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
-                    if (live) {
-#pragma unroll
-                        for (int c16 = 0; c16 < NCH; ++c16) {
-                            // position of 16-byte vector c16 of row `tok` in the swizzled tile
-                            int o;
-                            if constexpr (ROWB == 64) {
-                                o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
-                            } else {
-                                o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
-                            }
-                            const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
-                            float f[EPV];
-                            Vec16<T>::unpack(u, f);
-                            if constexpr (QREG) {
-#pragma unroll
-                                for (int e = 0; e < EPV; ++e) dot[0] = fmaf(qv[c16 * EPV + e], f[e], dot[0]);
-                            } else {
-#pragma unroll
-                                for (int gl = 0; gl < GPS; ++gl) {
-                                    const float *qq = q_s + gl * DI + c16 * EPV;
-#pragma unroll
-                                    for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qq[e], f[e], dot[gl]);
-                                }
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int gl = 0; gl < GPS; ++gl) {
-                        const float sc = live ? dot[gl] : -INFINITY;
-                        m[gl] = fmaxf(m[gl], sc);
-                        if (a.token_scores != nullptr && live) {
-                            const int g = p.hik + Hik * gl;
-                            a.token_scores[((size_t)p.b * a.G + g) * a.L_max + tok_base + tok] = sc;
-                        }
-                    }
-                }
+                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, p.b, p.hik, n * Bk + c * CT, qv, q_s, m);
                 __syncwarp();
                 ++consumed;
                 if (prod.valid && !failed) issue(slot);
@@ -327,6 +346,136 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
             __syncthreads();
         }
     }
+
+    // ------------------------------------------------ the shared tail, one block at a time
+    // Every warp takes tail blocks until the pools are empty; a block leaves only its scores
+    // (block_scores).  The pools hold the tail positions i * kTailPools + pool of the tails
+    // concatenated over (b, index-K head); a warp turns to the next pool after each block.
+    const long long total_t = offt[B];
+    if (a.sched != nullptr && total_t > 0) {
+        int pool = (int)(((long long)blockIdx.x * W + w) % kTailPools);
+        auto grab = [&]() -> long long {
+            long long x = -1;
+            if (lane == 0) {
+                for (int t = 0; t < kTailPools && x < 0; ++t, pool = (pool + 1) % kTailPools) {
+                    if (*reinterpret_cast<volatile int *>(&exh[pool])) continue;
+                    const long long y = (long long)atomicAdd(&a.sched[pool], 1u) * kTailPools + pool;
+                    if (y < total_t)
+                        x = y;
+                    else
+                        *reinterpret_cast<volatile int *>(&exh[pool]) = 1;
+                }
+            }
+            return __shfl_sync(FULL, x, 0);
+        };
+        // tail position -> (b, index-K head, block, chunks)
+        auto locate = [&](long long x) -> int4 {
+            int lo = 0, hi = B - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (offt[mid] <= x) lo = mid; else hi = mid - 1;
+            }
+            const int nt = nbs[lo] - nba[lo];
+            const int r = (int)(x - offt[lo]);
+            const int hik = r / nt;
+            const int n = nba[lo] + (r - hik * nt);
+            int bt = lens[lo] - n * Bk;
+            bt = bt < Bk ? bt : Bk;
+            return make_int4(lo, hik, n, (bt + CT - 1) / CT);
+        };
+        int4 *my_rec = trec + w * 4;  // blocks with chunks issued, in order (at most S + 1 live)
+        int t_head = 0, t_tail = 0, pc = 0;
+        bool more = !failed, have = false;
+        int4 pr = make_int4(0, 0, 0, 0);
+        auto t_issue = [&]() {
+            while (more && !failed && issued - consumed < S) {
+                if (!have) {
+                    const long long x = grab();
+                    if (x < 0) {
+                        more = false;
+                        break;
+                    }
+                    pr = locate(x);
+                    if (lane == 0) my_rec[t_tail & 3] = pr;
+                    __syncwarp();
+                    ++t_tail;
+                    have = true;
+                    pc = 0;
+                }
+                if (lane == 0) {
+                    const int slot = issued % S;
+                    const int row = (pr.x * Hik + pr.y) * a.L_max + pr.z * Bk + pc * CT;
+                    unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
+                    mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
+                    tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
+                    if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
+                }
+                ++issued;
+                if (++pc == pr.w) have = false;
+            }
+        };
+        float *my_q = q_w + (QREG ? 0 : w * GPS * DI);
+        int qb = -1, qh = -1;
+        t_issue();
+        while (t_head < t_tail) {
+            const int4 r = my_rec[t_head & 3];
+            if (r.x != qb || r.y != qh) {
+                qb = r.x;
+                qh = r.y;
+                if constexpr (QREG) {
+                    const T *src = qg + ((size_t)qb * a.G + qh) * DI;
+#pragma unroll
+                    for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
+                } else {
+                    __syncwarp();
+                    for (int i = lane; i < GPS * DI; i += 32) {
+                        const int g = qh + Hik * (i / DI);
+                        my_q[i] = load_elem(qg + ((size_t)qb * a.G + g) * DI + i % DI);
+                    }
+                    __syncwarp();
+                }
+            }
+            int bt = lens[r.x] - r.z * Bk;
+            bt = bt < Bk ? bt : Bk;
+            float m[GPS];
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) m[gl] = -INFINITY;
+            for (int c = 0; c < r.w; ++c) {
+                const int slot = consumed % S;
+                if (!failed && !mbar_wait(&my_bars[slot], (consumed / S) & 1, a.status)) {
+                    failed = true;
+                    for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
+                }
+                int nt = bt - c * CT;
+                nt = nt < CT ? nt : CT;
+                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, r.x, r.y, r.z * Bk + c * CT, qv, my_q, m);
+                __syncwarp();
+                ++consumed;
+                t_issue();
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], __shfl_xor_sync(FULL, m[gl], o));
+            if (a.block_scores != nullptr && lane == 0)
+#pragma unroll
+                for (int gl = 0; gl < GPS; ++gl)
+                    a.block_scores[((size_t)r.x * a.G + r.y + Hik * gl) * a.nb_max + r.z] = m[gl];
+            ++t_head;
+            t_issue();
+        }
+    }
+
+    // the CTA that finishes last returns the pool counters to zero for the next call
+    __syncthreads();
+    if (a.sched != nullptr && tid == 0) {
+        __threadfence();
+        if (atomicAdd(&a.sched[kTailPools], 1u) == gridDim.x - 1) {
+            for (int i = 0; i < kTailPools; ++i) a.sched[i] = 0;
+            __threadfence();
+            a.sched[kTailPools] = 0;
+        }
+    }
 }
 
 __global__ void fill_neg_inf_kernel(const FillArgs a) {
@@ -337,8 +486,11 @@ __global__ void fill_neg_inf_kernel(const FillArgs a) {
 template <typename T, int GPS, int ROWB>
 cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
     constexpr int W = ScanShape<GPS>::W, S = ScanShape<GPS>::S;
+    constexpr int DI = ROWB / (int)sizeof(T);
+    constexpr bool QREG = GPS == 1 && DI <= 64;
     const size_t smem = 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 +
-                        (size_t)GPS * (ROWB / sizeof(T)) * 4 + (size_t)(a.B + 1) * 8 + (size_t)a.B * 8;
+                        (size_t)GPS * DI * 4 + (size_t)W * 4 * 16 + (QREG ? 0 : (size_t)W * GPS * DI * 4) +
+                        (size_t)(a.B + 1) * 16 + (size_t)a.B * 12 + kTailPools * 4 + 64;
     static size_t attr_bytes = 0;  // opt-in raised on demand (smem grows with the batch)
     if (smem > attr_bytes) {
         cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB>,

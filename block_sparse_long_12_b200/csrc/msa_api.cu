@@ -166,6 +166,8 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
         off += round256(cand);
         L.cand_i = off;
         off += round256(cand);
+        L.tail_scores = off;
+        off += round256((size_t)p.batch * p.n_kv_heads * nb_max_of(p) * 4);
     }
     if (attend) {
         if (p.flags & MSA_DENSE) {
@@ -301,7 +303,8 @@ msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t str
 
 msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream) {
     if (ws == nullptr) return fail(MSA_ERR_INVALID_ARG, "ws is NULL");
-    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), (cudaStream_t)stream);
+    // the status word and the scan's counters (left non-zero by a scan that did not end normally)
+    cudaError_t e = cudaMemsetAsync(ws, 0, (kSchedWord + kTailPools + 1) * sizeof(unsigned), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
     return MSA_OK;
 }
@@ -334,6 +337,7 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
     a.n_cta = decode_ws_layout(*p, true, false, n_sm).n_cta;
     a.token_scores = mode == MSA_SCORES_TOKEN ? scores_out : nullptr;
     a.block_scores = mode == MSA_SCORES_BLOCKMAX ? scores_out : nullptr;
+    a.sched = reinterpret_cast<unsigned *>(ws) + kSchedWord;
     a.status = reinterpret_cast<int *>(ws);
     e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
@@ -373,6 +377,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
         a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
         a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
         a.seg_info = reinterpret_cast<const SegInfo *>(wsb + L.seg_info);
+        a.tail_scores = reinterpret_cast<const float *>(wsb + L.tail_scores);
         a.ids_out = ids_out;
     }
     a.n_cta = L.n_cta;
@@ -447,6 +452,8 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.cand_s = reinterpret_cast<float *>(wsb + L.cand_s);
     a.cand_i = reinterpret_cast<int *>(wsb + L.cand_i);
     a.seg_info = reinterpret_cast<SegInfo *>(wsb + L.seg_info);
+    a.block_scores = reinterpret_cast<float *>(wsb + L.tail_scores);  // read back for the tails' blocks
+    a.sched = reinterpret_cast<unsigned *>(wsb) + kSchedWord;
     a.counters = reinterpret_cast<int *>(wsb + L.counters);
     a.status = reinterpret_cast<int *>(wsb);
     cudaError_t e = stage_mark(0, s);

@@ -17,7 +17,14 @@ constexpr int kMaxBatch = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxGroupsPerSeg = 8;   // n_kv_heads / n_idx_k_heads handled by one index-K stream
 constexpr int kMaxPiecesPerSeg = 256; // lists merged per (segment, group) by one warp (8 per lane)
-constexpr size_t kStatusBytes = 256;  // workspace head: device status word + padding
+constexpr size_t kStatusBytes = 256;  // workspace head: device status word, scan counters, padding
+constexpr int kSchedWord = 4;          // ws words 4..4+kTailPools: tail-pool counters, then finished CTAs
+constexpr int kTailPools = 4;          // interleaved pools (counters) of the scan's shared tail
+
+// Blocks of a segment of nb blocks that the index scan hands out dynamically
+// (the last quarter); the first nb - scan_tail_blocks(nb) are split equally
+// between the CTAs.
+__host__ __device__ inline int scan_tail_blocks(int nb) { return nb / 4; }
 
 // ---- decode index scan (Step 1 for decode): persistent, 1 CTA per SM
 constexpr int kScanChunkBytes = 8192;   // ring stage: bytes of index keys per TMA copy
@@ -45,6 +52,7 @@ struct ScanArgs {
     float *cand_s;  // [n_seg, n_cta, G/Hik, k] per-piece sorted top-k (nullable)
     int *cand_i;
     SegInfo *seg_info;     // [n_seg] (written by CTA 0 when cand_s != nullptr)
+    unsigned *sched;       // [kTailPools + 1] tail-pool counters and finished CTAs (workspace head)
     float *token_scores;   // [B, 1, G, L_max] (nullable)
     float *block_scores;   // [B, 1, G, nb_max] (nullable)
     int *counters;         // [B, G] attention arrival counters, zeroed by CTA 0 (nullable)
@@ -60,6 +68,7 @@ struct AttnArgs {
     const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]: select in the kernel (fused decode)
     const int *cand_i;
     const SegInfo *seg_info;
+    const float *tail_scores;  // [B, G, nb_max] block scores of the segments' tails (fused decode)
     int n_cta;
     int *ids_out;              // nullable (fused decode)
     float *top_scores_out;     // nullable (fused decode)
@@ -138,7 +147,7 @@ struct FillArgs {
 
 // Workspace layout of the decode entries (offsets in bytes from ws).
 struct DecodeWs {
-    size_t seg_info, cand_s, cand_i, counters, part_o, part_lse, total;
+    size_t seg_info, cand_s, cand_i, tail_scores, counters, part_o, part_lse, total;
     int n_cta, S, blocks_per_split;
 };
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);

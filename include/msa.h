@@ -42,6 +42,10 @@
  *   - Scratch memory comes from the caller: `ws` of at least
  *     msa_workspace_size(params, entry) bytes (256-byte aligned).  Each call
  *     overwrites the workspace; calls that share a workspace must not overlap.
+ *     Its first 256 bytes hold the device status word and the index scan's
+ *     work counters (msa_index_score, msa_decode_fused), which the scan
+ *     returns to zero when it ends: zero-fill a workspace once before its
+ *     first use (a cudaMemset or a zeroed allocation).
  *   - Arguments are checked before anything is enqueued; on error nothing is
  *     launched and the call returns the status (text: msa_last_error_string).
  *   - A CUDA launch error returns MSA_ERR_CUDA.  Devices other than
@@ -226,7 +230,9 @@ MSA_API const char *msa_status_string(msa_status_t status);
 
 /* Device status word kept in a workspace (first 4 bytes): MSA_OK, or
  * MSA_ERR_TIMEOUT after a bounded wait ran out.  Copies it to *status after
- * synchronising `stream`; msa_clear_device_status resets it asynchronously. */
+ * synchronising `stream`; msa_clear_device_status resets it asynchronously,
+ * together with the scan's work counters (left non-zero by a scan that did
+ * not end normally). */
 MSA_API msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t stream);
 MSA_API msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream);
 

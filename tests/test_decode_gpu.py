@@ -204,6 +204,30 @@ def test_repeat_calls_same_workspace():
     assert _lib.msa_get_device_status(ws) == 0
 
 
+def test_workspace_reused_across_shapes():
+    """One workspace serves calls of different shapes in turn (its layout moves with the
+    shape): every call equals a call on a fresh workspace, and the status stays clean."""
+    api = _api()
+    from block_sparse_long_12_b200 import _lib
+    wa, wb = small(batch=4, seed=5), small(batch=1, max_seq_len=7000, seed=6, n_kv_heads=2, n_q_heads=8,
+                                           n_idx_k_heads=2)
+    ia, ib = make_inputs(wa, device="cuda"), make_inputs(wb, device="cuda")
+
+    def params(inp, w):
+        return api.params_from(inp["q"], inp["q_idx"], inp["k"], inp["k_idx"], block_size=w.block_size,
+                               top_k=w.top_k, seq_lens=inp["seq_lens"])
+
+    shared = api.workspace([params(ia, wa), params(ib, wb)], api.MSA_ENTRY_DECODE_FUSED, "cuda")
+    for inp, w in ((ia, wa), (ib, wb), (ia, wa), (ib, wb)):
+        got = api.decode(inp["q"], inp["q_idx"], inp["k"], inp["v"], inp["k_idx"], inp["seq_lens"],
+                         block_size=w.block_size, top_k=w.top_k, ws=shared)
+        got = [t.clone() for t in got]
+        ref = run_fused(inp, w)
+        for t1, t2 in zip(got, ref):
+            assert torch.equal(t1, t2)
+    assert _lib.msa_get_device_status(shared) == 0
+
+
 @pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m"])
 def test_full_size_decode(name):
     """The benchmark workloads at full size, checked against the oracle on every (sequence, group)."""
