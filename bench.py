@@ -37,8 +37,9 @@ METRIC = "MSA decode us/step/layer @1M ctx; prefill tok/s; % of HBM/tensor roofl
 UNIT = "us/step/layer"
 L2_FLUSH_BYTES = 512 << 20
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_index_scan_traffic.json")
-SCAN_SOURCES = ["block_sparse_long_12_b200/csrc/decode_index.cu", "block_sparse_long_12_b200/csrc/msa_device.cuh",
-                "block_sparse_long_12_b200/csrc/msa_internal.h"]
+# the index scan kernel's own sources: a committed DRAM-traffic capture counts only while they are unchanged
+SCAN_SOURCES = ["block_sparse_long_12_b200/csrc/decode_index.cu", "block_sparse_long_12_b200/csrc/scan_args.h",
+                "block_sparse_long_12_b200/csrc/msa_device.cuh", "block_sparse_long_12_b200/csrc/tcgen05.cuh"]
 
 
 def scan_source_hash() -> str:

@@ -88,23 +88,100 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
 }
 
 
-// Final TopK of group g of sequence b from the scan's per-piece sorted lists
-// (the fused decode step).  The candidates are staged in `scratch` (at least
-// 16 * n_cta * k + 16 bytes) by the whole CTA.  A threshold that the final k
-// all reach is the k-th best of a subset (the heads of the pieces' lists);
-// only candidates at least that good are kept, and each is ranked by
-// counting the survivors that beat it.  Leaves the list in sel_s /
+// (score, block id) as one 64-bit key whose unsigned order is the selection
+// order (higher score first, then lower id): the score's bits made
+// order-preserving in the high word, the complemented id in the low word.
+__device__ inline unsigned long long sel_key(float s, int id) {
+    uint32_t u = __float_as_uint(s + 0.0f);  // -0 -> +0: equal scores compare by id
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)u << 32) | (uint32_t)~(uint32_t)id;
+}
+__device__ inline void sel_unkey(unsigned long long key, float &s, int &id) {
+    uint32_t u = (uint32_t)(key >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    s = __uint_as_float(u);
+    id = (int)~(uint32_t)key;
+}
+
+// Descending bitonic sort of keys[0, P) (P a power of two) by the whole CTA.
+__device__ inline void block_sort_desc(unsigned long long *keys, int P) {
+    for (int size = 2; size <= P; size <<= 1)
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const unsigned long long x = keys[lo], y = keys[hi];
+                const bool desc = (lo & size) == 0;
+                if (desc ? x < y : x > y) {
+                    keys[lo] = y;
+                    keys[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+}
+
+// Descending bitonic sort of 64 keys held by one warp, element lane + 32 * j
+// in v[j]; the element of rank r ends in lane r % 32, v[r / 32].
+__device__ inline void warp_sort64_desc(unsigned long long (&v)[2], int lane) {
+#pragma unroll
+    for (int size = 2; size <= 64; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride == 32) {
+                if (v[0] < v[1]) {  // size 64: one descending run
+                    const unsigned long long t = v[0];
+                    v[0] = v[1];
+                    v[1] = t;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int idx = lane + 32 * j;
+                    const unsigned long long o = __shfl_xor_sync(FULL, v[j], stride);
+                    const bool keep_max = ((idx & stride) == 0) == ((idx & size) == 0);
+                    v[j] = keep_max ? (v[j] > o ? v[j] : o) : (v[j] < o ? v[j] : o);
+                }
+            }
+        }
+}
+
+constexpr int kSortCap = 512;  // survivors sorted at once; more go the counting way
+
+// Final TopK of group g of sequence b (the fused decode step) from the scan's
+// per-piece sorted lists and the block scores of the stream's tail.  The
+// lists are staged in `scratch` (select_scratch_bytes) by the whole CTA.  The
+// k-th best of a subset of the candidates (the first entries of some lists)
+// is a floor that the final k all reach: the list entries and tail blocks at
+// or above it are sorted as 64-bit keys and the first k kept.  If too many
+// reach the floor, counting ranks take over.  Leaves the list in sel_s /
 // sel_i[0..32), padded with (-inf, -1).  Called by every thread of the CTA.
 __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int cap = a.n_cta * a.k;
+    // scratch: lists [cap] scores | [cap] ids | 32 state words | one region for the survivors
+    // (sort keys, or scores and ids) and for the tail merge's lists
     float *ls = reinterpret_cast<float *>(scratch);
     int *li = reinterpret_cast<int *>(ls + cap);
-    float *ss = reinterpret_cast<float *>(li + cap);
+    int *st = li + cap;  // [0] survivors, [1] threshold id, [2] threshold score (bits), [4..] per-warp floors
+    float *ss = reinterpret_cast<float *>(st + 32);
     int *si = reinterpret_cast<int *>(ss + cap);
-    int *st = si + cap;  // [0] survivors, [1] threshold id, [2] threshold score (bits)
     const int gps = a.G / a.Hik;
     const int seg = b * a.Hik + g % a.Hik, gl = g / a.Hik;
+    // the first batch of the tail's block scores (merged at the end) is loaded now, so that its
+    // latency overlaps the work on the ranges' lists
+    constexpr int kBatch = 16;  // loads in flight per lane
+    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int nb = (L + a.Bk - 1) / a.Bk, nt = a.tail_scores != nullptr ? scan_tail_blocks(nb) : 0;
+    const float *tsc = a.tail_scores + ((size_t)b * a.G + g) * ((a.L_max + a.Bk - 1) / a.Bk);
+    const int base0 = nb - nt + warp * 32 * kBatch;
+    float v0[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+        const int n = base0 + u * 32 + lane;
+        v0[u] = n < nb ? tsc[n] : -INFINITY;
+    }
     const SegInfo info = a.seg_info[seg];
     const int k = a.k, np = info.n_pieces, n = np * k;
     for (int i = tid; i < n; i += nthr) {
@@ -122,6 +199,69 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
         sel_i[tid] = -1;
     }
     __syncthreads();
+    {
+        // floor: the k-th best of the first J entries of up to 64 / J lists, sorted by one warp;
+        // the k-th best of any subset is no better than the k-th best of all candidates
+        if (warp == 0) {
+            const int J = np > 0 ? min(k, max(1, (2 * k + np - 1) / np)) : 1;
+            const int nl = min(np, 64 / J);
+            unsigned long long v[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = lane + 32 * j, l = e / J, pos = e - l * J;
+                v[j] = 0ull;
+                if (l < nl && li[l * k + pos] >= 0) v[j] = sel_key(ls[l * k + pos], li[l * k + pos]);
+            }
+            warp_sort64_desc(v, lane);
+            const unsigned long long kth = __shfl_sync(FULL, (k - 1) < 32 ? v[0] : v[1], (k - 1) & 31);
+            if (lane == 0) {
+                st[4] = (int)(uint32_t)kth;
+                st[5] = (int)(uint32_t)(kth >> 32);
+            }
+        }
+        __syncthreads();
+        // 0 (fewer than k entries in the subset): no floor
+        const unsigned long long fk = ((unsigned long long)(uint32_t)st[5] << 32) | (uint32_t)st[4];
+        // survivors: list prefixes and tail blocks at or above the floor, as sort keys
+        unsigned long long *keys = reinterpret_cast<unsigned long long *>(ss);  // [max(cap, kSortCap)]
+        const int key_cap = cap > kSortCap ? cap : kSortCap;
+        for (int l = tid; l < np; l += nthr)
+            for (int j = 0; j < k; ++j) {
+                const int id = li[l * k + j];
+                if (id < 0) break;
+                const unsigned long long key = sel_key(ls[l * k + j], id);
+                if (key < fk) break;
+                const int at = atomicAdd(&st[0], 1);
+                if (at < key_cap) keys[at] = key;
+            }
+        for (int base = base0; base < nb; base += nwarps * 32 * kBatch) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int n = base + u * 32 + lane;
+                const float v = base == base0 ? v0[u] : (n < nb ? tsc[n] : -INFINITY);
+                const unsigned long long key = sel_key(v, n);
+                if (n < nb && key >= fk) {
+                    const int at = atomicAdd(&st[0], 1);
+                    if (at < key_cap) keys[at] = key;
+                }
+            }
+        }
+        __syncthreads();
+        const int m = st[0];
+        if (m <= kSortCap) {
+            int P = 32;
+            while (P < m) P <<= 1;
+            for (int i = m + tid; i < P; i += nthr) keys[i] = 0ull;  // below every real key
+            __syncthreads();
+            block_sort_desc(keys, P);
+            if (tid < k && tid < m) sel_unkey(keys[tid], sel_s[tid], sel_i[tid]);
+            __syncthreads();
+            return;
+        }
+        // too many at the floor: the counting way below (its state starts afresh)
+        if (tid == 0) st[0] = 0;
+        __syncthreads();
+    }
     // Threshold: the k-th best among the first J entries of every piece.  The k-th best of any
     // subset is no better than the k-th best of all candidates, so the whole top-k passes it;
     // taking each piece's head makes it tight, and few candidates survive.
@@ -171,25 +311,18 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
     // The tail of the stream (blocks [nb - nt, nb)) left block scores only: every warp keeps
     // the k best of its share of those that beat the k-th entry so far (the others cost one
     // comparison), and one warp merges these lists with the ranges' k best.
-    int L = a.seq_lens[b];
-    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
-    const int nb = (L + a.Bk - 1) / a.Bk, nt = scan_tail_blocks(nb);
-    const int nb_max = (a.L_max + a.Bk - 1) / a.Bk;
-    const float *tsc = a.tail_scores + ((size_t)b * a.G + g) * nb_max;
-    const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
     WarpTopK t;
     t.reset();
     // floor: a tail block must beat the k-th entry of the ranges' list (while the warp's own
     // list is not full its threshold is below that)
     const float fl_s = sel_s[k - 1];
     const int fl_i = sel_i[k - 1];
-    constexpr int kBatch = 16;  // loads in flight per lane
-    for (int base = nb - nt + warp * 32 * kBatch; base < nb; base += nwarps * 32 * kBatch) {
+    for (int base = base0; base < nb; base += nwarps * 32 * kBatch) {
         float v[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int n = base + u * 32 + lane;
-            v[u] = n < nb ? tsc[n] : -INFINITY;
+            v[u] = base == base0 ? v0[u] : (n < nb ? tsc[n] : -INFINITY);
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
@@ -203,8 +336,8 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
             }
         }
     }
-    float *tl_s = ls;  // [1 + nwarps][32] lists (the staging area is free now)
-    int *tl_i = li;
+    float *tl_s = ss;  // [1 + nwarps][32] lists (the survivors are ranked by now)
+    int *tl_i = reinterpret_cast<int *>(tl_s + 9 * 32);
     tl_s[(1 + warp) * 32 + lane] = t.s;
     tl_i[(1 + warp) * 32 + lane] = t.id;
     if (warp == 0) {
@@ -214,6 +347,12 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
     __syncthreads();
     if (warp == 0) warp_merge_sorted_lists<1>(tl_s, tl_i, 1 + nwarps, k, 32, k, sel_s, sel_i, lane);
     __syncthreads();
+}
+
+// Scratch bytes select_group_topk needs (lists of n_cta pieces of k entries).
+__host__ __device__ inline size_t select_scratch_bytes(int n_cta, int k) {
+    const size_t cap = (size_t)n_cta * k;
+    return cap * 8 + 32 * 4 + (cap > (size_t)kSortCap ? cap : (size_t)kSortCap) * 8;
 }
 
 // The last split CTA of (b, g) merges the normalised partial outputs of all
@@ -572,7 +711,7 @@ constexpr int kMmaThreads = 128;  // 4 warps
 constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
 
 template <int D>
-__global__ void __launch_bounds__(kMmaThreads) decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                       const __grid_constant__ CUtensorMap vmap,
                                                                       const AttnArgs a) {
     constexpr int NH = D / 64;     // 64-dim halves of a K/V row
@@ -869,7 +1008,7 @@ cudaError_t launch_attn_t(AttnArgs a, cudaStream_t s, bool pdl) {
     using Cfg = AttnCfg<T, D, R>;
     const int KT = a.Bk < Cfg::KT_MAX ? a.Bk : Cfg::KT_MAX;
     const size_t ring = (size_t)Cfg::NST * 2 * KT * D * Cfg::ES;
-    const size_t scratch = a.cand_s != nullptr ? max((size_t)16 * a.n_cta * a.k + 16, (size_t)2 * 9 * 32 * 4) : 0;
+    const size_t scratch = a.cand_s != nullptr ? select_scratch_bytes(a.n_cta, a.k) : 0;
     a.ring_bytes = (int)((ring > scratch ? ring : scratch) + 15) / 16 * 16;
     // p_s doubles as the [S][r] merge weights of the last split: R * max(KT, kMaxSplits) floats
     const size_t smem = (size_t)a.ring_bytes + Cfg::NST * 8 + 64 * 4 + 3 * R * 4 +
@@ -913,7 +1052,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     const bool one_tile = a.blocks_per_split == 1 && a.Bk <= 128;
     a.nst = one_tile ? 1 : 2;
     const size_t ring = a.nst * stage;
-    const size_t scratch = a.cand_s != nullptr ? max((size_t)16 * a.n_cta * a.k + 16, (size_t)2 * 9 * 32 * 4) : 0;
+    const size_t scratch = a.cand_s != nullptr ? select_scratch_bytes(a.n_cta, a.k) : 0;
     const size_t wgt = (size_t)a.S * a.r * 4 > (size_t)kMmaRows * D * 4 + 64 ? (size_t)a.S * a.r * 4
                                                                             : (size_t)kMmaRows * D * 4 + 64;
     size_t rb = ring > scratch ? ring : scratch;

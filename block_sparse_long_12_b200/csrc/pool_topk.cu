@@ -18,7 +18,7 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const PoolTopkArgs a) {
     __shared__ float out_s[32];
     __shared__ int out_i[32];
     const int row = blockIdx.x;
-    const int g = row % a.G, t = (row / a.G) % a.q_len, b = row / (a.G * a.q_len);
+    const int t = (row / a.G) % a.q_len, b = row / (a.G * a.q_len);
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int pos;
     if (a.prefill) {
