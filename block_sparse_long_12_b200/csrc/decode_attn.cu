@@ -147,6 +147,52 @@ __device__ inline void warp_sort64_desc(unsigned long long (&v)[2], int lane) {
 
 constexpr int kSortCap = 512;  // survivors sorted at once; more go the counting way
 
+// The scan's pieces of segment (b, hik): which CTA's list comes first and how
+// many CTAs hold one.  The same split the scan makes (equal ranges over the
+// streams' first nb - scan_tail_blocks(nb) blocks), recomputed from seq_lens
+// so that it is known before the scan has finished.  Called by every thread.
+__device__ SegInfo seg_pieces(const AttnArgs &a, int b, int hik) {
+    __shared__ long long red[2][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    long long tot = 0, pre = 0;
+    for (int bb = threadIdx.x; bb < a.B; bb += blockDim.x) {
+        int L = a.seq_lens[bb];
+        L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+        const int nb = (L + a.Bk - 1) / a.Bk;
+        const long long na = (long long)(nb - scan_tail_blocks(nb)) * a.Hik;
+        tot += na;
+        if (bb < b) pre += na;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(FULL, tot, o);
+        pre += __shfl_xor_sync(FULL, pre, o);
+    }
+    if (lane == 0) {
+        red[0][warp] = tot;
+        red[1][warp] = pre;
+    }
+    __syncthreads();
+    tot = 0;
+    pre = 0;
+    for (int w2 = 0; w2 < nwarps; ++w2) {
+        tot += red[0][w2];
+        pre += red[1][w2];
+    }
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int nb = (L + a.Bk - 1) / a.Bk, nba = nb - scan_tail_blocks(nb);
+    __syncthreads();  // red is free again
+    SegInfo si{-1, 0};
+    const long long per = tot > 0 ? (tot + a.n_cta - 1) / a.n_cta : 1;
+    if (nba > 0) {
+        const long long st = pre + (long long)hik * nba;
+        si.first_cta = (int)(st / per);
+        si.n_pieces = (int)((st + nba - 1) / per) - si.first_cta + 1;
+    }
+    return si;
+}
+
 // Final TopK of group g of sequence b (the fused decode step) from the scan's
 // per-piece sorted lists and the block scores of the stream's tail.  The
 // lists are staged in `scratch` (select_scratch_bytes) by the whole CTA.  The
@@ -155,7 +201,8 @@ constexpr int kSortCap = 512;  // survivors sorted at once; more go the counting
 // or above it are sorted as 64-bit keys and the first k kept.  If too many
 // reach the floor, counting ranks take over.  Leaves the list in sel_s /
 // sel_i[0..32), padded with (-inf, -1).  Called by every thread of the CTA.
-__device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
+__device__ void select_group_topk(const AttnArgs &a, int b, int g, const SegInfo info, unsigned char *scratch,
+                                  float *sel_s, int *sel_i) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int cap = a.n_cta * a.k;
     // scratch: lists [cap] scores | [cap] ids | 32 state words | one region for the survivors
@@ -182,7 +229,6 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
         const int n = base0 + u * 32 + lane;
         v0[u] = n < nb ? tsc[n] : -INFINITY;
     }
-    const SegInfo info = a.seg_info[seg];
     const int k = a.k, np = info.n_pieces, n = np * k;
     for (int i = tid; i < n; i += nthr) {
         const size_t src = (((size_t)seg * a.n_cta + i / k) * gps + gl) * k + i % k;
@@ -248,6 +294,18 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, unsigned char
         }
         __syncthreads();
         const int m = st[0];
+        if (m <= 64) {
+            // one warp sorts them in registers
+            if (warp == 0) {
+                unsigned long long v[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) v[j] = lane + 32 * j < m ? keys[lane + 32 * j] : 0ull;
+                warp_sort64_desc(v, lane);
+                if (lane < k && lane < m) sel_unkey(v[0], sel_s[lane], sel_i[lane]);
+            }
+            __syncthreads();
+            return;
+        }
         if (m <= kSortCap) {
             int P = 32;
             while (P < m) P <<= 1;
@@ -437,10 +495,11 @@ __device__ inline bool last_split(const AttnArgs &a, int b, int g, int *flag) {
 }
 
 // Obtain the group's list: fused selection from the scan, or a given ids tensor.
-__device__ inline void group_list(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
+__device__ inline void group_list(const AttnArgs &a, int b, int g, const SegInfo info, unsigned char *scratch,
+                                  float *sel_s, int *sel_i) {
     if (a.dense) return;
     if (a.cand_s != nullptr) {
-        select_group_topk(a, b, g, scratch, sel_s, sel_i);
+        select_group_topk(a, b, g, info, scratch, sel_s, sel_i);
         if (blockIdx.x == 0 && threadIdx.x < a.k) {
             const size_t o = ((size_t)b * a.G + g) * a.k + threadIdx.x;
             if (a.ids_out != nullptr) a.ids_out[o] = sel_i[threadIdx.x];
@@ -505,10 +564,12 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const int pos = L - 1;
     const int nb = (L + a.Bk - 1) / a.Bk;
 
+    // where the scan leaves this group's lists is known from seq_lens alone
+    const SegInfo info = (!a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
     __shared__ int last_flag;
-    group_list(a, b, g, ring, sel_s, sel_i);
+    group_list(a, b, g, info, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1)
     const int bps = a.blocks_per_split;
@@ -698,17 +759,16 @@ __device__ inline int cluster_rank() {
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return (int)r;
 }
-// load a float from the shared memory of CTA `rank` of the cluster, at the same offset as `local`
-__device__ inline float ld_peer(const float *local, int rank) {
+// store a float into the shared memory of CTA `rank` of the cluster, at the same offset as `local`
+__device__ inline void st_peer(float *local, int rank, float v) {
     uint32_t ra;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 constexpr int kMmaThreads = 128;  // 4 warps
 constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
+constexpr int kMaxCluster = 8;    // splits of a group that form one cluster
 
 template <int D>
 __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -733,6 +793,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     int *red_i = reinterpret_cast<int *>(red_s + 32);                              // [32]
     int *misc = red_i + 32;                                                        // [4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 4);                       // [2]
+    float *recv = reinterpret_cast<float *>(bars + 2);   // [cluster][slice] partials pushed to this CTA
+    float *recv_l = recv + kMmaRows * D + kMaxCluster;   // [cluster][16] their log2 normalisers
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int grp = lane >> 2, tig = lane & 3;  // fragment row group / thread in group
@@ -764,9 +826,11 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     const int pos = L - 1;
     const int nb = (L + a.Bk - 1) / a.Bk;
 
+    // where the scan leaves this group's lists is known from seq_lens alone
+    const SegInfo info = (!a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
-    group_list(a, b, g, ring, sel_s, sel_i);
+    group_list(a, b, g, info, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1), each cut into tiles of KT keys
     const int j0 = s * a.blocks_per_split;
@@ -934,43 +998,45 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     }
 
     if (a.cluster > 1) {
-        // the splits of (b, g) form one thread-block cluster: partials stay in shared memory and
-        // every CTA merges a slice of the output reading its peers' partials directly
-        float *po_s = reinterpret_cast<float *>(ring);  // [16][D], the ring is idle now
-        float *pl_s = po_s + kMmaRows * D;               // [16]
+        // The splits of (b, g) form one thread-block cluster.  CTA c owns a slice of the r * D
+        // outputs; every CTA stores its normalised partial of each slice, and its log2
+        // normalisers, straight into the owner's shared memory, and after one cluster barrier
+        // each owner merges its slice from local memory (nothing is read remotely).
+        const int cs = a.cluster, rank = cluster_rank();
+        const int n_out = r * D, per = (n_out + cs - 1) / cs;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int row = grp + 8 * h;
+            if (row >= r) continue;
             const float inv = l_run[h] > 0.f ? 1.f / l_run[h] : 0.f;
 #pragma unroll
             for (int dt = 0; dt < DT; ++dt) {
-                const int d = (w + 4 * dt) * 8 + tig * 2;
-                *reinterpret_cast<float2 *>(po_s + row * D + d) =
-                    make_float2(oacc[dt][2 * h] * inv, oacc[dt][2 * h + 1] * inv);
+                const int f = row * D + (w + 4 * dt) * 8 + tig * 2;
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int owner = (f + e) / per;
+                    st_peer(recv + rank * per + (f + e - owner * per), owner, oacc[dt][2 * h + e] * inv);
+                }
             }
-            if (w == 0 && tig == 0) pl_s[row] = l_run[h] > 0.f ? m_run[h] + log2f(l_run[h]) : -INFINITY;
+            if (w == 0 && tig == 0) {
+                const float lse2 = l_run[h] > 0.f ? m_run[h] + log2f(l_run[h]) : -INFINITY;
+                for (int c = 0; c < cs; ++c) st_peer(recv_l + rank * kMmaRows + row, c, lse2);
+            }
         }
         cluster_sync_all();
-        const int cs = a.cluster, rank = cluster_rank();
-        const int n_out = r * D, per = (n_out + cs - 1) / cs;
         const int f_end = (rank + 1) * per < n_out ? (rank + 1) * per : n_out;
         __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + ((size_t)b * a.Hq + (size_t)g * r) * D;
         for (int f = rank * per + tid; f < f_end; f += kMmaThreads) {
             const int h = f / D;
-            float ls[8];
             float M = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                ls[c] = c < cs ? ld_peer(pl_s + h, c) : -INFINITY;
-                M = fmaxf(M, ls[c]);
-            }
+            for (int c = 0; c < cs; ++c) M = fmaxf(M, recv_l[c * kMmaRows + h]);
             float num = 0.f, den = 0.f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                if (c < cs && ls[c] > -INFINITY) {
-                    const float wgt = exp2f(ls[c] - M);
+            for (int c = 0; c < cs; ++c) {
+                const float lc = recv_l[c * kMmaRows + h];
+                if (lc > -INFINITY) {
+                    const float wgt = exp2f(lc - M);
                     den += wgt;
-                    num = fmaf(wgt, ld_peer(po_s + h * D + f % D, c), num);
+                    num = fmaf(wgt, recv[c * per + (f - rank * per)], num);
                 }
             }
             o[f] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
@@ -978,8 +1044,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
                 a.lse[(size_t)b * a.Hq + (size_t)g * r + h] =
                     den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
         }
-        cluster_sync_all();  // peers may still be reading this CTA's partials
-        return;
+        return;  // no peer touches this CTA's shared memory after the barrier
     }
 
     // normalised partial output and log2 normaliser of this split
@@ -1045,7 +1110,7 @@ cudaError_t launch_attn_r(const AttnArgs &a, cudaStream_t s, bool pdl) {
 
 template <int D>
 cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
-    a.cluster = (!a.dense && a.S <= 8) ? a.S : 1;
+    a.cluster = (!a.dense && a.S <= kMaxCluster) ? a.S : 1;
     const int KT = a.Bk < 128 ? a.Bk : 128;
     const size_t stage = (size_t)2 * (D / 64) * KT * 128;
     // one stage when every split is a single tile, two otherwise
@@ -1058,7 +1123,8 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     size_t rb = ring > scratch ? ring : scratch;
     rb = rb > wgt ? rb : wgt;
     a.ring_bytes = (int)((rb + 1023) / 1024 * 1024);
-    const size_t smem = 1024 + (size_t)a.ring_bytes + (size_t)kMmaRows * (KT + 8) * 2 + (64 + 64 + 32 * 4 + 4) * 4 + 64;
+    const size_t smem = 1024 + (size_t)a.ring_bytes + (size_t)kMmaRows * (KT + 8) * 2 + (64 + 64 + 32 * 4 + 4) * 4 + 16 +
+                        ((size_t)kMmaRows * D + kMaxCluster + (size_t)kMaxCluster * kMmaRows) * 4 + 64;
     static size_t attr_bytes = 0;
     if (smem > attr_bytes) {
         cudaError_t e = cudaFuncSetAttribute(decode_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

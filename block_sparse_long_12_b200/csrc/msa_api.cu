@@ -376,7 +376,6 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
     if (after_scan) {  // select the group's list inside the attention kernel
         a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
         a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
-        a.seg_info = reinterpret_cast<const SegInfo *>(wsb + L.seg_info);
         a.tail_scores = reinterpret_cast<const float *>(wsb + L.tail_scores);
         a.ids_out = ids_out;
     }

@@ -32,7 +32,6 @@ struct AttnArgs {
     const int *ids_in;         // [B, 1, G, k] given selection (unused with dense or cand_s)
     const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]: select in the kernel (fused decode)
     const int *cand_i;
-    const SegInfo *seg_info;
     const float *tail_scores;  // [B, G, nb_max] block scores of the segments' tails (fused decode)
     int n_cta;
     int *ids_out;              // nullable (fused decode)
