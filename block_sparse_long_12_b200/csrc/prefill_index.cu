@@ -112,7 +112,7 @@ __device__ inline float chunk_max_masked(const uint32_t (&r)[32], int j0, int po
     return m;
 }
 
-template <int K>
+template <int K, int BK>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_index_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                          const PrefillIdxArgs a) {
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // consumes the phases of one accumulator buffer in order (the piece-end barriers keep the
         // groups in step across pieces).  Blocks spanning two tiles go to group 0 alone: a group
         // skipping tiles of its own buffer could otherwise wait on a phase two steps ahead.
-        const bool two_groups = a.Bk <= kKeys;
+        constexpr bool two_groups = BK <= kKeys;
         SmemTopK<K> top{list_s, list_i, e * 32 + lane};
         int ti = 0;
         bool ok = true;
@@ -287,14 +287,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int j0 = kb + 32 * c;
-                    bm = fmaxf(bm, cm[c]);
-                    if (((j0 + 32) & (a.Bk - 1)) == 0) {  // last chunk of block j0 / Bk
-                        const int blk = j0 / a.Bk;
-                        if (blk * a.Bk <= pos) top.insert(bm, blk);
+                // block maxima (BK is a compile-time block size: the block ends fold away); only the
+                // diagonal tiles can hold blocks that start after the row
+                if constexpr (BK >= kKeys) {
+                    bm = fmaxf(bm, tc::fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])));
+                    if ((n + 1) % (BK / kKeys) == 0) {  // last tile of block n / (BK / kKeys)
+                        const int blk = n / (BK / kKeys);
+                        if (!diag || blk * BK <= pos) top.insert(bm, blk);
                         bm = -INFINITY;
+                    }
+                } else {
+                    constexpr int CPB = BK / 32;  // 32-column chunks per block
+#pragma unroll
+                    for (int q = 0; q < 4 / CPB; ++q) {
+                        float v = cm[q * CPB];
+#pragma unroll
+                        for (int c = 1; c < CPB; ++c) v = fmaxf(v, cm[q * CPB + c]);
+                        const int blk = n * (kKeys / BK) + q;
+                        if (!diag || blk * BK <= pos) top.insert(v, blk);
                     }
                 }
             }
@@ -364,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int K>
+template <int K, int BK>
 cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid,
                      cudaStream_t s) {
     const size_t smem = 1024 + kAccs * kABytes + PiShape<K>::S * kTileBytes + (size_t)K * kEpiThreads * 8 +
@@ -372,12 +382,23 @@ cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUten
     static bool attr = false;
     if (!attr) {
         cudaError_t e =
-            cudaFuncSetAttribute(prefill_index_kernel<K>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            cudaFuncSetAttribute(prefill_index_kernel<K, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    prefill_index_kernel<K><<<grid, kThreads, smem, s>>>(qm, km, a);
+    prefill_index_kernel<K, BK><<<grid, kThreads, smem, s>>>(qm, km, a);
     return cudaGetLastError();
+}
+
+template <int K>
+cudaError_t launch_kb(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid, cudaStream_t s) {
+    switch (a.Bk) {
+        case 32: return launch_k<K, 32>(a, qm, km, grid, s);
+        case 64: return launch_k<K, 64>(a, qm, km, grid, s);
+        case 128: return launch_k<K, 128>(a, qm, km, grid, s);
+        case 256: return launch_k<K, 256>(a, qm, km, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -402,9 +423,8 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
     }
     const int grid = n_sm;  // the plan's CTA count (at most one per SM)
     *why = "prefill index kernel launch";
-    if (a.k <= 8) return launch_k<8>(a, qm, km, grid, s);
-    if (a.k <= 16) return launch_k<16>(a, qm, km, grid, s);
-    return launch_k<32>(a, qm, km, grid, s);
+    return a.k <= 8 ? launch_kb<8>(a, qm, km, grid, s) : a.k <= 16 ? launch_kb<16>(a, qm, km, grid, s)
+                                                             : launch_kb<32>(a, qm, km, grid, s);
 }
 
 }  // namespace msa
