@@ -352,9 +352,12 @@ def run_ours(args, world, rank, local):
         del x
 
     lens_host = lens.tolist()
+    del inp, q, q_idx, k, v, k_idx, ws, wsd, o, od
+    torch.cuda.empty_cache()
+    shared = None if args.no_shared_index else run_shared_index(args, world, rank, local, stream, flush)
     prefill = None
     if not args.no_prefill:
-        del inp, q, q_idx, k, v, k_idx, ws, wsd, o, od, flush_buf
+        del flush_buf
         torch.cuda.empty_cache()
         prefill = run_prefill(world, rank, local, stream)
 
@@ -386,11 +389,65 @@ def run_ours(args, world, rank, local):
         "dense_gqa_us": round(dense_us, 2), "sparse_vs_dense_speedup": round(dense_us / step_us, 2),
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
+        "shared_index_head": shared,
         "prefill": prefill,
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
+
+
+def run_shared_index(args, world, rank, local, stream, flush):
+    """The 1M decode step with one index-K head shared by the 8 groups: the index stream is 1/8
+    as long, so the step is no longer dominated by the scan.  Same timing as the main step."""
+    from block_sparse_long_12_b200 import _lib, api
+    w = WORKLOADS["decode_ctx1m_shared_idx"]
+    dev = torch.device("cuda", local)
+    inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
+    q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
+    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
+    ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, dev)
+    o = torch.empty_like(q)
+    ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
+
+    def step():
+        _lib.msa_decode_fused(p, q, q_idx, k, v, k_idx, o, ids, None, ws, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 500))
+    barrier(world)
+    step_us = max_over_ranks(statistics.mean(timed_steps(step, n, flush, stream)), world)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    for e in evs:
+        e.record(stream)
+    torch.cuda.synchronize()
+    _lib.msa_set_stage_events(evs)
+    stage = [[], []]
+    try:
+        for _ in range(n):
+            flush()
+            step()
+            torch.cuda.synchronize()
+            for i in range(2):
+                stage[i].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
+    finally:
+        _lib.msa_set_stage_events(None)
+    assert _lib.msa_get_device_status(ws) == 0
+    scan_us = max_over_ranks(statistics.mean(stage[0]), world)
+    attn_us = max_over_ranks(statistics.mean(stage[1]), world)
+    peaks, kind = measured_peaks()
+    idx_bytes = sum(lens.tolist()) * w.n_idx_k_heads * w.idx_dim * 2
+    kv_bytes = w.batch * w.n_kv_heads * w.top_k * w.block_size * w.head_dim * 2 * 2
+    del inp, q, q_idx, k, v, k_idx, ws, o
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "value": round(step_us, 2), "unit": UNIT, "n_idx_k_heads": w.n_idx_k_heads,
+            "stages_us": {"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)},
+            "algorithmic_bytes": idx_bytes + kv_bytes,
+            "step_roofline_frac": round((idx_bytes + kv_bytes) / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "scan_gbs": round(idx_bytes / (scan_us * 1e-6) / 1e9, 1), "peak_kind": kind}
 
 
 def run_prefill(world, rank, local, stream):
@@ -477,6 +534,7 @@ def main():
                                                                     "decode_b8_ctx128k_ragged"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-shared-index", action="store_true", help="skip the shared index-K head decode step")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -106,18 +106,24 @@ struct ChunkCursor {
 // on one stream (GPS > 1) read it from shared memory and use 8 warps.
 template <int GPS> struct ScanShape {
     static constexpr int W = GPS == 1 ? 12 : 8;
-    static constexpr int S = 2;
 };
+// several groups on one bf16 stream of 128- or 256-byte rows are scored on tensor cores
+template <typename T, int GPS, int ROWB> constexpr bool scan_mma() { return GPS > 1 && sizeof(T) == 2 && ROWB >= 128; }
 
-template <typename T, int GPS, int ROWB>
+// S: ring stages per warp (2; 3 when tensor-core scoring leaves the room and the batch allows)
+template <typename T, int GPS, int ROWB, int S>
 __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     decode_scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
-    constexpr int W = ScanShape<GPS>::W, S = ScanShape<GPS>::S;
+    constexpr int W = ScanShape<GPS>::W;
     constexpr int ES = (int)sizeof(T);
     constexpr int EPV = Vec16<T>::N;      // elements per 16-byte vector
     constexpr int NCH = ROWB / 16;        // 16-byte vectors per index-key row
     constexpr int DI = ROWB / ES;         // index dim
     constexpr bool QREG = GPS == 1 && DI <= 64;
+    // several groups on one bf16 stream: the scores of a chunk are a small GEMM (the groups' index
+    // queries, padded to 16 rows, times the chunk's keys) on mma.sync tensor-core fragments
+    constexpr bool MMA = scan_mma<T, GPS, ROWB>();
+    constexpr int KS = DI / 16;           // k-steps of 16 index dims
     const int CT = a.chunk_tokens;        // tokens per chunk (<= block size, 8 KB at most)
 
     extern __shared__ unsigned char smem_raw[];
@@ -128,7 +134,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     float *q_s = reinterpret_cast<float *>(lists_i + W * GPS * 32);           // [GPS][DI] (QREG: unused)
     int4 *trec = reinterpret_cast<int4 *>(q_s + GPS * DI);                    // [W][4] tail blocks in flight
     float *q_w = reinterpret_cast<float *>(trec + W * 4);                     // [W][GPS][DI] (QREG: unused)
-    long long *off = reinterpret_cast<long long *>(q_w + (QREG ? 0 : W * GPS * DI));  // [B+1] ranges' prefix
+    long long *off = reinterpret_cast<long long *>(q_w + (QREG || MMA ? 0 : W * GPS * DI));  // [B+1] ranges' prefix
     long long *offt = off + a.B + 1;                                          // [B+1] tail pool prefix
     int *nbs = reinterpret_cast<int *>(offt + a.B + 1);                       // [B] blocks
     int *lens = nbs + a.B;                                                    // [B] clamped lengths
@@ -218,10 +224,62 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     };
     for (int st = 0; st < S && prod.valid; ++st) issue(st);
 
+    // A fragments of the groups' index queries (rows = the GPS groups of the stream, zero rows up to
+    // 16; columns = index dims), loaded when the warp moves to another stream
+    uint32_t qa[MMA ? KS : 1][4];
+    auto load_qa = [&](int b, int hik) {
+        if constexpr (MMA) {
+            const int grp = lane >> 2, tig = lane & 3;
+            const uint16_t *src = reinterpret_cast<const uint16_t *>(a.q_idx) +
+                                  ((size_t)b * a.G + hik + (size_t)Hik * (grp < GPS ? grp : 0)) * DI;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                const int c0 = ks * 16 + tig * 2;
+                qa[ks][0] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0) : 0u;
+                qa[ks][1] = 0u;
+                qa[ks][2] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0 + 8) : 0u;
+                qa[ks][3] = 0u;
+            }
+        }
+    };
+
     // one chunk of nt index-key rows of segment (b, hik) starting at token tok_base: fp32 dot
-    // products with the index query (qv in registers, or qsrc in shared memory), running max m
+    // products with the index query (qv in registers, or qsrc in shared memory, or the qa
+    // fragments on tensor cores), running max m
     auto scan_chunk = [&](const unsigned char *base, int nt, int b, int hik, int tok_base, const float *qv_,
                           const float *qsrc, float *m) {
+        if constexpr (MMA) {
+            // S = Q_idx K^T for 8 keys at a time; lane (grp, tig) holds S[grp][2 tig, 2 tig + 1]
+            const uint32_t tile = smem_u32(base);
+            const int grp = lane >> 2, tig = lane & 3, mi = lane >> 3;
+            float cmax = -INFINITY;
+            for (int kn = 0; kn * 8 < nt; ++kn) {
+                float sv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < KS; ks += 2) {
+                    const int key = kn * 8 + (lane & 7);
+                    const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(tile + (d0 >> 6) * (CT * 128) + sw128(key, (d0 & 63) >> 3), b0, b1, b2, b3);
+                    mma_16816(sv, qa[ks], b0, b1);
+                    mma_16816(sv, qa[ks + 1], b2, b3);
+                }
+                const int k0 = kn * 8 + tig * 2;
+                const float s0 = (k0 < nt && !failed) ? sv[0] : -INFINITY;
+                const float s1 = (k0 + 1 < nt && !failed) ? sv[1] : -INFINITY;
+                cmax = tc::fmax3(cmax, s0, s1);
+                if (a.token_scores != nullptr && grp < GPS && !failed) {
+                    float *ts = a.token_scores + ((size_t)b * a.G + hik + Hik * grp) * a.L_max + tok_base;
+                    if (k0 < nt) ts[k0] = s0;
+                    if (k0 + 1 < nt) ts[k0 + 1] = s1;
+                }
+            }
+            cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
+            cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], gl == grp ? cmax : -INFINITY);
+            return;
+        }
         for (int t0 = 0; t0 < nt; t0 += 32) {
             const int tok = t0 + lane;  // one index-key row per lane
             const bool live = tok < nt && !failed;
@@ -279,6 +337,8 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 const T *src = qg + ((size_t)p.b * a.G + p.hik) * DI;
 #pragma unroll
                 for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
+            } else if constexpr (MMA) {
+                load_qa(p.b, p.hik);
             } else {
                 __syncthreads();  // every warp is done with the previous segment's query
                 for (int i = tid; i < GPS * DI; i += blockDim.x) {
@@ -414,7 +474,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 if (++pc == pr.w) have = false;
             }
         };
-        float *my_q = q_w + (QREG ? 0 : w * GPS * DI);
+        float *my_q = q_w + (QREG || MMA ? 0 : w * GPS * DI);
         int qb = -1, qh = -1;
         t_issue();
         while (t_head < t_tail) {
@@ -426,6 +486,8 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                     const T *src = qg + ((size_t)qb * a.G + qh) * DI;
 #pragma unroll
                     for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
+                } else if constexpr (MMA) {
+                    load_qa(qb, qh);
                 } else {
                     __syncwarp();
                     for (int i = lane; i < GPS * DI; i += 32) {
@@ -483,17 +545,24 @@ __global__ void fill_neg_inf_kernel(const FillArgs a) {
         a.scores[i] = -INFINITY;
 }
 
-template <typename T, int GPS, int ROWB>
-cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
-    constexpr int W = ScanShape<GPS>::W, S = ScanShape<GPS>::S;
+template <typename T, int GPS, int ROWB, int S>
+size_t scan_smem_bytes(int B) {
+    constexpr bool MMA = scan_mma<T, GPS, ROWB>();
+    constexpr int W = ScanShape<GPS>::W;
     constexpr int DI = ROWB / (int)sizeof(T);
     constexpr bool QREG = GPS == 1 && DI <= 64;
-    const size_t smem = 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 +
-                        (size_t)GPS * DI * 4 + (size_t)W * 4 * 16 + (QREG ? 0 : (size_t)W * GPS * DI * 4) +
-                        (size_t)(a.B + 1) * 16 + (size_t)a.B * 12 + kTailPools * 4 + 64;
+    return 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 + (size_t)GPS * DI * 4 +
+           (size_t)W * 4 * 16 + (QREG || MMA ? 0 : (size_t)W * GPS * DI * 4) + (size_t)(B + 1) * 16 + (size_t)B * 12 +
+           kTailPools * 4 + 64;
+}
+
+template <typename T, int GPS, int ROWB, int S>
+cudaError_t launch_scan_s(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
+    constexpr int W = ScanShape<GPS>::W;
+    const size_t smem = scan_smem_bytes<T, GPS, ROWB, S>(a.B);
     static size_t attr_bytes = 0;  // opt-in raised on demand (smem grows with the batch)
     if (smem > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB>,
+        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB, S>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_bytes = smem;
@@ -508,7 +577,15 @@ cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, ROWB>, km, a);
+    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, ROWB, S>, km, a);
+}
+
+template <typename T, int GPS, int ROWB>
+cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
+    if constexpr (scan_mma<T, GPS, ROWB>()) {
+        if (scan_smem_bytes<T, GPS, ROWB, 3>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 3>(a, km, s, pdl);
+    }
+    return launch_scan_s<T, GPS, ROWB, 2>(a, km, s, pdl);
 }
 
 template <typename T, int ROWB>

@@ -62,8 +62,9 @@ class Workload:
         return replace(self, **kw)
 
 
-# The five workloads: tiny fp32 decode, 16K causal prefill, ragged batched
-# 128K decode, 1M decode (batch 1 and 4), 1M chunked causal prefill.
+# The workloads: tiny fp32 decode, 16K causal prefill, ragged batched 128K
+# decode, 1M decode (batch 1 and 4), 1M chunked causal prefill, and 1M decode
+# with one index-K head shared by every group.
 WORKLOADS = {
     "decode_fp32_ctx4k": Workload("decode_fp32_ctx4k", "decode", 1, 4096, 4, 1, 1, 64, 32, 64, 8,
                                   "f32", seed=1001),
@@ -77,6 +78,9 @@ WORKLOADS = {
                                 hot_blocks=32, seed=1004),
     "prefill_causal_1m": Workload("prefill_causal_1m", "prefill", 1, 1048576, 64, 8, 8, 128, 64, 128, 16,
                                   "bf16", hot_blocks=32, chunk=8192, seed=1005),
+    # one index-K head shared by the 8 groups (the pages' literal reading): 1/8 of the index bytes
+    "decode_ctx1m_shared_idx": Workload("decode_ctx1m_shared_idx", "decode", 1, 1048576, 64, 8, 1, 128, 64, 128,
+                                        16, "bf16", hot_blocks=32, seed=1006),
 }
 
 

@@ -63,6 +63,11 @@ def test_tiny_fp32_decode_full():
     dict(idx_dim=128, dtype="bf16"),                                   # 256-byte index rows
     dict(idx_dim=32, dtype="bf16"),                                    # 64-byte index rows
     dict(batch=9, max_seq_len=700, min_seq_len=1, seed=5),             # many short sequences
+    # several groups on one index-K stream: tensor-core scores for bf16 rows of 128 / 256 bytes,
+    # CUDA-core dot products for fp32 and for 64-byte rows
+    dict(idx_dim=128, dtype="bf16", n_idx_k_heads=1),
+    dict(dtype="f32", idx_dim=32, head_dim=64, n_idx_k_heads=1),
+    dict(idx_dim=32, dtype="bf16", n_idx_k_heads=1),
 ], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()) or "base")
 def test_decode_fused_variants(case):
     w = small(**case)
@@ -84,10 +89,12 @@ def test_decode_exact_lengths_edges():
     assert idn[0, 0, :, 0].tolist() == [0] * 4 and (idn[0, 0, :, 1:] == -1).all()
 
 
-def test_index_scores_and_pool_topk():
-    """Stored token / block scores, then the stand-alone pool + TopK entry."""
+@pytest.mark.parametrize("hik", [4, 1], ids=["hik4", "hik1"])
+def test_index_scores_and_pool_topk(hik):
+    """Stored token / block scores, then the stand-alone pool + TopK entry (hik 1: the four groups
+    share one index-K stream and are scored together on tensor cores)."""
     api = _api()
-    w = small(dtype="bf16", hot_blocks=4)
+    w = small(dtype="bf16", hot_blocks=4, n_idx_k_heads=hik)
     inp = make_inputs(w, device="cuda")
     x = to_np(inp)
     p = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
@@ -228,7 +235,8 @@ def test_workspace_reused_across_shapes():
     assert _lib.msa_get_device_status(shared) == 0
 
 
-@pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m"])
+@pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m",
+                                  "decode_ctx1m_shared_idx"])
 def test_full_size_decode(name):
     """The benchmark workloads at full size, checked against the oracle on every (sequence, group)."""
     w = WORKLOADS[name]
