@@ -88,21 +88,6 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
 }
 
 
-// (score, block id) as one 64-bit key whose unsigned order is the selection
-// order (higher score first, then lower id): the score's bits made
-// order-preserving in the high word, the complemented id in the low word.
-__device__ inline unsigned long long sel_key(float s, int id) {
-    uint32_t u = __float_as_uint(s + 0.0f);  // -0 -> +0: equal scores compare by id
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    return ((unsigned long long)u << 32) | (uint32_t)~(uint32_t)id;
-}
-__device__ inline void sel_unkey(unsigned long long key, float &s, int &id) {
-    uint32_t u = (uint32_t)(key >> 32);
-    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
-    s = __uint_as_float(u);
-    id = (int)~(uint32_t)key;
-}
-
 // Descending bitonic sort of keys[0, P) (P a power of two) by the whole CTA.
 __device__ inline void block_sort_desc(unsigned long long *keys, int P) {
     for (int size = 2; size <= P; size <<= 1)

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     int *lens = nbs + a.B;                                                    // [B] clamped lengths
     int *nba = lens + a.B;                                                    // [B] blocks before the tail
     int *exh = nba + a.B;                                                     // [kTailPools] pool is empty
+    int *arrived = exh + kTailPools;                                          // warps done with their pieces
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int B = a.B, Hik = a.Hik, Bk = a.Bk, C = a.n_cta;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
         nba[b] = nbs[b] - scan_tail_blocks(nbs[b]);
     }
     if (tid < kTailPools) exh[tid] = 0;
+    if (tid == 0) *arrived = 0;
     if (tid < W * S) mbar_init(&bars[tid], 1);
     if (tid == 0) tc::prefetch_tmap(&kmap);
     fence_mbar_init();
@@ -204,25 +206,91 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     const bool want_cand = a.cand_s != nullptr;
     const uint32_t chunk_bytes = (uint32_t)CT * ROWB;
 
-    // producer cursor (lane 0 issues, every lane tracks it to stay uniform)
+    // The shared tail (the last quarter of every stream's blocks): every warp takes tail blocks,
+    // one at a time, until the pools are empty; a tail block leaves only its scores
+    // (block_scores).  The pools hold the tail positions i * kTailPools + pool of the tails
+    // concatenated over (b, index-K head); a warp turns to the next pool after each block.
+    const long long total_t = a.sched != nullptr ? offt[B] : 0;
+    int pool = (int)(((long long)blockIdx.x * W + w) % kTailPools);
+    auto grab = [&]() -> long long {
+        long long x = -1;
+        if (lane == 0) {
+            for (int t = 0; t < kTailPools && x < 0; ++t, pool = (pool + 1) % kTailPools) {
+                if (*reinterpret_cast<volatile int *>(&exh[pool])) continue;
+                const long long y = (long long)atomicAdd(&a.sched[pool], 1u) * kTailPools + pool;
+                if (y < total_t)
+                    x = y;
+                else
+                    *reinterpret_cast<volatile int *>(&exh[pool]) = 1;
+            }
+        }
+        return __shfl_sync(FULL, x, 0);
+    };
+    // tail position -> (b, index-K head, block, chunks)
+    auto locate = [&](long long x) -> int4 {
+        int lo = 0, hi = B - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (offt[mid] <= x) lo = mid; else hi = mid - 1;
+        }
+        const int nt = nbs[lo] - nba[lo];
+        const int r = (int)(x - offt[lo]);
+        const int hik = r / nt;
+        const int n = nba[lo] + (r - hik * nt);
+        int bt = lens[lo] - n * Bk;
+        bt = bt < Bk ? bt : Bk;
+        return make_int4(lo, hik, n, (bt + CT - 1) / CT);
+    };
+
+    // One producer per warp (lane 0 issues, every lane tracks it to stay uniform) keeps the
+    // warp's ring full: first the chunks of the warp's blocks of its CTA's range, then, with no
+    // gap, chunks of tail blocks, so that the copies of the first tail blocks are in flight
+    // while the range's last chunks are scored.
     ChunkCursor prod;
     prod.pw = PieceWalker{x0, x1};
     prod.w = w; prod.W = W; prod.Bk = Bk; prod.ct = CT;
     prod.start(off, nba, lens, B, Hik);
     bool failed = false;
-    int issued = 0;
-    auto issue = [&](int slot) {
-        if (lane == 0) {
-            const int row = (prod.p.b * Hik + prod.p.hik) * a.L_max + prod.n * Bk + prod.c * CT;
-            unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
-            mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
-            tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
-            if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
+    int issued = 0, consumed = 0;
+    int4 *my_rec = trec + w * 4;  // tail blocks with chunks issued, in order (at most S + 1 live)
+    int t_head = 0, t_tail = 0, pc = 0;
+    bool more = total_t > 0, have = false;
+    int4 pr = make_int4(0, 0, 0, 0);
+    auto refill = [&]() {
+        while (!failed && issued - consumed < S) {
+            int row;
+            if (prod.valid) {
+                row = (prod.p.b * Hik + prod.p.hik) * a.L_max + prod.n * Bk + prod.c * CT;
+                prod.advance(off, nba, lens, B, Hik);
+            } else {
+                if (!more) break;
+                if (!have) {
+                    const long long x = grab();
+                    if (x < 0) {
+                        more = false;
+                        break;
+                    }
+                    pr = locate(x);
+                    if (lane == 0) my_rec[t_tail & 3] = pr;
+                    __syncwarp();
+                    ++t_tail;
+                    have = true;
+                    pc = 0;
+                }
+                row = (pr.x * Hik + pr.y) * a.L_max + pr.z * Bk + pc * CT;
+                if (++pc == pr.w) have = false;
+            }
+            if (lane == 0) {
+                const int slot = issued % S;
+                unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
+                mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
+                tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
+                if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
+            }
+            ++issued;
         }
-        ++issued;
-        prod.advance(off, nba, lens, B, Hik);
     };
-    for (int st = 0; st < S && prod.valid; ++st) issue(st);
+    refill();
 
     // A fragments of the groups' index queries (rows = the GPS groups of the stream, zero rows up to
     // 16; columns = index dims), loaded when the warp moves to another stream
@@ -249,24 +317,33 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
     auto scan_chunk = [&](const unsigned char *base, int nt, int b, int hik, int tok_base, const float *qv_,
                           const float *qsrc, float *m) {
         if constexpr (MMA) {
-            // S = Q_idx K^T for 8 keys at a time; lane (grp, tig) holds S[grp][2 tig, 2 tig + 1]
+            // S = Q_idx K^T, 8 keys per tile; lane (grp, tig) holds S[grp][2 tig, 2 tig + 1] of each
+            // tile.  The k-steps run over all tiles in turn, so consecutive MMAs are independent.
+            constexpr int NTL = kScanChunkBytes / ROWB / 8;  // key tiles of a full chunk
             const uint32_t tile = smem_u32(base);
             const int grp = lane >> 2, tig = lane & 3, mi = lane >> 3;
-            float cmax = -INFINITY;
-            for (int kn = 0; kn * 8 < nt; ++kn) {
-                float sv[4] = {0.f, 0.f, 0.f, 0.f};
+            float sv[NTL][4];
 #pragma unroll
-                for (int ks = 0; ks < KS; ks += 2) {
-                    const int key = kn * 8 + (lane & 7);
-                    const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(tile + (d0 >> 6) * (CT * 128) + sw128(key, (d0 & 63) >> 3), b0, b1, b2, b3);
-                    mma_16816(sv, qa[ks], b0, b1);
-                    mma_16816(sv, qa[ks + 1], b2, b3);
+            for (int kn = 0; kn < NTL; ++kn) sv[kn][0] = sv[kn][1] = sv[kn][2] = sv[kn][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ks += 2) {
+                const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
+#pragma unroll
+                for (int kn = 0; kn < NTL; ++kn) {
+                    if (kn * 8 < nt) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(tile + (d0 >> 6) * (CT * 128) + sw128(kn * 8 + (lane & 7), (d0 & 63) >> 3), b0, b1, b2, b3);
+                        mma_16816(sv[kn], qa[ks], b0, b1);
+                        mma_16816(sv[kn], qa[ks + 1], b2, b3);
+                    }
                 }
+            }
+            float cmax = -INFINITY;
+#pragma unroll
+            for (int kn = 0; kn < NTL; ++kn) {
                 const int k0 = kn * 8 + tig * 2;
-                const float s0 = (k0 < nt && !failed) ? sv[0] : -INFINITY;
-                const float s1 = (k0 + 1 < nt && !failed) ? sv[1] : -INFINITY;
+                const float s0 = (k0 < nt && !failed) ? sv[kn][0] : -INFINITY;
+                const float s1 = (k0 + 1 < nt && !failed) ? sv[kn][1] : -INFINITY;
                 cmax = tc::fmax3(cmax, s0, s1);
                 if (a.token_scores != nullptr && grp < GPS && !failed) {
                     float *ts = a.token_scores + ((size_t)b * a.G + hik + Hik * grp) * a.L_max + tok_base;
@@ -274,60 +351,96 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                     if (k0 + 1 < nt) ts[k0 + 1] = s1;
                 }
             }
-            cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 1));
-            cmax = fmaxf(cmax, __shfl_xor_sync(FULL, cmax, 2));
+            // the 4 lanes of a group reduce at the block end
 #pragma unroll
             for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], gl == grp ? cmax : -INFINITY);
-            return;
-        }
-        for (int t0 = 0; t0 < nt; t0 += 32) {
-            const int tok = t0 + lane;  // one index-key row per lane
-            const bool live = tok < nt && !failed;
-            float dot[GPS];
+        } else {
+            for (int t0 = 0; t0 < nt; t0 += 32) {
+                const int tok = t0 + lane;  // one index-key row per lane
+                const bool live = tok < nt && !failed;
+                float dot[GPS];
 #pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
-            if (live) {
+                for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
+                if (live) {
 #pragma unroll
-                for (int c16 = 0; c16 < NCH; ++c16) {
-                    // position of 16-byte vector c16 of row `tok` in the swizzled tile
-                    int o;
-                    if constexpr (ROWB == 64) {
-                        o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
-                    } else {
-                        o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
-                    }
-                    const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
-                    float f[EPV];
-                    Vec16<T>::unpack(u, f);
-                    if constexpr (QREG) {
+                    for (int c16 = 0; c16 < NCH; ++c16) {
+                        // position of 16-byte vector c16 of row `tok` in the swizzled tile
+                        int o;
+                        if constexpr (ROWB == 64) {
+                            o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
+                        } else {
+                            o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
+                        }
+                        const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
+                        float f[EPV];
+                        Vec16<T>::unpack(u, f);
+                        if constexpr (QREG) {
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e) dot[0] = fmaf(qv_[c16 * EPV + e], f[e], dot[0]);
-                    } else {
+                            for (int e = 0; e < EPV; ++e) dot[0] = fmaf(qv_[c16 * EPV + e], f[e], dot[0]);
+                        } else {
 #pragma unroll
-                        for (int gl = 0; gl < GPS; ++gl) {
-                            const float *qq = qsrc + gl * DI + c16 * EPV;
+                            for (int gl = 0; gl < GPS; ++gl) {
+                                const float *qq = qsrc + gl * DI + c16 * EPV;
 #pragma unroll
-                            for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qq[e], f[e], dot[gl]);
+                                for (int e = 0; e < EPV; ++e) dot[gl] = fmaf(qq[e], f[e], dot[gl]);
+                            }
                         }
                     }
                 }
-            }
 #pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) {
-                const float sc = live ? dot[gl] : -INFINITY;
-                m[gl] = fmaxf(m[gl], sc);
-                if (a.token_scores != nullptr && live) {
-                    const int g = hik + Hik * gl;
-                    a.token_scores[((size_t)b * a.G + g) * a.L_max + tok_base + tok] = sc;
+                for (int gl = 0; gl < GPS; ++gl) {
+                    const float sc = live ? dot[gl] : -INFINITY;
+                    m[gl] = fmaxf(m[gl], sc);
+                    if (a.token_scores != nullptr && live) {
+                        const int g = hik + Hik * gl;
+                        a.token_scores[((size_t)b * a.G + g) * a.L_max + tok_base + tok] = sc;
+                    }
                 }
             }
         }
     };
 
-    int consumed = 0;
+    // every lane ends with the block's max of each group: a butterfly over the lanes, or, with
+    // tensor-core scores (lanes 4 g .. 4 g + 3 hold group g), a reduction over those 4 lanes
+    // and one broadcast per group
+    auto block_max = [&](float *m) {
+        if constexpr (MMA) {
+            float mine = -INFINITY;
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) mine = gl == (lane >> 2) ? m[gl] : mine;
+            mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 1));
+            mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 2));
+#pragma unroll
+            for (int gl = 0; gl < GPS; ++gl) m[gl] = __shfl_sync(FULL, mine, gl * 4);
+        } else {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], __shfl_xor_sync(FULL, m[gl], o));
+        }
+    };
+
     float qv[QREG ? DI : 1];
     int q_b = -1, q_h = -1;
     WarpTopK lst[GPS];
+    bool merged = false;
+    int def_seg = -1, def_piece = 0;  // the piece whose merge waits for the kernel's end
+    // group w's W lists pairwise, the pairs' results pairwise, ... (a tree of top-32 merges
+    // whose merges of one level are independent) into the candidates of piece `piece` of
+    // segment `seg`
+    auto merge_piece = [&](int seg, int piece) {
+        const int gl = GPS == 1 ? 0 : w;
+        unsigned long long key[W];
+#pragma unroll
+        for (int j = 0; j < W; ++j)
+            key[j] = sel_key(lists_s[(j * GPS + gl) * 32 + lane], lists_i[(j * GPS + gl) * 32 + lane]);
+#pragma unroll
+        for (int st = 1; st < W; st *= 2)
+#pragma unroll
+            for (int j = 0; j + st < W; j += 2 * st) key[j] = warp_merge_top32(key[j], key[j + st], lane);
+        const size_t o = (((size_t)seg * C + piece) * GPS + gl) * a.k;
+        if (lane < a.k) sel_unkey(key[0], a.cand_s[o + lane], a.cand_i[o + lane]);
+    };
     PieceWalker pw{x0, x1};
     Piece p;
     while (pw.next(off, nba, B, Hik, p)) {
@@ -372,111 +485,57 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, p.b, p.hik, n * Bk + c * CT, qv, q_s, m);
                 __syncwarp();
                 ++consumed;
-                if (prod.valid && !failed) issue(slot);
+                refill();
             }
+            block_max(m);
+            if (a.block_scores != nullptr && lane == 0)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], __shfl_xor_sync(FULL, m[gl], o));
-#pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) {
-                if (a.block_scores != nullptr && lane == 0) {
-                    const int g = p.hik + Hik * gl;
-                    a.block_scores[((size_t)p.b * a.G + g) * a.nb_max + n] = m[gl];
-                }
-                if (want_cand) lst[gl].insert(m[gl], n, a.k, lane);
-            }
+                for (int gl = 0; gl < GPS; ++gl)
+                    a.block_scores[((size_t)p.b * a.G + p.hik + Hik * gl) * a.nb_max + n] = m[gl];
+            if (want_cand) warp_topk_insert_all<GPS>(lst, m, n, a.k, lane);
         }
         if (want_cand) {
-            // merge the warps' sorted lists into this piece's candidates
+            // The warps' sorted lists of this piece merge into its candidates.  One group: the
+            // warp that finishes last merges them, and no warp waits for another.  Several
+            // groups: one warp per group, after every warp is done; for the CTA's last piece
+            // that is at the kernel's end, so that no warp waits before it goes on to the tail.
+            if (merged) __syncthreads();  // the previous piece's merge has read the lists
 #pragma unroll
             for (int gl = 0; gl < GPS; ++gl) {
                 lists_s[(w * GPS + gl) * 32 + lane] = lst[gl].s;
                 lists_i[(w * GPS + gl) * 32 + lane] = lst[gl].id;
             }
-            __syncthreads();
-            if (w < GPS) {
-                const int gl = w;
-                const int seg = p.b * Hik + p.hik;
-                const int piece = blockIdx.x - cta_of(p.seg_start, per);
-                const size_t o = (((size_t)seg * C + piece) * GPS + gl) * a.k;
-                warp_merge_sorted_lists<1>(lists_s + gl * 32, lists_i + gl * 32, W, a.k, GPS * 32, a.k,
-                                           a.cand_s + o, a.cand_i + o, lane);
+            const int seg = p.b * Hik + p.hik;
+            const int piece = blockIdx.x - cta_of(p.seg_start, per);
+            if constexpr (GPS == 1) {
+                __syncwarp();
+                int ticket = 0;
+                if (lane == 0) {
+                    __threadfence_block();  // this warp's list before its arrival
+                    ticket = atomicAdd(arrived, 1);
+                }
+                ticket = __shfl_sync(FULL, ticket, 0);
+                if (ticket % W == W - 1) {
+                    __threadfence_block();  // every warp's list after their arrivals
+                    merge_piece(seg, piece);
+                }
+                merged = true;
+            } else if (pw.x >= pw.x1) {
+                def_seg = seg;
+                def_piece = piece;
+            } else {
+                __syncthreads();
+                if (w < GPS) merge_piece(seg, piece);
+                merged = true;
             }
-            __syncthreads();
         }
     }
 
     // ------------------------------------------------ the shared tail, one block at a time
-    // Every warp takes tail blocks until the pools are empty; a block leaves only its scores
-    // (block_scores).  The pools hold the tail positions i * kTailPools + pool of the tails
-    // concatenated over (b, index-K head); a warp turns to the next pool after each block.
-    const long long total_t = offt[B];
-    if (a.sched != nullptr && total_t > 0) {
-        int pool = (int)(((long long)blockIdx.x * W + w) % kTailPools);
-        auto grab = [&]() -> long long {
-            long long x = -1;
-            if (lane == 0) {
-                for (int t = 0; t < kTailPools && x < 0; ++t, pool = (pool + 1) % kTailPools) {
-                    if (*reinterpret_cast<volatile int *>(&exh[pool])) continue;
-                    const long long y = (long long)atomicAdd(&a.sched[pool], 1u) * kTailPools + pool;
-                    if (y < total_t)
-                        x = y;
-                    else
-                        *reinterpret_cast<volatile int *>(&exh[pool]) = 1;
-                }
-            }
-            return __shfl_sync(FULL, x, 0);
-        };
-        // tail position -> (b, index-K head, block, chunks)
-        auto locate = [&](long long x) -> int4 {
-            int lo = 0, hi = B - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (offt[mid] <= x) lo = mid; else hi = mid - 1;
-            }
-            const int nt = nbs[lo] - nba[lo];
-            const int r = (int)(x - offt[lo]);
-            const int hik = r / nt;
-            const int n = nba[lo] + (r - hik * nt);
-            int bt = lens[lo] - n * Bk;
-            bt = bt < Bk ? bt : Bk;
-            return make_int4(lo, hik, n, (bt + CT - 1) / CT);
-        };
-        int4 *my_rec = trec + w * 4;  // blocks with chunks issued, in order (at most S + 1 live)
-        int t_head = 0, t_tail = 0, pc = 0;
-        bool more = !failed, have = false;
-        int4 pr = make_int4(0, 0, 0, 0);
-        auto t_issue = [&]() {
-            while (more && !failed && issued - consumed < S) {
-                if (!have) {
-                    const long long x = grab();
-                    if (x < 0) {
-                        more = false;
-                        break;
-                    }
-                    pr = locate(x);
-                    if (lane == 0) my_rec[t_tail & 3] = pr;
-                    __syncwarp();
-                    ++t_tail;
-                    have = true;
-                    pc = 0;
-                }
-                if (lane == 0) {
-                    const int slot = issued % S;
-                    const int row = (pr.x * Hik + pr.y) * a.L_max + pr.z * Bk + pc * CT;
-                    unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
-                    mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
-                    tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
-                    if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
-                }
-                ++issued;
-                if (++pc == pr.w) have = false;
-            }
-        };
+    {
         float *my_q = q_w + (QREG || MMA ? 0 : w * GPS * DI);
         int qb = -1, qh = -1;
-        t_issue();
+        refill();
         while (t_head < t_tail) {
             const int4 r = my_rec[t_head & 3];
             if (r.x != qb || r.y != qh) {
@@ -513,23 +572,21 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, r.x, r.y, r.z * Bk + c * CT, qv, my_q, m);
                 __syncwarp();
                 ++consumed;
-                t_issue();
+                refill();
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-                for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], __shfl_xor_sync(FULL, m[gl], o));
+            block_max(m);
             if (a.block_scores != nullptr && lane == 0)
 #pragma unroll
                 for (int gl = 0; gl < GPS; ++gl)
                     a.block_scores[((size_t)r.x * a.G + r.y + Hik * gl) * a.nb_max + r.z] = m[gl];
             ++t_head;
-            t_issue();
+            refill();
         }
     }
 
-    // the CTA that finishes last returns the pool counters to zero for the next call
     __syncthreads();
+    if (def_seg >= 0 && w < GPS) merge_piece(def_seg, def_piece);
+    // the CTA that finishes last returns the pool counters to zero for the next call
     if (a.sched != nullptr && tid == 0) {
         __threadfence();
         if (atomicAdd(&a.sched[kTailPools], 1u) == gridDim.x - 1) {
@@ -553,7 +610,7 @@ size_t scan_smem_bytes(int B) {
     constexpr bool QREG = GPS == 1 && DI <= 64;
     return 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 + (size_t)GPS * DI * 4 +
            (size_t)W * 4 * 16 + (QREG || MMA ? 0 : (size_t)W * GPS * DI * 4) + (size_t)(B + 1) * 16 + (size_t)B * 12 +
-           kTailPools * 4 + 64;
+           kTailPools * 4 + 4 + 64;
 }
 
 template <typename T, int GPS, int ROWB, int S>

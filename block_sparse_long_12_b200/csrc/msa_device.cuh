@@ -144,6 +144,66 @@ struct WarpTopK {
     }
 };
 
+// insert(cs[g], ci, ...) into l[g] for every g, the N lists in lockstep: one candidate id
+// with N scores (the block's max for each of N groups), so that the shuffles of different
+// lists are independent instructions.  cs/ci must be warp-uniform.
+template <int N>
+__device__ inline void warp_topk_insert_all(WarpTopK (&l)[N], const float (&cs)[N], int ci, int k, int lane) {
+    bool any = false;
+#pragma unroll
+    for (int g = 0; g < N; ++g) any |= better(cs[g], ci, l[g].thr_s, l[g].thr_i);
+    if (!any) return;
+    unsigned m[N];
+    float us[N];
+    int ui[N];
+#pragma unroll
+    for (int g = 0; g < N; ++g) {
+        m[g] = __ballot_sync(FULL, lane < k && better(cs[g], ci, l[g].s, l[g].id));
+        us[g] = __shfl_up_sync(FULL, l[g].s, 1);
+        ui[g] = __shfl_up_sync(FULL, l[g].id, 1);
+    }
+#pragma unroll
+    for (int g = 0; g < N; ++g) {
+        const int p = m[g] != 0 ? __ffs(m[g]) - 1 : 32;
+        if (lane == p) { l[g].s = cs[g]; l[g].id = ci; }
+        else if (lane > p && lane < k) { l[g].s = us[g]; l[g].id = ui[g]; }
+    }
+#pragma unroll
+    for (int g = 0; g < N; ++g) {
+        l[g].thr_s = __shfl_sync(FULL, l[g].s, k - 1);
+        l[g].thr_i = __shfl_sync(FULL, l[g].id, k - 1);
+    }
+}
+
+// (score, block id) as one 64-bit key whose unsigned order is the selection
+// order (higher score first, then lower id): the score's bits made
+// order-preserving in the high word, the complemented id in the low word.
+__device__ inline unsigned long long sel_key(float s, int id) {
+    uint32_t u = __float_as_uint(s + 0.0f);  // -0 -> +0: equal scores compare by id
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)u << 32) | (uint32_t)~(uint32_t)id;
+}
+__device__ inline void sel_unkey(unsigned long long key, float &s, int &id) {
+    uint32_t u = (uint32_t)(key >> 32);
+    u = (u & 0x80000000u) ? (u & 0x7fffffffu) : ~u;
+    s = __uint_as_float(u);
+    id = (int)~(uint32_t)key;
+}
+
+// The 32 best of two lists of distinct keys, each held descending one key per lane: the
+// elementwise max of one list and the other reversed is a bitonic sequence holding the 32
+// largest keys, which five half-cleaner steps sort descending.
+__device__ inline unsigned long long warp_merge_top32(unsigned long long a, unsigned long long b, int lane) {
+    const unsigned long long br = __shfl_sync(FULL, b, 31 - lane);
+    unsigned long long c = a > br ? a : br;
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) {
+        const unsigned long long o = __shfl_xor_sync(FULL, c, d);
+        c = (lane & d) ? (c < o ? c : o) : (c > o ? c : o);
+    }
+    return c;
+}
+
 // Warp argmax of (s, i) under `better`; every lane receives the winner.
 __device__ inline void warp_best(float &s, int &i) {
 #pragma unroll

@@ -3,6 +3,7 @@
   python -m block_sparse_long_12_b200.profile_run decode --context 262144 --steps 3
   python -m block_sparse_long_12_b200.profile_run prefill_index --context 65536 --chunk 8192 --steps 1
   python -m block_sparse_long_12_b200.profile_run prefill_attn --context 65536 --chunk 8192 --steps 1
+  python -m block_sparse_long_12_b200.profile_run scan_shared --context 1048576 --steps 3
 
 Inputs are the seeded synthetic workloads of ``inputs`` at the requested
 size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
@@ -72,15 +73,31 @@ def run_prefill_attn(args):
     print("prefill attention done", int(_lib.msa_get_device_status(ws_a)))
 
 
+def run_scan_shared(args):
+    """The index scan of one index-K head shared by the 8 groups (stored block scores, so that only
+    the index keys are on the device)."""
+    w = WORKLOADS["decode_ctx1m_shared_idx"].scaled(max_seq_len=args.context, batch=args.batch)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(w.seed)
+    q_idx = torch.randn(w.batch, 1, w.n_kv_heads, w.idx_dim, generator=gen, device="cuda").to(torch.bfloat16)
+    k_idx = torch.randn(w.batch, 1, w.max_seq_len, w.idx_dim, generator=gen, device="cuda").to(torch.bfloat16)
+    lens = torch.full((w.batch,), w.max_seq_len, dtype=torch.int32, device="cuda")
+    for _ in range(args.steps):
+        out = api.index_scores(q_idx, k_idx, lens, n_kv_heads=w.n_kv_heads, block_size=w.block_size, mode="block")
+    torch.cuda.synchronize()
+    print("scan done", float(out[0, 0, 0, :4].sum()))
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn"])
+    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "scan_shared"])
     ap.add_argument("--context", type=int, default=262144)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=8192)
     ap.add_argument("--steps", type=int, default=3)
     args = ap.parse_args()
-    {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn}[args.what](args)
+    {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn,
+     "scan_shared": run_scan_shared}[args.what](args)
 
 
 if __name__ == "__main__":
