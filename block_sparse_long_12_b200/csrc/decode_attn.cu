@@ -214,11 +214,29 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, const SegInfo
         const int n = base0 + u * 32 + lane;
         v0[u] = n < nb ? tsc[n] : -INFINITY;
     }
+    // the pieces' lists into shared memory, kLists loads in flight per thread and array
+    constexpr int kLists = 8;
     const int k = a.k, np = info.n_pieces, n = np * k;
-    for (int i = tid; i < n; i += nthr) {
-        const size_t src = (((size_t)seg * a.n_cta + i / k) * gps + gl) * k + i % k;
-        ls[i] = a.cand_s[src];
-        li[i] = a.cand_i[src];
+    for (int i0 = tid; i0 < n; i0 += nthr * kLists) {
+        float sv[kLists];
+        int iv[kLists];
+#pragma unroll
+        for (int u = 0; u < kLists; ++u) {
+            const int i = i0 + u * nthr;
+            if (i < n) {
+                const size_t src = (((size_t)seg * a.n_cta + i / k) * gps + gl) * k + i % k;
+                sv[u] = a.cand_s[src];
+                iv[u] = a.cand_i[src];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kLists; ++u) {
+            const int i = i0 + u * nthr;
+            if (i < n) {
+                ls[i] = sv[u];
+                li[i] = iv[u];
+            }
+        }
     }
     if (tid == 0) {
         st[0] = 0;
