@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT = range(6)
 MSA_F32, MSA_BF16 = 0, 1
-MSA_SCORES_TOKEN, MSA_SCORES_BLOCKMAX, MSA_DENSE = 1, 2, 8
+MSA_SCORES_TOKEN, MSA_SCORES_BLOCKMAX, MSA_DENSE, MSA_FORCE_SINK_LOCAL = 1, 2, 8, 16
 (MSA_ENTRY_INDEX_SCORE, MSA_ENTRY_MAXPOOL_TOPK, MSA_ENTRY_ATTN_DECODE, MSA_ENTRY_ATTN_PREFILL,
  MSA_ENTRY_DECODE_FUSED, MSA_ENTRY_PREFILL_INDEX_TOPK) = range(6)
 

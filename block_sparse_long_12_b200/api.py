@@ -13,7 +13,7 @@ import torch
 from . import _lib
 from ._lib import (MSA_BF16, MSA_DENSE, MSA_ENTRY_ATTN_DECODE, MSA_ENTRY_ATTN_PREFILL, MSA_ENTRY_DECODE_FUSED,
                    MSA_ENTRY_INDEX_SCORE, MSA_ENTRY_MAXPOOL_TOPK, MSA_ENTRY_PREFILL_INDEX_TOPK, MSA_F32,
-                   MSA_SCORES_BLOCKMAX, MSA_SCORES_TOKEN, Params)
+                   MSA_FORCE_SINK_LOCAL, MSA_SCORES_BLOCKMAX, MSA_SCORES_TOKEN, Params)
 
 
 def dtype_code(t: torch.Tensor) -> int:
@@ -51,10 +51,11 @@ def workspace(params, entry: int, device) -> torch.Tensor:
 
 
 def decode(q, q_idx, k, v, k_idx, seq_lens, *, block_size, top_k, softmax_scale=None, ws=None, out=None,
-           stream=None):
-    """One fused MSA decode step.  Returns (o [B,1,Hq,D], ids [B,1,G,k], lse [B,1,Hq])."""
+           stream=None, force_sink_local=False):
+    """One fused MSA decode step.  Returns (o [B,1,Hq,D], ids [B,1,G,k], lse [B,1,Hq]).
+    force_sink_local: the selection always keeps block 0 and the query's own block."""
     p = params_from(q, q_idx, k, k_idx, block_size=block_size, top_k=top_k, seq_lens=seq_lens,
-                    softmax_scale=softmax_scale)
+                    softmax_scale=softmax_scale, flags=MSA_FORCE_SINK_LOCAL if force_sink_local else 0)
     B, _, Hq, D = q.shape
     G = k.shape[1]
     if ws is None:
@@ -98,12 +99,14 @@ def index_scores(q_idx, k_idx, seq_lens, *, n_kv_heads, block_size, top_k=1, mod
     return out
 
 
-def pool_topk(scores, seq_lens, *, block_size, top_k, max_seq_len, is_block, q_start=0, stream=None):
+def pool_topk(scores, seq_lens, *, block_size, top_k, max_seq_len, is_block, q_start=0, stream=None,
+              force_sink_local=False):
     """Block max pool + TopK of stored scores [B, Tq, G, n].  Returns (ids, top_scores)."""
     B, Tq, G, _ = scores.shape
     p = make_params(batch=B, n_q_heads=G, n_kv_heads=G, n_idx_k_heads=G, head_dim=64, idx_dim=32,
                     block_size=block_size, top_k=top_k, max_seq_len=max_seq_len, dtype=MSA_F32, q_len=Tq,
-                    q_start=q_start, seq_lens=seq_lens, flags=MSA_SCORES_BLOCKMAX if is_block else 0)
+                    q_start=q_start, seq_lens=seq_lens,
+                    flags=(MSA_SCORES_BLOCKMAX if is_block else 0) | (MSA_FORCE_SINK_LOCAL if force_sink_local else 0))
     ids = torch.empty(B, Tq, G, top_k, dtype=torch.int32, device=scores.device)
     ts = torch.empty(B, Tq, G, top_k, dtype=torch.float32, device=scores.device)
     ws = workspace(p, MSA_ENTRY_MAXPOOL_TOPK, scores.device)

@@ -498,11 +498,45 @@ __device__ inline bool last_split(const AttnArgs &a, int b, int g, int *flag) {
 }
 
 // Obtain the group's list: fused selection from the scan, or a given ids tensor.
+// MSA_FORCE_SINK_LOCAL applied to a finished selection: block 0 and the sequence's last block
+// first (by id, score +inf), then the list's other blocks in their order.  The list holds the k
+// best of all blocks, so its other blocks, in order, are the best of the others.  Called by
+// every thread of the CTA; sel_s / sel_i stay padded with (-inf, -1).
+__device__ inline void force_sink_local(const AttnArgs &a, int b, float *sel_s, int *sel_i) {
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int nb = (L + a.Bk - 1) / a.Bk, nf = nb < 2 ? nb : 2, k = a.k;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const float s = sel_s[lane];
+        const int id = sel_i[lane];
+        const bool keep = lane < k && id >= 0 && id != 0 && id != nb - 1;
+        const unsigned m = __ballot_sync(FULL, keep);
+        const int dst = nf + __popc(m & ((1u << lane) - 1u));
+        const int n_keep = __popc(m);
+        __syncwarp();
+        if (keep && dst < k) {
+            sel_s[dst] = s;
+            sel_i[dst] = id;
+        }
+        if (lane < nf && lane < k) {
+            sel_s[lane] = INFINITY;
+            sel_i[lane] = lane == 0 ? 0 : nb - 1;
+        }
+        if (lane >= nf + n_keep || lane >= k) {
+            sel_s[lane] = -INFINITY;
+            sel_i[lane] = -1;
+        }
+    }
+    __syncthreads();
+}
+
 __device__ inline void group_list(const AttnArgs &a, int b, int g, const SegInfo info, unsigned char *scratch,
                                   float *sel_s, int *sel_i) {
     if (a.dense) return;
     if (a.cand_s != nullptr) {
         select_group_topk(a, b, g, info, scratch, sel_s, sel_i);
+        if (a.force) force_sink_local(a, b, sel_s, sel_i);
         if (blockIdx.x == 0 && threadIdx.x < a.k) {
             const size_t o = ((size_t)b * a.G + g) * a.k + threadIdx.x;
             if (a.ids_out != nullptr) a.ids_out[o] = sel_i[threadIdx.x];

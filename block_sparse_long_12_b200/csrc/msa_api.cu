@@ -94,7 +94,7 @@ msa_status_t check_params(const msa_params_t *p, Mode mode) {
         return fail(MSA_ERR_UNSUPPORTED, "batch * n_kv_heads * max_seq_len must stay below 2^31 cache rows");
     if (!(p->softmax_scale > 0.f) || !std::isfinite(p->softmax_scale))
         return fail(MSA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
-    if (p->flags & ~(MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_DENSE))
+    if (p->flags & ~(MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_DENSE | MSA_FORCE_SINK_LOCAL))
         return fail(MSA_ERR_INVALID_ARG, "unknown flags 0x%x", p->flags);
     if (p->q_len < 1) return fail(MSA_ERR_INVALID_ARG, "q_len %d < 1", p->q_len);
     if (mode == DECODE_ONLY && p->q_len != 1) return fail(MSA_ERR_INVALID_ARG, "decode entries take q_len = 1");
@@ -315,7 +315,8 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
     const int mode = p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX);
     if (mode != MSA_SCORES_TOKEN && mode != MSA_SCORES_BLOCKMAX)
         return fail(MSA_ERR_INVALID_ARG, "exactly one of MSA_SCORES_TOKEN / MSA_SCORES_BLOCKMAX must be set");
-    if (p->flags & MSA_DENSE) return fail(MSA_ERR_INVALID_ARG, "MSA_DENSE does not apply to index scores");
+    if (p->flags & (MSA_DENSE | MSA_FORCE_SINK_LOCAL))
+        return fail(MSA_ERR_INVALID_ARG, "MSA_DENSE and MSA_FORCE_SINK_LOCAL do not apply to index scores");
     MSA_TRY(check_ptr(q_idx, "q_idx"));
     MSA_TRY(check_ptr(k_idx, "k_idx"));
     MSA_TRY(check_ptr(scores_out, "scores_out"));
@@ -348,7 +349,8 @@ msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_i
                                     float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
     MSA_TRY(check_params(p, ANY_ROWS));
     if (p->flags & (MSA_SCORES_TOKEN | MSA_DENSE))
-        return fail(MSA_ERR_INVALID_ARG, "only MSA_SCORES_BLOCKMAX may be set for msa_block_maxpool_topk");
+        return fail(MSA_ERR_INVALID_ARG,
+                    "only MSA_SCORES_BLOCKMAX and MSA_FORCE_SINK_LOCAL may be set for msa_block_maxpool_topk");
     MSA_TRY(check_ptr(scores_in, "scores_in"));
     MSA_TRY(check_ptr(ids_out, "ids_out"));
     MSA_TRY(check_ptr(top_scores_out, "top_scores_out", true));
@@ -361,6 +363,7 @@ msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_i
     a.B = p->batch; a.q_len = p->q_len; a.q_start = p->q_start; a.G = p->n_kv_heads; a.Bk = p->block_size;
     a.k = p->top_k; a.L_max = p->max_seq_len; a.nb_max = nb_max_of(*p);
     a.is_block = (p->flags & MSA_SCORES_BLOCKMAX) != 0;
+    a.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
     a.prefill = p->q_len > 1;
     cudaError_t e = launch_pool_topk(a, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "pool/topk launch");
@@ -387,6 +390,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
     a.B = p->batch; a.Hq = p->n_q_heads; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.D = p->head_dim;
     a.Bk = p->block_size; a.k = p->top_k; a.L_max = p->max_seq_len; a.r = p->n_q_heads / p->n_kv_heads;
     a.S = L.S; a.blocks_per_split = L.blocks_per_split; a.dense = (p->flags & MSA_DENSE) != 0;
+    a.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(wsb);
     cudaError_t e;
@@ -404,8 +408,8 @@ msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const 
                                     const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
                                     msa_stream_t stream) {
     MSA_TRY(check_params(p, DECODE_ONLY));
-    if (p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX))
-        return fail(MSA_ERR_INVALID_ARG, "score flags do not apply to attention");
+    if (p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_FORCE_SINK_LOCAL))
+        return fail(MSA_ERR_INVALID_ARG, "score and selection flags do not apply to attention from given ids");
     const bool dense = (p->flags & MSA_DENSE) != 0;
     MSA_TRY(check_ptr(q, "q"));
     MSA_TRY(check_ptr(k_cache, "k_cache"));
@@ -426,8 +430,9 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
                               const void *v_cache, const void *k_idx, void *o, int32_t *ids_out, float *lse, void *ws,
                               size_t ws_bytes, msa_stream_t stream) {
     MSA_TRY(check_params(p, DECODE_ONLY));
-    if (p->flags != 0)
-        return fail(MSA_ERR_INVALID_ARG, "msa_decode_fused takes no flags (dense decode: msa_sparse_attn_decode + MSA_DENSE)");
+    if (p->flags & ~MSA_FORCE_SINK_LOCAL)
+        return fail(MSA_ERR_INVALID_ARG,
+                    "msa_decode_fused takes only MSA_FORCE_SINK_LOCAL (dense decode: msa_sparse_attn_decode + MSA_DENSE)");
     MSA_TRY(check_ptr(q, "q"));
     MSA_TRY(check_ptr(q_idx, "q_idx"));
     MSA_TRY(check_ptr(k_cache, "k_cache"));
@@ -502,7 +507,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
 msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, const void *k_idx, int32_t *ids_out,
                                     float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
     MSA_TRY(check_params(p, PREFILL_ONLY));
-    if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes no flags");
+    if (p->flags & ~MSA_FORCE_SINK_LOCAL)
+        return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes only MSA_FORCE_SINK_LOCAL");
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->idx_dim != 64) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes idx_dim 64");
     if (p->block_size < 32) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes block_size >= 32");
@@ -518,6 +524,7 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     PrefillIdxArgs a{};
     a.B = p->batch; a.T = p->q_len; a.G = p->n_kv_heads; a.Hik = p->n_idx_k_heads; a.Bk = p->block_size;
     a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len;
+    a.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
     a.n_mt = L.n_mt;
     a.n_seg = L.n_seg;
     a.ids_out = ids_out; a.top_scores_out = top_scores_out;

@@ -46,6 +46,7 @@ struct AttnArgs {
     float scale_log2;          // softmax_scale * log2(e)
     int ring_bytes, nst;       // set by the launcher
     int cluster;               // > 1: the S splits of a (b, g) form one cluster and merge in shared memory
+    int force;                 // MSA_FORCE_SINK_LOCAL: the selection keeps block 0 and the last block
     int *status;
 };
 
@@ -55,10 +56,12 @@ struct PoolTopkArgs {
     int32_t *ids_out;
     float *top_scores_out;
     int B, q_len, q_start, G, Bk, k, L_max, nb_max, is_block, prefill;
+    int force;                 // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank first
 };
 
 struct PrefillIdxArgs {
     int B, T, G, Hik, Bk, k, q_start, L_max;
+    int force;                 // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank first
     int n_mt;                  // 256-row query tiles per (b, g)
     int n_seg;                 // key segments per unit
     int32_t *ids_out;          // [B, T, G, k]

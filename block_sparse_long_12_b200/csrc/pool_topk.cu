@@ -5,7 +5,8 @@
 // keeps the best blocks for the group.  This entry works on scores that an
 // earlier call stored (token or block granularity), one CTA per
 // (sequence, query row, group); eight warps take blocks round-robin, keep
-// warp-distributed sorted lists, and warp 0 merges them.
+// warp-distributed sorted lists, and warp 0 merges them.  With
+// MSA_FORCE_SINK_LOCAL block 0 and the row's own block take the score +inf.
 #include "msa_device.cuh"
 
 namespace msa {
@@ -44,6 +45,8 @@ __global__ void __launch_bounds__(256) pool_topk_kernel(const PoolTopkArgs a) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
         }
+        // forced sink / local blocks rank above every score
+        if (a.force && (n == 0 || n == nb - 1)) m = INFINITY;
         lst.insert(m, n, a.k, lane);
     }
     ls[w * 32 + lane] = lst.s;

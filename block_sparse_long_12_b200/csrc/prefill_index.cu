@@ -257,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = m0 + rl;
             const int pos = a.q_start + t;
             const int pos_min = a.q_start + m0;  // smallest position of the unit
+            // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank above every score
+            auto forced = [&](int blk) { return a.force && (blk == 0 || blk == pos / BK); };
             top.reset();
             float bm = -INFINITY;
             for (int n = w.n0; n < w.n1 && ok; ++n, ++ti) {
@@ -293,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bm = fmaxf(bm, tc::fmax3(cm[0], cm[1], fmaxf(cm[2], cm[3])));
                     if ((n + 1) % (BK / kKeys) == 0) {  // last tile of block n / (BK / kKeys)
                         const int blk = n / (BK / kKeys);
-                        if (!diag || blk * BK <= pos) top.insert(bm, blk);
+                        if (!diag || blk * BK <= pos) top.insert(forced(blk) ? INFINITY : bm, blk);
                         bm = -INFINITY;
                     }
                 } else {
@@ -304,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int c = 1; c < CPB; ++c) v = fmaxf(v, cm[q * CPB + c]);
                         const int blk = n * (kKeys / BK) + q;
-                        if (!diag || blk * BK <= pos) top.insert(v, blk);
+                        if (!diag || blk * BK <= pos) top.insert(forced(blk) ? INFINITY : v, blk);
                     }
                 }
             }

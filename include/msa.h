@@ -87,8 +87,22 @@ typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype_t;
 enum {
     MSA_SCORES_TOKEN = 1,    /* token scores s_j  [B, q_len, G, max_seq_len]  */
     MSA_SCORES_BLOCKMAX = 2, /* block scores S_n  [B, q_len, G, nb_max]       */
-    MSA_DENSE = 8            /* attend every visible block (plain GQA), ids unused */
+    MSA_DENSE = 8,           /* attend every visible block (plain GQA), ids unused */
+    MSA_FORCE_SINK_LOCAL = 16 /* TopK always keeps block 0 and the query's own block */
 };
+/*
+ * MSA_FORCE_SINK_LOCAL (accepted by msa_decode_fused, msa_decode_fused_noalloc,
+ * msa_block_maxpool_topk and msa_prefill_index_topk): the selection of a query at
+ * position pos always holds the sink block 0 and the local block floor(pos / Bk),
+ * the block of the query itself.  They rank above every other block, between
+ * themselves by block id (sink first), and their reported score is +inf; the
+ * remaining top_k - 2 places (top_k - 1 when pos < Bk, where the two are one
+ * block) go to the best other blocks in the usual order.  With top_k = 1 only
+ * the sink is kept.  No page fixes such a rule: the atlascloud.ai page, section 2
+ * ("Drei bewusste Abgrenzungen", third point), only guesses that an attention
+ * sink and positional encoding stand in for NSA's dropped sliding window.  It is
+ * offered here as an option, off by default.
+ */
 
 /* entry ids for msa_workspace_size */
 enum {
@@ -115,7 +129,7 @@ typedef struct {
     const int32_t *seq_lens; /* device int32[B]: cached length incl. current token(s) */
     float softmax_scale;  /* > 0; 1/sqrt(head_dim) in the usual attention      */
     int dtype;            /* msa_dtype_t; prefill entries take MSA_BF16 only   */
-    int flags;            /* MSA_SCORES_* / MSA_DENSE                          */
+    int flags;            /* MSA_SCORES_* / MSA_DENSE / MSA_FORCE_SINK_LOCAL   */
 } msa_params_t;
 
 /*

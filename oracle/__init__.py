@@ -50,7 +50,8 @@ class _Params(ctypes.Structure):
         ("n_idx_k_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("idx_dim", ctypes.c_int),
         ("block_size", ctypes.c_int), ("top_k", ctypes.c_int), ("q_len", ctypes.c_int),
         ("q_start", ctypes.c_int), ("max_seq_len", ctypes.c_int), ("dtype", ctypes.c_int),
-        ("dense", ctypes.c_int), ("prefill", ctypes.c_int), ("softmax_scale", ctypes.c_double),
+        ("dense", ctypes.c_int), ("prefill", ctypes.c_int), ("force_sink_local", ctypes.c_int),
+        ("softmax_scale", ctypes.c_double),
     ]
 
 
@@ -72,12 +73,14 @@ class Params:
     softmax_scale: float
     prefill: bool = False
     dense: bool = False
+    force_sink_local: bool = False  # block 0 and the query's own block always selected
 
     def c(self) -> _Params:
         return _Params(self.batch, self.n_q_heads, self.n_kv_heads, self.n_idx_k_heads,
                        self.head_dim, self.idx_dim, self.block_size, self.top_k, self.q_len,
                        self.q_start, self.max_seq_len, 0 if self.dtype == "f32" else 1,
-                       int(self.dense), int(self.prefill), float(self.softmax_scale))
+                       int(self.dense), int(self.prefill), int(self.force_sink_local),
+                       float(self.softmax_scale))
 
 
 def _load():

@@ -36,7 +36,12 @@
  *   - index-K head for group g is g mod n_idx_k_heads (1 shared head, or one
  *     per KV group);
  *   - softmax scale is a parameter (1/sqrt(head_dim) in every workload);
- *   - the query at position pos sees keys 0..pos (its own K/V included).
+ *   - the query at position pos sees keys 0..pos (its own K/V included);
+ *   - optional forced blocks (off unless force_sink_local is set): the page's
+ *     section 2, third point, guesses that an attention sink stands in for the
+ *     dropped sliding window; when asked for, block 0 (the sink) and the block
+ *     holding pos (the local block) rank above every score, between
+ *     themselves by id, and are reported with the score +inf.
  *
  * Layouts (all contiguous, element type f32 or bf16 given by `dtype`):
  *   q      [B, Tq, Hq,  D]       q_idx [B, Tq, G,   di]
@@ -57,6 +62,7 @@ typedef struct {
     int dtype;   /* 0: float32, 1: bfloat16 (raw 16-bit patterns) */
     int dense;   /* 1: select every causally valid block (plain GQA) */
     int prefill; /* 1: pos = q_start + t; 0: pos = seq_len - 1 */
+    int force_sink_local; /* 1: block 0 and the query's own block are always selected */
     double softmax_scale;
 } oracle_params;
 
@@ -126,7 +132,12 @@ void oracle_topk(const oracle_params *p, const double *S, int nb, int *ids_out,
 {
     const int k = p->top_k;
     scored_block *all = (scored_block *)malloc(sizeof(scored_block) * (size_t)(nb > 0 ? nb : 1));
-    for (int n = 0; n < nb; ++n) { all[n].score = S[n]; all[n].id = n; }
+    for (int n = 0; n < nb; ++n) {
+        all[n].score = S[n];
+        all[n].id = n;
+        /* forced blocks: the sink (0) and the query's own block, the last valid one */
+        if (p->force_sink_local && (n == 0 || n == nb - 1)) all[n].score = INFINITY;
+    }
     qsort(all, (size_t)nb, sizeof(scored_block), by_score_then_id);
     for (int i = 0; i < k; ++i) {
         ids_out[i] = i < nb ? all[i].id : -1;

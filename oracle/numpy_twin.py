@@ -40,7 +40,12 @@ def rank_of(S: np.ndarray) -> np.ndarray:
     return beats.sum(axis=1)
 
 
-def topk(S: np.ndarray, k: int) -> np.ndarray:
+def topk(S: np.ndarray, k: int, force_sink_local: bool = False) -> np.ndarray:
+    """Ids of the k best blocks in order, padded with -1.  With ``force_sink_local`` the first
+    block (the sink) and the last one (the query's own) are raised to +inf before ranking."""
+    if force_sink_local and len(S):
+        S = S.copy()
+        S[[0, -1]] = np.inf
     rank = rank_of(S)
     ids = np.full(k, -1, np.int32)
     for n in np.nonzero(rank < k)[0]:
@@ -71,7 +76,7 @@ def msa_row(cfg: dict, q, q_idx, k, v, k_idx, b: int, t: int, pos: int, dense: b
     for g in range(Hkv):
         s = token_scores(qif[b, t, g], kif[b, g % Hik], pos)
         S = block_scores(s, cfg["block_size"])
-        ids = topk(S, cfg["top_k"])
+        ids = topk(S, cfg["top_k"], cfg.get("force_sink_local", False))
         ids_all.append(ids)
         use = np.arange(len(S), dtype=np.int32) if dense else ids
         for h in range(g * r, (g + 1) * r):

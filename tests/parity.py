@@ -22,13 +22,30 @@ TOL_O = {"f32": 1e-4, "bf16": 2e-2}
 TOL_LSE = {"f32": 1e-4, "bf16": 1e-3}
 
 
-def oracle_params(x: dict, *, block_size, top_k, prefill=False, q_start=0, dense=False, softmax_scale=None):
+def oracle_params(x: dict, *, block_size, top_k, prefill=False, q_start=0, dense=False, softmax_scale=None,
+                  force_sink_local=False):
     B, Tq, Hq, D = x["q"].shape
     G, L = x["k"].shape[1], x["k"].shape[2]
     dtype = "f32" if x["q"].dtype == np.float32 else "bf16"
     return oracle.Params(B, Hq, G, x["k_idx"].shape[1], D, x["q_idx"].shape[-1], block_size, top_k, Tq, q_start, L,
                          dtype, softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D),
-                         prefill=prefill, dense=dense)
+                         prefill=prefill, dense=dense, force_sink_local=force_sink_local)
+
+
+def check_forced(ids: np.ndarray, pos_of, block_size: int, top_k: int):
+    """Every row of ids [B, T, G, k] holds block 0 first and the row's own block second (when it
+    has two valid blocks and k >= 2); pos_of(b, t) gives the row's position."""
+    B, T, G, _ = ids.shape
+    for b in range(B):
+        for t in range(T):
+            pos = pos_of(b, t)
+            if pos < 0:
+                continue
+            own = pos // block_size
+            for g in range(G):
+                assert ids[b, t, g, 0] == 0, (b, t, g, ids[b, t, g])
+                if own > 0 and top_k >= 2:
+                    assert ids[b, t, g, 1] == own, (b, t, g, ids[b, t, g])
 
 
 def to_np(inputs: dict) -> dict:

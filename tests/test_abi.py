@@ -40,6 +40,14 @@ def test_library_exports_every_declared_symbol(lib):
     assert {s for s in exported if s.startswith("msa_")} == set(declared_symbols())
 
 
+def test_flag_values_match_the_header(lib):
+    hdr = open(os.path.join(ROOT, "include", "msa.h")).read()
+    for name in ("MSA_SCORES_TOKEN", "MSA_SCORES_BLOCKMAX", "MSA_DENSE", "MSA_FORCE_SINK_LOCAL"):
+        m = re.search(r"\b" + name + r"\s*=\s*(\d+)", hdr)
+        assert m is not None, name
+        assert int(m.group(1)) == getattr(lib, name), name
+
+
 def test_status_strings(lib):
     L = lib.lib()
     for code, name in enumerate(["MSA_OK", "MSA_ERR_INVALID_ARG", "MSA_ERR_UNSUPPORTED", "MSA_ERR_WORKSPACE",
@@ -116,9 +124,16 @@ def test_bad_pointers_rejected_before_launch(lib):
     assert rc == lib.MSA_ERR_INVALID_ARG
     ps = good_params(lib, flags=lib.MSA_SCORES_TOKEN | lib.MSA_SCORES_BLOCKMAX)
     assert L.msa_index_score(ctypes.byref(ps), a, a, a, a, ws, None) == lib.MSA_ERR_INVALID_ARG
-    # fused decode takes no flags
+    # fused decode takes only the forced-block flag
     pd = good_params(lib, flags=lib.MSA_DENSE)
     assert L.msa_decode_fused(ctypes.byref(pd), *ptrs, ws, None) == lib.MSA_ERR_INVALID_ARG
+    pd = good_params(lib, flags=lib.MSA_DENSE | lib.MSA_FORCE_SINK_LOCAL)
+    assert L.msa_decode_fused(ctypes.byref(pd), *ptrs, ws, None) == lib.MSA_ERR_INVALID_ARG
+    # forcing blocks applies to selections, not to scores or to attention from given ids
+    pf = good_params(lib, flags=lib.MSA_SCORES_BLOCKMAX | lib.MSA_FORCE_SINK_LOCAL)
+    assert L.msa_index_score(ctypes.byref(pf), a, a, a, a, ws, None) == lib.MSA_ERR_INVALID_ARG
+    pf = good_params(lib, flags=lib.MSA_FORCE_SINK_LOCAL)
+    assert L.msa_sparse_attn_decode(ctypes.byref(pf), a, a, a, a, a, None, a, ws, None) == lib.MSA_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")

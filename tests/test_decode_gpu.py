@@ -17,7 +17,7 @@ from block_sparse_long_12_b200.inputs import WORKLOADS, Workload, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-from parity import compare_decode, oracle_params, to_np  # noqa: E402
+from parity import check_forced, compare_decode, oracle_params, to_np  # noqa: E402
 
 
 def _api():
@@ -25,10 +25,10 @@ def _api():
     return api
 
 
-def run_fused(inp, w):
+def run_fused(inp, w, force_sink_local=False):
     api = _api()
     o, ids, lse = api.decode(inp["q"], inp["q_idx"], inp["k"], inp["v"], inp["k_idx"], inp["seq_lens"],
-                             block_size=w.block_size, top_k=w.top_k)
+                             block_size=w.block_size, top_k=w.top_k, force_sink_local=force_sink_local)
     torch.cuda.synchronize()
     return o, ids, lse
 
@@ -75,6 +75,26 @@ def test_decode_fused_variants(case):
     o, ids, lse = run_fused(inp, w)
     x = to_np(inp)
     compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+
+
+@pytest.mark.parametrize("case", [
+    dict(),                                                           # ragged, partial last blocks
+    dict(n_idx_k_heads=1, hot_blocks=0),                               # groups on one shared stream (tensor cores)
+    dict(dtype="f32", idx_dim=32, head_dim=64),                        # fp32
+    dict(block_size=128, top_k=20, max_seq_len=1500, min_seq_len=1),  # fewer valid blocks than k
+    dict(block_size=256, top_k=1, max_seq_len=9000),                   # k = 1: the sink alone
+    dict(block_size=16, top_k=32, max_seq_len=3000),                   # small blocks, largest k
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()) or "base")
+def test_decode_forced_sink_local(case):
+    """MSA_FORCE_SINK_LOCAL: block 0 and the query's own block lead every list, the rest is the
+    best of the other blocks; ids and outputs against the oracle with the same option."""
+    w = small(**case)
+    inp = make_inputs(w, device="cuda")
+    inp["seq_lens"][0] = 1  # one visible token: the two forced blocks are one
+    o, ids, lse = run_fused(inp, w, force_sink_local=True)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k, force_sink_local=True), o, ids, lse)
+    check_forced(ids.cpu().numpy(), lambda b, t: int(x["seq_lens"][b]) - 1, w.block_size, w.top_k)
 
 
 def test_decode_exact_lengths_edges():
@@ -127,6 +147,40 @@ def test_index_scores_and_pool_topk(hik):
                 ref_ids, ref_sc, _, _ = oracle.topk(p, S)
                 assert ids_n[b, 0, g].tolist() == ref_ids.tolist()
                 np.testing.assert_array_equal(ts_n[b, 0, g][ref_ids >= 0], ref_sc[ref_ids >= 0].astype(np.float32))
+
+
+def test_pool_topk_forced_sink_local():
+    """The stand-alone TopK entry with MSA_FORCE_SINK_LOCAL, decode rows (block scores) and prefill
+    rows (token scores): exact against the oracle on the same fp32 values, forced scores +inf."""
+    api = _api()
+    B, G, L, bk, k = 3, 2, 700, 16, 6
+    gen = torch.Generator(device="cuda").manual_seed(8)
+    lens = torch.tensor([700, 17, 5], dtype=torch.int32, device="cuda")
+    nb = -(-L // bk)
+    blk = torch.randn(B, 1, G, nb, device="cuda", generator=gen).round(decimals=1)
+    ids, ts = api.pool_topk(blk, lens, block_size=bk, top_k=k, max_seq_len=L, is_block=True, force_sink_local=True)
+    torch.cuda.synchronize()
+    p = oracle.Params(B, G, G, G, 64, 32, bk, k, 1, 0, L, "f32", 0.125, force_sink_local=True)
+    bn, idn, tsn = blk.cpu().numpy(), ids.cpu().numpy(), ts.cpu().numpy()
+    for b in range(B):
+        n_valid = (int(lens[b]) - 1) // bk + 1
+        for g in range(G):
+            ref_ids, ref_sc, _, _ = oracle.topk(p, bn[b, 0, g, :n_valid].astype(np.float64))
+            assert idn[b, 0, g].tolist() == ref_ids.tolist()
+            np.testing.assert_array_equal(tsn[b, 0, g][ref_ids >= 0], ref_sc[ref_ids >= 0].astype(np.float32))
+    check_forced(idn, lambda b, t: int(lens[b]) - 1, bk, k)
+    T = 40
+    sc = torch.randn(1, T, G, 300, device="cuda", generator=gen).round(decimals=1)
+    ids, _ = api.pool_topk(sc, None, block_size=bk, top_k=k, max_seq_len=300, is_block=False, q_start=0,
+                           force_sink_local=True)
+    torch.cuda.synchronize()
+    pp = oracle.Params(1, G, G, G, 64, 32, bk, k, T, 0, 300, "f32", 0.125, prefill=True, force_sink_local=True)
+    scn, idn = sc.cpu().numpy(), ids.cpu().numpy()
+    for t in range(T):
+        for g in range(G):
+            S = oracle.block_scores(pp, scn[0, t, g, :t + 1].astype(np.float64), t)
+            assert idn[0, t, g].tolist() == oracle.topk(pp, S)[0].tolist()
+    check_forced(idn, lambda b, t: t, bk, k)
 
 
 def test_pool_topk_prefill_rows():

@@ -46,7 +46,8 @@ class COracle:
         return oracle.Params(cfg["batch"], cfg["n_q_heads"], cfg["n_kv_heads"], cfg["n_idx_k_heads"],
                              cfg["head_dim"], cfg["idx_dim"], cfg["block_size"], cfg["top_k"], cfg["q_len"],
                              cfg["q_start"], cfg["max_seq_len"], cfg["dtype"], cfg["softmax_scale"],
-                             prefill=cfg["prefill"], dense=dense)
+                             prefill=cfg["prefill"], dense=dense,
+                             force_sink_local=cfg.get("force_sink_local", False))
 
     def token_scores(self, cfg, x, b, t, g, pos):
         return oracle.token_scores(self.params(cfg), x["q_idx"], x["k_idx"], b, t, g, pos)
@@ -79,7 +80,7 @@ class Twin:
         return tw.block_scores(s[: pos + 1], cfg["block_size"])
 
     def topk(self, cfg, S):
-        return tw.topk(S, cfg["top_k"])
+        return tw.topk(S, cfg["top_k"], cfg.get("force_sink_local", False))
 
     def attend(self, cfg, qh, K, V, ids, pos):
         return tw.attention(qh, K, V, ids, pos, cfg["block_size"], cfg["softmax_scale"])
@@ -174,9 +175,32 @@ class MutIndexHeadOfGroupZero(Twin):
         return tw.token_scores(qi, ki, pos)
 
 
+class MutForcedLocalIsPrevious(Twin):
+    name = "mut_forced_local_is_previous_block"
+
+    def topk(self, cfg, S):
+        if cfg.get("force_sink_local", False) and len(S):
+            S = S.copy()
+            S[[0, max(len(S) - 2, 0)]] = np.inf
+        return tw.topk(S, cfg["top_k"])
+
+
+class MutForcedKeepRealScoreOrder(Twin):
+    name = "mut_forced_blocks_ranked_by_score"
+
+    def topk(self, cfg, S):
+        if not (cfg.get("force_sink_local", False) and len(S)):
+            return tw.topk(S, cfg["top_k"])
+        forced = sorted({0, len(S) - 1}, key=lambda n: (-S[n], n))
+        rest = [n for n in tw.topk(S, len(S)) if n not in forced]
+        out = (forced + rest)[: cfg["top_k"]]
+        return np.array(out + [-1] * (cfg["top_k"] - len(out)), np.int32)
+
+
 GOOD = [COracle(), Twin()]
 MUTANTS = [MutGroupModulo(), MutTieHigherId(), MutPoolSeesFuture(), MutMeanPool(), MutNoScale(),
-           MutAttendFuture(), MutDropIndexDim(), MutIndexHeadOfGroupZero()]
+           MutAttendFuture(), MutDropIndexDim(), MutIndexHeadOfGroupZero(), MutForcedLocalIsPrevious(),
+           MutForcedKeepRealScoreOrder()]
 
 
 # --------------------------------------------------------------------------
@@ -432,9 +456,52 @@ def pin_planted_hot_blocks(impl):
             assert set(ids[g].tolist()) <= hot, (b, g, ids[g], hot)
 
 
+def pin_forced_sink_local_brute_force(impl):
+    """Forced blocks: block 0 and the last valid block (the query's own) come first, by id, then the
+    best k - 2 of the other blocks by exhaustive search; with k = 1 the sink alone."""
+    rng = np.random.default_rng(29)
+    for trial in range(300):
+        nb = int(rng.integers(1, 13))
+        k = int(rng.integers(1, 6))
+        S = rng.integers(-3, 4, nb).astype(np.float64) if trial % 2 else rng.standard_normal(nb)
+        cfg = make_cfg(top_k=k, force_sink_local=True)
+        forced = [0] if nb == 1 else [0, nb - 1]
+        head = forced[:k]
+        others = [n for n in range(nb) if n not in forced]
+        m = min(k - len(head), len(others))
+        best = max((sorted(((S[n], -n) for n in comb), reverse=True)
+                    for comb in itertools.combinations(others, m)), default=[])
+        want = head + [-neg for (_, neg) in best]
+        want += [-1] * (k - len(want))
+        got = list(impl.topk(cfg, S))
+        assert got == want, (S, k, got, want)
+
+
+def pin_forced_rows(impl):
+    """On whole rows (decode and prefill) the forced flag keeps block 0 and block pos // Bk in every
+    group's list, the list stays valid, and with k >= the valid blocks the output is the dense one."""
+    for prefill in (False, True):
+        cfg = make_cfg(n_q_heads=4, n_kv_heads=2, n_idx_k_heads=2, max_seq_len=40, block_size=4, top_k=4,
+                       prefill=prefill, q_len=40 if prefill else 1, force_sink_local=True)
+        x = rand_inputs(cfg, 31, seq_lens=[37])
+        for t in ((0, 3, 4, 17, 36) if prefill else (0,)):
+            pos = t if prefill else 36
+            ids, o, _ = impl.row(cfg, x, 0, t)
+            nv = pos // 4 + 1
+            for g in range(2):
+                sel = [n for n in ids[g] if n >= 0]
+                assert ids[g][0] == 0 and (nv == 1 or ids[g][1] == nv - 1), (t, ids[g])
+                assert len(sel) == min(nv, 4) and len(set(sel)) == len(sel)
+                assert all(0 <= n < nv for n in sel)
+            if nv <= 4:
+                _, od, _ = impl.row(cfg, x, 0, t, dense=True)
+                np.testing.assert_allclose(o, od, rtol=0, atol=1e-12)
+
+
 PINS = [pin_golden_hand_worked, pin_topk_brute_force, pin_block_pool_properties, pin_index_score_projection,
         pin_dense_equals_sdpa, pin_sparse_equals_masked_sdpa, pin_diagram_grouping, pin_uniform_when_query_zero,
-        pin_single_key, pin_causality, pin_selection_valid_and_scale_free, pin_planted_hot_blocks]
+        pin_single_key, pin_causality, pin_selection_valid_and_scale_free, pin_planted_hot_blocks,
+        pin_forced_sink_local_brute_force, pin_forced_rows]
 
 
 @pytest.mark.parametrize("impl", GOOD, ids=lambda i: i.name)
@@ -473,6 +540,7 @@ def test_c_oracle_matches_numpy_twin(oracle_lib, dtype, mode):
     c, n = COracle(), Twin()
     for (b, t_) in rows:
         for dense in (False, True):
+            cfg["force_sink_local"] = not dense and t_ % 2 == 0
             i1, o1, l1 = c.row(cfg, x, b, t_, dense)
             i2, o2, l2 = n.row(cfg, x, b, t_, dense)
             np.testing.assert_array_equal(i1, i2)

@@ -15,10 +15,10 @@ from block_sparse_long_12_b200.inputs import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
 
-from parity import check_ids_row  # noqa: E402
+from parity import check_forced, check_ids_row  # noqa: E402
 
 
-def prefill_ids(inp, w, q_start, T, top_k=None, block_size=None, scores=False):
+def prefill_ids(inp, w, q_start, T, top_k=None, block_size=None, scores=False, force=False):
     from block_sparse_long_12_b200 import _lib, api
     k = top_k or w.top_k
     bk = block_size or w.block_size
@@ -26,7 +26,8 @@ def prefill_ids(inp, w, q_start, T, top_k=None, block_size=None, scores=False):
     qi = inp["q_idx"][:, q_start:q_start + T].contiguous()
     p = api.make_params(batch=B, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
                         head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=bk, top_k=k, max_seq_len=w.max_seq_len,
-                        dtype=_lib.MSA_BF16, q_len=T, q_start=q_start)
+                        dtype=_lib.MSA_BF16, q_len=T, q_start=q_start,
+                        flags=_lib.MSA_FORCE_SINK_LOCAL if force else 0)
     ids = torch.full((B, T, w.n_kv_heads, k), -7, dtype=torch.int32, device="cuda")
     ts = torch.empty(B, T, w.n_kv_heads, k, dtype=torch.float32, device="cuda") if scores else None
     ws = api.workspace(p, _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, "cuda")
@@ -36,7 +37,7 @@ def prefill_ids(inp, w, q_start, T, top_k=None, block_size=None, scores=False):
     return ids, ts
 
 
-def check_rows(inp, w, q_start, T, ids, rows, top_k=None, block_size=None):
+def check_rows(inp, w, q_start, T, ids, rows, top_k=None, block_size=None, force=False):
     """Compare GPU ids with the oracle on the given chunk rows (t relative to the chunk)."""
     from block_sparse_long_12_b200.inputs import to_numpy_raw
     k = top_k or w.top_k
@@ -45,7 +46,7 @@ def check_rows(inp, w, q_start, T, ids, rows, top_k=None, block_size=None):
     xo = {"q_idx": to_numpy_raw(inp["q_idx"][:, q_start:q_start + T]), "k_idx": to_numpy_raw(inp["k_idx"])}
     unused = np.zeros(8, np.uint16)  # Step 1 only: q, k, v are not read
     p = oracle.Params(B, w.n_q_heads, w.n_kv_heads, w.n_idx_k_heads, w.head_dim, w.idx_dim, bk, k, T, q_start,
-                      w.max_seq_len, "bf16", w.softmax_scale, prefill=True)
+                      w.max_seq_len, "bf16", w.softmax_scale, prefill=True, force_sink_local=force)
     ref = oracle.msa_rows(p, None, unused, xo["q_idx"], unused, unused, xo["k_idx"], rows, attention=False)
     idn = ids.cpu().numpy()
     ties = 0
@@ -150,3 +151,25 @@ def test_prefill_index_key_segments(case):
     tsn, idn = ts.cpu().numpy(), ids.cpu().numpy()
     assert ((idn == -1) == np.isneginf(tsn)).all()
     assert (idn >= -1).all() and (idn <= (q_start + T - 1) // case["block_size"]).all()
+
+
+@pytest.mark.parametrize("case", [
+    dict(block_size=128, top_k=16, q_start=0, T=700),      # first rows: one or few valid blocks
+    dict(block_size=64, top_k=8, q_start=1500, T=1000),
+    dict(block_size=128, top_k=1, q_start=1500, T=1000),   # k = 1: the sink alone
+    dict(block_size=32, top_k=32, q_start=39000, T=1000),  # long context: split key segments
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()))
+def test_prefill_index_forced_sink_local(case):
+    """MSA_FORCE_SINK_LOCAL in the fused prefill index: block 0 and each row's own (diagonal) block
+    lead the row's list, reported with +inf; the rest against the oracle with the same option."""
+    L = 40000 if case["q_start"] >= 39000 else 3000
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=L, batch=1, hot_blocks=5, seed=31)
+    inp = make_inputs(w, device="cuda")
+    q_start, T, k, bk = case["q_start"], case["T"], case["top_k"], case["block_size"]
+    ids, ts = prefill_ids(inp, w, q_start, T, top_k=k, block_size=bk, scores=True, force=True)
+    rng = np.random.default_rng(9)
+    rows = [(0, int(t)) for t in sorted(set(rng.choice(T, 200, replace=False).tolist()) | {0, 1, 255, 256, T - 1})]
+    check_rows(inp, w, q_start, T, ids, rows, top_k=k, block_size=bk, force=True)
+    idn, tsn = ids.cpu().numpy(), ts.cpu().numpy()
+    check_forced(idn, lambda b, t: q_start + t, bk, k)
+    assert np.isposinf(tsn[..., 0]).all()
