@@ -355,6 +355,8 @@ def run_ours(args, world, rank, local):
     del inp, q, q_idx, k, v, k_idx, ws, wsd, o, od
     torch.cuda.empty_cache()
     shared = None if args.no_shared_index else run_shared_index(args, world, rank, local, stream, flush)
+    large_k = None if args.no_large_k else run_shared_index(args, world, rank, local, stream, flush,
+                                                            name="decode_ctx1m_large_k")
     prefill = None
     if not args.no_prefill:
         del flush_buf
@@ -390,6 +392,7 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
         "shared_index_head": shared,
+        "large_k": large_k,
         "prefill": prefill,
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -397,11 +400,13 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def run_shared_index(args, world, rank, local, stream, flush):
+def run_shared_index(args, world, rank, local, stream, flush, name="decode_ctx1m_shared_idx"):
     """The 1M decode step with one index-K head shared by the 8 groups: the index stream is 1/8
-    as long, so the step is no longer dominated by the scan.  Same timing as the main step."""
+    as long, so the step is no longer dominated by the scan.  Same timing as the main step.
+    With name="decode_ctx1m_large_k": the large-k regime (64-token blocks, k 1024 of 16,384; the
+    middle stage is then the radix select, the last the attention over 268 MB of K/V)."""
     from block_sparse_long_12_b200 import _lib, api
-    w = WORKLOADS["decode_ctx1m_shared_idx"]
+    w = WORKLOADS[name]
     dev = torch.device("cuda", local)
     inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
@@ -443,8 +448,11 @@ def run_shared_index(args, world, rank, local, stream, flush):
     kv_bytes = w.batch * w.n_kv_heads * w.top_k * w.block_size * w.head_dim * 2 * 2
     del inp, q, q_idx, k, v, k_idx, ws, o
     torch.cuda.empty_cache()
+    stages = ({"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)}
+              if w.top_k <= 32 else
+              {"index_scan": round(scan_us, 2), "radix_select_and_sparse_attention": round(attn_us, 2)})
     return {"workload": w.name, "value": round(step_us, 2), "unit": UNIT, "n_idx_k_heads": w.n_idx_k_heads,
-            "stages_us": {"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)},
+            "block_size": w.block_size, "top_k": w.top_k, "stages_us": stages,
             "algorithmic_bytes": idx_bytes + kv_bytes,
             "step_roofline_frac": round((idx_bytes + kv_bytes) / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
             "scan_gbs": round(idx_bytes / (scan_us * 1e-6) / 1e9, 1), "peak_kind": kind}
@@ -535,6 +543,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-shared-index", action="store_true", help="skip the shared index-K head decode step")
+    ap.add_argument("--no-large-k", action="store_true", help="skip the large-k (k 1024 of 16,384 blocks) decode step")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -88,23 +88,6 @@ __device__ inline float reduce_scatter(float (&x)[R], int lane, int &head) {
 }
 
 
-// Descending bitonic sort of keys[0, P) (P a power of two) by the whole CTA.
-__device__ inline void block_sort_desc(unsigned long long *keys, int P) {
-    for (int size = 2; size <= P; size <<= 1)
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const unsigned long long x = keys[lo], y = keys[hi];
-                const bool desc = (lo & size) == 0;
-                if (desc ? x < y : x > y) {
-                    keys[lo] = y;
-                    keys[hi] = x;
-                }
-            }
-            __syncthreads();
-        }
-}
-
 // Descending bitonic sort of 64 keys held by one warp, element lane + 32 * j
 // in v[j]; the element of rank r ends in lane r % 32, v[r / 32].
 __device__ inline void warp_sort64_desc(unsigned long long (&v)[2], int lane) {
@@ -543,7 +526,7 @@ __device__ inline void group_list(const AttnArgs &a, int b, int g, const SegInfo
             if (a.top_scores_out != nullptr) a.top_scores_out[o] = sel_s[threadIdx.x];
         }
     } else {
-        if (threadIdx.x < a.k) sel_i[threadIdx.x] = a.ids_in[((size_t)b * a.G + g) * a.k + threadIdx.x];
+        if (threadIdx.x < a.k && a.k <= 32) sel_i[threadIdx.x] = a.ids_in[((size_t)b * a.G + g) * a.k + threadIdx.x];
         __syncthreads();
     }
 }
@@ -616,7 +599,8 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     if (j1 > jmax) j1 = jmax;
 
     auto block_at = [&](int j) -> int {
-        const int id = a.dense ? j : sel_i[j];
+        // more than 32 given ids stay in global memory (each split reads its own range)
+        const int id = a.dense ? j : (a.k > 32 ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
         return (id >= 0 && id < nb) ? id : -1;
     };
     auto tiles_of = [&](int id) -> int {
@@ -855,7 +839,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     const int jmax = a.dense ? nb : a.k;
     if (j1 > jmax) j1 = jmax;
     auto block_at = [&](int j) -> int {
-        const int id = a.dense ? j : sel_i[j];
+        // more than 32 given ids stay in global memory (each split reads its own range)
+        const int id = a.dense ? j : (a.k > 32 ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
         return (id >= 0 && id < nb) ? id : -1;
     };
     auto tiles_of = [&](int id) -> int {

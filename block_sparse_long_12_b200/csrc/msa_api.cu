@@ -158,20 +158,26 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
     const int n_seg = p.batch * p.n_idx_k_heads, gps = p.n_kv_heads / p.n_idx_k_heads;
     const int r = p.n_q_heads / p.n_kv_heads;
     size_t off = kStatusBytes;
+    const bool large = p.top_k > kMaxTopKList;
     if (scan) {
         L.seg_info = off;
         off += round256((size_t)n_seg * sizeof(SegInfo));
-        const size_t cand = (size_t)n_seg * L.n_cta * gps * p.top_k * 4;
+        // large k: no per-piece lists; the scan leaves every block's score and a radix select
+        // writes the ids
+        const size_t cand = large ? 0 : (size_t)n_seg * L.n_cta * gps * p.top_k * 4;
         L.cand_s = off;
         off += round256(cand);
         L.cand_i = off;
         off += round256(cand);
         L.tail_scores = off;
         off += round256((size_t)p.batch * p.n_kv_heads * nb_max_of(p) * 4);
+        L.large_ids = off;
+        off += round256(large ? (size_t)p.batch * p.n_kv_heads * p.top_k * 4 : 0);
     }
     if (attend) {
-        if (p.flags & MSA_DENSE) {
-            const int nb = nb_max_of(p);
+        if ((p.flags & MSA_DENSE) || large) {
+            // many blocks per group: about two CTAs per SM over all (sequence, group) pairs
+            const int nb = (p.flags & MSA_DENSE) ? nb_max_of(p) : p.top_k;
             const long long want = 2LL * n_sm;
             long long S = (want + (long long)p.batch * p.n_kv_heads - 1) / ((long long)p.batch * p.n_kv_heads);
             if (S < 1) S = 1;
@@ -230,6 +236,13 @@ PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm) {
     return L;
 }
 
+// The stand-alone TopK keeps warp lists up to kMaxTopKList; beyond, a radix select per row reads
+// block scores, which token scores first become in the workspace.
+size_t maxpool_topk_ws_bytes(const msa_params_t &p) {
+    if (p.top_k <= kMaxTopKList || (p.flags & MSA_SCORES_BLOCKMAX)) return kStatusBytes;
+    return kStatusBytes + round256((size_t)p.batch * p.q_len * p.n_kv_heads * nb_max_of(p) * 4);
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -254,9 +267,11 @@ size_t msa_workspace_size(const msa_params_t *p, int entry) {
     int n_sm = 0;
     switch (entry) {
         case MSA_ENTRY_INDEX_SCORE:
-        case MSA_ENTRY_MAXPOOL_TOPK:
             if (check_params(p, ANY_ROWS) != MSA_OK) return (size_t)-1;
             return kStatusBytes;
+        case MSA_ENTRY_MAXPOOL_TOPK:
+            if (check_params(p, ANY_ROWS) != MSA_OK) return (size_t)-1;
+            return maxpool_topk_ws_bytes(*p);
         case MSA_ENTRY_ATTN_DECODE:
             if (check_params(p, DECODE_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
             return decode_ws_layout(*p, false, true, n_sm).total;
@@ -355,9 +370,29 @@ msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_i
     MSA_TRY(check_ptr(ids_out, "ids_out"));
     MSA_TRY(check_ptr(top_scores_out, "top_scores_out", true));
     MSA_TRY(check_ptr(ws, "ws"));
-    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    const size_t need = maxpool_topk_ws_bytes(*p);
+    if (ws_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
     int n_sm = 0;
     MSA_TRY(check_device(&n_sm));
+    if (p->top_k > kMaxTopKList) {
+        LargeTopkArgs la{};
+        la.seq_lens = p->seq_lens; la.rows = p->batch * p->q_len * p->n_kv_heads; la.q_len = p->q_len;
+        la.q_start = p->q_start; la.G = p->n_kv_heads; la.Bk = p->block_size; la.k = p->top_k;
+        la.L_max = p->max_seq_len; la.prefill = p->q_len > 1; la.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
+        la.ids_out = ids_out; la.top_scores_out = top_scores_out;
+        la.stride = nb_max_of(*p);
+        cudaError_t e;
+        if (p->flags & MSA_SCORES_BLOCKMAX) {
+            la.scores = scores_in;
+        } else {
+            float *blk = reinterpret_cast<float *>(static_cast<unsigned char *>(ws) + kStatusBytes);
+            if ((e = launch_token_block_max(la, scores_in, blk, (cudaStream_t)stream)) != cudaSuccess)
+                return cuda_fail(e, "block max launch");
+            la.scores = blk;
+        }
+        if ((e = launch_large_topk(la, (cudaStream_t)stream)) != cudaSuccess) return cuda_fail(e, "topk launch");
+        return MSA_OK;
+    }
     PoolTopkArgs a{};
     a.scores = scores_in; a.seq_lens = p->seq_lens; a.ids_out = ids_out; a.top_scores_out = top_scores_out;
     a.B = p->batch; a.q_len = p->q_len; a.q_start = p->q_start; a.G = p->n_kv_heads; a.Bk = p->block_size;
@@ -376,7 +411,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
     AttnArgs a{};
     a.q = q; a.k_cache = k_cache; a.v_cache = v_cache; a.seq_lens = p->seq_lens;
     a.ids_in = ids;
-    if (after_scan) {  // select the group's list inside the attention kernel
+    if (after_scan && ids == nullptr) {  // select the group's list inside the attention kernel
         a.cand_s = reinterpret_cast<const float *>(wsb + L.cand_s);
         a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
         a.tail_scores = reinterpret_cast<const float *>(wsb + L.tail_scores);
@@ -460,10 +495,30 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.sched = reinterpret_cast<unsigned *>(wsb) + kSchedWord;
     a.counters = reinterpret_cast<int *>(wsb + L.counters);
     a.status = reinterpret_cast<int *>(wsb);
+    const bool large = p->top_k > kMaxTopKList;
+    if (large) {
+        // every block's score (static ranges and tails alike) into the block-score region
+        a.cand_s = nullptr;
+        a.cand_i = nullptr;
+    }
     cudaError_t e = stage_mark(0, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
+    if (large) {
+        if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+        int32_t *ids = reinterpret_cast<int32_t *>(wsb + L.large_ids);
+        LargeTopkArgs la{};
+        la.scores = reinterpret_cast<const float *>(wsb + L.tail_scores);
+        la.stride = nb_max_of(*p);
+        la.seq_lens = p->seq_lens; la.rows = p->batch * p->n_kv_heads; la.q_len = 1; la.q_start = 0;
+        la.G = p->n_kv_heads; la.Bk = p->block_size; la.k = p->top_k; la.L_max = p->max_seq_len;
+        la.prefill = 0; la.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
+        la.ids_out = ids;
+        la.ids_copy = ids_out;
+        if ((e = launch_large_topk(la, s)) != cudaSuccess) return cuda_fail(e, "topk launch");
+        return attend_decode(p, q, k_cache, v_cache, ids, true, L, wsb, o, nullptr, lse, s);
+    }
     if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return attend_decode(p, q, k_cache, v_cache, nullptr, true, L, wsb, o, ids_out, lse, s);
 }
@@ -473,6 +528,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
                                      msa_stream_t stream) {
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_sparse_attn_prefill takes no flags");
+    if (p->top_k > kMaxTopKList)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes at most %d blocks per row", kMaxTopKList);
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->block_size != 64 && p->block_size != 128)
         return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes block_size 64 or 128");
@@ -509,6 +566,8 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags & ~MSA_FORCE_SINK_LOCAL)
         return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes only MSA_FORCE_SINK_LOCAL");
+    if (p->top_k > kMaxTopKList)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill index TopK keeps at most %d blocks per row", kMaxTopKList);
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->idx_dim != 64) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes idx_dim 64");
     if (p->block_size < 32) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes block_size >= 32");

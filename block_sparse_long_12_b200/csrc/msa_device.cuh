@@ -190,6 +190,23 @@ __device__ inline void sel_unkey(unsigned long long key, float &s, int &id) {
     id = (int)~(uint32_t)key;
 }
 
+// Descending bitonic sort of keys[0, P) (P a power of two) by the whole CTA.
+__device__ inline void block_sort_desc(unsigned long long *keys, int P) {
+    for (int size = 2; size <= P; size <<= 1)
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const unsigned long long x = keys[lo], y = keys[hi];
+                const bool desc = (lo & size) == 0;
+                if (desc ? x < y : x > y) {
+                    keys[lo] = y;
+                    keys[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+}
+
 // The 32 best of two lists of distinct keys, each held descending one key per lane: the
 // elementwise max of one list and the other reversed is a bitonic sequence holding the 32
 // largest keys, which five half-cleaner steps sort descending.

@@ -15,7 +15,8 @@ namespace msa {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 constexpr int kMaxBatch = 1024;
-constexpr int kMaxTopK = 32;
+constexpr int kMaxTopK = 1024;          // largest top_k (decode entries and the stand-alone TopK)
+constexpr int kMaxTopKList = 32;        // largest top_k of the warp-list paths (fused prefill index, its attention)
 constexpr int kMaxGroupsPerSeg = 8;   // n_kv_heads / n_idx_k_heads handled by one index-K stream
 constexpr int kMaxPiecesPerSeg = 256; // lists merged per (segment, group) by one warp (8 per lane)
 
@@ -57,6 +58,17 @@ struct PoolTopkArgs {
     float *top_scores_out;
     int B, q_len, q_start, G, Bk, k, L_max, nb_max, is_block, prefill;
     int force;                 // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank first
+};
+
+// Large-k TopK of stored block scores, one CTA per row (b, t, g).
+struct LargeTopkArgs {
+    const float *scores;       // block scores: row r at scores + r * stride
+    long long stride;          // nb_max
+    const int *seq_lens;       // decode rows: pos = seq_lens[b] - 1
+    int rows, q_len, q_start, G, Bk, k, L_max, prefill, force;
+    int32_t *ids_out;          // [rows, k]
+    int32_t *ids_copy;         // nullable: a second copy of ids_out
+    float *top_scores_out;     // nullable
 };
 
 struct PrefillIdxArgs {
@@ -114,7 +126,7 @@ struct FillArgs {
 
 // Workspace layout of the decode entries (offsets in bytes from ws).
 struct DecodeWs {
-    size_t seg_info, cand_s, cand_i, tail_scores, counters, part_o, part_lse, total;
+    size_t seg_info, cand_s, cand_i, tail_scores, large_ids, counters, part_o, part_lse, total;
     int n_cta, S, blocks_per_split;
 };
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);
@@ -124,6 +136,8 @@ cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);
 cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl);
 cudaError_t launch_pool_topk(const PoolTopkArgs &a, cudaStream_t s);
+cudaError_t launch_large_topk(const LargeTopkArgs &a, cudaStream_t s);
+cudaError_t launch_token_block_max(const LargeTopkArgs &a, const float *tok, float *blk, cudaStream_t s);
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_cache, const void *v_cache, int n_sm,
                                 cudaStream_t s, const char **why);
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,

@@ -81,6 +81,10 @@ WORKLOADS = {
     # one index-K head shared by the 8 groups (the pages' literal reading): 1/8 of the index bytes
     "decode_ctx1m_shared_idx": Workload("decode_ctx1m_shared_idx", "decode", 1, 1048576, 64, 8, 1, 128, 64, 128,
                                         16, "bf16", hot_blocks=32, seed=1006),
+    # the large-k regime the pages back-calculate (section 3): 64-token blocks, 16,384 of them at
+    # 1M tokens, about 6 % selected (k 1024)
+    "decode_ctx1m_large_k": Workload("decode_ctx1m_large_k", "decode", 1, 1048576, 64, 8, 8, 128, 64, 64, 1024,
+                                     "bf16", hot_blocks=32, seed=1007),
 }
 
 

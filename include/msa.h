@@ -122,7 +122,7 @@ typedef struct {
     int head_dim;         /* D: 64 or 128                                      */
     int idx_dim;          /* di: idx_dim * sizeof(elem) in {64, 128, 256} bytes */
     int block_size;       /* Bk: 16..256, power of two                         */
-    int top_k;            /* 1..32                                             */
+    int top_k;            /* 1..1024; the prefill entries take 1..32           */
     int q_len;            /* decode entries: 1; prefill: chunk length          */
     int q_start;          /* prefill: absolute position of query row 0         */
     int max_seq_len;      /* Lmax, the caches' token stride                    */
@@ -151,7 +151,11 @@ MSA_API msa_status_t msa_index_score(const msa_params_t *params, const void *q_i
  * MSA_SCORES_BLOCKMAX, block scores ([B, q_len, G, nb_max]); only entries of
  * visible tokens/blocks are read.  ids_out [B, q_len, G, top_k] int32 in
  * selection order; top_scores_out (nullable) the matching fp32 scores
- * (-inf for padding).
+ * (-inf for padding).  top_k up to 32 keeps warp-distributed lists; larger
+ * top_k (the atlascloud.ai page, section 3: about 6-7 % of 16,384 blocks at
+ * 1M tokens) takes a radix select per row, and token scores then need
+ * msa_workspace_size(params, MSA_ENTRY_MAXPOOL_TOPK) bytes of ws for the
+ * rows' block maxima.
  */
 MSA_API msa_status_t msa_block_maxpool_topk(const msa_params_t *params, const float *scores_in,
                                     int32_t *ids_out, float *top_scores_out, void *ws,
@@ -178,6 +182,10 @@ MSA_API msa_status_t msa_sparse_attn_prefill(const msa_params_t *params, const v
 /*
  * One decode step, Steps 1 and 2 fused into back-to-back kernels on `stream`
  * (the block list never leaves the device).  ids_out and lse are nullable.
+ * top_k up to 32: the scan keeps per-range candidate lists and the attention
+ * kernel finishes the TopK; larger top_k: the scan stores every block's score
+ * in ws, a radix select per (sequence, group) writes the list, and the
+ * attention splits each group's blocks over about two CTAs per SM.
  */
 MSA_API msa_status_t msa_decode_fused(const msa_params_t *params, const void *q, const void *q_idx,
                               const void *k_cache, const void *v_cache, const void *k_idx, void *o,

@@ -71,11 +71,19 @@ def check_ids_row(p, x, b, t, g, pos, gpu_ids, ref_ids, kth, kth_next, where="",
     ref_ids = [int(i) for i in ref_ids]
     if gpu_ids == ref_ids:
         return True
+    cache = {}
+
+    def block_score(i):
+        # the row's block scores, computed once (long rows and large k make per-id calls costly)
+        if "S" not in cache:
+            s = oracle.token_scores(p, x["q_idx"], x["k_idx"], b, t, g, pos)
+            cache["S"] = oracle.block_scores(p, s, pos)
+        return float(cache["S"][i])
     if sorted(gpu_ids) == sorted(ref_ids):
         def score(i):
             if ref_scores is not None:
                 return float(ref_scores[ref_ids.index(i)])
-            return oracle_block_score(p, x, b, t, g, pos, i)
+            return block_score(i)
         for a_, r_ in zip(gpu_ids, ref_ids):
             if a_ != r_:
                 assert a_ >= 0 and r_ >= 0 and _close(score(a_), score(r_)), \
@@ -90,12 +98,13 @@ def check_ids_row(p, x, b, t, g, pos, gpu_ids, ref_ids, kth, kth_next, where="",
     assert all(0 <= i < nb for i in sel), f"{where}: gpu id not causal-valid {gpu_ids}"
     band_lo = kth_next - TIE_REL * max(abs(kth), abs(kth_next))
     band_hi = kth + TIE_REL * max(abs(kth), abs(kth_next))
+    sel_set, ref_set = set(sel), set(ref_ids)
     for i in ref_ids:
-        if i >= 0 and oracle_block_score(p, x, b, t, g, pos, i) > band_hi:
-            assert i in sel, f"{where}: block {i} above the tie band missing from gpu ids {gpu_ids}"
+        if i >= 0 and block_score(i) > band_hi:
+            assert i in sel_set, f"{where}: block {i} above the tie band missing from gpu ids {gpu_ids}"
     for i in sel:
-        if i not in ref_ids:
-            sc = oracle_block_score(p, x, b, t, g, pos, i)
+        if i not in ref_set:
+            sc = block_score(i)
             assert band_lo <= sc <= band_hi, f"{where}: gpu block {i} (score {sc}) outside the tie band"
     return False
 

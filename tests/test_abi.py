@@ -75,7 +75,7 @@ BAD = [
     (dict(block_size=100), "UNSUPPORTED"),
     (dict(block_size=512), "UNSUPPORTED"),
     (dict(top_k=0), "INVALID_ARG"),
-    (dict(top_k=33), "UNSUPPORTED"),
+    (dict(top_k=1025), "UNSUPPORTED"),
     (dict(max_seq_len=0), "INVALID_ARG"),
     (dict(softmax_scale=-1.0), "INVALID_ARG"),
     (dict(softmax_scale=float("inf")), "INVALID_ARG"),
@@ -119,6 +119,10 @@ def test_bad_pointers_rejected_before_launch(lib):
     pp = good_params(lib, q_len=100, q_start=4000)
     rc = L.msa_prefill_index_topk(ctypes.byref(pp), a, a, a, None, a, ws, None)
     assert rc == lib.MSA_ERR_INVALID_ARG
+    # prefill entries keep warp lists: at most 32 blocks per row
+    pk = good_params(lib, q_len=100, top_k=64)
+    assert L.msa_prefill_index_topk(ctypes.byref(pk), a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
+    assert L.msa_sparse_attn_prefill(ctypes.byref(pk), a, a, a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
     # index scores need exactly one score granularity
     rc = L.msa_index_score(ctypes.byref(p), a, a, a, a, ws, None)
     assert rc == lib.MSA_ERR_INVALID_ARG

@@ -183,6 +183,82 @@ def test_pool_topk_forced_sink_local():
     check_forced(idn, lambda b, t: t, bk, k)
 
 
+@pytest.mark.parametrize("k", [33, 100, 1024])
+def test_pool_topk_large_k(k):
+    """TopK beyond the warp lists (radix select per row) from stored block and token scores,
+    decode rows with ragged lengths (fewer valid blocks than k included), many exact ties; with
+    and without forced blocks; exact against the oracle on the same fp32 values."""
+    api = _api()
+    B, G, L, bk = 3, 2, 40000, 16
+    gen = torch.Generator(device="cuda").manual_seed(k)
+    lens = torch.tensor([40000, 5000, 700], dtype=torch.int32, device="cuda")
+    nb = -(-L // bk)
+    tok = torch.randn(B, 1, G, L, device="cuda", generator=gen).round(decimals=2)
+    for force in (False, True):
+        p = oracle.Params(B, G, G, G, 64, 32, bk, k, 1, 0, L, "f32", 0.125, force_sink_local=force)
+        tok_n = tok.cpu().numpy()
+        want = {}
+        for b in range(B):
+            Lb = int(lens[b])
+            for g in range(G):
+                S = oracle.block_scores(p, tok_n[b, 0, g, :Lb].astype(np.float64), Lb - 1)
+                want[b, g] = (S, oracle.topk(p, S))
+        blk = torch.full((B, 1, G, nb), float("nan"), device="cuda")  # entries past a row's blocks are not read
+        for (b, g), (S, _) in want.items():
+            blk[b, 0, g, :len(S)] = torch.from_numpy(S.astype(np.float32))
+        for is_block, sc in ((True, blk), (False, tok)):
+            ids, ts = api.pool_topk(sc, lens, block_size=bk, top_k=k, max_seq_len=L, is_block=is_block,
+                                    force_sink_local=force)
+            torch.cuda.synchronize()
+            idn, tsn = ids.cpu().numpy(), ts.cpu().numpy()
+            for (b, g), (S, (ref_ids, ref_sc, _, _)) in want.items():
+                assert idn[b, 0, g].tolist() == ref_ids.tolist(), (is_block, force, b, g)
+                np.testing.assert_array_equal(tsn[b, 0, g][ref_ids >= 0], ref_sc[ref_ids >= 0].astype(np.float32))
+                assert np.isneginf(tsn[b, 0, g][ref_ids < 0]).all()
+            if force:
+                check_forced(idn, lambda b, t: int(lens[b]) - 1, bk, k)
+
+
+def test_pool_topk_large_k_prefill_rows():
+    """The large-k TopK on prefill rows (pos = q_start + t) from stored token scores."""
+    api = _api()
+    B, T, G, L, bk, k = 1, 24, 2, 3000, 16, 64
+    gen = torch.Generator(device="cuda").manual_seed(12)
+    sc = torch.randn(B, T, G, L, device="cuda", generator=gen).round(decimals=1)
+    ids, _ = api.pool_topk(sc, None, block_size=bk, top_k=k, max_seq_len=L, is_block=False, q_start=2000)
+    torch.cuda.synchronize()
+    p = oracle.Params(B, G, G, G, 64, 32, bk, k, T, 2000, L, "f32", 0.125, prefill=True)
+    scn, idn = sc.cpu().numpy(), ids.cpu().numpy()
+    for t in range(T):
+        pos = 2000 + t
+        for g in range(G):
+            S = oracle.block_scores(p, scn[0, t, g, :pos + 1].astype(np.float64), pos)
+            assert idn[0, t, g].tolist() == oracle.topk(p, S)[0].tolist()
+
+
+@pytest.mark.parametrize("case", [
+    dict(block_size=64, top_k=100, max_seq_len=20000),                       # ragged batch of 3
+    dict(block_size=64, top_k=1024, max_seq_len=100000, batch=2, hot_blocks=40),  # k 1024
+    dict(block_size=64, top_k=300, max_seq_len=12000, min_seq_len=1),         # fewer valid blocks than k
+    dict(block_size=64, top_k=48, dtype="f32", idx_dim=32, head_dim=64),      # fp32 attention kernel
+    dict(block_size=128, top_k=64, n_idx_k_heads=1, hot_blocks=0),             # shared stream (tensor cores)
+    dict(block_size=64, top_k=128, max_seq_len=30000, force=True),            # forced sink / local blocks
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()))
+def test_decode_fused_large_k(case):
+    """Fused decode with k beyond the warp lists: the scan stores every block score, a radix select
+    writes each group's list, the attention splits the blocks over many CTAs; ids and outputs
+    against the oracle."""
+    case = dict(case)
+    force = case.pop("force", False)
+    w = small(**case)
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w, force_sink_local=force)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k, force_sink_local=force), o, ids, lse)
+    if force:
+        check_forced(ids.cpu().numpy(), lambda b, t: int(x["seq_lens"][b]) - 1, w.block_size, w.top_k)
+
+
 def test_pool_topk_prefill_rows():
     """The stand-alone TopK entry on prefill rows (pos = q_start + t) from stored token scores."""
     api = _api()
@@ -289,7 +365,7 @@ def test_workspace_reused_across_shapes():
     assert _lib.msa_get_device_status(shared) == 0
 
 
-@pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m",
+@pytest.mark.parametrize("name", ["decode_b8_ctx128k_ragged", "decode_ctx1m", "decode_b4_ctx1m", "decode_ctx1m_large_k",
                                   "decode_ctx1m_shared_idx"])
 def test_full_size_decode(name):
     """The benchmark workloads at full size, checked against the oracle on every (sequence, group)."""
@@ -301,8 +377,9 @@ def test_full_size_decode(name):
     del inp
     torch.cuda.empty_cache()
     compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
-    # planted data: every selected block is hot
+    # planted data: every selected block is hot (k <= hot blocks), or every hot block is selected
     idn = ids.cpu().numpy()
     for b in range(w.batch):
         for g in range(w.n_kv_heads):
-            assert set(idn[b, 0, g].tolist()) <= set(hot[b, g % w.n_idx_k_heads].tolist())
+            sel, hb = set(idn[b, 0, g].tolist()), set(hot[b, g % w.n_idx_k_heads].tolist()) - {-1}
+            assert sel <= hb if w.top_k <= len(hb) else hb <= sel
