@@ -768,6 +768,7 @@ __device__ inline void st_peer(float *local, int rank, float v) {
 }
 
 constexpr int kMmaThreads = 128;  // 4 warps
+constexpr int kMaxStages = 4;     // K/V ring stages (mbarriers reserved)
 constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
 constexpr int kMaxCluster = 8;    // splits of a group that form one cluster
 
@@ -793,8 +794,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     float *red_s = reinterpret_cast<float *>(sel_i + 32);                          // [32]
     int *red_i = reinterpret_cast<int *>(red_s + 32);                              // [32]
     int *misc = red_i + 32;                                                        // [4]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 4);                       // [2]
-    float *recv = reinterpret_cast<float *>(bars + 2);   // [cluster][slice] partials pushed to this CTA
+    uint64_t *bars = reinterpret_cast<uint64_t *>(misc + 4);                       // [kMaxStages]
+    float *recv = reinterpret_cast<float *>(bars + kMaxStages);  // [cluster][slice] partials pushed to this CTA
     float *recv_l = recv + kMmaRows * D + kMaxCluster;   // [cluster][16] their log2 normalisers
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
@@ -1115,9 +1116,11 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     a.cluster = (!a.dense && a.S <= kMaxCluster) ? a.S : 1;
     const int KT = a.Bk < 128 ? a.Bk : 128;
     const size_t stage = (size_t)2 * (D / 64) * KT * 128;
-    // one stage when every split is a single tile, two otherwise
+    // one stage when every split is a single tile; three for long splits of small tiles (large
+    // k, 64-key blocks: two CTAs per SM then keep 192 KB of K/V in flight per SM), two otherwise
     const bool one_tile = a.blocks_per_split == 1 && a.Bk <= 128;
-    a.nst = one_tile ? 1 : 2;
+    const int tiles = a.blocks_per_split * ((a.Bk + KT - 1) / KT);
+    a.nst = one_tile ? 1 : (stage <= 32768 && tiles >= 3 ? 3 : 2);
     const size_t ring = a.nst * stage;
     const size_t scratch = a.cand_s != nullptr ? select_scratch_bytes(a.n_cta, a.k) : 0;
     const size_t wgt = (size_t)a.S * a.r * 4 > (size_t)kMmaRows * D * 4 + 64 ? (size_t)a.S * a.r * 4
@@ -1125,7 +1128,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     size_t rb = ring > scratch ? ring : scratch;
     rb = rb > wgt ? rb : wgt;
     a.ring_bytes = (int)((rb + 1023) / 1024 * 1024);
-    const size_t smem = 1024 + (size_t)a.ring_bytes + (size_t)kMmaRows * (KT + 8) * 2 + (64 + 64 + 32 * 4 + 4) * 4 + 16 +
+    const size_t smem = 1024 + (size_t)a.ring_bytes + (size_t)kMmaRows * (KT + 8) * 2 + (64 + 64 + 32 * 4 + 4) * 4 + kMaxStages * 8 +
                         ((size_t)kMmaRows * D + kMaxCluster + (size_t)kMaxCluster * kMmaRows) * 4 + 64;
     static size_t attr_bytes = 0;
     if (smem > attr_bytes) {
@@ -1165,9 +1168,302 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     return cudaLaunchKernelEx(&cfg, decode_attn_mma_kernel<D>, km, vm, a);
 }
 
+
+// ---------------------------------------------------------------- bf16, many tiles per split
+// Large k and MSA_DENSE give every split tens to hundreds of key tiles.  One CTA per SM; each of
+// its NW warps owns SPW ring stages (K and V of TK keys each) and runs its own tiles
+// t = w, w + NW, ... from copy to output with no barrier: while it works on one tile its next
+// one is on the way.  S = Q K^T on mma.sync fragments, the online softmax on the quad's
+// registers, P handed to P V straight from the S accumulators (the accumulator layout of two
+// 8-key tiles is the A-fragment layout of one 16-key step).  NW x SPW stages keep ~192 KB of
+// K/V in flight per SM.  The warps' (m, l, O) are combined in shared memory at the end; splits
+// merge by log-sum-exp as in the other kernels.
+constexpr int kWideRing = 196608;  // bytes of ring per CTA
+
+template <int D> struct WideShape {
+    static constexpr int TK = D == 128 ? 32 : 64;        // keys per tile
+    static constexpr int STAGE = 2 * D * TK * 2;         // K and V of one tile, bf16 (16 KB)
+    static constexpr int SPW = 2;                        // stages per warp
+    static constexpr int NW = kWideRing / (STAGE * SPW); // warps
+};
+
+template <int D>
+__global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
+    decode_attn_wide_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                            const AttnArgs a) {
+    constexpr int NW = WideShape<D>::NW, STAGE = WideShape<D>::STAGE, SPW = WideShape<D>::SPW;
+    constexpr int TK = WideShape<D>::TK;
+    constexpr int NH = D / 64;          // 64-dim halves of a K/V row
+    constexpr int KS = D / 16;          // k-steps of Q.K^T
+    constexpr int NT = TK / 8;          // 8-key tiles of S
+    constexpr int DN = D / 8;           // 8-dim output tiles
+    constexpr int KVH = TK * 128;       // bytes of one 64-dim half tile
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + NW * SPW * STAGE);  // [NW][SPW]
+    float *cm = reinterpret_cast<float *>(bars + NW * SPW);                   // [NW][16] warps' row maxima
+    float *cl = cm + NW * 16;                                                 // [NW][16] warps' row sums
+    int *misc = reinterpret_cast<int *>(cl + NW * 16);                        // [4]
+
+    const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+    const int grp = lane >> 2, tig = lane & 3;
+    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int r = a.r;
+    uint64_t *my_bars = bars + w * SPW;
+    if (lane < SPW) mbar_init(&my_bars[lane], 1);
+    if (tid == 0) {
+        tc::prefetch_tmap(&kmap);
+        tc::prefetch_tmap(&vmap);
+    }
+    fence_mbar_init();
+    __syncwarp();
+    uint32_t qa[KS][4];
+    {
+        const __nv_bfloat16 *qg = reinterpret_cast<const __nv_bfloat16 *>(a.q) + ((size_t)b * a.Hq + (size_t)g * r) * D;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int c0 = ks * 16 + tig * 2;
+            qa[ks][0] = grp < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)grp * D + c0) : 0u;
+            qa[ks][1] = grp + 8 < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)(grp + 8) * D + c0) : 0u;
+            qa[ks][2] = grp < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)grp * D + c0 + 8) : 0u;
+            qa[ks][3] = grp + 8 < r ? *reinterpret_cast<const uint32_t *>(qg + (size_t)(grp + 8) * D + c0 + 8) : 0u;
+        }
+    }
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int pos = L - 1;
+    const int nb = (L + a.Bk - 1) / a.Bk;
+    pdl_wait_prior_grid();  // the selection (large k) is complete from here on
+    pdl_allow_next_grid();
+
+    // this split's list positions [j0, j1), each block cut into TPB tiles of TK keys
+    const int TPB = (a.Bk + TK - 1) / TK;
+    const int j0 = s * a.blocks_per_split;
+    int j1 = j0 + a.blocks_per_split;
+    const int jmax = a.dense ? nb : a.k;
+    if (j1 > jmax) j1 = jmax;
+    const int n_tiles = j1 > j0 ? (j1 - j0) * TPB : 0;
+    const int *ids = a.dense ? nullptr : a.ids_in + ((size_t)b * a.G + g) * a.k;
+    // first key and visible key count of tile t of the split (0 keys: nothing to do)
+    auto tile_of = [&](int t, int &key0) -> int {
+        const int j = j0 + t / TPB;
+        const int id = a.dense ? j : ids[j];
+        if (id < 0 || id >= nb) return 0;
+        key0 = id * a.Bk + (t % TPB) * TK;
+        const int blk_end = (id + 1) * a.Bk < pos + 1 ? (id + 1) * a.Bk : pos + 1;
+        const int nk = blk_end - key0;
+        return nk < TK ? (nk > 0 ? nk : 0) : TK;
+    };
+    const int row0 = (b * a.G + g) * a.L_max;
+    unsigned char *my_ring = ring + (size_t)w * SPW * STAGE;
+    // the warp's tiles in order: the next one with keys is copied into the next stage
+    int t_next = w, issued = 0, consumed = 0;
+    int nk_slot[SPW];
+#pragma unroll
+    for (int i = 0; i < SPW; ++i) nk_slot[i] = 0;
+    auto issue = [&]() {
+        int key0 = 0, nk = 0;
+        for (; t_next < n_tiles; t_next += NW) {
+            nk = tile_of(t_next, key0);
+            if (nk > 0) break;
+        }
+        if (t_next >= n_tiles) return;
+        t_next += NW;
+        const int slot = issued % SPW;
+#pragma unroll
+        for (int i = 0; i < SPW; ++i)
+            if (i == slot) nk_slot[i] = nk;
+        if (lane == 0) {
+            unsigned char *st = my_ring + (size_t)slot * STAGE;
+            mbar_arrive_expect_tx(&my_bars[slot], STAGE);
+#pragma unroll
+            for (int h = 0; h < NH; ++h) {
+                tc::tma_load_2d(st + h * KVH, &kmap, h * 64, row0 + key0, &my_bars[slot]);
+                tc::tma_load_2d(st + (NH + h) * KVH, &vmap, h * 64, row0 + key0, &my_bars[slot]);
+            }
+        }
+        ++issued;
+    };
+#pragma unroll
+    for (int i = 0; i < SPW; ++i) issue();
+
+    float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+    float oacc[DN][4];
+#pragma unroll
+    for (int dn = 0; dn < DN; ++dn) oacc[dn][0] = oacc[dn][1] = oacc[dn][2] = oacc[dn][3] = 0.f;
+    bool failed = false;
+    while (consumed < issued) {
+        const int slot = consumed % SPW;
+        if (!mbar_wait(&my_bars[slot], (consumed / SPW) & 1, a.status)) {
+            // give up: wait (bounded) for the warp's copies in flight, issue nothing more
+            failed = true;
+            for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % SPW], (q2 / SPW) & 1, nullptr);
+            break;
+        }
+        int nk = 0;
+#pragma unroll
+        for (int i = 0; i < SPW; ++i)
+            if (i == slot) nk = nk_slot[i];
+        const uint32_t k_addr = smem_u32(my_ring + (size_t)slot * STAGE), v_addr = k_addr + NH * KVH;
+        // S = Q K^T (scaled to the log2 domain), keys past the row masked
+        float sv[NT][4];
+#pragma unroll
+        for (int kn = 0; kn < NT; ++kn) sv[kn][0] = sv[kn][1] = sv[kn][2] = sv[kn][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ks += 2) {
+            const int mi = lane >> 3;
+            const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
+#pragma unroll
+            for (int kn = 0; kn < NT; ++kn) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(k_addr + (d0 >> 6) * KVH + sw128(kn * 8 + (lane & 7), (d0 & 63) >> 3), b0, b1, b2, b3);
+                mma_16816(sv[kn], qa[ks], b0, b1);
+                mma_16816(sv[kn], qa[ks + 1], b2, b3);
+            }
+        }
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int kn = 0; kn < NT; ++kn)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int key = kn * 8 + tig * 2 + (e & 1);
+                sv[kn][e] = key < nk ? sv[kn][e] * a.scale_log2 : -INFINITY;
+                mx[e >> 1] = fmaxf(mx[e >> 1], sv[kn][e]);
+            }
+        float alpha[2], m_new[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(FULL, mx[h], 1));
+            mx[h] = fmaxf(mx[h], __shfl_xor_sync(FULL, mx[h], 2));
+            m_new[h] = fmaxf(m_run[h], mx[h]);
+            alpha[h] = m_run[h] > -INFINITY ? exp2f(m_run[h] - m_new[h]) : 0.f;
+            m_run[h] = m_new[h];
+            l_part[h] *= alpha[h];
+        }
+#pragma unroll
+        for (int dn = 0; dn < DN; ++dn) {
+            oacc[dn][0] *= alpha[0]; oacc[dn][1] *= alpha[0];
+            oacc[dn][2] *= alpha[1]; oacc[dn][3] *= alpha[1];
+        }
+        // O += P V, 16 keys per step; P's A fragments come from the S accumulators of two 8-key tiles
+#pragma unroll
+        for (int kc = 0; kc < TK / 16; ++kc) {
+            uint32_t pa[4];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {      // the two 8-key tiles of the step
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {     // rows grp, grp + 8
+                    const float x0 = sv[2 * kc + hh][2 * h], x1 = sv[2 * kc + hh][2 * h + 1];
+                    const float p0 = x0 > -INFINITY ? exp2f(x0 - m_new[h]) : 0.f;
+                    const float p1 = x1 > -INFINITY ? exp2f(x1 - m_new[h]) : 0.f;
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    l_part[h] += __low2float(pb) + __high2float(pb);
+                    pa[hh * 2 + h] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+            }
+#pragma unroll
+            for (int dp = 0; dp < DN; dp += 2) {
+                const int mi = lane >> 3;
+                const int d0 = (dp + (mi >> 1)) * 8;
+                const int key = kc * 16 + (mi & 1) * 8 + (lane & 7);
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(v_addr + (d0 >> 6) * KVH + sw128(key, (d0 & 63) >> 3), b0, b1, b2, b3);
+                mma_16816(oacc[dp], pa, b0, b1);
+                mma_16816(oacc[dp + 1], pa, b2, b3);
+            }
+        }
+        __syncwarp();  // every lane is done with the stage before it is refilled
+        ++consumed;
+        issue();
+    }
+    (void)failed;
+
+    // the warp's rows: quad sums, then every warp's (m, l, O) combined in shared memory
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        l_part[h] += __shfl_xor_sync(FULL, l_part[h], 1);
+        l_part[h] += __shfl_xor_sync(FULL, l_part[h], 2);
+    }
+    __syncthreads();  // every warp is done with the ring: it holds the warps' O now
+    float *co = reinterpret_cast<float *>(ring);  // [NW][16][D]
+    if (tig == 0) {
+        cm[w * 16 + grp] = m_run[0];
+        cm[w * 16 + grp + 8] = m_run[1];
+        cl[w * 16 + grp] = l_part[0];
+        cl[w * 16 + grp + 8] = l_part[1];
+    }
+#pragma unroll
+    for (int dn = 0; dn < DN; ++dn) {
+        const int d = dn * 8 + tig * 2;
+        *reinterpret_cast<float2 *>(co + ((size_t)w * 16 + grp) * D + d) = make_float2(oacc[dn][0], oacc[dn][1]);
+        *reinterpret_cast<float2 *>(co + ((size_t)w * 16 + grp + 8) * D + d) = make_float2(oacc[dn][2], oacc[dn][3]);
+    }
+    __syncthreads();
+    const size_t split = ((size_t)b * a.G + g) * a.S + s;
+    for (int f = tid; f < r * D; f += NW * 32) {
+        const int row = f / D, d = f % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) M = fmaxf(M, cm[ww * 16 + row]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < NW; ++ww) {
+            const float mw = cm[ww * 16 + row];
+            if (mw > -INFINITY) {
+                const float e = exp2f(mw - M);
+                num = fmaf(e, co[((size_t)ww * 16 + row) * D + d], num);
+                den = fmaf(e, cl[ww * 16 + row], den);
+            }
+        }
+        a.part_o[(split * r + row) * D + d] = den > 0.f ? num / den : 0.f;
+        if (d == 0) a.part_lse[split * r + row] = den > 0.f ? M + log2f(den) : -INFINITY;
+    }
+    if (!last_split(a, b, g, &misc[0])) return;
+    merge_splits<__nv_bfloat16>(a, b, g, reinterpret_cast<float *>(ring));
+}
+
+template <int D>
+cudaError_t launch_wide(const AttnArgs &a, cudaStream_t s, bool pdl) {
+    constexpr int NW = WideShape<D>::NW, STAGE = WideShape<D>::STAGE, SPW = WideShape<D>::SPW;
+    constexpr int TK = WideShape<D>::TK;
+    const size_t smem = 1024 + (size_t)NW * SPW * STAGE + NW * SPW * 8 + (size_t)NW * 16 * 4 * 2 + 16;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(decode_attn_wide_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap km, vm;
+    const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
+    if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.k_cache), D, rows, D * 2, 64, TK,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.v_cache), D, rows, D * 2, 64, TK,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.S, a.G, a.B);
+    cfg.blockDim = dim3(NW * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_attn_wide_kernel<D>, km, vm, a);
+}
 }  // namespace
 
+// bf16 splits of many tiles (large k, MSA_DENSE) take the warp-per-stage kernel; the sparse step
+// with k <= 32 (a few blocks per split, the selection inside) takes decode_attn_mma_kernel.
+bool wide_attention(const msa_params_t &p) {
+    return p.dtype == MSA_BF16 && ((p.flags & MSA_DENSE) || p.top_k > kMaxTopKList);
+}
+
 cudaError_t launch_decode_attn(const AttnArgs &a, int dtype, cudaStream_t s, bool pdl) {
+    if (dtype == MSA_BF16 && (a.dense || a.k > kMaxTopKList))
+        return a.D == 64 ? launch_wide<64>(a, s, pdl) : launch_wide<128>(a, s, pdl);
     if (dtype == MSA_BF16) return a.D == 64 ? launch_mma<64>(a, s, pdl) : launch_mma<128>(a, s, pdl);
     return a.D == 64 ? launch_attn_r<float, 64>(a, s, pdl) : launch_attn_r<float, 128>(a, s, pdl);
 }

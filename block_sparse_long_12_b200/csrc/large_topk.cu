@@ -4,19 +4,19 @@
 // Page "MiniMax wird duenn" (atlascloud.ai), section 1, Step 1: block scores (the block maxima
 // of the index scores) go through TopK per group.  Section 3 back-calculates that a query
 // touches about 6-7 % of the blocks at 1M tokens (k near 1000 of 16,384 blocks of 64 tokens),
-// far beyond what per-warp sorted lists hold.  One CTA per row finds the k-th best score by a
-// radix select on the scores' order-preserving bits (four passes of 8 bits, a shared histogram
-// each), takes every block above it and, among the blocks equal to it, the lowest ids (an
-// ordered block-wide count), then sorts the k taken blocks once (bitonic, 64-bit keys: score
-// bits above the complemented id).  The row's scores are read from global memory in every pass
-// (L2 keeps them), so the number of blocks is not bounded by shared memory.
+// far beyond what per-warp sorted lists hold.  One CTA per row forms every block's 64-bit key
+// (the score's order-preserving bits above the complemented id: all distinct, ordered as the
+// selection), finds the k-th largest key exactly by a radix select (eight passes of 8 bits, a
+// shared histogram each), takes the k keys at or above it and sorts them once (bitonic).  Rows of
+// up to 16,384 blocks keep their keys in registers; longer rows re-read the scores from global
+// memory in every pass (L2 keeps them).
 #include "msa_device.cuh"
 
 namespace msa {
 
 namespace {
 
-constexpr int kLargeThreads = 1024;
+constexpr int kLargeThreads = 1024;  // = kMaxTopK: one sorted slot per thread
 
 // order-preserving image of a float: larger score, larger unsigned value (-0 taken as +0)
 __device__ inline uint32_t score_bits(float v) {
@@ -27,36 +27,10 @@ __device__ inline float bits_score(uint32_t u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-// Inclusive sum over the CTA of one value per thread; `tot` receives the total.
-__device__ inline int block_inclusive_sum(int v, int *warp_sums, int &tot) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(FULL, v, o);
-        if (lane >= o) v += u;
-    }
-    if (lane == 31) warp_sums[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int x = lane < nw ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(FULL, x, o);
-            if (lane >= o) x += u;
-        }
-        if (lane < nw) warp_sums[lane] = x;
-    }
-    __syncthreads();
-    tot = warp_sums[nw - 1];
-    const int before = warp > 0 ? warp_sums[warp - 1] : 0;
-    __syncthreads();  // warp_sums free again
-    return v + before;
-}
-
 __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTopkArgs a) {
+    constexpr int KPT = 16;  // keys per thread held in registers (rows of up to 16,384 blocks)
     __shared__ unsigned hist[256];
     __shared__ unsigned long long keys[kMaxTopK];
-    __shared__ int warp_sums[32];
     __shared__ int st[4];  // [0] chosen digit, [1] remaining rank, [2] taken blocks
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
     const int row = blockIdx.x;
@@ -73,22 +47,43 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
     const int nb = pos >= 0 ? pos / a.Bk + 1 : 0;
     const int kk = a.k < nb ? a.k : nb;
     const float *src = a.scores + (size_t)row * a.stride;
-    auto key_of = [&](int n) -> uint32_t {
+    // the selection key of block n: score bits above the complemented id, so that keys are
+    // distinct and their order is the selection order (higher score, then lower id)
+    auto key_of = [&](int n) -> unsigned long long {
         // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank above every score
         const float v = (a.force && (n == 0 || n == nb - 1)) ? INFINITY : src[n];
-        return score_bits(v);
+        return ((unsigned long long)score_bits(v) << 32) | (uint32_t)~(uint32_t)n;
     };
+    const bool in_regs = nb <= KPT * nthr;
+    unsigned long long kr[KPT];
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int n = tid + j * nthr;
+        kr[j] = (in_regs && n < nb) ? key_of(n) : 0ull;
+    }
 
     // the kk-th largest key T (exactly): one 8-bit digit per pass, from the top
-    uint32_t prefix = 0, mask = 0;
+    unsigned long long prefix = 0, mask = 0;
     int rem = kk;  // rank of T among the keys that match the prefix so far
     if (kk < nb) {
-        for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int shift = 56; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += nthr) hist[i] = 0;
             __syncthreads();
-            for (int n = tid; n < nb; n += nthr) {
-                const uint32_t u = key_of(n);
-                if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
+            // lanes with the same digit add once (the high digits of nearby scores coincide, and
+            // one atomic per lane would serialise on a few bins)
+            auto count = [&](unsigned long long u, bool valid) {
+                const unsigned d = valid && (u & mask) == prefix ? ((unsigned)(u >> shift) & 255u) : 256u;
+                const unsigned peers = __match_any_sync(FULL, d);
+                if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
+            };
+            if (in_regs) {
+#pragma unroll
+                for (int j = 0; j < KPT; ++j) count(kr[j], tid + j * nthr < nb);
+            } else {
+                for (int n0 = 0; n0 < nb; n0 += nthr) {
+                    const int n = n0 + tid;
+                    count(n < nb ? key_of(n) : 0ull, n < nb);
+                }
             }
             __syncthreads();
             if (warp == 0) {
@@ -107,8 +102,7 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
                     if (lane >= o) incl += u;
                 }
                 const unsigned excl = incl - sum;
-                const bool here = excl < (unsigned)rem && (unsigned)rem <= incl;
-                if (here) {
+                if (excl < (unsigned)rem && (unsigned)rem <= incl) {
                     unsigned above = excl;
                     int d = 255 - 8 * lane;
 #pragma unroll
@@ -124,56 +118,55 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
                 }
             }
             __syncthreads();
-            prefix |= (uint32_t)st[0] << shift;
-            mask |= 255u << shift;
+            prefix |= (unsigned long long)st[0] << shift;
+            mask |= 255ull << shift;
             rem = st[1];
             __syncthreads();
         }
     }
-    const uint32_t T = prefix;  // with kk == nb every block is taken (mask 0 keeps all)
-
-    // take every key above T and the `rem` lowest ids equal to T: each thread scans a contiguous
-    // range of ids, so an inclusive sum of the per-thread counts ranks the equal keys by id
+    // keys are distinct, so exactly kk of them are >= T (with kk == nb, T = 0 takes every block)
+    const unsigned long long T = prefix;
     if (tid == 0) st[2] = 0;
-    const int chunk = (nb + nthr - 1) / nthr;
-    const int n0 = tid * chunk, n1 = n0 + chunk < nb ? n0 + chunk : nb;
-    int eq = 0;
-    if (kk < nb)
-        for (int n = n0; n < n1; ++n) eq += key_of(n) == T;
-    int tot = 0;
-    const int eq_incl = block_inclusive_sum(eq, warp_sums, tot);
-    int rank = eq_incl - eq;  // equal keys with lower ids
-    for (int n = n0; n < n1; ++n) {
-        const uint32_t u = key_of(n);
-        bool take;
-        if (kk == nb) {
-            take = true;
-        } else if (u > T) {
-            take = true;
-        } else if (u == T) {
-            take = rank < rem;
-            ++rank;
-        } else {
-            take = false;
-        }
-        if (take) {
+    __syncthreads();
+    auto take = [&](unsigned long long u) {
+        if (u >= T) {
             const int at = atomicAdd(&st[2], 1);
-            if (at < kMaxTopK) keys[at] = ((unsigned long long)u << 32) | (uint32_t)~(uint32_t)n;
+            if (at < kMaxTopK) keys[at] = u;
         }
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int j = 0; j < KPT; ++j)
+            if (tid + j * nthr < nb) take(kr[j]);
+    } else {
+        for (int n = tid; n < nb; n += nthr) take(key_of(n));
     }
     __syncthreads();
-    int P = 1;
-    while (P < kk) P <<= 1;
-    for (int i = kk + tid; i < P; i += nthr) keys[i] = 0ull;  // below every real key
-    __syncthreads();
-    if (P > 1) block_sort_desc(keys, P);
-    for (int i = tid; i < a.k; i += nthr) {
-        const size_t o = (size_t)row * a.k + i;
-        const unsigned long long key = i < kk ? keys[i] : 0ull;
-        const int id = i < kk ? (int)~(uint32_t)key : -1;
+    // descending bitonic sort of the kMaxTopK slots (one per thread, zero padding below every
+    // real key): strides below 32 exchange through shuffles, larger ones through shared memory
+    unsigned long long v = tid < kk ? keys[tid] : 0ull;
+    if (kk > 1) {
+        for (int size = 2; size <= kMaxTopK; size <<= 1)
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                unsigned long long o;
+                if (stride >= 32) {
+                    __syncthreads();
+                    keys[tid] = v;
+                    __syncthreads();
+                    o = keys[tid ^ stride];
+                } else {
+                    o = __shfl_xor_sync(FULL, v, stride);
+                }
+                const bool keep_max = ((tid & stride) == 0) == ((tid & size) == 0);
+                v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+            }
+    }
+    if (tid < a.k) {  // thread i holds the i-th key (a.k <= kMaxTopK = blockDim.x)
+        const size_t o = (size_t)row * a.k + tid;
+        const int id = tid < kk ? (int)~(uint32_t)v : -1;
         a.ids_out[o] = id;
         if (a.ids_copy != nullptr) a.ids_copy[o] = id;
-        if (a.top_scores_out != nullptr) a.top_scores_out[o] = i < kk ? bits_score((uint32_t)(key >> 32)) : -INFINITY;
+        if (a.top_scores_out != nullptr) a.top_scores_out[o] = tid < kk ? bits_score((uint32_t)(v >> 32)) : -INFINITY;
     }
 }
 

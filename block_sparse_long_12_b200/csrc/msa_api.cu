@@ -176,9 +176,10 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
     }
     if (attend) {
         if ((p.flags & MSA_DENSE) || large) {
-            // many blocks per group: about two CTAs per SM over all (sequence, group) pairs
+            // many blocks per group: one CTA per SM (the bf16 warp-per-stage kernel) or about two
+            // (fp32) over all (sequence, group) pairs
             const int nb = (p.flags & MSA_DENSE) ? nb_max_of(p) : p.top_k;
-            const long long want = 2LL * n_sm;
+            const long long want = (wide_attention(p) ? 1LL : 2LL) * n_sm;
             long long S = (want + (long long)p.batch * p.n_kv_heads - 1) / ((long long)p.batch * p.n_kv_heads);
             if (S < 1) S = 1;
             if (S > kMaxSplits) S = kMaxSplits;

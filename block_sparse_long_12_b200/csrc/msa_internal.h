@@ -130,6 +130,7 @@ struct DecodeWs {
     int n_cta, S, blocks_per_split;
 };
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm);
+bool wide_attention(const msa_params_t &p);  // bf16 and (MSA_DENSE or top_k > kMaxTopKList)
 
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_fill_neg_inf(float *p, long long n, cudaStream_t s);

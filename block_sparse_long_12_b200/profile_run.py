@@ -4,10 +4,12 @@
   python -m block_sparse_long_12_b200.profile_run prefill_index --context 65536 --chunk 8192 --steps 1
   python -m block_sparse_long_12_b200.profile_run prefill_attn --context 65536 --chunk 8192 --steps 1
   python -m block_sparse_long_12_b200.profile_run scan_shared --context 1048576 --steps 3
+  python -m block_sparse_long_12_b200.profile_run large_k --context 262144 --steps 3
 
 Inputs are the seeded synthetic workloads of ``inputs`` at the requested
 size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
-64, block 128, top-k 16), kept small enough for a profiler's replay passes.
+64, block 128, top-k 16; large_k: block 64, top-k 1024), kept small enough
+for a profiler's replay passes.
 """
 from __future__ import annotations
 
@@ -19,8 +21,8 @@ from . import _lib, api
 from .inputs import WORKLOADS, make_inputs
 
 
-def run_decode(args):
-    w = WORKLOADS["decode_ctx1m"].scaled(max_seq_len=args.context, batch=args.batch)
+def run_decode(args, name="decode_ctx1m"):
+    w = WORKLOADS[name].scaled(max_seq_len=args.context, batch=args.batch)
     inp = make_inputs(w, device="cuda")
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
     p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
@@ -90,14 +92,15 @@ def run_scan_shared(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "scan_shared"])
+    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "scan_shared", "large_k"])
     ap.add_argument("--context", type=int, default=262144)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=8192)
     ap.add_argument("--steps", type=int, default=3)
     args = ap.parse_args()
     {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn,
-     "scan_shared": run_scan_shared}[args.what](args)
+     "scan_shared": run_scan_shared,
+     "large_k": lambda a: run_decode(a, "decode_ctx1m_large_k")}[args.what](args)
 
 
 if __name__ == "__main__":
