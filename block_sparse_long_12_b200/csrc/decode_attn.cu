@@ -1204,6 +1204,7 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
     float *cm = reinterpret_cast<float *>(bars + NW * SPW);                   // [NW][16] warps' row maxima
     float *cl = cm + NW * 16;                                                 // [NW][16] warps' row sums
     int *misc = reinterpret_cast<int *>(cl + NW * 16);                        // [4]
+    int *sid = misc + 4;                                                      // [kMaxTopK] the split's ids
 
     const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
     const int grp = lane >> 2, tig = lane & 3;
@@ -1243,11 +1244,17 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
     const int jmax = a.dense ? nb : a.k;
     if (j1 > jmax) j1 = jmax;
     const int n_tiles = j1 > j0 ? (j1 - j0) * TPB : 0;
-    const int *ids = a.dense ? nullptr : a.ids_in + ((size_t)b * a.G + g) * a.k;
+    if (!a.dense) {
+        // the split's ids into shared memory once (a global load per tile would sit on the
+        // issue path of every copy)
+        const int *ids = a.ids_in + ((size_t)b * a.G + g) * a.k;
+        for (int j = j0 + tid; j < j1; j += NW * 32) sid[j - j0] = ids[j];
+        __syncthreads();
+    }
     // first key and visible key count of tile t of the split (0 keys: nothing to do)
     auto tile_of = [&](int t, int &key0) -> int {
         const int j = j0 + t / TPB;
-        const int id = a.dense ? j : ids[j];
+        const int id = a.dense ? j : sid[j - j0];
         if (id < 0 || id >= nb) return 0;
         key0 = id * a.Bk + (t % TPB) * TK;
         const int blk_end = (id + 1) * a.Bk < pos + 1 ? (id + 1) * a.Bk : pos + 1;
@@ -1426,7 +1433,7 @@ template <int D>
 cudaError_t launch_wide(const AttnArgs &a, cudaStream_t s, bool pdl) {
     constexpr int NW = WideShape<D>::NW, STAGE = WideShape<D>::STAGE, SPW = WideShape<D>::SPW;
     constexpr int TK = WideShape<D>::TK;
-    const size_t smem = 1024 + (size_t)NW * SPW * STAGE + NW * SPW * 8 + (size_t)NW * 16 * 4 * 2 + 16;
+    const size_t smem = 1024 + (size_t)NW * SPW * STAGE + NW * SPW * 8 + (size_t)NW * 16 * 4 * 2 + 16 + kMaxTopK * 4;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_attn_wide_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -6,8 +6,9 @@
 // touches about 6-7 % of the blocks at 1M tokens (k near 1000 of 16,384 blocks of 64 tokens),
 // far beyond what per-warp sorted lists hold.  One CTA per row forms every block's 64-bit key
 // (the score's order-preserving bits above the complemented id: all distinct, ordered as the
-// selection), finds the k-th largest key exactly by a radix select (eight passes of 8 bits, a
-// shared histogram each), takes the k keys at or above it and sorts them once (bitonic).  Rows of
+// selection), finds the k-th largest key exactly by a radix select (passes of 8 bits with a
+// shared histogram each: four over the score bits, four more over the id bits only when blocks
+// tie at the k-th score), takes the k keys at or above it and sorts them once (bitonic).  Rows of
 // up to 16,384 blocks keep their keys in registers; longer rows re-read the scores from global
 // memory in every pass (L2 keeps them).
 #include "msa_device.cuh"
@@ -31,7 +32,7 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
     constexpr int KPT = 16;  // keys per thread held in registers (rows of up to 16,384 blocks)
     __shared__ unsigned hist[256];
     __shared__ unsigned long long keys[kMaxTopK];
-    __shared__ int st[4];  // [0] chosen digit, [1] remaining rank, [2] taken blocks
+    __shared__ int st[4];  // [0] chosen digit, [1] remaining rank, [2] taken blocks, [3] prefix all taken
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
     const int row = blockIdx.x;
     const int t = (row / a.G) % a.q_len, b = row / (a.G * a.q_len);
@@ -115,13 +116,18 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
                     }
                     st[0] = d;
                     st[1] = rem - (int)above;
+                    st[3] = hist[d] == (unsigned)(rem - (int)above);  // every key with this prefix is taken
                 }
             }
             __syncthreads();
             prefix |= (unsigned long long)st[0] << shift;
             mask |= 255ull << shift;
             rem = st[1];
+            const bool all_taken = st[3] != 0;
             __syncthreads();
+            // once the score bits are fixed and every block with that score is taken, the id bits
+            // need no passes: T is that score with the lowest id bits
+            if (shift == 32 && all_taken) break;
         }
     }
     // keys are distinct, so exactly kk of them are >= T (with kk == nb, T = 0 takes every block)

@@ -179,8 +179,10 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
             // many blocks per group: one CTA per SM (the bf16 warp-per-stage kernel) or about two
             // (fp32) over all (sequence, group) pairs
             const int nb = (p.flags & MSA_DENSE) ? nb_max_of(p) : p.top_k;
-            const long long want = (wide_attention(p) ? 1LL : 2LL) * n_sm;
-            long long S = (want + (long long)p.batch * p.n_kv_heads - 1) / ((long long)p.batch * p.n_kv_heads);
+            const long long bg = (long long)p.batch * p.n_kv_heads;
+            // one CTA per SM: no more splits than fill one wave (a second, short wave would
+            // double the kernel's time); two per SM: round up
+            long long S = wide_attention(p) ? n_sm / bg : (2LL * n_sm + bg - 1) / bg;
             if (S < 1) S = 1;
             if (S > kMaxSplits) S = kMaxSplits;
             if (S > nb) S = nb;
