@@ -17,8 +17,10 @@
 //
 // bf16: decode_attn_mma_kernel runs both products on mma.sync tensor-core
 // fragments (the r <= 16 heads padded to 16 rows), K/V tiles in the 128-byte
-// swizzle layout written by TMA tensor copies.  fp32: decode_attn_kernel on
-// CUDA cores (exact fp32 products).
+// swizzle layout written by TMA tensor copies; splits of many tiles (large k,
+// MSA_DENSE) take decode_attn_wide_kernel, whose warps run their own tiles
+// without barriers.  fp32: decode_attn_kernel on CUDA cores (exact fp32
+// products).
 #include "tcgen05.cuh"
 
 namespace msa {
@@ -526,7 +528,8 @@ __device__ inline void group_list(const AttnArgs &a, int b, int g, const SegInfo
             if (a.top_scores_out != nullptr) a.top_scores_out[o] = sel_s[threadIdx.x];
         }
     } else {
-        if (threadIdx.x < a.k && a.k <= 32) sel_i[threadIdx.x] = a.ids_in[((size_t)b * a.G + g) * a.k + threadIdx.x];
+        if (threadIdx.x < a.k && a.k <= kMaxTopKList)
+            sel_i[threadIdx.x] = a.ids_in[((size_t)b * a.G + g) * a.k + threadIdx.x];
         __syncthreads();
     }
 }
@@ -600,7 +603,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
 
     auto block_at = [&](int j) -> int {
         // more than 32 given ids stay in global memory (each split reads its own range)
-        const int id = a.dense ? j : (a.k > 32 ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
+        const int id = a.dense ? j : (a.k > kMaxTopKList ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
         return (id >= 0 && id < nb) ? id : -1;
     };
     auto tiles_of = [&](int id) -> int {
@@ -841,7 +844,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     if (j1 > jmax) j1 = jmax;
     auto block_at = [&](int j) -> int {
         // more than 32 given ids stay in global memory (each split reads its own range)
-        const int id = a.dense ? j : (a.k > 32 ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
+        const int id = a.dense ? j : (a.k > kMaxTopKList ? a.ids_in[((size_t)b * a.G + g) * a.k + j] : sel_i[j]);
         return (id >= 0 && id < nb) ? id : -1;
     };
     auto tiles_of = [&](int id) -> int {
@@ -1463,7 +1466,7 @@ cudaError_t launch_wide(const AttnArgs &a, cudaStream_t s, bool pdl) {
 }  // namespace
 
 // bf16 splits of many tiles (large k, MSA_DENSE) take the warp-per-stage kernel; the sparse step
-// with k <= 32 (a few blocks per split, the selection inside) takes decode_attn_mma_kernel.
+// with k <= kMaxTopKList (a few blocks per split, the selection inside) takes decode_attn_mma_kernel.
 bool wide_attention(const msa_params_t &p) {
     return p.dtype == MSA_BF16 && ((p.flags & MSA_DENSE) || p.top_k > kMaxTopKList);
 }
