@@ -219,6 +219,30 @@ def test_pool_topk_large_k(k):
                 check_forced(idn, lambda b, t: int(lens[b]) - 1, bk, k)
 
 
+def test_pool_topk_large_k_long_rows():
+    """Rows of more blocks than the select keeps in registers (40,000 and 20,001 blocks): the keys
+    are re-read from memory in every radix pass; exact against the oracle, ties included."""
+    api = _api()
+    B, G, bk, k = 2, 2, 16, 500
+    L = 40000 * bk
+    gen = torch.Generator(device="cuda").manual_seed(21)
+    lens = torch.tensor([L, 20001 * bk - 3], dtype=torch.int32, device="cuda")
+    nb = L // bk
+    blk = torch.randn(B, 1, G, nb, device="cuda", generator=gen).round(decimals=2)
+    for force in (False, True):
+        ids, ts = api.pool_topk(blk, lens, block_size=bk, top_k=k, max_seq_len=L, is_block=True,
+                                force_sink_local=force)
+        torch.cuda.synchronize()
+        p = oracle.Params(B, G, G, G, 64, 32, bk, k, 1, 0, L, "f32", 0.125, force_sink_local=force)
+        bn, idn, tsn = blk.cpu().numpy(), ids.cpu().numpy(), ts.cpu().numpy()
+        for b in range(B):
+            n_valid = (int(lens[b]) - 1) // bk + 1
+            for g in range(G):
+                ref_ids, ref_sc, _, _ = oracle.topk(p, bn[b, 0, g, :n_valid].astype(np.float64))
+                assert idn[b, 0, g].tolist() == ref_ids.tolist(), (force, b, g)
+                np.testing.assert_array_equal(tsn[b, 0, g], ref_sc.astype(np.float32))
+
+
 def test_pool_topk_large_k_prefill_rows():
     """The large-k TopK on prefill rows (pos = q_start + t) from stored token scores."""
     api = _api()
@@ -276,9 +300,15 @@ def test_pool_topk_prefill_rows():
             assert idn[0, t, g].tolist() == oracle.topk(p, S)[0].tolist()
 
 
-def test_attend_decode_given_ids_and_dense():
+@pytest.mark.parametrize("case", [
+    dict(),                                              # D 128, block 64, k 6
+    dict(head_dim=64, block_size=128),                   # D 64 (the many-tile kernel's 64-key tiles)
+    dict(block_size=16, top_k=40),                       # k > 32 given: ids read by split; tiles of 16 keys
+    dict(head_dim=64, block_size=256, top_k=48),         # D 64, 256-token blocks, k > 32, lists mostly -1
+], ids=lambda c: ",".join(f"{k}={v}" for k, v in c.items()) or "base")
+def test_attend_decode_given_ids_and_dense(case):
     api = _api()
-    w = small(batch=4, max_seq_len=3000, top_k=6, hot_blocks=0)
+    w = small(batch=4, max_seq_len=3000, **{"top_k": 6, "hot_blocks": 0, **case})
     inp = make_inputs(w, device="cuda")
     x = to_np(inp)
     gen = np.random.default_rng(5)
