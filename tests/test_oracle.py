@@ -555,3 +555,22 @@ def test_kth_gap_reported(oracle_lib):
     assert ids.tolist() == [1, 2] and sc.tolist() == [5.0, 3.0] and kth == 3.0 and kn == 3.0
     ids, sc, kth, kn = oracle.topk(p, np.array([1.0]))
     assert ids.tolist() == [0, -1] and math.isnan(kth) and math.isnan(kn)
+
+
+@pytest.mark.parametrize("k", [33, 100, 1024])
+def test_large_k_topk_matches_twin(oracle_lib, k):
+    """TopK far beyond a warp list (the large-k regime): the C oracle's sort and the twin's rank
+    counting agree on rows with many exact ties, fewer blocks than k, and forced blocks."""
+    rng = np.random.default_rng(k)
+    for trial in range(12):
+        nb = int(rng.integers(1, 2500))
+        S = rng.integers(-20, 21, nb).astype(np.float64) if trial % 2 else rng.standard_normal(nb)
+        for force in (False, True):
+            cfg = make_cfg(top_k=k, force_sink_local=force)
+            got = COracle().topk(cfg, S)
+            want = Twin().topk(cfg, S)
+            np.testing.assert_array_equal(got, want)
+            sel = [n for n in got if n >= 0]
+            assert len(sel) == min(k, nb) and len(set(sel)) == len(sel)
+            if force:
+                assert got[0] == 0 and (nb == 1 or got[1] == nb - 1)
