@@ -6,9 +6,9 @@
 // touches about 6-7 % of the blocks at 1M tokens (k near 1000 of 16,384 blocks of 64 tokens),
 // far beyond what per-warp sorted lists hold.  One CTA per row forms every block's 64-bit key
 // (the score's order-preserving bits above the complemented id: all distinct, ordered as the
-// selection), finds the k-th largest key exactly by a radix select (passes of 8 bits with a
-// shared histogram each: four over the score bits, four more over the id bits only when blocks
-// tie at the k-th score), takes the k keys at or above it and sorts them once (bitonic).  Rows of
+// selection), finds the k-th largest key exactly by a radix select (a shared histogram per pass:
+// digits of 12, 12 and 8 bits over the score bits, the same over the id bits only when blocks tie
+// at the k-th score), takes the k keys at or above it and sorts them once (bitonic).  Rows of
 // up to 16,384 blocks keep their keys in registers; longer rows re-read the scores from global
 // memory in every pass (L2 keeps them).
 #include "msa_device.cuh"
@@ -28,9 +28,38 @@ __device__ inline float bits_score(uint32_t u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
+// Inclusive sum over the CTA of one value per thread; `tot` receives the total.
+__device__ inline int block_inclusive_sum(int v, int *warp_sums, int &tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(FULL, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) warp_sums[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int x = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(FULL, x, o);
+            if (lane >= o) x += u;
+        }
+        if (lane < nw) warp_sums[lane] = x;
+    }
+    __syncthreads();
+    tot = warp_sums[nw - 1];
+    const int before = warp > 0 ? warp_sums[warp - 1] : 0;
+    __syncthreads();  // warp_sums free again
+    return v + before;
+}
+
+constexpr int kHistBins = 4096;  // the widest digit: 12 bits
+
 __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTopkArgs a) {
     constexpr int KPT = 16;  // keys per thread held in registers (rows of up to 16,384 blocks)
-    __shared__ unsigned hist[256];
+    __shared__ unsigned hist[kHistBins];
+    __shared__ int warp_sums[32];
     __shared__ unsigned long long keys[kMaxTopK];
     __shared__ int st[4];  // [0] chosen digit, [1] remaining rank, [2] taken blocks, [3] prefix all taken
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
@@ -63,19 +92,27 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
         kr[j] = (in_regs && n < nb) ? key_of(n) : 0ull;
     }
 
-    // the kk-th largest key T (exactly): one 8-bit digit per pass, from the top
+    // the kk-th largest key T (exactly): digits of 12, 12 and 8 bits from the top, first over the
+    // score bits, then over the id bits when the k-th score is tied.  12-bit digits spread the
+    // first pass (sign, exponent and 3 mantissa bits) over more bins than 8 would.
     unsigned long long prefix = 0, mask = 0;
     int rem = kk;  // rank of T among the keys that match the prefix so far
     if (kk < nb) {
-        for (int shift = 56; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += nthr) hist[i] = 0;
+#pragma unroll 1
+        for (int ps = 0; ps < 6; ++ps) {
+            // passes 0-2: bits 63-52, 51-40, 39-32 (score); passes 3-5: bits 31-20, 19-8, 7-0 (id)
+            const int within = ps % 3;
+            const int shift = 32 * (1 - ps / 3) + (within == 0 ? 20 : within == 1 ? 8 : 0);
+            const int nbins = within == 2 ? 256 : 4096;
+            const unsigned dmask = (unsigned)nbins - 1u;
+            for (int i = tid; i < nbins; i += nthr) hist[i] = 0;
             __syncthreads();
             // lanes with the same digit add once (the high digits of nearby scores coincide, and
             // one atomic per lane would serialise on a few bins)
             auto count = [&](unsigned long long u, bool valid) {
-                const unsigned d = valid && (u & mask) == prefix ? ((unsigned)(u >> shift) & 255u) : 256u;
+                const unsigned d = valid && (u & mask) == prefix ? ((unsigned)(u >> shift) & dmask) : 0xffffffffu;
                 const unsigned peers = __match_any_sync(FULL, d);
-                if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
+                if (d != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
             };
             if (in_regs) {
 #pragma unroll
@@ -87,41 +124,38 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
                 }
             }
             __syncthreads();
-            if (warp == 0) {
-                // lane l holds digits 255 - 8 l .. 248 - 8 l (from the top)
-                unsigned c[8];
-                unsigned sum = 0;
+            // thread t sums the bins nbins - 1 - (t * bpt ... t * bpt + bpt - 1) (from the top); the
+            // thread whose running count crosses rem holds T's digit
+            const int bpt = nbins > nthr ? nbins / nthr : 1;
+            unsigned c[kHistBins / kLargeThreads];
+            unsigned sum = 0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    c[j] = hist[255 - 8 * lane - j];
-                    sum += c[j];
-                }
-                unsigned incl = sum;
+            for (int i = 0; i < kHistBins / kLargeThreads; ++i) {
+                const int bin = nbins - 1 - (tid * bpt + i);
+                c[i] = (i < bpt && bin >= 0) ? hist[bin] : 0u;
+                sum += c[i];
+            }
+            int tot = 0;
+            const unsigned incl = (unsigned)block_inclusive_sum((int)sum, warp_sums, tot);
+            const unsigned excl = incl - sum;
+            if (sum > 0 && excl < (unsigned)rem && (unsigned)rem <= incl) {
+                unsigned above = excl;
+                int d = nbins - 1 - tid * bpt;
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const unsigned u = __shfl_up_sync(FULL, incl, o);
-                    if (lane >= o) incl += u;
-                }
-                const unsigned excl = incl - sum;
-                if (excl < (unsigned)rem && (unsigned)rem <= incl) {
-                    unsigned above = excl;
-                    int d = 255 - 8 * lane;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (above + c[j] >= (unsigned)rem) {
-                            d = 255 - 8 * lane - j;
-                            break;
-                        }
-                        above += c[j];
+                for (int i = 0; i < kHistBins / kLargeThreads; ++i) {
+                    if (i < bpt && above + c[i] >= (unsigned)rem) {
+                        d = nbins - 1 - (tid * bpt + i);
+                        st[3] = c[i] == (unsigned)rem - above;  // every key with this prefix is taken
+                        break;
                     }
-                    st[0] = d;
-                    st[1] = rem - (int)above;
-                    st[3] = hist[d] == (unsigned)(rem - (int)above);  // every key with this prefix is taken
+                    above += c[i];
                 }
+                st[0] = d;
+                st[1] = rem - (int)above;
             }
             __syncthreads();
             prefix |= (unsigned long long)st[0] << shift;
-            mask |= 255ull << shift;
+            mask |= (unsigned long long)dmask << shift;
             rem = st[1];
             const bool all_taken = st[3] != 0;
             __syncthreads();
