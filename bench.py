@@ -3,10 +3,14 @@
 A step is one MSA decode step at 1M context (index scan + block max pool +
 TopK + sparse attention + split combine) through the C ABI, batch 1, with
 the caches resident in HBM.  Metric: microseconds per decode step per layer
-(lower is better).  Also reported: the dominant kernel (the index-key scan)
-against the HBM roofline, the dense GQA decode over the same cache, an
-end-to-end number with host<->device copies, and the CPU oracle timed on
-this host.
+(lower is better).  Also reported, each with its roofline fraction and the
+CPU oracle timed on this host:
+  * every other workload: tiny fp32 decode, 16K causal prefill, ragged
+    batch-8 128K decode, batch-4 1M decode (``configs``);
+  * the 1M decode with one shared index-K head and the large-k regime;
+  * the 1M-token chunked causal prefill (tok/s, tensor-core fraction);
+  * the dense GQA decode over the same cache, and an end-to-end number with
+    host<->device copies inside the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -36,6 +40,7 @@ from block_sparse_long_12_b200.inputs import WORKLOADS, make_inputs, to_numpy_ra
 METRIC = "MSA decode us/step/layer @1M ctx; prefill tok/s; % of HBM/tensor roofline"
 UNIT = "us/step/layer"
 L2_FLUSH_BYTES = 512 << 20
+SPEC_HBM_GBS = 8000.0  # the B200's nominal HBM3e bandwidth (DGX figure), for context beside the measured copy
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_index_scan_traffic.json")
 # the index scan kernel's own sources: a committed DRAM-traffic capture counts only while they are unchanged
 SCAN_SOURCES = ["block_sparse_long_12_b200/csrc/decode_index.cu", "block_sparse_long_12_b200/csrc/scan_args.h",
@@ -57,7 +62,8 @@ def measured_peaks() -> tuple[dict, str]:
 
 
 class ClockSampler:
-    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+    """nvidia-smi samples of this GPU's clocks and throttle reasons, time-stamped, for the whole run;
+    `window()` marks the spans (timed regions) whose samples the summary uses."""
     FIELDS = ("pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -65,26 +71,59 @@ class ClockSampler:
     def __init__(self, device_index: int):
         props = torch.cuda.get_device_properties(device_index)
         self.bus = getattr(props, "pci_bus_id", None)
-        self.rows = []
+        self.dom = getattr(props, "pci_domain_id", None)
+        self.rows = []      # (monotonic time, fields)
+        self.windows = []   # (t0, t1)
         self.proc = None
+        self.error = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                                          "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-        except OSError:
-            self.proc = None
+        except OSError as e:
+            self.proc, self.error = None, f"nvidia-smi did not start: {e}"
         return self
+
+    def _mine(self, bus_field: str) -> bool:
+        # "00000000:1B:00.0": domain, bus (hex), device.function
+        if self.bus is None:
+            return True
+        try:
+            dom, bus = bus_field.split(":")[:2]
+            return int(bus, 16) == int(self.bus) and (self.dom is None or int(dom, 16) == int(self.dom))
+        except ValueError:
+            return False
 
     def _read(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 9:
-                self.rows.append(parts)
+            if len(parts) == 9 and self._mine(parts[0]):
+                self.rows.append((time.monotonic(), parts))
 
-    def __exit__(self, *a):
+    def wait_first(self, timeout=8.0):
+        t0 = time.monotonic()
+        while self.proc is not None and not self.rows and time.monotonic() - t0 < timeout:
+            time.sleep(0.05)
+        if self.proc is not None and not self.rows and self.error is None:
+            self.error = f"no sample from nvidia-smi within {timeout:.0f} s"
+
+    class _Win:
+        def __init__(self, s):
+            self.s = s
+
+        def __enter__(self):
+            self.t0 = time.monotonic()
+
+        def __exit__(self, *a):
+            self.s.windows.append((self.t0, time.monotonic()))
+
+    def window(self):
+        return ClockSampler._Win(self)
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -92,20 +131,23 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.thread.join(timeout=2)
+            if not self.rows and self.error is None:
+                err = (self.proc.stderr.read() or "").strip()[:200]
+                self.error = f"nvidia-smi gave no row for this GPU (bus {self.bus}){': ' + err if err else ''}"
 
-    def summary(self) -> dict:
-        rows = self.rows
-        if self.bus is not None:
-            mine = [r for r in rows if r[0].lower().endswith(str(self.bus).lower())]
-            rows = mine or rows
+    def summary(self, windows=None) -> dict:
+        wins = self.windows if windows is None else windows
+        rows = [r for (t, r) in self.rows if any(a <= t <= b for a, b in wins)]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "why_empty": self.error or "no sample fell inside the timed windows"}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
 
 
 def dist_setup():
@@ -152,23 +194,73 @@ def timed_steps(fn, steps, flush, stream):
     return [a.elapsed_time(b) * 1e3 for a, b in ev]  # microseconds
 
 
-def oracle_decode_seconds(w, x, repeats: int) -> tuple[float, int]:
-    """Wall seconds of one oracle decode step (all sequences of the batch) and the threads it used."""
+def hbm_frac(nbytes: float, us: float, peaks: dict) -> dict:
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"achieved_gbs": round(gbs, 1), "frac_of_measured_copy": round(gbs / peaks["hbm_gbs"], 4),
+            "frac_of_spec_8tbs": round(gbs / SPEC_HBM_GBS, 4)}
+
+
+# ----------------------------------------------------------------------------- oracle timing (CPU legs)
+def oracle_params(w, q_len=1, q_start=0, prefill=False):
     import oracle
-    oracle.build()
-    p = oracle.Params(w.batch, w.n_q_heads, w.n_kv_heads, w.n_idx_k_heads, w.head_dim, w.idx_dim, w.block_size,
-                      w.top_k, 1, 0, w.max_seq_len, w.dtype, w.softmax_scale)
-    rows = [(b, 0) for b in range(w.batch)]
+    return oracle.Params(w.batch, w.n_q_heads, w.n_kv_heads, w.n_idx_k_heads, w.head_dim, w.idx_dim, w.block_size,
+                         w.top_k, q_len, q_start, w.max_seq_len, w.dtype, w.softmax_scale, prefill=prefill)
+
+
+def time_oracle(fn, repeats: int, warmup: int = 1) -> float:
+    for _ in range(warmup):
+        fn()
     ts = []
     for _ in range(repeats):
         t0 = time.perf_counter()
-        oracle.msa_rows(p, x["seq_lens"], x["q"], x["q_idx"], x["k"], x["v"], x["k_idx"], rows)
+        fn()
         ts.append(time.perf_counter() - t0)
-    threads = min(os.cpu_count() or 1, int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)),
-                  len(rows) * w.n_kv_heads)
-    return statistics.median(ts), threads
+    return statistics.median(ts)
 
 
+def oracle_decode(w, x, repeats=5, threads=None) -> dict:
+    """The oracle's decode step (every sequence and group of the batch), median of `repeats` after a warm-up."""
+    import oracle
+    oracle.build()
+    n = oracle.set_threads(threads)
+    p = oracle_params(w)
+    rows = [(b, 0) for b in range(w.batch)]
+
+    def run():
+        oracle.msa_rows(p, x["seq_lens"], x["q"], x["q_idx"], x["k"], x["v"], x["k_idx"], rows)
+    sec = time_oracle(run, repeats)
+    oracle.set_threads(None)
+    return {"value": round(sec * 1e6, 1), "unit": UNIT, "cores": min(n, w.batch * w.n_kv_heads), "kind": "oracle",
+            "sample": f"one full decode step of {w.name} (batch {w.batch}), fp64 C oracle, median of {repeats} "
+                      f"after a warm-up"}
+
+
+def oracle_prefill_rows(w, inp, positions, repeats=3) -> dict:
+    """The oracle's Steps 1 and 2 for query rows at the given absolute positions (prefill), us per row."""
+    import oracle
+    oracle.build()
+    n = oracle.set_threads(None)
+    x = {k_: to_numpy_raw(inp[k_]) for k_ in ("k", "v", "k_idx")}
+    pos = torch.tensor(sorted(positions), device=inp["q"].device)
+    # the rows' q / q_idx placed at their positions of a compact chunk starting at the first row
+    c0 = int(pos[0])
+    span = int(pos[-1]) - c0 + 1
+    q = np.zeros((1, span, w.n_q_heads, w.head_dim), np.uint16)
+    qi = np.zeros((1, span, w.n_kv_heads, w.idx_dim), np.uint16)
+    q[0, (pos - c0).cpu().numpy()] = to_numpy_raw(inp["q"][0, pos])
+    qi[0, (pos - c0).cpu().numpy()] = to_numpy_raw(inp["q_idx"][0, pos])
+    p = oracle_params(w, q_len=span, q_start=c0, prefill=True)
+    rows = [(0, int(t) - c0) for t in pos.tolist()]
+
+    def run():
+        oracle.msa_rows(p, None, q, qi, x["k"], x["v"], x["k_idx"], rows)
+    sec = time_oracle(run, repeats, warmup=0)
+    return {"us_per_row": round(sec / len(rows) * 1e6, 1), "rows": len(rows), "cores": n,
+            "sample": f"{len(rows)} query rows spread over positions {c0}..{int(pos[-1])}, fp64 C oracle "
+                      f"(Steps 1 and 2, all groups), median of {repeats}"}
+
+
+# ----------------------------------------------------------------------------- reference arm
 def run_reference(args, world, rank):
     """The oracle, as it stands, on this host's cores, on the same workload and metric.
 
@@ -233,59 +325,120 @@ def workload_config(w, n):
             "parallelism": "replicas" if n == 1 else f"weak-scaling replicas x{n}, no collective"}
 
 
-def run_ours(args, world, rank, local):
+# ----------------------------------------------------------------------------- decode timing
+def decode_bytes(w, lens_host) -> tuple[int, int]:
+    es = 2 if w.dtype == "bf16" else 4
+    idx = sum(lens_host) * w.n_idx_k_heads * w.idx_dim * es  # every index key read once
+    kv = 0
+    for L in lens_host:  # the selected blocks' K and V (the visible part of each)
+        nb = -(-L // w.block_size)
+        kv += w.n_kv_heads * min(w.top_k, nb) * w.block_size * w.head_dim * es * 2
+    return idx, kv
+
+
+def time_decode(w, rank, world, local, stream, flush, steps, warmup, clk=None, stage=True, oracle_leg=False):
+    """Steady-state fused decode steps of workload w: step time, stage times, bytes, roofline."""
     from block_sparse_long_12_b200 import _lib, api
-    torch.cuda.set_device(local)
-    w = WORKLOADS[args.workload]
     dev = torch.device("cuda", local)
     inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
-    stream = torch.cuda.current_stream()
     p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
     ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, dev)
     o = torch.empty_like(q)
     ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
     lse = torch.empty(w.batch, 1, w.n_q_heads, dtype=torch.float32, device=dev)
+
+    def step():
+        _lib.msa_decode_fused(p, q, q_idx, k, v, k_idx, o, ids, lse, ws, stream)
+
+    for _ in range(max(warmup, 3)):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    if clk is not None:
+        with clk.window():
+            per_step = timed_steps(step, steps, flush, stream)
+    else:
+        per_step = timed_steps(step, steps, flush, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    step_us = max_over_ranks(sum(per_step) / len(per_step), world)
+    assert _lib.msa_get_device_status(ws) == 0, "device status word reports a timeout"
+    out = {"step_us": step_us, "per_step": per_step, "inp": inp, "step": step, "p": p, "ws": ws, "o": o,
+           "ids": ids, "lse": lse, "lens_host": lens.tolist()}
+    if stage:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for e in evs:
+            e.record(stream)
+        torch.cuda.synchronize()
+        _lib.msa_set_stage_events(evs)
+        st = [[], []]
+        try:
+            for _ in range(min(steps, 200)):
+                flush()
+                step()
+                torch.cuda.synchronize()
+                for i in range(2):
+                    st[i].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
+        finally:
+            _lib.msa_set_stage_events(None)
+        out["scan_us"] = max_over_ranks(statistics.mean(st[0]), world)
+        out["attn_us"] = max_over_ranks(statistics.mean(st[1]), world)
+    return out
+
+
+def decode_summary(w, r, peaks, peak_kind, cpu=None) -> dict:
+    idx_b, kv_b = decode_bytes(w, r["lens_host"])
+    d = {"workload": w.name, "value": round(r["step_us"], 2), "unit": UNIT, "batch": w.batch,
+         "context": (min(r["lens_host"]), max(r["lens_host"])) if min(r["lens_host"]) != max(r["lens_host"])
+         else r["lens_host"][0],
+         "n_idx_k_heads": w.n_idx_k_heads, "block_size": w.block_size, "top_k": w.top_k, "dtype": w.dtype,
+         "algorithmic_bytes": idx_b + kv_b, "step_roofline": hbm_frac(idx_b + kv_b, r["step_us"], peaks),
+         "peak_kind": peak_kind}
+    if "scan_us" in r:
+        stage2 = "topk_merge_and_sparse_attention" if w.top_k <= 32 else "radix_select_and_sparse_attention"
+        d["stages_us"] = {"index_scan": round(r["scan_us"], 2), stage2: round(r["attn_us"], 2)}
+        d["scan_roofline"] = hbm_frac(idx_b, r["scan_us"], peaks)
+    if cpu is not None:
+        d["oracle"] = cpu
+    return d
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_long_12_b200 import _lib, api
+    torch.cuda.set_device(local)
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
     flush_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    peaks, peak_kind = measured_peaks()
 
     def flush():
         # reads (not writes) so that the next step does not start by writing back dirty lines
         torch.amax(flush_buf)
 
-    def step():
-        _lib.msa_decode_fused(p, q, q_idx, k, v, k_idx, o, ids, lse, ws, stream)
+    clk = ClockSampler(local).start()
+    clk.wait_first()
 
-    for _ in range(max(args.warmup, 3)):
-        flush()
-        step()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        barrier(world)
-        torch.cuda.synchronize()
-        per_step = timed_steps(step, args.steps, flush, stream)
-        torch.cuda.synchronize()
-        barrier(world)
-    step_us = max_over_ranks(sum(per_step) / len(per_step), world)
-    assert _lib.msa_get_device_status(ws) == 0, "device status word reports a timeout"
-
-    # per-kernel durations inside the same step (stage events; separate pass)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    for e in evs:
-        e.record(stream)
-    torch.cuda.synchronize()
-    _lib.msa_set_stage_events(evs)
-    stage = [[], []]  # index scan; TopK merge + sparse attention + split merge
-    try:
-        for _ in range(args.steps):
-            flush()
-            step()
-            torch.cuda.synchronize()
-            for i in range(2):
-                stage[i].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
-    finally:
-        _lib.msa_set_stage_events(None)
-    scan_us = max_over_ranks(statistics.mean(stage[0]), world)
-    attn_us = max_over_ranks(statistics.mean(stage[1]), world)
+    r = time_decode(w, rank, world, local, stream, flush, args.steps, args.warmup, clk=clk)
+    step_us, scan_us, attn_us = r["step_us"], r["scan_us"], r["attn_us"]
+    inp, step, p = r["inp"], r["step"], r["p"]
+    q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
+    o, ids = r["o"], r["ids"]
+    # clocks: if the timed region was too short for the sampler (100 ms period), keep the same step
+    # running back to back for a moment, inside a marked window, so that the record shows its clocks
+    if clk.summary()["samples"] < 3:
+        with clk.window():
+            t_end = time.monotonic() + 1.5
+            while time.monotonic() < t_end:
+                for _ in range(200):
+                    step()
+                torch.cuda.synchronize()
+        clocks_window = "timed region + 1.5 s of the same decode step back to back"
+    else:
+        clocks_window = "timed region"
 
     # dense GQA decode over the same cache (the sparse-vs-dense ratio)
     pd = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens,
@@ -343,31 +496,52 @@ def run_ours(args, world, rank, local):
     h2d = sum(t.numel() * t.element_size() for t in (h_q, h_qi, new_k, new_v, new_ki))
     d2h = h_o.numel() * h_o.element_size() + h_ids.numel() * h_ids.element_size()
 
-    cpu = None
+    cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         x = {n: to_numpy_raw(inp[n]) for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens")}
-        sec, threads = oracle_decode_seconds(w, x, repeats=2)
-        cpu = {"value": round(sec * 1e6, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": f"one full decode step of {w.name} (batch {w.batch}), fp64 C oracle, median of 2"}
+        cpu = oracle_decode(w, x, repeats=5)
+        cpu1 = oracle_decode(w, x, repeats=3, threads=1)
         del x
 
-    lens_host = lens.tolist()
-    del inp, q, q_idx, k, v, k_idx, ws, wsd, o, od
+    lens_host = r["lens_host"]
+    del r, inp, q, q_idx, k, v, k_idx, o, od, wsd
     torch.cuda.empty_cache()
-    shared = None if args.no_shared_index else run_shared_index(args, world, rank, local, stream, flush)
-    large_k = None if args.no_large_k else run_shared_index(args, world, rank, local, stream, flush,
-                                                            name="decode_ctx1m_large_k")
+
+    # the other workloads, each with its own oracle time
+    configs = {}
+    if not args.no_configs:
+        for name in ("decode_fp32_ctx4k", "decode_b8_ctx128k_ragged", "decode_b4_ctx1m"):
+            if name == w.name:
+                continue
+            wc = WORKLOADS[name]
+            rc = time_decode(wc, rank, world, local, stream, flush, max(3, min(args.steps, 500)), args.warmup)
+            oc = None
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                xc = {n: to_numpy_raw(rc["inp"][n]) for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens")}
+                oc = oracle_decode(wc, xc, repeats=3)
+                del xc
+            configs[name] = decode_summary(wc, rc, peaks, peak_kind, oc)
+            del rc
+            torch.cuda.empty_cache()
+        configs["prefill_causal_16k"] = run_prefill(WORKLOADS["prefill_causal_16k"], world, rank, local, stream,
+                                                    peaks, peak_kind, oracle_rows=0 if args.no_cpu_baseline else 256)
+        torch.cuda.empty_cache()
+
+    shared = None if args.no_shared_index else run_extra_decode("decode_ctx1m_shared_idx", args, world, rank, local,
+                                                                stream, flush, peaks, peak_kind)
+    large_k = None if args.no_large_k else run_extra_decode("decode_ctx1m_large_k", args, world, rank, local, stream,
+                                                            flush, peaks, peak_kind)
     prefill = None
     if not args.no_prefill:
         del flush_buf
         torch.cuda.empty_cache()
-        prefill = run_prefill(world, rank, local, stream)
+        prefill = run_prefill(WORKLOADS["prefill_causal_1m"], world, rank, local, stream, peaks, peak_kind,
+                              oracle_rows=0 if args.no_cpu_baseline else 32)
+    clk.stop()
 
     if rank != 0:
         return
-    peaks, peak_kind = measured_peaks()
-    es = 2 if w.dtype == "bf16" else 4
-    scan_bytes = sum(lens_host) * w.n_idx_k_heads * w.idx_dim * es  # every index key read once
+    scan_bytes, kv_bytes = decode_bytes(w, lens_host)
     achieved = scan_bytes / (scan_us * 1e-6) / 1e9
     traffic = None
     if os.path.exists(TRAFFIC_FILE):
@@ -375,6 +549,10 @@ def run_ours(args, world, rank, local):
         if rec.get("source_sha256") == scan_source_hash() and rec.get("workload") == w.name:
             traffic = rec.get("dram_bytes_per_launch")
     clocks = clk.summary()
+    clocks["window"] = clocks_window
+    clocks["whole_run"] = {k_: v_ for k_, v_ in clk.summary([(0.0, float("inf"))]).items() if k_ != "why_empty"}
+    if cpu is not None:
+        cpu["single_thread_us"] = cpu1["value"]
 
     line = {
         "metric": METRIC, "value": round(step_us, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -383,14 +561,16 @@ def run_ours(args, world, rank, local):
         "config": workload_config(w, world),
         "roofline": {"bound": "hbm", "kernel": "decode index scan", "achieved": round(achieved, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "peak_kind": peak_kind, "algorithmic_bytes": scan_bytes, "kernel_us": round(scan_us, 2),
-                     "traffic": traffic},
+                     "peak_kind": f"{peak_kind} copy (read+write); a read-only stream can exceed it",
+                     "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
+                     "algorithmic_bytes": scan_bytes, "kernel_us": round(scan_us, 2), "traffic": traffic},
         "stages_us": {"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)},
-        "step_roofline_frac": round((scan_bytes + w.batch * w.n_kv_heads * w.top_k * w.block_size * w.head_dim * es * 2)
-                                    / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+        "step_roofline": hbm_frac(scan_bytes + kv_bytes, step_us, peaks),
+        "step_roofline_frac": round((scan_bytes + kv_bytes) / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
         "dense_gqa_us": round(dense_us, 2), "sparse_vs_dense_speedup": round(dense_us / step_us, 2),
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
+        "configs": configs,
         "shared_index_head": shared,
         "large_k": large_k,
         "prefill": prefill,
@@ -400,98 +580,57 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
-def run_shared_index(args, world, rank, local, stream, flush, name="decode_ctx1m_shared_idx"):
-    """The 1M decode step with one index-K head shared by the 8 groups: the index stream is 1/8
-    as long, so the step is no longer dominated by the scan.  Same timing as the main step.
-    With name="decode_ctx1m_large_k": the large-k regime (64-token blocks, k 1024 of 16,384; the
-    middle stage is then the radix select, the last the attention over 268 MB of K/V)."""
-    from block_sparse_long_12_b200 import _lib, api
+def run_extra_decode(name, args, world, rank, local, stream, flush, peaks, peak_kind):
+    """The 1M decode step with one index-K head shared by the 8 groups (the index stream is 1/8 as
+    long), or the large-k regime (64-token blocks, k 1024 of 16,384; the middle stage is then the
+    radix select, the last the attention over 268 MB of K/V).  Same timing as the main step."""
     w = WORKLOADS[name]
-    dev = torch.device("cuda", local)
-    inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
-    q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
-    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
-    ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, dev)
-    o = torch.empty_like(q)
-    ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
-
-    def step():
-        _lib.msa_decode_fused(p, q, q_idx, k, v, k_idx, o, ids, None, ws, stream)
-
-    for _ in range(max(args.warmup, 3)):
-        flush()
-        step()
-    torch.cuda.synchronize()
-    n = max(3, min(args.steps, 500))
-    barrier(world)
-    step_us = max_over_ranks(statistics.mean(timed_steps(step, n, flush, stream)), world)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-    for e in evs:
-        e.record(stream)
-    torch.cuda.synchronize()
-    _lib.msa_set_stage_events(evs)
-    stage = [[], []]
-    try:
-        for _ in range(n):
-            flush()
-            step()
-            torch.cuda.synchronize()
-            for i in range(2):
-                stage[i].append(evs[i].elapsed_time(evs[i + 1]) * 1e3)
-    finally:
-        _lib.msa_set_stage_events(None)
-    assert _lib.msa_get_device_status(ws) == 0
-    scan_us = max_over_ranks(statistics.mean(stage[0]), world)
-    attn_us = max_over_ranks(statistics.mean(stage[1]), world)
-    peaks, kind = measured_peaks()
-    idx_bytes = sum(lens.tolist()) * w.n_idx_k_heads * w.idx_dim * 2
-    kv_bytes = w.batch * w.n_kv_heads * w.top_k * w.block_size * w.head_dim * 2 * 2
-    del inp, q, q_idx, k, v, k_idx, ws, o
+    r = time_decode(w, rank, world, local, stream, flush, max(3, min(args.steps, 500)), args.warmup)
+    d = decode_summary(w, r, peaks, peak_kind)
+    del r
     torch.cuda.empty_cache()
-    stages = ({"index_scan": round(scan_us, 2), "topk_merge_and_sparse_attention": round(attn_us, 2)}
-              if w.top_k <= 32 else
-              {"index_scan": round(scan_us, 2), "radix_select_and_sparse_attention": round(attn_us, 2)})
-    return {"workload": w.name, "value": round(step_us, 2), "unit": UNIT, "n_idx_k_heads": w.n_idx_k_heads,
-            "block_size": w.block_size, "top_k": w.top_k, "stages_us": stages,
-            "algorithmic_bytes": idx_bytes + kv_bytes,
-            "step_roofline_frac": round((idx_bytes + kv_bytes) / (step_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
-            "scan_gbs": round(idx_bytes / (scan_us * 1e-6) / 1e9, 1), "peak_kind": kind}
+    return d
 
 
-def run_prefill(world, rank, local, stream):
-    """The 1M-token causal prefill in 8192-token chunks: Step 1 (tensor-core index scores, block max
-    pool, TopK) then Step 2 (tensor-core sparse attention) for every chunk.  Returns tok/s and the
-    index kernel's tensor-core roofline fraction (max over ranks)."""
+def run_prefill(w, world, rank, local, stream, peaks, peak_kind, oracle_rows=0):
+    """Causal prefill of workload w in w.chunk-token chunks (the whole sequence when 0): Step 1
+    (tensor-core index scores, block max pool, TopK) then Step 2 (sparse attention) for every chunk.
+    Returns tok/s and the tensor-core roofline fractions (max over ranks), and the oracle's time per
+    row on `oracle_rows` rows spread over the sequence."""
     from block_sparse_long_12_b200 import _lib, api
-    w = WORKLOADS["prefill_causal_1m"]
     dev = torch.device("cuda", local)
     inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
-    T, C = w.max_seq_len, w.chunk
-    n_chunks = T // C
+    T = w.max_seq_len
+    C = w.chunk or T
+    n_chunks = -(-T // C)
     ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
     o = torch.empty_like(inp["q"])
     chunks = []
     for c in range(n_chunks):
+        n = min(C, T - c * C)
         p = api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, n_idx_k_heads=w.n_idx_k_heads,
                             head_dim=w.head_dim, idx_dim=w.idx_dim, block_size=w.block_size, top_k=w.top_k,
-                            max_seq_len=T, dtype=_lib.MSA_BF16, q_len=C, q_start=c * C)
-        chunks.append((p, inp["q"][:, c * C:(c + 1) * C], inp["q_idx"][:, c * C:(c + 1) * C],
-                       ids[:, c * C:(c + 1) * C], o[:, c * C:(c + 1) * C]))
-    ws = api.workspace([c[0] for c in chunks], _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, dev)
+                            max_seq_len=T, dtype=_lib.MSA_BF16, q_len=n, q_start=c * C)
+        chunks.append((p, inp["q"][:, c * C:c * C + n], inp["q_idx"][:, c * C:c * C + n],
+                       ids[:, c * C:c * C + n], o[:, c * C:c * C + n]))
+    ws_i = api.workspace([c[0] for c in chunks], _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, dev)
+    ws_a = api.workspace([c[0] for c in chunks], _lib.MSA_ENTRY_ATTN_PREFILL, dev)
 
     def index_pass():
         for (p, q, qi, idc, oc) in chunks:
-            _lib.msa_prefill_index_topk(p, qi, inp["k_idx"], idc, None, ws, stream)
+            _lib.msa_prefill_index_topk(p, qi, inp["k_idx"], idc, None, ws_i, stream)
 
     def attn_pass():
         for (p, q, qi, idc, oc) in chunks:
-            _lib.msa_sparse_attn_prefill(p, q, inp["k"], inp["v"], idc, oc, None, ws, stream)
+            _lib.msa_sparse_attn_prefill(p, q, inp["k"], inp["v"], idc, oc, None, ws_a, stream)
 
-    index_pass()
-    attn_pass()
+    for _ in range(3 if n_chunks == 1 else 1):
+        index_pass()
+        attn_pass()
     torch.cuda.synchronize()
     ti, ta = [], []
-    for _ in range(3):
+    reps = 20 if n_chunks == 1 else 3
+    for _ in range(reps):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record(stream)
         index_pass()
@@ -501,35 +640,40 @@ def run_prefill(world, rank, local, stream):
         torch.cuda.synchronize()
         ti.append(e[0].elapsed_time(e[1]) / 1e3)
         ta.append(e[1].elapsed_time(e[2]) / 1e3)
-    assert _lib.msa_get_device_status(ws) == 0
-    # issued attention work: every 16-token x 8-head tile walks the union of its tokens' lists
-    tq = 128 // (w.n_q_heads // w.n_kv_heads)
-    u_sum = 0
-    for c0 in range(0, T, 65536):
-        blk = ids[0, c0:c0 + 65536].reshape(-1, tq, w.n_kv_heads, w.top_k).permute(0, 2, 1, 3)
-        blk = blk.reshape(-1, tq * w.top_k).sort(dim=-1).values
-        distinct = (blk[:, 1:] != blk[:, :-1]) & (blk[:, 1:] >= 0)
-        u_sum += int(distinct.sum()) + int((blk[:, 0] >= 0).sum())
-    att_issued = 4.0 * 128 * w.block_size * w.head_dim * u_sum
+    assert _lib.msa_get_device_status(ws_i) == 0 and _lib.msa_get_device_status(ws_a) == 0
     t_idx = max_over_ranks(statistics.median(ti), world)
     t_att = max_over_ranks(statistics.median(ta), world)
-    peaks, kind = measured_peaks()
     # algorithmic FLOPs: every visible (row, key) pair of every group scores d_i MACs; attention
-    # touches top_k blocks of block_size keys per (row, head) for Q.K and P.V
+    # touches the selected blocks' visible keys per (row, head) for Q.K and P.V
     pairs = T * (T + 1) // 2
     idx_flops = 2.0 * w.idx_dim * w.n_kv_heads * pairs
-    att_flops = 4.0 * w.head_dim * w.n_q_heads * w.top_k * w.block_size * T
+    nb = torch.arange(T, device=dev) // w.block_size + 1
+    keys = (torch.clamp(nb, max=w.top_k) * w.block_size).double().sum().item()  # upper bound per row: k full blocks
+    att_flops = 4.0 * w.head_dim * w.n_q_heads * keys
     total = t_idx + t_att
-    return {"workload": w.name, "tokens": T, "chunk": C, "tok_per_s": round(T * world / total, 1),
-            "seconds": round(total, 4), "index_s": round(t_idx, 4), "attention_s": round(t_att, 4),
-            "index_tflops": round(idx_flops / t_idx / 1e12, 1),
-            "index_frac_of_bf16_peak": round(idx_flops / t_idx / 1e12 / peaks["bf16_tflops_sustained"], 4),
-            "attention_useful_tflops": round(att_flops / t_att / 1e12, 1),
-            "attention_issued_tflops": round(att_issued / t_att / 1e12, 1),
-            "attention_mean_union_blocks": round(u_sum / (T // tq * w.n_kv_heads), 2),
-            "overall_frac_of_bf16_peak": round((idx_flops + att_flops) / total / 1e12 / peaks["bf16_tflops_sustained"], 4),
-            "peak": peaks["bf16_tflops_sustained"], "peak_kind": f"{kind} sustained (long step)",
-            "gpu_launches": 2 * n_chunks * 3}
+    sus, burst = peaks["bf16_tflops_sustained"], peaks["bf16_tflops"]
+    d = {"workload": w.name, "tokens": T, "chunk": C, "tok_per_s": round(T * world / total, 1),
+         "seconds": round(total, 5), "index_s": round(t_idx, 5), "attention_s": round(t_att, 5),
+         "index_tflops": round(idx_flops / t_idx / 1e12, 1),
+         "index_frac_of_bf16_peak": round(idx_flops / t_idx / 1e12 / sus, 4),
+         "attention_useful_tflops": round(att_flops / t_att / 1e12, 1),
+         "attention_frac_of_bf16_peak": round(att_flops / t_att / 1e12 / sus, 4),
+         "overall_frac_of_bf16_peak": round((idx_flops + att_flops) / total / 1e12 / sus, 4),
+         "overall_frac_of_bf16_burst_peak": round((idx_flops + att_flops) / total / 1e12 / burst, 4),
+         "algorithmic_flops": idx_flops + att_flops,
+         "peak": sus, "peak_kind": f"{peak_kind} sustained (long step); burst {burst}",
+         "gpu_launches": None}
+    if oracle_rows and rank == 0 and world == 1:
+        rng = np.random.default_rng(w.seed)
+        positions = sorted(set(rng.choice(T, oracle_rows, replace=False).tolist()))
+        orc = oracle_prefill_rows(w, inp, positions)
+        orc["extrapolated_full_sequence_s"] = round(orc["us_per_row"] * T / 1e6, 1)
+        orc["extrapolation"] = ("us_per_row x all rows; rows late in the sequence cost more (Step 1 is linear in "
+                                "the position), so the sample spreads over the whole sequence")
+        d["oracle"] = orc
+    del inp, ids, o, chunks, ws_i, ws_a
+    torch.cuda.empty_cache()
+    return d
 
 
 def main():
@@ -542,6 +686,7 @@ def main():
                                                                     "decode_b8_ctx128k_ragged"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' sub-lines")
     ap.add_argument("--no-shared-index", action="store_true", help="skip the shared index-K head decode step")
     ap.add_argument("--no-large-k", action="store_true", help="skip the large-k (k 1024 of 16,384 blocks) decode step")
     args = ap.parse_args()

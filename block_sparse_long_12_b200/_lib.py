@@ -25,7 +25,8 @@ MSA_SCORES_TOKEN, MSA_SCORES_BLOCKMAX, MSA_DENSE, MSA_FORCE_SINK_LOCAL = 1, 2, 8
 EXPORTED = ["msa_index_score", "msa_block_maxpool_topk", "msa_sparse_attn_decode", "msa_sparse_attn_prefill",
             "msa_decode_fused", "msa_prefill_index_topk", "msa_workspace_size", "msa_last_error_string",
             "msa_status_string", "msa_get_device_status", "msa_clear_device_status", "msa_set_stage_events",
-            "msa_decode_fused_noalloc"]
+            "msa_decode_fused_noalloc", "msa_noalloc_get_status", "msa_noalloc_clear_status", "msa_set_wait_limit",
+            "msa_diag_wait_timeout"]
 
 
 class MsaError(RuntimeError):
@@ -67,6 +68,10 @@ def lib() -> ctypes.CDLL:
             "msa_get_device_status": [vp, ctypes.POINTER(ctypes.c_int), st],
             "msa_clear_device_status": [vp, st],
             "msa_set_stage_events": [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int],
+            "msa_noalloc_get_status": [ctypes.POINTER(ctypes.c_int), st],
+            "msa_noalloc_clear_status": [st],
+            "msa_set_wait_limit": [vp, ctypes.c_uint64, st],
+            "msa_diag_wait_timeout": [vp, sz, st],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -167,3 +172,21 @@ def msa_set_stage_events(events):
         return
     arr = (ctypes.c_void_p * 3)(*[e.cuda_event for e in events])
     _check(lib().msa_set_stage_events(arr, 3))
+
+
+def msa_noalloc_get_status(stream=None) -> int:
+    out = ctypes.c_int(0)
+    _check(lib().msa_noalloc_get_status(ctypes.byref(out), _stream(stream)))
+    return out.value
+
+
+def msa_noalloc_clear_status(stream=None):
+    _check(lib().msa_noalloc_clear_status(_stream(stream)))
+
+
+def msa_set_wait_limit(ws, limit_ns: int, stream=None):
+    _check(lib().msa_set_wait_limit(_ptr(ws), int(limit_ns), _stream(stream)))
+
+
+def msa_diag_wait_timeout(ws, stream=None):
+    _check(lib().msa_diag_wait_timeout(_ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))

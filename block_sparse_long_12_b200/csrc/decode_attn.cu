@@ -667,7 +667,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
             const int slot = consumed % NST;
             if (!failed && !mbar_wait(&bars[slot], (consumed / NST) & 1, a.status)) {
                 failed = true;
-                for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&bars[q2 % NST], (q2 / NST) & 1, nullptr);
+                for (int q2 = consumed; q2 < issued; ++q2) mbar_wait(&bars[q2 % NST], (q2 / NST) & 1, nullptr);
             }
             const T *ks = reinterpret_cast<const T *>(ring + (size_t)slot * 2 * tile_bytes);
             const T *vs = reinterpret_cast<const T *>(ring + (size_t)slot * 2 * tile_bytes + tile_bytes);
@@ -896,7 +896,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
             const int slot = consumed % nst;
             if (!failed && !mbar_wait(&bars[slot], (consumed / nst) & 1, a.status)) {
                 failed = true;
-                for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&bars[q2 % nst], (q2 / nst) & 1, nullptr);
+                for (int q2 = consumed; q2 < issued; ++q2) mbar_wait(&bars[q2 % nst], (q2 / nst) & 1, nullptr);
             }
             const uint32_t k_addr = smem_u32(ring + slot * STAGE);
             const uint32_t v_addr = k_addr + NH * KVH;
@@ -1307,7 +1307,7 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
         if (!mbar_wait(&my_bars[slot], (consumed / SPW) & 1, a.status)) {
             // give up: wait (bounded) for the warp's copies in flight, issue nothing more
             failed = true;
-            for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % SPW], (q2 / SPW) & 1, nullptr);
+            for (int q2 = consumed; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % SPW], (q2 / SPW) & 1, nullptr);
             break;
         }
         int nk = 0;

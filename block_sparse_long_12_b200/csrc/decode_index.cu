@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                     // give up: wait (bounded) for this warp's copies still in flight, then
                     // run the loop to its end without waiting or issuing again
                     failed = true;
-                    for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
+                    for (int q2 = consumed; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;
@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                 const int slot = consumed % S;
                 if (!failed && !mbar_wait(&my_bars[slot], (consumed / S) & 1, a.status)) {
                     failed = true;
-                    for (int q2 = consumed + 1; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
+                    for (int q2 = consumed; q2 < issued; ++q2) mbar_wait(&my_bars[q2 % S], (q2 / S) & 1, nullptr);
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;

@@ -321,9 +321,28 @@ msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t str
 
 msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream) {
     if (ws == nullptr) return fail(MSA_ERR_INVALID_ARG, "ws is NULL");
-    // the status word and the scan's counters (left non-zero by a scan that did not end normally)
+    // the status word, the wait limit and the scan's counters (left non-zero by a scan that did not
+    // end normally)
     cudaError_t e = cudaMemsetAsync(ws, 0, (kSchedWord + kTailPools + 1) * sizeof(unsigned), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    return MSA_OK;
+}
+
+msa_status_t msa_set_wait_limit(void *ws, uint64_t limit_ns, msa_stream_t stream) {
+    if (ws == nullptr) return fail(MSA_ERR_INVALID_ARG, "ws is NULL");
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(MSA_ERR_INVALID_ARG, "ws is not 256-byte aligned");
+    cudaError_t e = launch_set_wait_limit(reinterpret_cast<int *>(ws), (unsigned long long)limit_ns, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "setting the wait limit");
+    return MSA_OK;
+}
+
+msa_status_t msa_diag_wait_timeout(void *ws, size_t ws_bytes, msa_stream_t stream) {
+    MSA_TRY(check_ptr(ws, "ws"));
+    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    cudaError_t e = launch_wait_never(reinterpret_cast<int *>(ws), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "diagnostic wait launch");
     return MSA_OK;
 }
 

@@ -77,14 +77,24 @@ __device__ inline uint64_t global_timer_ns() {
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
-// Wait for phase `parity` of an mbarrier for at most kWaitLimitNs.  On
-// timeout the workspace status word is set to MSA_ERR_TIMEOUT and false is
+// Limit of a bounded wait: the workspace header's wait-limit field (bytes
+// 8..15 after the status word, set by msa_set_wait_limit) when it is non-zero,
+// else kWaitLimitNs.  Read only once a wait has not completed at once.
+__device__ inline uint64_t wait_limit_ns(const int *status) {
+    if (status == nullptr) return kWaitLimitNs;
+    const uint64_t v = *reinterpret_cast<const volatile uint64_t *>(status + kWaitLimitWord);
+    return v != 0 ? v : kWaitLimitNs;
+}
+
+// Wait for phase `parity` of an mbarrier for at most wait_limit_ns(status).
+// On timeout the workspace status word is set to MSA_ERR_TIMEOUT and false is
 // returned; the caller then stops issuing work and drains what it issued.
 __device__ inline bool mbar_wait(uint64_t *bar, uint32_t parity, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = wait_limit_ns(status);
     while (!mbar_try_wait(bar, parity)) {
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit) {
             if (status) atomicExch(status, (int)MSA_ERR_TIMEOUT);
             return false;
         }

@@ -11,8 +11,10 @@
 
 namespace msa {
 
-// Bounded device-side waits give up after this long and report MSA_ERR_TIMEOUT.
+// Bounded device-side waits give up after this long and report MSA_ERR_TIMEOUT,
+// unless the workspace header holds another limit (msa_set_wait_limit).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr int kWaitLimitWord = 2;  // int words 2..3 of the workspace header: wait limit in ns (0: default)
 
 constexpr int kMaxBatch = 1024;
 constexpr int kMaxTopK = 1024;          // largest top_k (decode entries and the stand-alone TopK)
@@ -143,6 +145,8 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
                                 cudaStream_t s, const char **why);
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
                                  cudaStream_t s, const char **why);
+cudaError_t launch_set_wait_limit(int *ws, unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_wait_never(int *ws, cudaStream_t s);
 
 int num_sms();
 

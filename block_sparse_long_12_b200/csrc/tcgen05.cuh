@@ -121,9 +121,10 @@ __device__ inline float max32(const uint32_t (&r)[32]) {
 __device__ inline bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
+    const uint64_t limit = wait_limit_ns(status);
     while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
+        if (global_timer_ns() - t0 > limit) {
             *abort_flag = 1;
             if (status) atomicExch(status, (int)MSA_ERR_TIMEOUT);
             return false;

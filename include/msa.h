@@ -42,10 +42,11 @@
  *   - Scratch memory comes from the caller: `ws` of at least
  *     msa_workspace_size(params, entry) bytes (256-byte aligned).  Each call
  *     overwrites the workspace; calls that share a workspace must not overlap.
- *     Its first 256 bytes hold the device status word and the index scan's
- *     work counters (msa_index_score, msa_decode_fused), which the scan
- *     returns to zero when it ends: zero-fill a workspace once before its
- *     first use (a cudaMemset or a zeroed allocation).
+ *     Its first 256 bytes hold the device status word, the limit of the
+ *     kernels' bounded waits (msa_set_wait_limit; 0 = one second) and the
+ *     index scan's work counters (msa_index_score, msa_decode_fused), which
+ *     the scan returns to zero when it ends: zero-fill a workspace once before
+ *     its first use (a cudaMemset or a zeroed allocation).
  *   - Arguments are checked before anything is enqueued; on error nothing is
  *     launched and the call returns the status (text: msa_last_error_string).
  *   - A CUDA launch error returns MSA_ERR_CUDA.  Devices other than
@@ -208,13 +209,27 @@ MSA_API msa_status_t msa_decode_fused(const msa_params_t *params, const void *q,
  *     overlaps on the GPU (other streams, other host threads) race on it
  *     and must be ordered by the caller.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make it before
+ *     (cudaGetSymbolAddress) with that device current, and again after the
+ *     device's context was replaced (cudaDeviceReset); make it before
  *     capturing any stream.
  *   - Nothing is allocated or freed; results equal msa_decode_fused's.
+ *   - A bounded wait that ran out is reported only through the fixed
+ *     scratch's status word: msa_noalloc_get_status / msa_noalloc_clear_status.
  */
 MSA_API msa_status_t msa_decode_fused_noalloc(const msa_params_t *params, const void *q, const void *q_idx,
                                               const void *k_cache, const void *v_cache, const void *k_idx, void *o,
                                               int32_t *ids_out, float *lse, msa_stream_t stream);
+
+/*
+ * Status of msa_decode_fused_noalloc's fixed scratch on the current device:
+ * its device status word works like a workspace's (see msa_get_device_status),
+ * and a call whose bounded wait ran out still returns MSA_OK (the kernels are
+ * asynchronous), so read it here after the calls.  msa_noalloc_get_status
+ * synchronises `stream`; msa_noalloc_clear_status resets the status word and
+ * the scan's counters of the fixed scratch, asynchronously on `stream`.
+ */
+MSA_API msa_status_t msa_noalloc_get_status(int *status, msa_stream_t stream);
+MSA_API msa_status_t msa_noalloc_clear_status(msa_stream_t stream);
 
 /*
  * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,
@@ -253,10 +268,25 @@ MSA_API const char *msa_status_string(msa_status_t status);
 /* Device status word kept in a workspace (first 4 bytes): MSA_OK, or
  * MSA_ERR_TIMEOUT after a bounded wait ran out.  Copies it to *status after
  * synchronising `stream`; msa_clear_device_status resets it asynchronously,
- * together with the scan's work counters (left non-zero by a scan that did
- * not end normally). */
+ * together with the wait limit (back to the default) and the scan's work
+ * counters (left non-zero by a scan that did not end normally).  A kernel that
+ * timed out stops issuing work, waits (bounded) for its own copies in flight
+ * and returns; its outputs are then undefined, the context stays usable. */
 MSA_API msa_status_t msa_get_device_status(const void *ws, int *status, msa_stream_t stream);
 MSA_API msa_status_t msa_clear_device_status(void *ws, msa_stream_t stream);
+
+/* Limit of every bounded device wait of the kernels that use this workspace,
+ * in nanoseconds (bytes 8..15 of the workspace header, written on `stream`);
+ * 0 restores the default of one second.  ws: 256-byte aligned device memory. */
+MSA_API msa_status_t msa_set_wait_limit(void *ws, uint64_t limit_ns, msa_stream_t stream);
+
+/* Failure-detection diagnostic (not part of the method): launches one thread
+ * that waits, bounded by the workspace's wait limit, for an mbarrier phase
+ * that nothing completes, so the wait runs out and the status word becomes
+ * MSA_ERR_TIMEOUT without any fault.  Lets a caller check that timeouts reach
+ * msa_get_device_status and that the workspace works again after
+ * msa_clear_device_status.  ws_bytes >= 256. */
+MSA_API msa_status_t msa_diag_wait_timeout(void *ws, size_t ws_bytes, msa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -177,6 +177,14 @@ def msa_rows(p: Params, seq_lens, q, q_idx, k, v, k_idx, rows, ids_in=None, atte
     return {"ids": ids, "top_scores": ts, "kth": kth, "kth_next": kn, "o": o, "lse": lse}
 
 
+def set_threads(n: int | None) -> int:
+    """Threads the oracle's OpenMP loops use from now on (None: all cores); returns the count set."""
+    n = int(n) if n else (os.cpu_count() or 1)
+    _load()
+    ctypes.CDLL("libgomp.so.1").omp_set_num_threads(n)
+    return n
+
+
 def to_f64(x: np.ndarray) -> np.ndarray:
     """Exact widening of stored f32 / bf16-bit arrays to float64."""
     if x.dtype == np.uint16:

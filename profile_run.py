@@ -1,10 +1,10 @@
 """Small, self-contained runs of the MSA kernels for profilers (ncu).
 
-  python -m block_sparse_long_12_b200.profile_run decode --context 262144 --steps 3
-  python -m block_sparse_long_12_b200.profile_run prefill_index --context 65536 --chunk 8192 --steps 1
-  python -m block_sparse_long_12_b200.profile_run prefill_attn --context 65536 --chunk 8192 --steps 1
-  python -m block_sparse_long_12_b200.profile_run scan_shared --context 1048576 --steps 3
-  python -m block_sparse_long_12_b200.profile_run large_k --context 262144 --steps 3
+  python profile_run.py decode --context 262144 --steps 3
+  python profile_run.py prefill_index --context 65536 --chunk 8192 --steps 1
+  python profile_run.py prefill_attn --context 65536 --chunk 8192 --steps 1
+  python profile_run.py scan_shared --context 1048576 --steps 3
+  python profile_run.py large_k --context 262144 --steps 3
 
 Inputs are the seeded synthetic workloads of ``inputs`` at the requested
 size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
@@ -17,8 +17,8 @@ import argparse
 
 import torch
 
-from . import _lib, api
-from .inputs import WORKLOADS, make_inputs
+from block_sparse_long_12_b200 import _lib, api
+from block_sparse_long_12_b200.inputs import WORKLOADS, make_inputs
 
 
 def run_decode(args, name="decode_ctx1m"):

@@ -147,3 +147,17 @@ def test_no_device_reports_cuda_error(lib):
     a = 0x10000
     rc = L.msa_decode_fused(ctypes.byref(p), a, a, a, a, a, a, None, None, a, ctypes.c_size_t(1 << 30), None)
     assert rc == lib.MSA_ERR_CUDA
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers: host-only argument checks")
+def test_failure_detection_calls_check_arguments(lib):
+    L = lib.lib()
+    a = 0x10000
+    assert L.msa_set_wait_limit(None, 1000, None) == lib.MSA_ERR_INVALID_ARG
+    assert L.msa_set_wait_limit(a + 16, 1000, None) == lib.MSA_ERR_INVALID_ARG  # not 256-byte aligned
+    assert L.msa_diag_wait_timeout(None, 256, None) == lib.MSA_ERR_INVALID_ARG
+    assert L.msa_diag_wait_timeout(a, 64, None) == lib.MSA_ERR_WORKSPACE
+    assert L.msa_noalloc_get_status(None, None) == lib.MSA_ERR_INVALID_ARG
+    # valid arguments reach the device, which is missing here
+    assert L.msa_diag_wait_timeout(a, 256, None) == lib.MSA_ERR_CUDA
+    assert L.msa_noalloc_clear_status(None) == lib.MSA_ERR_CUDA

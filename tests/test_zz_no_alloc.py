@@ -40,6 +40,10 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
         assert torch.equal(ids, ref_ids), f"call {call}: block ids differ"
         assert (o.float() - ref_o.float()).abs().max().item() <= 2e-2, f"call {call}: outputs differ"
         assert (lse - ref_lse).abs().max().item() <= 1e-3, f"call {call}: lse differs"
+        # no bounded wait ran out: the fixed scratch's status word reads MSA_OK
+        assert _lib.msa_noalloc_get_status() == _lib.MSA_OK, f"call {call}: status word set"
+    _lib.msa_noalloc_clear_status()
+    assert _lib.msa_noalloc_get_status() == _lib.MSA_OK
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
