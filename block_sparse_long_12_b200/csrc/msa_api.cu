@@ -283,7 +283,7 @@ size_t msa_workspace_size(const msa_params_t *p, int entry) {
             return decode_ws_layout(*p, true, true, n_sm).total;
         case MSA_ENTRY_ATTN_PREFILL:
             if (check_params(p, PREFILL_ONLY) != MSA_OK) return (size_t)-1;
-            return kStatusBytes;
+            return prefill_attn_plan(*p).total;
         case MSA_ENTRY_PREFILL_INDEX_TOPK:
             if (check_params(p, PREFILL_ONLY) != MSA_OK || check_device(&n_sm) != MSA_OK) return (size_t)-1;
             return prefill_index_plan(*p, n_sm).total;
@@ -557,10 +557,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
         return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes block_size 64 or 128");
     const int r = p->n_q_heads / p->n_kv_heads;
     if (128 % r != 0) return fail(MSA_ERR_UNSUPPORTED, "prefill attention needs a group size dividing 128");
-    if ((128 / r) * p->top_k > 512)
-        return fail(MSA_ERR_UNSUPPORTED, "prefill attention: (128 / group size) * top_k must not exceed 512");
-    if ((((long long)p->max_seq_len + p->block_size - 1) / p->block_size + 31) / 32 > 2048)
-        return fail(MSA_ERR_UNSUPPORTED, "prefill attention: at most 65536 blocks per sequence");
+    if ((long long)p->batch * p->q_len * p->n_q_heads >= (1LL << 31))
+        return fail(MSA_ERR_UNSUPPORTED, "prefill attention: batch * q_len * n_q_heads must stay below 2^31 rows");
     MSA_TRY(check_ptr(q, "q"));
     MSA_TRY(check_ptr(k_cache, "k_cache"));
     MSA_TRY(check_ptr(v_cache, "v_cache"));
@@ -568,7 +566,8 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
     MSA_TRY(check_ptr(o, "o"));
     MSA_TRY(check_ptr(lse, "lse", true));
     MSA_TRY(check_ptr(ws, "ws"));
-    if (ws_bytes < kStatusBytes) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, kStatusBytes);
+    const PrefillAttnPlan L = prefill_attn_plan(*p);
+    if (ws_bytes < L.total) return fail(MSA_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
     int n_sm = 0;
     MSA_TRY(check_device(&n_sm));
     PrefillAttnArgs a{};
@@ -577,6 +576,15 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
     a.Bk = p->block_size; a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len; a.r = r;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(ws);
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    a.counts = reinterpret_cast<int *>(w + L.counts);
+    a.offsets = reinterpret_cast<int *>(w + L.offsets);
+    a.n_tiles = reinterpret_cast<int *>(w + L.n_tiles);
+    a.rank = reinterpret_cast<int *>(w + L.rank);
+    a.members = reinterpret_cast<int *>(w + L.members);
+    a.tiles = reinterpret_cast<int4 *>(w + L.tiles);
+    a.part_lse = reinterpret_cast<float *>(w + L.part_lse);
+    a.part_o = reinterpret_cast<__half *>(w + L.part_o);
     const char *why = "";
     cudaError_t e = launch_prefill_attn(a, q, k_cache, v_cache, n_sm, (cudaStream_t)stream, &why);
     if (e != cudaSuccess) return cuda_fail(e, why);

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -111,15 +112,39 @@ struct PrefillIdxPlan {
 };
 PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm);
 
+// Prefill sparse attention, block-major: the (row, selected block) pairs of up to
+// kPrefillRowsPerPass query rows are bucketed by block; a tile is up to 128 / r member
+// rows' r heads against one block, giving one partial output per pair that a merge
+// combines per row by log-sum-exp.
+constexpr int kPrefillRowsPerPass = 8192;
+
 struct PrefillAttnArgs {
     const int *ids;            // [B, T, G, k]
     void *o;                   // [B, T, Hq, D] bf16
     float *lse;                // [B, T, Hq] nullable
     int B, T, Hq, G, D, Bk, k, q_start, L_max, r;
     float scale_log2;
-    int max_union, mask_words, bitmap_words;  // set by the launcher
     int *status;
+    // one pass over query rows [t0, t0 + Tn)
+    int t0, Tn;
+    int nbv;                   // blocks visible to the pass's last row: buckets per (b, g)
+    int tt;                    // member rows per tile, 128 / r
+    int *counts;               // [B*G*nbv] pairs per bucket (zeroed before the pass)
+    int *offsets;              // [B*G*nbv] first member of each bucket
+    int *rank;                 // [B*Tn*G*k] rank of each pair in its bucket (-1: not attended)
+    int *members;              // [pairs] member tt * k + slot, grouped by bucket
+    int4 *tiles;               // [max_tiles] (bucket, first member, member count, 0)
+    int *n_tiles;
+    __half *part_o;            // [B*Tn*G*k][r][D] per-pair output, normalised by the pair's sum
+    float *part_lse;           // [B*Tn*G*k][r] per-pair log2 normaliser
 };
+
+// Workspace of one prefill attention call (offsets in bytes).
+struct PrefillAttnPlan {
+    int rows, nbv_max, max_tiles;
+    size_t counts, offsets, n_tiles, rank, members, tiles, part_lse, part_o, total;
+};
+PrefillAttnPlan prefill_attn_plan(const msa_params_t &p);
 
 struct FillArgs {
     float *scores;

@@ -2,58 +2,95 @@
 // head attends over its group's selected blocks of the real K/V.
 //
 // Page "MiniMax wird duenn" (atlascloud.ai), section 1, Step 2: the heads of
-// a group share one block list, so one set of KV blocks serves all of them
-// (Q1/Q2/Q3 -> I1, Q4/Q5/Q6 -> I2).  In prefill every token has its own list;
-// a work unit packs TQ = 128 / r consecutive tokens x the r heads of group g
-// into one 128-row query tile (row = token * r + head) and walks the sorted
-// union of the TQ tokens' lists.  Per union block:
-//   S = Q K^T      tcgen05.mma (M=128, N=block, K=16 steps over head_dim),
-//                  fp32 accumulator in TMEM (double-buffered);
-//   softmax        two warps per TMEM lane quadrant, each on half of the
-//                  block's columns: tcgen05.ld of S, mask (block not in this
-//                  token's list, or key after the token), row max exchanged
-//                  between the two warps through shared memory, running max
-//                  with lazy rescaling (the output is rescaled in TMEM only
-//                  when the max grows by more than 2^8), P = 2^(z*c - m) as
-//                  bf16 into shared memory in the 128-byte swizzle layout;
-//   O += P V       tcgen05.mma with V as an MN-major operand, O in TMEM.
-// K and V tiles have their own stages: a K stage is refilled as soon as its
-// Q K^T has completed, a V stage once its P V has.
-// Warp roles: 0 TMA producer of Q and K, 1 MMA issuer and TMEM owner, 2
-// builds the per-unit block union and per-token membership masks, 3 TMA
-// producer of V, 4-11 softmax and the final normalisation.
+// a group share one block list, so one KV block serves all of them (Q1/Q2/Q3
+// -> I1, Q4/Q5/Q6 -> I2).  In prefill every token has its own list, and the
+// lists of neighbouring tokens need not overlap, so the work is organised by
+// block instead of by token: every (row, selected block) pair is put in the
+// bucket of its block, and a tile is up to 128 / r member rows of one bucket
+// with their r heads (M = 128) against that one block.  A pair's attention is
+// then exact within the block -- S = Q K^T, softmax over the block's visible
+// keys, O = P V normalised by the block's sum -- and its output and log2 sum
+// go to the workspace; a merge kernel combines each row's k pairs by
+// log-sum-exp into the row's output.  No tile computes a row that did not
+// select its block.
+//
+// Per pass over up to kPrefillRowsPerPass query rows:
+//   pa_count_kernel     pairs per bucket and each pair's rank in it;
+//   pa_scan_kernel      bucket offsets and the tile list (bucket order);
+//   pa_scatter_kernel   members grouped by bucket;
+//   pa_tile_kernel      the tiles, persistent, one contiguous range per SM:
+//     warp 0      TMA of the block's K and V tiles (2-stage ring, reloaded
+//                 only when the bucket changes);
+//     warp 1      TMEM owner, issues tcgen05.mma: S = Q K^T (M 128, N Bk)
+//                 into a double-buffered S buffer, and O = P V (N = D) with P
+//                 read from TMEM (it overwrites its own S buffer) into a
+//                 double-buffered O;
+//     warp 2      TMA gather of the members' query rows (one box of the r
+//                 heads per member and 64-dim half, 2-stage ring);
+//     warps 4-11  softmax, two warps per TMEM lane quadrant on half of the
+//                 block's keys each: mask keys after the row, row max
+//                 (exchanged between the two), P = 2^(z*c - m) as bf16 into
+//                 TMEM, row sums;
+//     warps 12-15 epilogue: O / sum as fp16 and the log2 sum per pair;
+//   pa_merge_kernel     per row and head: log-sum-exp of its pairs -> o, lse.
 #include "tcgen05.cuh"
 
 namespace msa {
 
 namespace {
 
-constexpr int kPaThreads = 384;
-constexpr int kPaRows = 128;
-constexpr int kPaSm0 = 4;    // first softmax warp
-constexpr int kPaSmWarps = 8;
-constexpr int kHalf = 16384; // one 128-row x 128-byte operand tile
+constexpr int kPtThreads = 512;
+constexpr int kPtRows = 128;
+constexpr int kPtSm0 = 4;       // first softmax warp
+constexpr int kPtSmWarps = 8;
+constexpr int kPtEpi0 = 12;     // first epilogue warp
+constexpr int kPtEpiWarps = 4;
+constexpr int kHalf = 16384;    // one 128-row x 128-byte operand tile
 
-struct PaBars {
-    uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+struct PtBars {
+    uint64_t kv_full[2], kv_empty[2];
+    uint64_t q_full[2], q_empty[2];
     uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, pv_done;
-    uint64_t q_full, q_empty;
-    uint64_t u_full[2], u_empty[2];
+    uint64_t p_full[2];
+    uint64_t o_full[2], o_empty[2];
+    uint64_t ml_full[2], ml_empty[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
-    int u_count[2];
-    float red_m[2][2][kPaRows];  // [block parity][column half][row]: raw row max of the half
-    float red_l[2][kPaRows];     // [column half][row]: row sum of the half
+    float red_m[2][2][kPtRows];  // [buffer][column half][row] raw max of the half row
+    float ml_m[2][kPtRows];      // [buffer][row] row max, log2 domain
+    float ml_l[2][2][kPtRows];   // [buffer][column half][row] sum of the half row
 };
 
 __device__ inline void mbar_arrive1(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-__device__ inline void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ inline void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+// D[tmem] (+)= A[tmem] * B[smem]: A (M x 16 bf16) read from tensor memory, lane i = row i,
+// two bf16 per 32-bit column, lower k in the low half.
+__device__ inline void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                   uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <int N>
+__device__ inline void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
+template <>
+__device__ inline void tmem_st<16>(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+template <>
+__device__ inline void tmem_st<32>(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
@@ -73,9 +110,9 @@ __device__ __forceinline__ float exp2_approx(float x) {
     return y;
 }
 
-// Barrier over the two softmax warps of one lane quadrant (64 threads) that
-// also ANDs a per-thread flag across them, so both warps leave a loop at the
-// same barrier when either has given up a wait.
+// Barrier over the two softmax warps of one lane quadrant (64 threads) that also ANDs a
+// per-thread flag across them, so both warps leave a loop at the same barrier when either
+// has given up a wait.
 __device__ inline bool pair_sync_and(int id, bool ok) {
     uint32_t r;
     __syncwarp();
@@ -90,10 +127,9 @@ __device__ inline bool pair_sync_and(int id, bool ok) {
     return r != 0;
 }
 
-// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle
-// layout: 64-element rows of 128 bytes along N, consecutive K rows 128 bytes
-// apart, 8-row groups 1024 bytes apart (stride byte offset), the next 64
-// elements of N `lbo` bytes further (leading byte offset).
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle layout: 64-element
+// rows of 128 bytes along N, consecutive K rows 128 bytes apart, 8-row groups 1024 bytes apart
+// (stride byte offset), the next 64 elements of N `lbo` bytes further (leading byte offset).
 __device__ inline uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) {
     uint64_t d = 0;
     d |= (uint64_t)((smem_addr >> 4) & 0x3fff);
@@ -104,47 +140,122 @@ __device__ inline uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo) 
     return d;
 }
 
+// A pair (row t of the pass, slot j of its list, group g, sequence b) is attended when its
+// block is visible to the row.
+__device__ inline bool pair_valid(int id, int bk, int pos) { return id >= 0 && id * bk <= pos; }
+
+// ------------------------------------------------------------------ bucketing
+__global__ void pa_count_kernel(const PrefillAttnArgs a) {
+    const long long n = (long long)a.B * a.Tn * a.G * a.k;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int j = (int)(i % a.k);
+        long long rest = i / a.k;
+        const int g = (int)(rest % a.G);
+        rest /= a.G;
+        const int tt = (int)(rest % a.Tn);
+        const int b = (int)(rest / a.Tn);
+        const int t = a.t0 + tt;
+        const int id = a.ids[(((size_t)b * a.T + t) * a.G + g) * a.k + j];
+        int rk = -1;
+        if (pair_valid(id, a.Bk, a.q_start + t) && id < a.nbv)
+            rk = atomicAdd(&a.counts[((size_t)b * a.G + g) * a.nbv + id], 1);
+        a.rank[i] = rk;
+    }
+}
+
+// One CTA: exclusive scan of the bucket counts (pairs and tiles), tile list in bucket order.
+__global__ void __launch_bounds__(1024) pa_scan_kernel(const PrefillAttnArgs a) {
+    __shared__ long long wsum_p[32], wsum_t[32];
+    const int nb = a.B * a.G * a.nbv;
+    const int per = (nb + 1023) / 1024;
+    const int s0 = threadIdx.x * per, s1 = s0 + per < nb ? s0 + per : nb;
+    long long lp = 0, lt = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int c = a.counts[s];
+        lp += c;
+        lt += (c + a.tt - 1) / a.tt;
+    }
+    // block-wide exclusive scan of (lp, lt)
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long ip = lp, it = lt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long vp = __shfl_up_sync(FULL, ip, o), vt = __shfl_up_sync(FULL, it, o);
+        if (lane >= o) { ip += vp; it += vt; }
+    }
+    if (lane == 31) { wsum_p[warp] = ip; wsum_t[warp] = it; }
+    __syncthreads();
+    if (warp == 0) {
+        long long xp = wsum_p[lane], xt = wsum_t[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long vp = __shfl_up_sync(FULL, xp, o), vt = __shfl_up_sync(FULL, xt, o);
+            if (lane >= o) { xp += vp; xt += vt; }
+        }
+        wsum_p[lane] = xp;
+        wsum_t[lane] = xt;
+    }
+    __syncthreads();
+    long long bp = ip - lp + (warp > 0 ? wsum_p[warp - 1] : 0);
+    long long bt = it - lt + (warp > 0 ? wsum_t[warp - 1] : 0);
+    for (int s = s0; s < s1; ++s) {
+        const int c = a.counts[s];
+        a.offsets[s] = (int)bp;
+        for (int q = 0; q * a.tt < c; ++q) {
+            const int m = c - q * a.tt < a.tt ? c - q * a.tt : a.tt;
+            a.tiles[bt++] = make_int4(s, (int)bp + q * a.tt, m, 0);
+        }
+        bp += c;
+    }
+    if (threadIdx.x == 1023) *a.n_tiles = (int)wsum_t[31];
+}
+
+__global__ void pa_scatter_kernel(const PrefillAttnArgs a) {
+    const long long n = (long long)a.B * a.Tn * a.G * a.k;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+        const int rk = a.rank[i];
+        if (rk < 0) continue;
+        const int j = (int)(i % a.k);
+        long long rest = i / a.k;
+        const int g = (int)(rest % a.G);
+        rest /= a.G;
+        const int tt = (int)(rest % a.Tn);
+        const int b = (int)(rest / a.Tn);
+        const int id = a.ids[(((size_t)b * a.T + a.t0 + tt) * a.G + g) * a.k + j];
+        a.members[a.offsets[((size_t)b * a.G + g) * a.nbv + id] + rk] = tt * a.k + j;
+    }
+}
+
+// ------------------------------------------------------------------ tiles
 template <int D, int BK>
-__global__ void __launch_bounds__(kPaThreads, 1)
-    prefill_attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
-                        const __grid_constant__ CUtensorMap vmap, const PrefillAttnArgs a) {
-    constexpr int NH = D / 64;        // 64-dim halves of a row
-    constexpr int PH = BK / 64;       // 64-key halves of a P row
-    constexpr int KVH = BK * 128;     // bytes of one 64-dim half of a K or V block tile
-    constexpr int STAGE = 2 * NH * KVH;
-    constexpr uint32_t TMEM_COLS = (2 * BK + D) <= 256 ? 256 : 512;
-    constexpr uint32_t O_COL = 2 * BK;
-    constexpr int CW = BK / 2;        // S columns of one softmax warp
-    constexpr int DW = D / 2;         // O columns of one softmax warp
+__global__ void __launch_bounds__(kPtThreads, 1)
+    pa_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, const PrefillAttnArgs a) {
+    constexpr int NH = D / 64;               // 64-dim halves of a row
+    constexpr int KVH = BK * 128;            // bytes of one 64-dim half of a K or V block tile
+    constexpr int KV_STAGE = 2 * NH * KVH;   // K halves, then V halves
+    constexpr int Q_STAGE = NH * kHalf;
+    constexpr int CW = BK / 2;               // S columns of one softmax warp
+    constexpr uint32_t O_COL = 2 * BK;       // TMEM: S/P buffers [0, 2 BK), O buffers [2 BK, 2 BK + 2 D)
+    constexpr uint32_t TMEM_COLS = 512;
+    static_assert(2 * BK + 2 * D <= 512, "TMEM budget");
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    unsigned char *smQ = base;                       // [NH][128 rows][128 B]
-    unsigned char *smP = smQ + NH * kHalf;           // [PH][128 rows][128 B]
-    unsigned char *smKV = smP + PH * kHalf;          // [2 stages][K halves | V halves]
-    PaBars &S = *reinterpret_cast<PaBars *>(smKV + 2 * STAGE);
-    int *u_ids = reinterpret_cast<int *>(&S + 1);    // [2][max_union]
-    uint32_t *u_mask = reinterpret_cast<uint32_t *>(u_ids + 2 * a.max_union);  // [2][max_union][MW]
-    uint32_t *bitmap = u_mask + 2 * a.max_union * a.mask_words;               // [bitmap_words]
-    int *prefix = reinterpret_cast<int *>(bitmap + a.bitmap_words);           // [bitmap_words]
+    unsigned char *smQ = base;                    // [2][NH][128 rows][128 B]
+    unsigned char *smKV = smQ + 2 * Q_STAGE;      // [2][K halves | V halves]
+    PtBars &S = *reinterpret_cast<PtBars *>(smKV + 2 * KV_STAGE);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int r = a.r, TQ = kPaRows / r, MW = a.mask_words;
-    const int n_tiles = (a.T + TQ - 1) / TQ;
-    const int n_units = a.B * a.G * n_tiles;
-
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&S.k_full[i], 1); mbar_init(&S.k_empty[i], 1);
-            mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1);
-            mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], kPaSmWarps);
-            // K producer, V producer, MMA issuer and the softmax warps release a union slot
-            mbar_init(&S.u_full[i], 1); mbar_init(&S.u_empty[i], 3 + kPaSmWarps);
+            mbar_init(&S.kv_full[i], 1); mbar_init(&S.kv_empty[i], 1);
+            mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1);
+            mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1);
+            mbar_init(&S.p_full[i], kPtSmWarps);
+            mbar_init(&S.o_full[i], 1); mbar_init(&S.o_empty[i], kPtEpiWarps);
+            mbar_init(&S.ml_full[i], kPtSmWarps); mbar_init(&S.ml_empty[i], kPtEpiWarps);
         }
-        mbar_init(&S.p_full, kPaSmWarps);
-        mbar_init(&S.pv_done, 1);
-        mbar_init(&S.q_full, 1);
-        mbar_init(&S.q_empty, 1);
         mbar_init(&S.mma_done, 1);
         S.abort_flag = 0;
         fence_mbar_init();
@@ -162,352 +273,247 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const uint32_t tmem = S.tmem_base;
     volatile int *abort_flag = &S.abort_flag;
 
-    auto unit_of = [&](int u, int &b, int &g, int &t0) {
-        const int tile = u % n_tiles;
-        const int bg = u / n_tiles;
+    // this CTA's contiguous range of tiles (bucket order: consecutive tiles mostly share a block)
+    const long long nt = *a.n_tiles;
+    const int tb = (int)(nt * blockIdx.x / gridDim.x), te = (int)(nt * (blockIdx.x + 1) / gridDim.x);
+    const int r = a.r;
+    auto bucket_block = [&](int bkt, int &b, int &g, int &n) {
+        const int bg = bkt / a.nbv;
+        n = bkt - bg * a.nbv;
         b = bg / a.G;
-        g = bg % a.G;
-        t0 = tile * TQ;
+        g = bg - b * a.G;
     };
 
-    if (warp == 2) {
-        // ------------------------------------------------ union of the tile's block lists
-        int ui = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-            int b, g, t0;
-            unit_of(u, b, g, t0);
-            const int slot = ui & 1;
-            bool ok = true;
-            if (lane == 0) ok = tc::wait_or_abort(&S.u_empty[slot], ((ui >> 1) & 1) ^ 1, abort_flag, a.status);
-            if (!__shfl_sync(FULL, ok, 0)) break;
-            const int nv = a.T - t0 < TQ ? a.T - t0 : TQ;
-            const int nbits = (a.q_start + t0 + nv - 1) / a.Bk + 1;
-            const int words = (nbits + 31) >> 5;
-            for (int i = lane; i < words; i += 32) bitmap[i] = 0;
-            __syncwarp();
-            const int *ids = a.ids + (((size_t)b * a.T + t0) * a.G + g) * a.k;
-            const size_t tok_stride = (size_t)a.G * a.k;
-            for (int i = lane; i < nv * a.k; i += 32) {
-                const int tq = i / a.k;
-                const int id = ids[tq * tok_stride + i % a.k];
-                if (id >= 0 && id * a.Bk <= a.q_start + t0 + tq) atomicOr(&bitmap[id >> 5], 1u << (id & 31));
-            }
-            __syncwarp();
-            int carry = 0;
-            for (int w0 = 0; w0 < words; w0 += 32) {
-                const int wi = w0 + lane;
-                const int c = wi < words ? __popc(bitmap[wi]) : 0;
-                int incl = c;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(FULL, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                if (wi < words) prefix[wi] = carry + incl - c;
-                carry += __shfl_sync(FULL, incl, 31);
-            }
-            const int U = carry;
-            __syncwarp();
-            int *uid = u_ids + slot * a.max_union;
-            uint32_t *um = u_mask + (size_t)slot * a.max_union * MW;
-            for (int wi = lane; wi < words; wi += 32) {
-                uint32_t bits = bitmap[wi];
-                int at = prefix[wi];
-                while (bits) {
-                    const int bit = __ffs(bits) - 1;
-                    uid[at++] = wi * 32 + bit;
-                    bits &= bits - 1;
-                }
-            }
-            for (int i = lane; i < U * MW; i += 32) um[i] = 0;
-            __syncwarp();
-            for (int i = lane; i < nv * a.k; i += 32) {
-                const int tq = i / a.k;
-                const int id = ids[tq * tok_stride + i % a.k];
-                if (id >= 0 && id * a.Bk <= a.q_start + t0 + tq) {
-                    const int wi = id >> 5;
-                    const int at = prefix[wi] + __popc(bitmap[wi] & ((1u << (id & 31)) - 1u));
-                    atomicOr(&um[at * MW + (tq >> 5)], 1u << (tq & 31));
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                S.u_count[slot] = U;
-                mbar_arrive1(&S.u_full[slot]);
+    if (warp == 0) {
+        // ------------------------------------------------ K/V producer: one load per new bucket
+        if (lane == 0) {
+            int kvi = -1, prev = -1;
+            for (int ti = tb; ti < te; ++ti) {
+                const int bkt = a.tiles[ti].x;
+                if (bkt == prev) continue;
+                prev = bkt;
+                ++kvi;
+                const int ks = kvi & 1;
+                if (!tc::wait_or_abort(&S.kv_empty[ks], ((kvi >> 1) & 1) ^ 1, abort_flag, a.status)) break;
+                int b, g, n;
+                bucket_block(bkt, b, g, n);
+                mbar_arrive_expect_tx(&S.kv_full[ks], 2 * NH * KVH);
+                const int row = (b * a.G + g) * a.L_max + n * BK;
+                unsigned char *dst = smKV + ks * KV_STAGE;
+                for (int h = 0; h < NH; ++h) tc::tma_load_2d(dst + h * KVH, &kmap, h * 64, row, &S.kv_full[ks]);
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_2d(dst + (NH + h) * KVH, &vmap, h * 64, row, &S.kv_full[ks]);
             }
         }
-    } else if (warp == 0 || warp == 3) {
-        // ------------------------------------------------ TMA producers: warp 0 the Q tile and K tiles, warp 3 V tiles
-        if (lane == 0) {
-            const bool is_k = warp == 0;
-            const CUtensorMap *map = is_k ? &kmap : &vmap;
-            uint64_t *full = is_k ? S.k_full : S.v_full;
-            uint64_t *empty = is_k ? S.k_empty : S.v_empty;
-            const int off = is_k ? 0 : NH * KVH;
-            int ui = 0, it = 0;
-            for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-                int b, g, t0;
-                unit_of(u, b, g, t0);
-                const int slot = ui & 1;
-                if (!tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status)) break;
-                const int U = S.u_count[slot];
-                if (is_k) {
-                    if (!tc::wait_or_abort(&S.q_empty, (ui & 1) ^ 1, abort_flag, a.status)) break;
-                    mbar_arrive_expect_tx(&S.q_full, NH * kHalf);
-                    for (int h = 0; h < NH; ++h)
-                        tc::tma_load_3d(smQ + h * kHalf, &qmap, h * 64, g * r, b * a.T + t0, &S.q_full);
-                }
-                const int *uid = u_ids + slot * a.max_union;
-                bool ok = true;
-                for (int j = 0; j < U; ++j, ++it) {
-                    const int st = it & 1;
-                    if (!tc::wait_or_abort(&empty[st], ((it >> 1) & 1) ^ 1, abort_flag, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full[st], NH * KVH);
-                    const int row = (b * a.G + g) * a.L_max + uid[j] * a.Bk;
-                    unsigned char *dst = smKV + st * STAGE + off;
-                    for (int h = 0; h < NH; ++h) tc::tma_load_2d(dst + h * KVH, map, h * 64, row, &full[st]);
-                }
-                mbar_arrive1(&S.u_empty[slot]);
-                if (!ok) break;
+    } else if (warp == 2) {
+        // ------------------------------------------------ Q gather: the members' r heads, one box per member and half
+        for (int ti = tb; ti < te; ++ti) {
+            const int il = ti - tb, qs = il & 1;
+            bool ok = true;
+            if (lane == 0) ok = tc::wait_or_abort(&S.q_empty[qs], ((il >> 1) & 1) ^ 1, abort_flag, a.status);
+            if (!__shfl_sync(FULL, ok, 0)) break;
+            const int4 tile = a.tiles[ti];
+            int b, g, n;
+            bucket_block(tile.x, b, g, n);
+            if (lane == 0) mbar_arrive_expect_tx(&S.q_full[qs], (uint32_t)tile.z * r * 128 * NH);
+            __syncwarp();
+            for (int m = lane; m < tile.z; m += 32) {
+                const int tt = a.members[tile.y + m] / a.k;
+                const int qrow = ((b * a.T + a.t0 + tt) * a.Hq) + g * r;
+                for (int h = 0; h < NH; ++h)
+                    tc::tma_load_2d(smQ + qs * Q_STAGE + h * kHalf + m * r * 128, &qmap, h * 64, qrow, &S.q_full[qs]);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_qk = tc::idesc_bf16_f32(kPaRows, BK);
-            const uint32_t idesc_pv = tc::idesc_bf16_f32(kPaRows, D) | (1u << 16);  // B (V) is MN-major
-            int ui = 0, it = 0, sc = 0, pc = 0;
-            for (int u = blockIdx.x; u < n_units && !*abort_flag; u += gridDim.x, ++ui) {
-                const int slot = ui & 1;
-                if (!tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status)) break;
-                const int U = S.u_count[slot];
-                if (!tc::wait_or_abort(&S.q_full, ui & 1, abort_flag, a.status)) break;
+            const uint32_t idesc_qk = tc::idesc_bf16_f32(kPtRows, BK);
+            const uint32_t idesc_pv = tc::idesc_bf16_f32(kPtRows, D) | (1u << 16);  // B (V) is MN-major
+            int kvi = -1, prev = -1;
+            int pend = -1, pend_ks = 0;
+            bool pend_last = false, ok = true;
+            // O = P V of tile `il` (its P overwrote its S buffer); frees the S buffer and, after a
+            // bucket's last tile, the K/V stage
+            auto issue_pv = [&](int il, int ks, bool last) -> bool {
+                const int ob = il & 1;
+                if (!tc::wait_or_abort(&S.p_full[ob], (il >> 1) & 1, abort_flag, a.status)) return false;
+                if (!tc::wait_or_abort(&S.o_empty[ob], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
                 tc::fence_after_sync();
-                const uint32_t q_addr = smem_u32(smQ);
-                bool ok = true;
-                // Q K^T of block j into S buffer (sc + j) & 1; its K stage is free once it completes
-                auto qk = [&](int j) -> bool {
-                    const int st = (it + j) & 1;
-                    const int sb = (sc + j) & 1;
-                    if (!tc::wait_or_abort(&S.k_full[st], ((it + j) >> 1) & 1, abort_flag, a.status)) return false;
-                    if (!tc::wait_or_abort(&S.s_empty[sb], (((sc + j) >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
-                    tc::fence_after_sync();
-                    const uint32_t k_addr = smem_u32(smKV + st * STAGE);
+                const uint32_t v_addr = smem_u32(smKV + ks * KV_STAGE + NH * KVH);
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (ks >> 2) * kHalf + (ks & 3) * 32),
-                                        tc::sw128_kmajor_desc(k_addr + (ks >> 2) * KVH + (ks & 3) * 32), idesc_qk, ks > 0);
-                    tc::mma_commit(&S.k_empty[st]);
-                    tc::mma_commit(&S.s_full[sb]);
-                    return true;
-                };
-                if (U > 0 && !qk(0)) break;
-                for (int j = 0; j < U; ++j) {
-                    if (j + 1 < U && !qk(j + 1)) { ok = false; break; }
-                    if (!tc::wait_or_abort(&S.p_full, pc & 1, abort_flag, a.status)) { ok = false; break; }
-                    ++pc;
-                    const int st = (it + j) & 1;
-                    if (!tc::wait_or_abort(&S.v_full[st], ((it + j) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-                    tc::fence_after_sync();
-                    const uint32_t v_addr = smem_u32(smKV + st * STAGE + NH * KVH);
-                    const uint32_t p_addr = smem_u32(smP);
-#pragma unroll
-                    for (int ks = 0; ks < BK / 16; ++ks)
-                        tc::mma_bf16_ss(tmem + O_COL, tc::sw128_kmajor_desc(p_addr + (ks >> 2) * kHalf + (ks & 3) * 32),
-                                        sw128_mnmajor_desc(v_addr + ks * 2048, KVH), idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-                    tc::mma_commit(&S.v_empty[st]);
-                    tc::mma_commit(&S.pv_done);
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    mma_bf16_ts(tmem + O_COL + ob * D, tmem + ob * BK + kk * 8, sw128_mnmajor_desc(v_addr + kk * 2048, KVH),
+                                idesc_pv, kk > 0 ? 1u : 0u);
+                tc::mma_commit(&S.o_full[ob]);
+                tc::mma_commit(&S.s_empty[ob]);
+                if (last) tc::mma_commit(&S.kv_empty[ks]);
+                return true;
+            };
+            for (int ti = tb; ti < te && ok; ++ti) {
+                const int il = ti - tb, sb = il & 1;
+                const int bkt = a.tiles[ti].x;
+                if (bkt != prev) { prev = bkt; ++kvi; }
+                const int ks = kvi & 1;
+                const bool last = ti + 1 == te || a.tiles[ti + 1].x != bkt;
+                if (!tc::wait_or_abort(&S.q_full[sb], (il >> 1) & 1, abort_flag, a.status) ||
+                    !tc::wait_or_abort(&S.kv_full[ks], (kvi >> 1) & 1, abort_flag, a.status) ||
+                    !tc::wait_or_abort(&S.s_empty[sb], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
-                it += U;
-                sc += U;
-                tc::mma_commit(&S.q_empty);
-                mbar_arrive1(&S.u_empty[slot]);
+                tc::fence_after_sync();
+                const uint32_t q_addr = smem_u32(smQ + sb * Q_STAGE), k_addr = smem_u32(smKV + ks * KV_STAGE);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32),
+                                    tc::sw128_kmajor_desc(k_addr + (kk >> 2) * KVH + (kk & 3) * 32), idesc_qk, kk > 0);
+                tc::mma_commit(&S.q_empty[sb]);
+                tc::mma_commit(&S.s_full[sb]);
+                if (pend >= 0 && !issue_pv(pend, pend_ks, pend_last)) {
+                    ok = false;
+                    break;
+                }
+                pend = il;
+                pend_ks = ks;
+                pend_last = last;
             }
+            if (ok && pend >= 0) issue_pv(pend, pend_ks, pend_last);
             tc::mma_commit(&S.mma_done);
             mbar_wait(&S.mma_done, 0, a.status);
         }
-    } else {
-        // ------------------------------------------------ softmax / epilogue
-        // Warps w and w + 4 share TMEM lane quadrant w % 4 (one query row per
-        // lane); warp half hf takes S columns [hf*CW, hf*CW + CW) and O
-        // columns [hf*DW, hf*DW + DW).  Every wait result is made uniform over
-        // the pair through pair_sync_and before either warp acts on it, so the
-        // two always execute the same sequence of pair barriers.
-        const int sw = warp - kPaSm0;
+    } else if (warp >= kPtSm0 && warp < kPtSm0 + kPtSmWarps) {
+        // ------------------------------------------------ softmax
+        // Warps w and w + 4 share TMEM lane quadrant w % 4 (one row per lane); half hf takes the
+        // block's keys [hf*CW, hf*CW + CW).  Every wait of a tile comes before the pair barrier,
+        // whose AND makes any failure uniform over the pair.
+        const int sw = warp - kPtSm0;
         const int qd = sw & 3, hf = sw >> 2;
         const int pair_bar = 1 + qd;
         const int row = qd * 32 + lane;
-        const int tq = row / r, hh = row % r;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
-        int ui = 0, sc = 0, pv_waits = 0;
-        bool p_zero = false;  // this warp's part of P already holds zeros
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++ui) {
-            int b, g, t0;
-            unit_of(u, b, g, t0);
-            const int slot = ui & 1;
-            bool ok = __all_sync(FULL, tc::wait_or_abort(&S.u_full[slot], (ui >> 1) & 1, abort_flag, a.status));
-            if (!pair_sync_and(pair_bar, ok)) break;
-            const int U = S.u_count[slot];
-            const int *uid = u_ids + slot * a.max_union;
-            const uint32_t *um = u_mask + (size_t)slot * a.max_union * MW;
-            const int t = t0 + tq;
-            const bool row_live = t < a.T;
-            const int pos = a.q_start + t;
-            float m = -INFINITY, l = 0.f;
-            for (int j = 0; j < U; ++j, ++sc) {
-                const int sb = sc & 1;
-                if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.s_full[sb], (sc >> 1) & 1, abort_flag, a.status));
-                const int id = uid[j];
-                const bool member = row_live && ((um[j * MW + (tq >> 5)] >> (tq & 31)) & 1u);
-                const bool active = __any_sync(FULL, member);
-                uint32_t zr[CW];
-                float mb = -INFINITY;
-                if (ok) {
-                    if (active) {
-                        tc::fence_after_sync();
-#pragma unroll
-                        for (int c = 0; c < CW / 32; ++c)
-                            tc::tmem_ld32(tmem + lane_addr + sb * BK + hf * CW + c * 32,
-                                          *reinterpret_cast<uint32_t(*)[32]>(&zr[c * 32]));
-                        tc::tmem_ld_wait();
-                        tc::fence_before_sync();
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive1(&S.s_empty[sb]);
-                    if (active) {
-                        // only the block holding the query needs the causal mask
-                        const int kb = id * a.Bk + hf * CW;
-                        if (member && kb + CW - 1 > pos) {
-#pragma unroll
-                            for (int c = 0; c < CW; ++c)
-                                if (kb + c > pos) zr[c] = __float_as_uint(-INFINITY);
-                        }
-                        float mx[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) mx[i] = -INFINITY;
-#pragma unroll
-                        for (int c = 0; c < CW; c += 8)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                mx[i] = tc::fmax3(mx[i], __uint_as_float(zr[c + 2 * i]), __uint_as_float(zr[c + 2 * i + 1]));
-                        mb = member ? fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) : -INFINITY;
-                    }
-                }
-                S.red_m[sc & 1][hf][row] = mb;
-                ok = pair_sync_and(pair_bar, ok);
-                if (!ok) break;
-                // row max of the block (raw scores), then the running max in the log2 domain
-                const float mraw = fmaxf(mb, S.red_m[sc & 1][hf ^ 1][row]);
-                const float m_new = fmaxf(m, mraw * a.scale_log2);
-                const bool grow = m_new > m + 8.f;  // rescale only when the max grows by more than 2^8
-                const float alpha = grow ? exp2_approx(m - m_new) : 1.f;
-                if (grow) m = m_new;
-                // P = 2^(z*c - m) as packed bf16 pairs; rows whose token did not select the block get 0
-                uint32_t pk[CW / 2];
-                float ps = 0.f;
-                if (active) {
-                    const float cz = member ? a.scale_log2 : 0.f;
-                    const float off = member ? -m : -INFINITY;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int e = 0; e < CW / 2; ++e) {
-                        const float p0 = exp2_approx(fmaf(__uint_as_float(zr[2 * e]), cz, off));
-                        const float p1 = exp2_approx(fmaf(__uint_as_float(zr[2 * e + 1]), cz, off));
-                        acc[e & 3] += p0 + p1;
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
-                    }
-                    ps = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                }
-                // the P buffer and O are free once the previous block's P.V has completed
-                if (j > 0) {
-                    ok = __all_sync(FULL, tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status));
-                    ++pv_waits;
-                    if (!ok) continue;  // both warps of the pair leave at the next pair barrier
-                    tc::fence_after_sync();
-                    if (__any_sync(FULL, alpha != 1.f)) {
-#pragma unroll 1
-                        for (int c = 0; c < DW / 32; ++c) {
-                            uint32_t ov[32];
-                            const uint32_t ta = tmem + lane_addr + O_COL + hf * DW + c * 32;
-                            tc::tmem_ld32(ta, ov);
-                            tc::tmem_ld_wait();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                            tmem_st32(ta, ov);
-                        }
-                        tmem_st_wait();
-                    }
-                }
-                if (active || !p_zero) {
-                    if (!active) {
-#pragma unroll
-                        for (int e = 0; e < CW / 2; ++e) pk[e] = 0u;
-                    }
-                    p_zero = !active;
-                    // this warp's CW keys of the row: 16-byte chunks of P half-tile (hf*CW)/64
-#pragma unroll
-                    for (int c16 = 0; c16 < CW / 8; ++c16) {
-                        const int kc = hf * CW + c16 * 8;  // first key of the chunk
-                        unsigned char *dst = smP + (kc >> 6) * kHalf + row * 128 + ((((kc & 63) >> 3) ^ (row & 7)) << 4);
-                        *reinterpret_cast<uint4 *>(dst) =
-                            make_uint4(pk[c16 * 4], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
-                    }
-                    fence_proxy_async_smem();
-                }
-                l = l * alpha + ps;
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive1(&S.p_full);
-            }
-            // final normalisation once the last P.V has completed
-            if (ok && U > 0) {
-                ok = __all_sync(FULL, tc::wait_or_abort(&S.pv_done, pv_waits & 1, abort_flag, a.status));
-                ++pv_waits;
-            }
-            S.red_l[hf][row] = l;
-            if (!pair_sync_and(pair_bar, ok)) break;
-            const float l_row = l + S.red_l[hf ^ 1][row];
-            float o_scale = 0.f;
-            if (U > 0) {
+        const int m_i = row / r;
+        const float c = a.scale_log2;
+        bool ok = true;
+        for (int ti = tb; ti < te; ++ti) {
+            const int il = ti - tb, sb = il & 1, par = (il >> 1) & 1;
+            const int4 tile = a.tiles[ti];
+            int b, g, n;
+            bucket_block(tile.x, b, g, n);
+            const bool valid = m_i < tile.z;
+            const bool any = __any_sync(FULL, valid);
+            int pos = 0;
+            if (valid) pos = a.q_start + a.t0 + a.members[tile.y + m_i] / a.k;
+            if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.s_full[sb], par, abort_flag, a.status));
+            if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.ml_empty[sb], par ^ 1, abort_flag, a.status));
+            uint32_t zr[CW];
+            float mb = -INFINITY;
+            if (ok && any) {
                 tc::fence_after_sync();
-                o_scale = l_row > 0.f ? 1.f / l_row : 0.f;
-            }
-            const int hq = g * r + hh;
-            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + hq) * D + hf * DW;
 #pragma unroll
-            for (int c = 0; c < DW / 32; ++c) {
-                uint32_t ov[32];
-                if (U > 0) {
-                    tc::tmem_ld32(tmem + lane_addr + O_COL + hf * DW + c * 32, ov);
-                    tc::tmem_ld_wait();
-                } else {
+                for (int cc = 0; cc < CW / 32; ++cc)
+                    tc::tmem_ld32(tmem + lane_addr + sb * BK + hf * CW + cc * 32,
+                                  *reinterpret_cast<uint32_t(*)[32]>(&zr[cc * 32]));
+                tc::tmem_ld_wait();
+                // only the block holding the row's own position needs the causal mask
+                const int key0 = n * BK + hf * CW;
+                if (valid && key0 + CW - 1 > pos) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] = 0u;
+                    for (int cc = 0; cc < CW; ++cc)
+                        if (key0 + cc > pos) zr[cc] = __float_as_uint(-INFINITY);
                 }
-                if (row_live) {
+                float mx[4];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t pk[4];
+                for (int i = 0; i < 4; ++i) mx[i] = -INFINITY;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(ov[q * 8 + 2 * e]) * o_scale,
-                                                                            __uint_as_float(ov[q * 8 + 2 * e + 1]) * o_scale);
-                            pk[e] = *reinterpret_cast<const uint32_t *>(&v2);
-                        }
-                        *reinterpret_cast<uint4 *>(o + c * 32 + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
-                }
+                for (int cc = 0; cc < CW; cc += 8)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        mx[i] = tc::fmax3(mx[i], __uint_as_float(zr[cc + 2 * i]), __uint_as_float(zr[cc + 2 * i + 1]));
+                mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             }
-            if (hf == 0 && row_live && a.lse != nullptr)
-                a.lse[((size_t)b * a.T + t) * a.Hq + hq] = l_row > 0.f ? (m + log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+            S.red_m[sb][hf][row] = mb;
+            ok = pair_sync_and(pair_bar, ok);
+            if (!ok) break;
+            // every lane of both warps has read its S half: P may now overwrite the S buffer
+            const float m2 = fmaxf(mb, S.red_m[sb][hf ^ 1][row]) * c;  // row max in the log2 domain
+            float ls = 0.f;
+            if (any) {
+                const float off = valid ? -m2 : 0.f;
+                uint32_t pk[CW / 2];
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < CW / 2; ++e) {
+                    const float p0 = exp2_approx(fmaf(__uint_as_float(zr[2 * e]), c, off));
+                    const float p1 = exp2_approx(fmaf(__uint_as_float(zr[2 * e + 1]), c, off));
+                    acc[e & 3] += p0 + p1;
+                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                    pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                }
+                ls = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                tmem_st<CW / 2>(tmem + lane_addr + sb * BK + hf * (CW / 2), pk);
+                tmem_st_wait();
+            }
+            if (hf == 0) S.ml_m[sb][row] = m2;
+            S.ml_l[sb][hf][row] = ls;
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive1(&S.u_empty[slot]);
+            if (lane == 0) {
+                mbar_arrive1(&S.p_full[sb]);
+                mbar_arrive1(&S.ml_full[sb]);
+            }
+        }
+    } else if (warp >= kPtEpi0) {
+        // ------------------------------------------------ epilogue: one pair row per lane
+        const int qd = warp & 3;
+        const int row = qd * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+        const int m_i = row / r, hh = row % r;
+        for (int ti = tb; ti < te; ++ti) {
+            const int il = ti - tb, ob = il & 1, par = (il >> 1) & 1;
+            const int4 tile = a.tiles[ti];
+            int b, g, n;
+            bucket_block(tile.x, b, g, n);
+            const bool valid = m_i < tile.z;
+            const bool any = __any_sync(FULL, valid);
+            int pl = 0;
+            if (valid) {
+                const int mem = a.members[tile.y + m_i];
+                pl = ((b * a.Tn + mem / a.k) * a.G + g) * a.k + mem % a.k;  // the pair's index in this pass
+            }
+            if (!__all_sync(FULL, tc::wait_or_abort(&S.ml_full[ob], par, abort_flag, a.status))) break;
+            const float m2 = S.ml_m[ob][row];
+            const float l = S.ml_l[ob][0][row] + S.ml_l[ob][1][row];
+            __syncwarp();
+            if (lane == 0) mbar_arrive1(&S.ml_empty[ob]);
+            if (!__all_sync(FULL, tc::wait_or_abort(&S.o_full[ob], par, abort_flag, a.status))) break;
+            tc::fence_after_sync();
+            if (any) {
+                const float inv = valid && l > 0.f ? 1.f / l : 0.f;
+                __half *dst = a.part_o + ((size_t)pl * r + hh) * D;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ov[32];
+                    tc::tmem_ld32(tmem + lane_addr + O_COL + ob * D + cc * 32, ov);
+                    tc::tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __half2 h2 = __floats2half2_rn(__uint_as_float(ov[q * 8 + 2 * e]) * inv,
+                                                                     __uint_as_float(ov[q * 8 + 2 * e + 1]) * inv);
+                                pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive1(&S.o_empty[ob]);
+            if (valid) a.part_lse[(size_t)pl * r + hh] = l > 0.f ? m2 + log2f(l) : -INFINITY;
         }
     }
     tc::fence_before_sync();
@@ -518,41 +524,148 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     }
 }
 
-template <int D, int BK>
-cudaError_t launch_pa(const PrefillAttnArgs &a, const CUtensorMap &qm, const CUtensorMap &km, const CUtensorMap &vm,
-                      int grid, cudaStream_t s) {
-    constexpr int NH = D / 64, PH = BK / 64;
-    const size_t smem = 1024 + (size_t)NH * kHalf + (size_t)PH * kHalf + 2 * (2 * NH * BK * 128) + sizeof(PaBars) +
-                        (size_t)2 * a.max_union * 4 + (size_t)2 * a.max_union * a.mask_words * 4 +
-                        (size_t)a.bitmap_words * 8 + 64;
-    if (smem > 232448) return cudaErrorInvalidValue;
-    static size_t attr_bytes = 0;
-    if (smem > attr_bytes) {
-        cudaError_t e =
-            cudaFuncSetAttribute(prefill_attn_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_bytes = smem;
+// ------------------------------------------------------------------ merge
+// One warp per (sequence, row, group, head): the log-sum-exp combination of the row's pairs.
+template <int D>
+__global__ void __launch_bounds__(256) pa_merge_kernel(const PrefillAttnArgs a) {
+    constexpr int DPL = D / 32;  // dims per lane
+    const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long n_rows = (long long)a.B * a.Tn * a.G * a.r;
+    if (w >= n_rows) return;
+    const int hh = (int)(w % a.r);
+    long long rest = w / a.r;
+    const int g = (int)(rest % a.G);
+    rest /= a.G;
+    const int tt = (int)(rest % a.Tn);
+    const int b = (int)(rest / a.Tn);
+    const int t = a.t0 + tt;
+    const int pos = a.q_start + t;
+    const size_t pl0 = (((size_t)b * a.Tn + tt) * a.G + g) * a.k;
+    float lj = -INFINITY;
+    if (lane < a.k) {
+        const int id = a.ids[(((size_t)b * a.T + t) * a.G + g) * a.k + lane];
+        if (pair_valid(id, a.Bk, pos) && id < a.nbv) lj = a.part_lse[(pl0 + lane) * a.r + hh];
     }
-    prefill_attn_kernel<D, BK><<<grid, kPaThreads, smem, s>>>(qm, km, vm, a);
+    float m = lj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+    const float wj = m > -INFINITY && lj > -INFINITY ? exp2_approx(lj - m) : 0.f;
+    float L = wj;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
+    float acc[DPL];
+#pragma unroll
+    for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
+    const unsigned valid_mask = __ballot_sync(FULL, wj > 0.f);
+    unsigned mask = valid_mask;
+    // a few partial rows in flight at once
+    while (mask) {
+        int js[4];
+        int nj = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            js[i] = -1;
+            if (mask) {
+                js[i] = __ffs(mask) - 1;
+                mask &= mask - 1;
+                ++nj;
+            }
+        }
+        uint2 raw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            raw[i] = make_uint2(0u, 0u);
+            if (js[i] >= 0) {
+                const __half *src = a.part_o + ((pl0 + js[i]) * a.r + hh) * D + lane * DPL;
+                if constexpr (DPL == 4) raw[i] = __ldcs(reinterpret_cast<const uint2 *>(src));
+                else raw[i].x = __ldcs(reinterpret_cast<const unsigned *>(src));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (js[i] < 0) continue;
+            const float wi = __shfl_sync(FULL, wj, js[i]);
+            const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw[i].x);
+            const float2 f0 = __half22float2(h0);
+            acc[0] = fmaf(wi, f0.x, acc[0]);
+            acc[1] = fmaf(wi, f0.y, acc[1]);
+            if constexpr (DPL == 4) {
+                const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw[i].y);
+                const float2 f1 = __half22float2(h1);
+                acc[2] = fmaf(wi, f1.x, acc[2]);
+                acc[3] = fmaf(wi, f1.y, acc[3]);
+            }
+        }
+        (void)nj;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const int hq = g * a.r + hh;
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + hq) * D + lane * DPL;
+    const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    if constexpr (DPL == 4) {
+        const __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2 *>(o) =
+            make_uint2(*reinterpret_cast<const uint32_t *>(&o0), *reinterpret_cast<const uint32_t *>(&o1));
+    } else {
+        *reinterpret_cast<uint32_t *>(o) = *reinterpret_cast<const uint32_t *>(&o0);
+    }
+    if (lane == 0 && a.lse != nullptr)
+        a.lse[((size_t)b * a.T + t) * a.Hq + hq] = L > 0.f ? (m + log2f(L)) * 0.69314718055994531f : -INFINITY;
+}
+
+template <int D, int BK>
+size_t tile_smem_bytes() {
+    return 1024 + 2 * (size_t)(D / 64) * kHalf + 2 * (size_t)(2 * (D / 64) * BK * 128) + sizeof(PtBars) + 64;
+}
+
+template <int D, int BK>
+cudaError_t launch_tiles(const PrefillAttnArgs &a, const CUtensorMap &qm, const CUtensorMap &km, const CUtensorMap &vm,
+                         int grid, cudaStream_t s) {
+    const size_t smem = tile_smem_bytes<D, BK>();
+    if (smem > 232448) return cudaErrorInvalidValue;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(pa_tile_kernel<D, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    pa_tile_kernel<D, BK><<<grid, kPtThreads, smem, s>>>(qm, km, vm, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+PrefillAttnPlan prefill_attn_plan(const msa_params_t &p) {
+    PrefillAttnPlan L{};
+    const int r = p.n_q_heads / p.n_kv_heads;
+    const int tt = 128 / r;
+    L.rows = p.q_len < kPrefillRowsPerPass ? p.q_len : kPrefillRowsPerPass;
+    L.nbv_max = (p.q_start + p.q_len - 1) / p.block_size + 1;
+    const size_t pairs = (size_t)p.batch * L.rows * p.n_kv_heads * p.top_k;
+    const size_t buckets = (size_t)p.batch * p.n_kv_heads * L.nbv_max;
+    L.max_tiles = (int)(pairs / tt + buckets + 1);
+    auto r256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+    size_t off = kStatusBytes;
+    L.counts = off; off += r256(buckets * 4);
+    L.offsets = off; off += r256(buckets * 4);
+    L.n_tiles = off; off += 256;
+    L.rank = off; off += r256(pairs * 4);
+    L.members = off; off += r256(pairs * 4);
+    L.tiles = off; off += r256((size_t)L.max_tiles * 16);
+    L.part_lse = off; off += r256(pairs * r * 4);
+    L.part_o = off; off += r256(pairs * r * p.head_dim * 2);
+    L.total = off;
+    return L;
+}
+
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_cache, const void *v_cache, int n_sm,
                                 cudaStream_t s, const char **why) {
-    const int TQ = kPaRows / a.r;
-    a.max_union = TQ * a.k;
-    a.mask_words = (TQ + 31) / 32;
-    const int nb_all = (a.L_max + a.Bk - 1) / a.Bk;
-    a.bitmap_words = (nb_all + 31) / 32;
     CUtensorMap qm, km, vm;
-    const unsigned long long qdim[3] = {(unsigned long long)a.D, (unsigned long long)a.Hq,
-                                        (unsigned long long)a.B * a.T};
-    const unsigned long long qstr[2] = {(unsigned long long)a.D * 2, (unsigned long long)a.Hq * a.D * 2};
-    const unsigned qbox[3] = {64, (unsigned)a.r, (unsigned)TQ};
+    // q as [B * T * Hq rows, D]: a box of 64 dims x r rows holds one member's r heads
     *why = "encoding the prefill attention tensor maps failed";
-    if (!encode_3d(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(q), qdim, qstr, qbox,
+    if (!encode_2d(&qm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(q), a.D,
+                   (unsigned long long)a.B * a.T * a.Hq, (unsigned long long)a.D * 2, 64, a.r,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
@@ -561,11 +674,35 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
         !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(v_cache), a.D, rows,
                    (unsigned long long)a.D * 2, 64, a.Bk, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    const int n_units = a.B * a.G * ((a.T + TQ - 1) / TQ);
-    const int grid = n_units < n_sm ? n_units : n_sm;
-    *why = "prefill attention launch (shared memory or shape out of range)";
-    if (a.D == 128) return a.Bk == 128 ? launch_pa<128, 128>(a, qm, km, vm, grid, s) : launch_pa<128, 64>(a, qm, km, vm, grid, s);
-    return a.Bk == 128 ? launch_pa<64, 128>(a, qm, km, vm, grid, s) : launch_pa<64, 64>(a, qm, km, vm, grid, s);
+    a.tt = 128 / a.r;
+    cudaError_t e = cudaSuccess;
+    for (int t0 = 0; t0 < a.T && e == cudaSuccess; t0 += kPrefillRowsPerPass) {
+        a.t0 = t0;
+        a.Tn = a.T - t0 < kPrefillRowsPerPass ? a.T - t0 : kPrefillRowsPerPass;
+        a.nbv = (a.q_start + t0 + a.Tn - 1) / a.Bk + 1;
+        const long long pairs = (long long)a.B * a.Tn * a.G * a.k;
+        const int pgrid = (int)((pairs + 255) / 256 < 4LL * n_sm ? (pairs + 255) / 256 : 4LL * n_sm);
+        *why = "prefill attention bucketing";
+        e = cudaMemsetAsync(a.counts, 0, (size_t)a.B * a.G * a.nbv * 4, s);
+        if (e != cudaSuccess) break;
+        pa_count_kernel<<<pgrid, 256, 0, s>>>(a);
+        pa_scan_kernel<<<1, 1024, 0, s>>>(a);
+        pa_scatter_kernel<<<pgrid, 256, 0, s>>>(a);
+        if ((e = cudaGetLastError()) != cudaSuccess) break;
+        *why = "prefill attention tile launch (shared memory or shape out of range)";
+        if (a.D == 128)
+            e = a.Bk == 128 ? launch_tiles<128, 128>(a, qm, km, vm, n_sm, s) : launch_tiles<128, 64>(a, qm, km, vm, n_sm, s);
+        else
+            e = a.Bk == 128 ? launch_tiles<64, 128>(a, qm, km, vm, n_sm, s) : launch_tiles<64, 64>(a, qm, km, vm, n_sm, s);
+        if (e != cudaSuccess) break;
+        *why = "prefill attention merge launch";
+        const long long warps = (long long)a.B * a.Tn * a.G * a.r;
+        const int mgrid = (int)((warps * 32 + 255) / 256);
+        if (a.D == 128) pa_merge_kernel<128><<<mgrid, 256, 0, s>>>(a);
+        else pa_merge_kernel<64><<<mgrid, 256, 0, s>>>(a);
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 }  // namespace msa
