@@ -580,11 +580,12 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
     a.counts = reinterpret_cast<int *>(w + L.counts);
     a.offsets = reinterpret_cast<int *>(w + L.offsets);
     a.n_tiles = reinterpret_cast<int *>(w + L.n_tiles);
+    a.block_sums = reinterpret_cast<int *>(w + L.block_sums);
     a.rank = reinterpret_cast<int *>(w + L.rank);
     a.members = reinterpret_cast<int *>(w + L.members);
     a.tiles = reinterpret_cast<int4 *>(w + L.tiles);
     a.part_lse = reinterpret_cast<float *>(w + L.part_lse);
-    a.part_o = reinterpret_cast<__half *>(w + L.part_o);
+    a.part_o = reinterpret_cast<__nv_bfloat16 *>(w + L.part_o);
     const char *why = "";
     cudaError_t e = launch_prefill_attn(a, q, k_cache, v_cache, n_sm, (cudaStream_t)stream, &why);
     if (e != cudaSuccess) return cuda_fail(e, why);

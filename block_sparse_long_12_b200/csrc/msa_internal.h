@@ -2,7 +2,7 @@
 #pragma once
 
 #include <cuda.h>
-#include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -135,14 +135,15 @@ struct PrefillAttnArgs {
     int *members;              // [pairs] member tt * k + slot, grouped by bucket
     int4 *tiles;               // [max_tiles] (bucket, first member, member count, 0)
     int *n_tiles;
-    __half *part_o;            // [B*Tn*G*k][r][D] per-pair output, normalised by the pair's sum
+    int *block_sums;           // [2 * scan blocks] pairs and tiles of each scan block's buckets
+    __nv_bfloat16 *part_o;     // [B*Tn*G*k][D/8][r][8] per-pair output (chunk-major), normalised by the pair's sum
     float *part_lse;           // [B*Tn*G*k][r] per-pair log2 normaliser
 };
 
 // Workspace of one prefill attention call (offsets in bytes).
 struct PrefillAttnPlan {
     int rows, nbv_max, max_tiles;
-    size_t counts, offsets, n_tiles, rank, members, tiles, part_lse, part_o, total;
+    size_t counts, offsets, n_tiles, block_sums, rank, members, tiles, part_lse, part_o, total;
 };
 PrefillAttnPlan prefill_attn_plan(const msa_params_t &p);
 

@@ -10,15 +10,18 @@
 // with their r heads (M = 128) against that one block.  A pair's attention is
 // then exact within the block -- S = Q K^T, softmax over the block's visible
 // keys, O = P V normalised by the block's sum -- and its output and log2 sum
-// go to the workspace; a merge kernel combines each row's k pairs by
+// (bf16) go to the workspace; a merge kernel combines each row's k pairs by
 // log-sum-exp into the row's output.  No tile computes a row that did not
 // select its block.
 //
 // Per pass over up to kPrefillRowsPerPass query rows:
 //   pa_count_kernel     pairs per bucket and each pair's rank in it;
-//   pa_scan_kernel      bucket offsets and the tile list (bucket order);
+//   pa_tilecount_kernel pairs and tiles per scan block of 1024 buckets;
+//   pa_emit_kernel      bucket offsets and the tile list (bucket order);
 //   pa_scatter_kernel   members grouped by bucket;
 //   pa_tile_kernel      the tiles, persistent, one contiguous range per SM:
+//     warp 3      stages each tile's descriptor and member list in a
+//                 shared-memory ring that every other role reads;
 //     warp 0      TMA of the block's K and V tiles (2-stage ring, reloaded
 //                 only when the bucket changes);
 //     warp 1      TMEM owner, issues tcgen05.mma: S = Q K^T (M 128, N Bk)
@@ -31,8 +34,10 @@
 //                 block's keys each: mask keys after the row, row max
 //                 (exchanged between the two), P = 2^(z*c - m) as bf16 into
 //                 TMEM, row sums;
-//     warps 12-15 epilogue: O / sum as fp16 and the log2 sum per pair;
-//   pa_merge_kernel     per row and head: log-sum-exp of its pairs -> o, lse.
+//     warps 12-15 epilogue: O / sum as bf16, stored chunk-major per pair so
+//                 that the r heads of a member (consecutive lanes) write
+//                 whole lines, and the log2 sum per pair;
+//   pa_merge_kernel     per row and group: log-sum-exp of its pairs -> o, lse.
 #include "tcgen05.cuh"
 
 namespace msa {
@@ -46,6 +51,18 @@ constexpr int kPtSmWarps = 8;
 constexpr int kPtEpi0 = 12;     // first epilogue warp
 constexpr int kPtEpiWarps = 4;
 constexpr int kHalf = 16384;    // one 128-row x 128-byte operand tile
+constexpr int kInfoSlots = 6;   // tiles staged ahead in shared memory
+// every role but the stager releases a tile's info slot: K/V producer, MMA issuer, Q gather,
+// the softmax warps, the epilogue warps
+constexpr int kInfoConsumers = 3 + kPtSmWarps + kPtEpiWarps;
+constexpr int kRun = 8;         // consecutive tiles of the list a CTA takes at a time
+
+// One tile as the roles read it: its block, members, and whether the next tile changes block.
+struct TileInfo {
+    int bkt, start, cnt, last;  // last: the CTA's next tile is another bucket (or none)
+    int b, g, n, pad;
+    int mem[kPtRows];           // member i: row tt * k + slot
+};
 
 struct PtBars {
     uint64_t kv_full[2], kv_empty[2];
@@ -54,12 +71,14 @@ struct PtBars {
     uint64_t p_full[2];
     uint64_t o_full[2], o_empty[2];
     uint64_t ml_full[2], ml_empty[2];
+    uint64_t info_full[kInfoSlots], info_empty[kInfoSlots];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
     float red_m[2][2][kPtRows];  // [buffer][column half][row] raw max of the half row
     float ml_m[2][kPtRows];      // [buffer][row] row max, log2 domain
     float ml_l[2][2][kPtRows];   // [buffer][column half][row] sum of the half row
+    TileInfo info[kInfoSlots];
 };
 
 __device__ inline void mbar_arrive1(uint64_t *bar) {
@@ -163,51 +182,85 @@ __global__ void pa_count_kernel(const PrefillAttnArgs a) {
     }
 }
 
-// One CTA: exclusive scan of the bucket counts (pairs and tiles), tile list in bucket order.
-__global__ void __launch_bounds__(1024) pa_scan_kernel(const PrefillAttnArgs a) {
-    __shared__ long long wsum_p[32], wsum_t[32];
-    const int nb = a.B * a.G * a.nbv;
-    const int per = (nb + 1023) / 1024;
-    const int s0 = threadIdx.x * per, s1 = s0 + per < nb ? s0 + per : nb;
-    long long lp = 0, lt = 0;
-    for (int s = s0; s < s1; ++s) {
-        const int c = a.counts[s];
-        lp += c;
-        lt += (c + a.tt - 1) / a.tt;
-    }
-    // block-wide exclusive scan of (lp, lt)
+// Block-wide sum of (x, y) over 1024 threads; every thread gets the totals.
+__device__ inline void block_sum2(long long &x, long long &y, long long (*sh)[2]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    long long ip = lp, it = lt;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        x += __shfl_xor_sync(FULL, x, o);
+        y += __shfl_xor_sync(FULL, y, o);
+    }
+    __syncthreads();
+    if (lane == 0) { sh[warp][0] = x; sh[warp][1] = y; }
+    __syncthreads();
+    x = lane < (int)(blockDim.x >> 5) ? sh[lane][0] : 0;
+    y = lane < (int)(blockDim.x >> 5) ? sh[lane][1] : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        x += __shfl_xor_sync(FULL, x, o);
+        y += __shfl_xor_sync(FULL, y, o);
+    }
+}
+
+// Pairs and tiles of the 1024 buckets of each scan block.
+__global__ void __launch_bounds__(1024) pa_tilecount_kernel(const PrefillAttnArgs a) {
+    __shared__ long long sh[32][2];
+    const int nb = a.B * a.G * a.nbv;
+    const int s = blockIdx.x * 1024 + threadIdx.x;
+    const int c = s < nb ? a.counts[s] : 0;
+    long long p = c, t = (c + a.tt - 1) / a.tt;
+    block_sum2(p, t, sh);
+    if (threadIdx.x == 0) {
+        a.block_sums[2 * blockIdx.x] = (int)p;
+        a.block_sums[2 * blockIdx.x + 1] = (int)t;
+    }
+}
+
+// Exclusive scan of the bucket counts (pairs and tiles): bucket offsets and the tile list in
+// bucket order.  Each block adds the totals of the blocks before it.
+__global__ void __launch_bounds__(1024) pa_emit_kernel(const PrefillAttnArgs a) {
+    __shared__ long long sh[32][2];
+    __shared__ long long wsum[32][2];
+    const int nb = a.B * a.G * a.nbv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long bp = 0, bt = 0;
+    for (int i = threadIdx.x; i < (int)blockIdx.x; i += 1024) {
+        bp += a.block_sums[2 * i];
+        bt += a.block_sums[2 * i + 1];
+    }
+    block_sum2(bp, bt, sh);
+    const int s = blockIdx.x * 1024 + threadIdx.x;
+    const int c = s < nb ? a.counts[s] : 0;
+    const long long nt = (c + a.tt - 1) / a.tt;
+    long long ip = c, it = nt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const long long vp = __shfl_up_sync(FULL, ip, o), vt = __shfl_up_sync(FULL, it, o);
         if (lane >= o) { ip += vp; it += vt; }
     }
-    if (lane == 31) { wsum_p[warp] = ip; wsum_t[warp] = it; }
+    if (lane == 31) { wsum[warp][0] = ip; wsum[warp][1] = it; }
     __syncthreads();
     if (warp == 0) {
-        long long xp = wsum_p[lane], xt = wsum_t[lane];
+        long long xp = wsum[lane][0], xt = wsum[lane][1];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const long long vp = __shfl_up_sync(FULL, xp, o), vt = __shfl_up_sync(FULL, xt, o);
             if (lane >= o) { xp += vp; xt += vt; }
         }
-        wsum_p[lane] = xp;
-        wsum_t[lane] = xt;
+        wsum[lane][0] = xp;
+        wsum[lane][1] = xt;
     }
     __syncthreads();
-    long long bp = ip - lp + (warp > 0 ? wsum_p[warp - 1] : 0);
-    long long bt = it - lt + (warp > 0 ? wsum_t[warp - 1] : 0);
-    for (int s = s0; s < s1; ++s) {
-        const int c = a.counts[s];
-        a.offsets[s] = (int)bp;
-        for (int q = 0; q * a.tt < c; ++q) {
+    long long p0 = bp + ip - c + (warp > 0 ? wsum[warp - 1][0] : 0);
+    long long t0 = bt + it - nt + (warp > 0 ? wsum[warp - 1][1] : 0);
+    if (s < nb) {
+        a.offsets[s] = (int)p0;
+        for (int q = 0; q < nt; ++q) {
             const int m = c - q * a.tt < a.tt ? c - q * a.tt : a.tt;
-            a.tiles[bt++] = make_int4(s, (int)bp + q * a.tt, m, 0);
+            a.tiles[t0 + q] = make_int4(s, (int)p0 + q * a.tt, m, 0);
         }
-        bp += c;
     }
-    if (threadIdx.x == 1023) *a.n_tiles = (int)wsum_t[31];
+    if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 1023) *a.n_tiles = (int)(bt + wsum[31][1]);
 }
 
 __global__ void pa_scatter_kernel(const PrefillAttnArgs a) {
@@ -256,6 +309,10 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             mbar_init(&S.o_full[i], 1); mbar_init(&S.o_empty[i], kPtEpiWarps);
             mbar_init(&S.ml_full[i], kPtSmWarps); mbar_init(&S.ml_empty[i], kPtEpiWarps);
         }
+        for (int i = 0; i < kInfoSlots; ++i) {
+            mbar_init(&S.info_full[i], 1);
+            mbar_init(&S.info_empty[i], kInfoConsumers);
+        }
         mbar_init(&S.mma_done, 1);
         S.abort_flag = 0;
         fence_mbar_init();
@@ -273,30 +330,66 @@ __global__ void __launch_bounds__(kPtThreads, 1)
     const uint32_t tmem = S.tmem_base;
     volatile int *abort_flag = &S.abort_flag;
 
-    // this CTA's contiguous range of tiles (bucket order: consecutive tiles mostly share a block)
-    const long long nt = *a.n_tiles;
-    const int tb = (int)(nt * blockIdx.x / gridDim.x), te = (int)(nt * (blockIdx.x + 1) / gridDim.x);
+    // This CTA's tiles: runs of kRun consecutive tiles of the list (bucket order), every gridDim.x-th
+    // run, so that consecutive tiles of a CTA mostly share a block (its K/V stays) while all CTAs
+    // sweep the list together (the query rows of one group at a time stay in L2).
+    const int nt = *a.n_tiles;
+    const int n_runs = (nt + kRun - 1) / kRun;
+    const int my_runs = (int)blockIdx.x < n_runs ? (n_runs - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    int n_my = my_runs * kRun;
+    if (my_runs > 0 && (int)blockIdx.x + (my_runs - 1) * (int)gridDim.x == n_runs - 1) n_my -= n_runs * kRun - nt;
+    auto tile_of = [&](int il) { return ((il / kRun) * (int)gridDim.x + (int)blockIdx.x) * kRun + il % kRun; };
     const int r = a.r;
-    auto bucket_block = [&](int bkt, int &b, int &g, int &n) {
-        const int bg = bkt / a.nbv;
-        n = bkt - bg * a.nbv;
-        b = bg / a.G;
-        g = bg - b * a.G;
+    // wait for tile il's info (whole warp; false if the CTA gives up)
+    auto info_wait = [&](int il) -> bool {
+        bool ok = true;
+        if (lane == 0) ok = tc::wait_or_abort(&S.info_full[il % kInfoSlots], (il / kInfoSlots) & 1, abort_flag, a.status);
+        return __shfl_sync(FULL, ok, 0) != 0;
+    };
+    auto info_release = [&](int il) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive1(&S.info_empty[il % kInfoSlots]);
     };
 
-    if (warp == 0) {
+    if (warp == 3) {
+        // ------------------------------------------------ tile info stager
+        for (int il = 0; il < n_my; ++il) {
+            const int ti = tile_of(il), slot = il % kInfoSlots;
+            bool ok = true;
+            if (lane == 0) ok = tc::wait_or_abort(&S.info_empty[slot], ((il / kInfoSlots) & 1) ^ 1, abort_flag, a.status);
+            if (!__shfl_sync(FULL, ok, 0)) break;
+            const int4 tile = a.tiles[ti];
+            TileInfo &I = S.info[slot];
+            for (int m = lane; m < tile.z; m += 32) I.mem[m] = a.members[tile.y + m];
+            if (lane == 0) {
+                const int bg = tile.x / a.nbv;
+                I.bkt = tile.x;
+                I.start = tile.y;
+                I.cnt = tile.z;
+                I.last = il + 1 == n_my || a.tiles[tile_of(il + 1)].x != tile.x;
+                I.n = tile.x - bg * a.nbv;
+                I.b = bg / a.G;
+                I.g = bg - I.b * a.G;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive1(&S.info_full[slot]);
+        }
+    } else if (warp == 0) {
         // ------------------------------------------------ K/V producer: one load per new bucket
-        if (lane == 0) {
-            int kvi = -1, prev = -1;
-            for (int ti = tb; ti < te; ++ti) {
-                const int bkt = a.tiles[ti].x;
-                if (bkt == prev) continue;
-                prev = bkt;
-                ++kvi;
-                const int ks = kvi & 1;
-                if (!tc::wait_or_abort(&S.kv_empty[ks], ((kvi >> 1) & 1) ^ 1, abort_flag, a.status)) break;
-                int b, g, n;
-                bucket_block(bkt, b, g, n);
+        int kvi = -1, prev = -1;
+        for (int il = 0; il < n_my; ++il) {
+            if (!info_wait(il)) break;
+            const TileInfo &I = S.info[il % kInfoSlots];
+            const int bkt = I.bkt, b = I.b, g = I.g, n = I.n;
+            info_release(il);
+            if (bkt == prev) continue;
+            prev = bkt;
+            ++kvi;
+            const int ks = kvi & 1;
+            bool ok = true;
+            if (lane == 0) ok = tc::wait_or_abort(&S.kv_empty[ks], ((kvi >> 1) & 1) ^ 1, abort_flag, a.status);
+            if (!__shfl_sync(FULL, ok, 0)) break;
+            if (lane == 0) {
                 mbar_arrive_expect_tx(&S.kv_full[ks], 2 * NH * KVH);
                 const int row = (b * a.G + g) * a.L_max + n * BK;
                 unsigned char *dst = smKV + ks * KV_STAGE;
@@ -304,79 +397,92 @@ __global__ void __launch_bounds__(kPtThreads, 1)
                 for (int h = 0; h < NH; ++h)
                     tc::tma_load_2d(dst + (NH + h) * KVH, &vmap, h * 64, row, &S.kv_full[ks]);
             }
+            __syncwarp();
         }
     } else if (warp == 2) {
         // ------------------------------------------------ Q gather: the members' r heads, one box per member and half
-        for (int ti = tb; ti < te; ++ti) {
-            const int il = ti - tb, qs = il & 1;
+        for (int il = 0; il < n_my; ++il) {
+            const int qs = il & 1;
+            if (!info_wait(il)) break;
+            const TileInfo &I = S.info[il % kInfoSlots];
+            const int cnt = I.cnt, b = I.b, g = I.g;
+            int mem[kPtRows / 32];
+#pragma unroll
+            for (int q = 0; q < kPtRows / 32; ++q) mem[q] = lane + 32 * q < cnt ? I.mem[lane + 32 * q] : 0;
+            info_release(il);
             bool ok = true;
             if (lane == 0) ok = tc::wait_or_abort(&S.q_empty[qs], ((il >> 1) & 1) ^ 1, abort_flag, a.status);
             if (!__shfl_sync(FULL, ok, 0)) break;
-            const int4 tile = a.tiles[ti];
-            int b, g, n;
-            bucket_block(tile.x, b, g, n);
-            if (lane == 0) mbar_arrive_expect_tx(&S.q_full[qs], (uint32_t)tile.z * r * 128 * NH);
+            if (lane == 0) mbar_arrive_expect_tx(&S.q_full[qs], (uint32_t)cnt * r * 128 * NH);
             __syncwarp();
-            for (int m = lane; m < tile.z; m += 32) {
-                const int tt = a.members[tile.y + m] / a.k;
-                const int qrow = ((b * a.T + a.t0 + tt) * a.Hq) + g * r;
-                for (int h = 0; h < NH; ++h)
-                    tc::tma_load_2d(smQ + qs * Q_STAGE + h * kHalf + m * r * 128, &qmap, h * 64, qrow, &S.q_full[qs]);
+#pragma unroll
+            for (int q = 0; q < kPtRows / 32; ++q) {
+                const int m = lane + 32 * q;
+                if (m < cnt) {
+                    const int qrow = ((b * a.T + a.t0 + mem[q] / a.k) * a.Hq) + g * r;
+                    for (int h = 0; h < NH; ++h)
+                        tc::tma_load_2d(smQ + qs * Q_STAGE + h * kHalf + m * r * 128, &qmap, h * 64, qrow,
+                                        &S.q_full[qs]);
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc_qk = tc::idesc_bf16_f32(kPtRows, BK);
-            const uint32_t idesc_pv = tc::idesc_bf16_f32(kPtRows, D) | (1u << 16);  // B (V) is MN-major
-            int kvi = -1, prev = -1;
-            int pend = -1, pend_ks = 0;
-            bool pend_last = false, ok = true;
-            // O = P V of tile `il` (its P overwrote its S buffer); frees the S buffer and, after a
-            // bucket's last tile, the K/V stage
-            auto issue_pv = [&](int il, int ks, bool last) -> bool {
-                const int ob = il & 1;
-                if (!tc::wait_or_abort(&S.p_full[ob], (il >> 1) & 1, abort_flag, a.status)) return false;
-                if (!tc::wait_or_abort(&S.o_empty[ob], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
-                tc::fence_after_sync();
-                const uint32_t v_addr = smem_u32(smKV + ks * KV_STAGE + NH * KVH);
+        const uint32_t idesc_qk = tc::idesc_bf16_f32(kPtRows, BK);
+        const uint32_t idesc_pv = tc::idesc_bf16_f32(kPtRows, D) | (1u << 16);  // B (V) is MN-major
+        int kvi = -1, prev = -1;
+        int pend = -1, pend_ks = 0;
+        bool pend_last = false, ok = true;
+        // O = P V of tile `il` (its P overwrote its S buffer); frees the S buffer and, after a
+        // bucket's last tile, the K/V stage
+        auto issue_pv = [&](int il, int ks, bool last) -> bool {
+            const int ob = il & 1;
+            if (!tc::wait_or_abort(&S.p_full[ob], (il >> 1) & 1, abort_flag, a.status)) return false;
+            if (!tc::wait_or_abort(&S.o_empty[ob], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+            tc::fence_after_sync();
+            const uint32_t v_addr = smem_u32(smKV + ks * KV_STAGE + NH * KVH);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_bf16_ts(tmem + O_COL + ob * D, tmem + ob * BK + kk * 8, sw128_mnmajor_desc(v_addr + kk * 2048, KVH),
-                                idesc_pv, kk > 0 ? 1u : 0u);
-                tc::mma_commit(&S.o_full[ob]);
-                tc::mma_commit(&S.s_empty[ob]);
-                if (last) tc::mma_commit(&S.kv_empty[ks]);
-                return true;
-            };
-            for (int ti = tb; ti < te && ok; ++ti) {
-                const int il = ti - tb, sb = il & 1;
-                const int bkt = a.tiles[ti].x;
-                if (bkt != prev) { prev = bkt; ++kvi; }
-                const int ks = kvi & 1;
-                const bool last = ti + 1 == te || a.tiles[ti + 1].x != bkt;
+            for (int kk = 0; kk < BK / 16; ++kk)
+                mma_bf16_ts(tmem + O_COL + ob * D, tmem + ob * BK + kk * 8, sw128_mnmajor_desc(v_addr + kk * 2048, KVH),
+                            idesc_pv, kk > 0 ? 1u : 0u);
+            tc::mma_commit(&S.o_full[ob]);
+            tc::mma_commit(&S.s_empty[ob]);
+            if (last) tc::mma_commit(&S.kv_empty[ks]);
+            return true;
+        };
+        for (int il = 0; il < n_my && ok; ++il) {
+            const int sb = il & 1;
+            if (!info_wait(il)) break;
+            const TileInfo &I = S.info[il % kInfoSlots];
+            const int bkt = I.bkt;
+            const bool last = I.last != 0;
+            info_release(il);
+            if (bkt != prev) { prev = bkt; ++kvi; }
+            const int ks = kvi & 1;
+            if (lane == 0) {
                 if (!tc::wait_or_abort(&S.q_full[sb], (il >> 1) & 1, abort_flag, a.status) ||
                     !tc::wait_or_abort(&S.kv_full[ks], (kvi >> 1) & 1, abort_flag, a.status) ||
                     !tc::wait_or_abort(&S.s_empty[sb], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) {
                     ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const uint32_t q_addr = smem_u32(smQ + sb * Q_STAGE), k_addr = smem_u32(smKV + ks * KV_STAGE);
+                } else {
+                    tc::fence_after_sync();
+                    const uint32_t q_addr = smem_u32(smQ + sb * Q_STAGE), k_addr = smem_u32(smKV + ks * KV_STAGE);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32),
-                                    tc::sw128_kmajor_desc(k_addr + (kk >> 2) * KVH + (kk & 3) * 32), idesc_qk, kk > 0);
-                tc::mma_commit(&S.q_empty[sb]);
-                tc::mma_commit(&S.s_full[sb]);
-                if (pend >= 0 && !issue_pv(pend, pend_ks, pend_last)) {
-                    ok = false;
-                    break;
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32),
+                                        tc::sw128_kmajor_desc(k_addr + (kk >> 2) * KVH + (kk & 3) * 32), idesc_qk,
+                                        kk > 0);
+                    tc::mma_commit(&S.q_empty[sb]);
+                    tc::mma_commit(&S.s_full[sb]);
+                    if (pend >= 0 && !issue_pv(pend, pend_ks, pend_last)) ok = false;
                 }
-                pend = il;
-                pend_ks = ks;
-                pend_last = last;
             }
+            ok = __shfl_sync(FULL, ok, 0) != 0;
+            pend = il;
+            pend_ks = ks;
+            pend_last = last;
+        }
+        if (lane == 0) {
             if (ok && pend >= 0) issue_pv(pend, pend_ks, pend_last);
             tc::mma_commit(&S.mma_done);
             mbar_wait(&S.mma_done, 0, a.status);
@@ -394,15 +500,19 @@ __global__ void __launch_bounds__(kPtThreads, 1)
         const int m_i = row / r;
         const float c = a.scale_log2;
         bool ok = true;
-        for (int ti = tb; ti < te; ++ti) {
-            const int il = ti - tb, sb = il & 1, par = (il >> 1) & 1;
-            const int4 tile = a.tiles[ti];
-            int b, g, n;
-            bucket_block(tile.x, b, g, n);
-            const bool valid = m_i < tile.z;
+        for (int il = 0; il < n_my; ++il) {
+            const int sb = il & 1, par = (il >> 1) & 1;
+            if (ok) ok = info_wait(il);
+            int n = 0, pos = 0;
+            bool valid = false;
+            if (ok) {
+                const TileInfo &I = S.info[il % kInfoSlots];
+                n = I.n;
+                valid = m_i < I.cnt;
+                if (valid) pos = a.q_start + a.t0 + I.mem[m_i] / a.k;
+                info_release(il);
+            }
             const bool any = __any_sync(FULL, valid);
-            int pos = 0;
-            if (valid) pos = a.q_start + a.t0 + a.members[tile.y + m_i] / a.k;
             if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.s_full[sb], par, abort_flag, a.status));
             if (ok) ok = __all_sync(FULL, tc::wait_or_abort(&S.ml_empty[sb], par ^ 1, abort_flag, a.status));
             uint32_t zr[CW];
@@ -464,22 +574,27 @@ __global__ void __launch_bounds__(kPtThreads, 1)
         }
     } else if (warp >= kPtEpi0) {
         // ------------------------------------------------ epilogue: one pair row per lane
+        // A pair's r x D outputs are stored chunk-major ([D / 8 chunks][r heads][8 dims]), so the r
+        // heads of a member -- r consecutive lanes -- write r * 16 contiguous bytes per store.
         const int qd = warp & 3;
         const int row = qd * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         const int m_i = row / r, hh = row % r;
-        for (int ti = tb; ti < te; ++ti) {
-            const int il = ti - tb, ob = il & 1, par = (il >> 1) & 1;
-            const int4 tile = a.tiles[ti];
-            int b, g, n;
-            bucket_block(tile.x, b, g, n);
-            const bool valid = m_i < tile.z;
-            const bool any = __any_sync(FULL, valid);
+        for (int il = 0; il < n_my; ++il) {
+            const int ob = il & 1, par = (il >> 1) & 1;
+            if (!info_wait(il)) break;
+            bool valid;
             int pl = 0;
-            if (valid) {
-                const int mem = a.members[tile.y + m_i];
-                pl = ((b * a.Tn + mem / a.k) * a.G + g) * a.k + mem % a.k;  // the pair's index in this pass
+            {
+                const TileInfo &I = S.info[il % kInfoSlots];
+                valid = m_i < I.cnt;
+                if (valid) {
+                    const int mem = I.mem[m_i];
+                    pl = ((I.b * a.Tn + mem / a.k) * a.G + I.g) * a.k + mem % a.k;  // the pair's index in this pass
+                }
+                info_release(il);
             }
+            const bool any = __any_sync(FULL, valid);
             if (!__all_sync(FULL, tc::wait_or_abort(&S.ml_full[ob], par, abort_flag, a.status))) break;
             const float m2 = S.ml_m[ob][row];
             const float l = S.ml_l[ob][0][row] + S.ml_l[ob][1][row];
@@ -489,31 +604,30 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             tc::fence_after_sync();
             if (any) {
                 const float inv = valid && l > 0.f ? 1.f / l : 0.f;
-                __half *dst = a.part_o + ((size_t)pl * r + hh) * D;
+                uint4 *dst = reinterpret_cast<uint4 *>(a.part_o + (size_t)pl * r * D) + hh;
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t ov[32];
                     tc::tmem_ld32(tmem + lane_addr + O_COL + ob * D + cc * 32, ov);
                     tc::tmem_ld_wait();
-                    if (valid) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t pk[4];
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t pk[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __half2 h2 = __floats2half2_rn(__uint_as_float(ov[q * 8 + 2 * e]) * inv,
-                                                                     __uint_as_float(ov[q * 8 + 2 * e + 1]) * inv);
-                                pk[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                            }
-                            *reinterpret_cast<uint4 *>(dst + cc * 32 + q * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(ov[q * 8 + 2 * e]) * inv,
+                                                                            __uint_as_float(ov[q * 8 + 2 * e + 1]) * inv);
+                            pk[e] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
+                        if (valid)  // read once, by the merge: stream past L2
+                            __stcs(dst + (cc * 4 + q) * r, make_uint4(pk[0], pk[1], pk[2], pk[3]));
                     }
                 }
             }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive1(&S.o_empty[ob]);
-            if (valid) a.part_lse[(size_t)pl * r + hh] = l > 0.f ? m2 + log2f(l) : -INFINITY;
+            if (valid) __stcs(a.part_lse + (size_t)pl * r + hh, l > 0.f ? m2 + log2f(l) : -INFINITY);
         }
     }
     tc::fence_before_sync();
@@ -525,93 +639,105 @@ __global__ void __launch_bounds__(kPtThreads, 1)
 }
 
 // ------------------------------------------------------------------ merge
-// One warp per (sequence, row, group, head): the log-sum-exp combination of the row's pairs.
-template <int D>
-__global__ void __launch_bounds__(256) pa_merge_kernel(const PrefillAttnArgs a) {
-    constexpr int DPL = D / 32;  // dims per lane
-    const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const long long n_rows = (long long)a.B * a.Tn * a.G * a.r;
-    if (w >= n_rows) return;
-    const int hh = (int)(w % a.r);
-    long long rest = w / a.r;
-    const int g = (int)(rest % a.G);
-    rest /= a.G;
+// One warp per (sequence, row, group): the log-sum-exp combination of the row's pairs for all r
+// heads of the group.  A pair's r x D bf16 partials are one contiguous block, chunk-major (16-byte
+// chunk c = dims 8 (c / r) .., head c % r), read with lane l on chunks l, l + 32, ... (PER per
+// lane); the r heads' outputs of the row are contiguous too (head-major), written back per chunk.
+template <int PER>
+__global__ void __launch_bounds__(256, 2) pa_merge_kernel(const PrefillAttnArgs a) {
+    __shared__ float s_lse[8][kMaxTopKList * 16];  // per warp: [slot][head] log2 sums
+    __shared__ float s_m[8][16], s_inv[8][16];     // per warp and head: max, 1 / sum of weights
+    const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long w = blockIdx.x * 8LL + wib;
+    if (w >= (long long)a.B * a.Tn * a.G) return;  // whole warps only; no block-wide barrier below
+    const int g = (int)(w % a.G);
+    const long long rest = w / a.G;
     const int tt = (int)(rest % a.Tn);
     const int b = (int)(rest / a.Tn);
     const int t = a.t0 + tt;
     const int pos = a.q_start + t;
-    const size_t pl0 = (((size_t)b * a.Tn + tt) * a.G + g) * a.k;
-    float lj = -INFINITY;
-    if (lane < a.k) {
-        const int id = a.ids[(((size_t)b * a.T + t) * a.G + g) * a.k + lane];
-        if (pair_valid(id, a.Bk, pos) && id < a.nbv) lj = a.part_lse[(pl0 + lane) * a.r + hh];
+    const int r = a.r, k = a.k, D = a.D;
+    const int rs = __ffs(r) - 1;  // r is a power of two (it divides 128)
+    const size_t pl0 = (((size_t)b * a.Tn + tt) * a.G + g) * k;
+    bool v = false;
+    if (lane < k) {
+        const int id = a.ids[(((size_t)b * a.T + t) * a.G + g) * k + lane];
+        v = pair_valid(id, a.Bk, pos) && id < a.nbv;
     }
-    float m = lj;
+    const unsigned vmask = __ballot_sync(FULL, v);
+    float *L = s_lse[wib];
+    for (int e = lane; e < k * r; e += 32) L[e] = (vmask >> (e >> rs)) & 1u ? a.part_lse[pl0 * r + e] : -INFINITY;
+    __syncwarp();
+    if (lane < r) {
+        float m = -INFINITY;
+        for (int j = 0; j < k; ++j) m = fmaxf(m, L[j * r + lane]);
+        float sum = 0.f;
+        if (m > -INFINITY)
+            for (int j = 0; j < k; ++j) sum += exp2_approx(L[j * r + lane] - m);
+        s_m[wib][lane] = m;
+        s_inv[wib][lane] = sum > 0.f ? 1.f / sum : 0.f;
+        if (a.lse != nullptr)
+            a.lse[((size_t)b * a.T + t) * a.Hq + g * r + lane] =
+                sum > 0.f ? (m + log2f(sum)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncwarp();
+    const int nch = r * D / 8, cph = D / 8;  // chunks per pair, per head row
+    float acc[PER][8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-    const float wj = m > -INFINITY && lj > -INFINITY ? exp2_approx(lj - m) : 0.f;
-    float L = wj;
+    for (int i = 0; i < PER; ++i)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
-    float acc[DPL];
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+    constexpr int NBATCH = PER >= 8 ? 1 : PER >= 4 ? 2 : 4;  // slots in flight (registers: NBATCH * PER uint4)
+    unsigned mk = vmask;
+    while (mk) {
+        int js[NBATCH];
 #pragma unroll
-    for (int d = 0; d < DPL; ++d) acc[d] = 0.f;
-    const unsigned valid_mask = __ballot_sync(FULL, wj > 0.f);
-    unsigned mask = valid_mask;
-    // a few partial rows in flight at once
-    while (mask) {
-        int js[4];
-        int nj = 0;
+        for (int q = 0; q < NBATCH; ++q) {
+            js[q] = mk ? __ffs(mk) - 1 : -1;
+            if (mk) mk &= mk - 1;
+        }
+        uint4 raw[NBATCH][PER];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            js[i] = -1;
-            if (mask) {
-                js[i] = __ffs(mask) - 1;
-                mask &= mask - 1;
-                ++nj;
+        for (int q = 0; q < NBATCH; ++q)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int c = lane + 32 * i;
+                raw[q][i] = make_uint4(0u, 0u, 0u, 0u);
+                if (js[q] >= 0 && c < nch)
+                    raw[q][i] = __ldcs(reinterpret_cast<const uint4 *>(a.part_o + (pl0 + js[q]) * r * D) + c);
+            }
+#pragma unroll
+        for (int q = 0; q < NBATCH; ++q) {
+            if (js[q] < 0) continue;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int c = lane + 32 * i;
+                if (c >= nch) continue;
+                const int hh = c & (r - 1);
+                const float wt = exp2_approx(L[js[q] * r + hh] - s_m[wib][hh]) * s_inv[wib][hh];
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw[q][i]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(h[e]);
+                    acc[i][2 * e] = fmaf(wt, f.x, acc[i][2 * e]);
+                    acc[i][2 * e + 1] = fmaf(wt, f.y, acc[i][2 * e + 1]);
+                }
             }
         }
-        uint2 raw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            raw[i] = make_uint2(0u, 0u);
-            if (js[i] >= 0) {
-                const __half *src = a.part_o + ((pl0 + js[i]) * a.r + hh) * D + lane * DPL;
-                if constexpr (DPL == 4) raw[i] = __ldcs(reinterpret_cast<const uint2 *>(src));
-                else raw[i].x = __ldcs(reinterpret_cast<const unsigned *>(src));
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (js[i] < 0) continue;
-            const float wi = __shfl_sync(FULL, wj, js[i]);
-            const __half2 h0 = *reinterpret_cast<const __half2 *>(&raw[i].x);
-            const float2 f0 = __half22float2(h0);
-            acc[0] = fmaf(wi, f0.x, acc[0]);
-            acc[1] = fmaf(wi, f0.y, acc[1]);
-            if constexpr (DPL == 4) {
-                const __half2 h1 = *reinterpret_cast<const __half2 *>(&raw[i].y);
-                const float2 f1 = __half22float2(h1);
-                acc[2] = fmaf(wi, f1.x, acc[2]);
-                acc[3] = fmaf(wi, f1.y, acc[3]);
-            }
-        }
-        (void)nj;
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    const int hq = g * a.r + hh;
-    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + hq) * D + lane * DPL;
-    const __nv_bfloat162 o0 = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    if constexpr (DPL == 4) {
-        const __nv_bfloat162 o1 = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-        *reinterpret_cast<uint2 *>(o) =
-            make_uint2(*reinterpret_cast<const uint32_t *>(&o0), *reinterpret_cast<const uint32_t *>(&o1));
-    } else {
-        *reinterpret_cast<uint32_t *>(o) = *reinterpret_cast<const uint32_t *>(&o0);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + g * r) * D;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int c = lane + 32 * i;
+        if (c >= nch) continue;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 o2 = __floats2bfloat162_rn(acc[i][2 * e], acc[i][2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&o2);
+        }
+        reinterpret_cast<uint4 *>(o)[(c & (r - 1)) * cph + (c >> rs)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
-    if (lane == 0 && a.lse != nullptr)
-        a.lse[((size_t)b * a.T + t) * a.Hq + hq] = L > 0.f ? (m + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
 template <int D, int BK>
@@ -650,6 +776,7 @@ PrefillAttnPlan prefill_attn_plan(const msa_params_t &p) {
     L.counts = off; off += r256(buckets * 4);
     L.offsets = off; off += r256(buckets * 4);
     L.n_tiles = off; off += 256;
+    L.block_sums = off; off += r256((buckets + 1023) / 1024 * 8);
     L.rank = off; off += r256(pairs * 4);
     L.members = off; off += r256(pairs * 4);
     L.tiles = off; off += r256((size_t)L.max_tiles * 16);
@@ -685,8 +812,10 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
         *why = "prefill attention bucketing";
         e = cudaMemsetAsync(a.counts, 0, (size_t)a.B * a.G * a.nbv * 4, s);
         if (e != cudaSuccess) break;
+        const int sgrid = (a.B * a.G * a.nbv + 1023) / 1024;
         pa_count_kernel<<<pgrid, 256, 0, s>>>(a);
-        pa_scan_kernel<<<1, 1024, 0, s>>>(a);
+        pa_tilecount_kernel<<<sgrid, 1024, 0, s>>>(a);
+        pa_emit_kernel<<<sgrid, 1024, 0, s>>>(a);
         pa_scatter_kernel<<<pgrid, 256, 0, s>>>(a);
         if ((e = cudaGetLastError()) != cudaSuccess) break;
         *why = "prefill attention tile launch (shared memory or shape out of range)";
@@ -696,10 +825,13 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
             e = a.Bk == 128 ? launch_tiles<64, 128>(a, qm, km, vm, n_sm, s) : launch_tiles<64, 64>(a, qm, km, vm, n_sm, s);
         if (e != cudaSuccess) break;
         *why = "prefill attention merge launch";
-        const long long warps = (long long)a.B * a.Tn * a.G * a.r;
-        const int mgrid = (int)((warps * 32 + 255) / 256);
-        if (a.D == 128) pa_merge_kernel<128><<<mgrid, 256, 0, s>>>(a);
-        else pa_merge_kernel<64><<<mgrid, 256, 0, s>>>(a);
+        const long long warps = (long long)a.B * a.Tn * a.G;
+        const int mgrid = (int)((warps + 7) / 8);
+        const int per = (a.r * a.D / 8 + 31) / 32;  // 16-byte chunks per lane
+        if (per <= 1) pa_merge_kernel<1><<<mgrid, 256, 0, s>>>(a);
+        else if (per <= 2) pa_merge_kernel<2><<<mgrid, 256, 0, s>>>(a);
+        else if (per <= 4) pa_merge_kernel<4><<<mgrid, 256, 0, s>>>(a);
+        else pa_merge_kernel<8><<<mgrid, 256, 0, s>>>(a);
         e = cudaGetLastError();
     }
     return e;

@@ -3,6 +3,7 @@
   python profile_run.py decode --context 262144 --steps 3
   python profile_run.py prefill_index --context 65536 --chunk 8192 --steps 1
   python profile_run.py prefill_attn --context 65536 --chunk 8192 --steps 1
+  python profile_run.py prefill_chunks --context 1048576 --chunks 16,64,127 --steps 1
   python profile_run.py scan_shared --context 1048576 --steps 3
   python profile_run.py large_k --context 262144 --steps 3
 
@@ -75,6 +76,33 @@ def run_prefill_attn(args):
     print("prefill attention done", int(_lib.msa_get_device_status(ws_a)))
 
 
+def run_prefill_chunks(args):
+    """Index branch, then the sparse branch, for a few 8192-token chunks of the 1M-token causal
+    prefill (the chunks listed in --chunks), so that a launch list shows every kernel of a chunk
+    early, in the middle and at the end of the sequence."""
+    w = WORKLOADS["prefill_causal_1m"].scaled(max_seq_len=args.context)
+    inp = make_inputs(w, device="cuda")
+    T = args.chunk
+    todo = [int(c) for c in args.chunks.split(",")]
+    plist = []
+    for c in todo:
+        plist.append(api.make_params(batch=1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                                     n_idx_k_heads=w.n_idx_k_heads, head_dim=w.head_dim, idx_dim=w.idx_dim,
+                                     block_size=w.block_size, top_k=w.top_k, max_seq_len=w.max_seq_len,
+                                     dtype=_lib.MSA_BF16, q_len=T, q_start=c * T))
+    ws_i = api.workspace(plist, _lib.MSA_ENTRY_PREFILL_INDEX_TOPK, "cuda")
+    ws_a = api.workspace(plist, _lib.MSA_ENTRY_ATTN_PREFILL, "cuda")
+    ids = torch.empty(1, T, w.n_kv_heads, w.top_k, dtype=torch.int32, device="cuda")
+    o = torch.empty(1, T, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")
+    for _ in range(args.steps):
+        for c, p in zip(todo, plist):
+            q0 = c * T
+            _lib.msa_prefill_index_topk(p, inp["q_idx"][:, q0:q0 + T], inp["k_idx"], ids, None, ws_i)
+            _lib.msa_sparse_attn_prefill(p, inp["q"][:, q0:q0 + T], inp["k"], inp["v"], ids, o, None, ws_a)
+    torch.cuda.synchronize()
+    print("prefill chunks done", todo, int(_lib.msa_get_device_status(ws_a)))
+
+
 def run_scan_shared(args):
     """The index scan of one index-K head shared by the 8 groups (stored block scores, so that only
     the index keys are on the device)."""
@@ -92,13 +120,16 @@ def run_scan_shared(args):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "scan_shared", "large_k"])
+    ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "prefill_chunks", "scan_shared",
+                                     "large_k"])
     ap.add_argument("--context", type=int, default=262144)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=8192)
     ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--chunks", default="16,64,127", help="prefill_chunks: chunk indices to run")
     args = ap.parse_args()
     {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn,
+     "prefill_chunks": run_prefill_chunks,
      "scan_shared": run_scan_shared,
      "large_k": lambda a: run_decode(a, "decode_ctx1m_large_k")}[args.what](args)
 
