@@ -454,37 +454,46 @@ def run_ours(args, world, rank, local):
         dense()
     dense_us = max_over_ranks(statistics.mean(timed_steps(dense, dense_steps, flush, stream)), world)
 
-    # end to end through the C ABI: pinned host inputs -> device, decode, result -> pinned host
-    h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q)
-    h_qi = torch.empty(q_idx.shape, dtype=q_idx.dtype, pin_memory=True).copy_(q_idx)
+    # end to end through the C ABI: every step brings the new token (q, q_idx and its K, V and index
+    # key) from pinned host memory in one copy, appends it to the caches (msa_decode_append), decodes,
+    # and takes the output and the block ids back in one copy; the host reads them before the next step
+    es = q.element_size()
+
+    def seg(n):  # 16-byte aligned segment lengths
+        return (n + 15) // 16 * 16
+    sizes_in = [q.numel() * es, q_idx.numel() * es, w.batch * w.n_kv_heads * w.head_dim * es,
+                w.batch * w.n_kv_heads * w.head_dim * es, w.batch * w.n_idx_k_heads * w.idx_dim * es]
+    offs_in = [sum(seg(n) for n in sizes_in[:i]) for i in range(len(sizes_in))]
+    h_in = torch.empty(offs_in[-1] + seg(sizes_in[-1]), dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty_like(h_in, device=dev)
+
+    def view(buf, i, shape, dtype):
+        return buf[offs_in[i]:offs_in[i] + sizes_in[i]].view(dtype).view(shape)
     pos = lens.long() - 1
-    new_k = torch.empty(w.batch, w.n_kv_heads, 1, w.head_dim, dtype=k.dtype, pin_memory=True)
-    new_v = torch.empty_like(new_k).pin_memory()
-    new_ki = torch.empty(w.batch, w.n_idx_k_heads, 1, w.idx_dim, dtype=k_idx.dtype, pin_memory=True)
-    for b in range(w.batch):
-        new_k[b].copy_(k[b, :, pos[b]:pos[b] + 1])
-        new_v[b].copy_(v[b, :, pos[b]:pos[b] + 1])
-        new_ki[b].copy_(k_idx[b, :, pos[b]:pos[b] + 1])
-    h_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    h_ids = torch.empty(ids.shape, dtype=ids.dtype, pin_memory=True)
-    pos_host = pos.tolist()
+    new_k = torch.stack([k[b, :, pos[b]] for b in range(w.batch)])
+    new_v = torch.stack([v[b, :, pos[b]] for b in range(w.batch)])
+    new_ki = torch.stack([k_idx[b, :, pos[b]] for b in range(w.batch)])
+    for i, t in enumerate((q, q_idx, new_k, new_v, new_ki)):
+        view(h_in, i, t.shape, t.dtype).copy_(t)
+    dq, dqi = view(d_in, 0, q.shape, q.dtype), view(d_in, 1, q_idx.shape, q_idx.dtype)
+    dk, dv, dki = (view(d_in, i, t.shape, t.dtype) for i, t in ((2, new_k), (3, new_v), (4, new_ki)))
+    o_bytes, id_bytes = o.numel() * es, ids.numel() * 4
+    d_out = torch.empty(seg(o_bytes) + id_bytes, dtype=torch.uint8, device=dev)
+    h_out = torch.empty_like(d_out, device="cpu").pin_memory()
+    do = d_out[:o_bytes].view(o.dtype).view(o.shape)
+    dids = d_out[seg(o_bytes):].view(torch.int32).view(ids.shape)
 
     def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        q_idx.copy_(h_qi, non_blocking=True)
-        for b in range(w.batch):  # append the new token's K, V and index key at its position
-            pb = pos_host[b]
-            k[b, :, pb:pb + 1].copy_(new_k[b], non_blocking=True)
-            v[b, :, pb:pb + 1].copy_(new_v[b], non_blocking=True)
-            k_idx[b, :, pb:pb + 1].copy_(new_ki[b], non_blocking=True)
-        step()
-        h_o.copy_(o, non_blocking=True)
-        h_ids.copy_(ids, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
+        _lib.msa_decode_append(p, dk, dv, dki, k, v, k_idx, stream)
+        _lib.msa_decode_fused(p, dq, dqi, k, v, k_idx, do, dids, None, r["ws"], stream)
+        h_out.copy_(d_out, non_blocking=True)
 
     e2e_n = max(3, min(args.steps, 200))
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize()
+    assert torch.equal(dids, ids), "the end-to-end step selected other blocks"
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_n)]
     for i in range(e2e_n):
         flush()
@@ -493,8 +502,8 @@ def run_ours(args, world, rank, local):
         e2e_ev[i][1].record(stream)
         e2e_ev[i][1].synchronize()  # the host reads the step's result before the next step
     e2e_us = max_over_ranks(statistics.mean(a.elapsed_time(b) * 1e3 for a, b in e2e_ev), world)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_qi, new_k, new_v, new_ki))
-    d2h = h_o.numel() * h_o.element_size() + h_ids.numel() * h_ids.element_size()
+    h2d = h_in.numel()
+    d2h = h_out.numel()
 
     cpu = cpu1 = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -570,6 +579,7 @@ def run_ours(args, world, rank, local):
         "dense_gqa_us": round(dense_us, 2), "sparse_vs_dense_speedup": round(dense_us / step_us, 2),
         "e2e": {"value": round(e2e_us, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
+        "e2e_launches_per_step": 3,
         "configs": configs,
         "shared_index_head": shared,
         "large_k": large_k,

@@ -26,7 +26,7 @@ EXPORTED = ["msa_index_score", "msa_block_maxpool_topk", "msa_sparse_attn_decode
             "msa_decode_fused", "msa_prefill_index_topk", "msa_workspace_size", "msa_last_error_string",
             "msa_status_string", "msa_get_device_status", "msa_clear_device_status", "msa_set_stage_events",
             "msa_decode_fused_noalloc", "msa_noalloc_get_status", "msa_noalloc_clear_status", "msa_set_wait_limit",
-            "msa_diag_wait_timeout"]
+            "msa_diag_wait_timeout", "msa_decode_append"]
 
 
 class MsaError(RuntimeError):
@@ -41,7 +41,7 @@ class Params(ctypes.Structure):
         ("n_idx_k_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("idx_dim", ctypes.c_int),
         ("block_size", ctypes.c_int), ("top_k", ctypes.c_int), ("q_len", ctypes.c_int), ("q_start", ctypes.c_int),
         ("max_seq_len", ctypes.c_int), ("seq_lens", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
-        ("dtype", ctypes.c_int), ("flags", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("flags", ctypes.c_int), ("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int),
     ]
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
             "msa_noalloc_clear_status": [st],
             "msa_set_wait_limit": [vp, ctypes.c_uint64, st],
             "msa_diag_wait_timeout": [vp, sz, st],
+            "msa_decode_append": [P, vp, vp, vp, vp, vp, vp, st],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -190,3 +191,8 @@ def msa_set_wait_limit(ws, limit_ns: int, stream=None):
 
 def msa_diag_wait_timeout(ws, stream=None):
     _check(lib().msa_diag_wait_timeout(_ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)))
+
+
+def msa_decode_append(params, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx, stream=None):
+    _check(lib().msa_decode_append(ctypes.byref(params), _ptr(k_new), _ptr(v_new), _ptr(k_idx_new), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(k_idx), _stream(stream)))

@@ -25,10 +25,13 @@ def dtype_code(t: torch.Tensor) -> int:
 
 
 def make_params(*, batch, n_q_heads, n_kv_heads, n_idx_k_heads, head_dim, idx_dim, block_size, top_k,
-                max_seq_len, dtype, q_len=1, q_start=0, seq_lens=None, softmax_scale=None, flags=0) -> Params:
+                max_seq_len, dtype, q_len=1, q_start=0, seq_lens=None, softmax_scale=None, flags=0,
+                block_table=None, n_pages=0) -> Params:
+    """block_table (int32 [B, ceil(max_seq_len / block_size)], device) selects paged caches of n_pages pages."""
     return Params(batch, n_q_heads, n_kv_heads, n_idx_k_heads, head_dim, idx_dim, block_size, top_k, q_len,
                   q_start, max_seq_len, seq_lens.data_ptr() if seq_lens is not None else None,
-                  float(softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(head_dim)), dtype, flags)
+                  float(softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(head_dim)), dtype, flags,
+                  block_table.data_ptr() if block_table is not None else None, int(n_pages))
 
 
 def params_from(q, q_idx, k, k_idx, *, block_size, top_k, seq_lens=None, q_start=0, softmax_scale=None,

@@ -618,7 +618,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     while (pj < j1 && tiles_of(block_at(pj)) == 0) ++pj;
     const unsigned char *kb = reinterpret_cast<const unsigned char *>(a.k_cache);
     const unsigned char *vb = reinterpret_cast<const unsigned char *>(a.v_cache);
-    const size_t head_off = ((size_t)b * a.G + g) * (size_t)a.L_max;
+
     int issued = 0;
     bool failed = false;
     auto issue = [&]() {
@@ -632,7 +632,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
         if (tid == 0) {
             const uint32_t bytes = (uint32_t)nk * D * ES;
             mbar_arrive_expect_tx(&bars[slot], 2 * bytes);
-            const size_t src = (head_off + (size_t)key0) * D * ES;
+            const size_t src = (size_t)a.cache.row(b, g, a.G, a.L_max, key0) * D * ES;
             unsigned char *dst = ring + (size_t)slot * 2 * tile_bytes;
             bulk_g2s(dst, kb + src, bytes, &bars[slot], l2_evict_first_policy());
             bulk_g2s(dst + tile_bytes, vb + src, bytes, &bars[slot], l2_evict_first_policy());
@@ -855,14 +855,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     };
     int pj = j0, pt = 0, issued = 0;
     while (pj < j1 && tiles_of(block_at(pj)) == 0) ++pj;
-    const int row0 = (b * a.G + g) * a.L_max;
     auto issue = [&]() {
         const int id = block_at(pj);
         const int slot = issued % nst;
         if (tid == 0) {
             unsigned char *dst = ring + slot * STAGE;
             mbar_arrive_expect_tx(&bars[slot], STAGE);
-            const int row = row0 + id * a.Bk + pt * KT;
+            const int row = a.cache.row(b, g, a.G, a.L_max, id * a.Bk + pt * KT);
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
                 tc::tma_load_2d(dst + h * KVH, &kmap, h * 64, row, &bars[slot]);
@@ -1141,7 +1140,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
         attr_bytes = smem;
     }
     CUtensorMap km, vm;
-    const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
+    const unsigned long long rows = a.cache.rows(a.B, a.G, a.L_max);
     if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.k_cache), D, rows, D * 2, 64, KT,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.v_cache), D, rows, D * 2, 64, KT,
@@ -1264,7 +1263,6 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
         const int nk = blk_end - key0;
         return nk < TK ? (nk > 0 ? nk : 0) : TK;
     };
-    const int row0 = (b * a.G + g) * a.L_max;
     unsigned char *my_ring = ring + (size_t)w * SPW * STAGE;
     // the warp's tiles in order: the next one with keys is copied into the next stage
     int t_next = w, issued = 0, consumed = 0;
@@ -1287,9 +1285,10 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
             unsigned char *st = my_ring + (size_t)slot * STAGE;
             mbar_arrive_expect_tx(&my_bars[slot], STAGE);
 #pragma unroll
+            const int row = a.cache.row(b, g, a.G, a.L_max, key0);
             for (int h = 0; h < NH; ++h) {
-                tc::tma_load_2d(st + h * KVH, &kmap, h * 64, row0 + key0, &my_bars[slot]);
-                tc::tma_load_2d(st + (NH + h) * KVH, &vmap, h * 64, row0 + key0, &my_bars[slot]);
+                tc::tma_load_2d(st + h * KVH, &kmap, h * 64, row, &my_bars[slot]);
+                tc::tma_load_2d(st + (NH + h) * KVH, &vmap, h * 64, row, &my_bars[slot]);
             }
         }
         ++issued;
@@ -1445,7 +1444,7 @@ cudaError_t launch_wide(const AttnArgs &a, cudaStream_t s, bool pdl) {
         attr_set = true;
     }
     CUtensorMap km, vm;
-    const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
+    const unsigned long long rows = a.cache.rows(a.B, a.G, a.L_max);
     if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.k_cache), D, rows, D * 2, 64, TK,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(a.v_cache), D, rows, D * 2, 64, TK,

@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
         while (!failed && issued - consumed < S) {
             int row;
             if (prod.valid) {
-                row = (prod.p.b * Hik + prod.p.hik) * a.L_max + prod.n * Bk + prod.c * CT;
+                row = a.cache.row(prod.p.b, prod.p.hik, Hik, a.L_max, prod.n * Bk + prod.c * CT);
                 prod.advance(off, nba, lens, B, Hik);
             } else {
                 if (!more) break;
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
                     have = true;
                     pc = 0;
                 }
-                row = (pr.x * Hik + pr.y) * a.L_max + pr.z * Bk + pc * CT;
+                row = a.cache.row(pr.x, pr.y, Hik, a.L_max, pr.z * Bk + pc * CT);
                 if (++pc == pr.w) have = false;
             }
             if (lane == 0) {
@@ -678,7 +678,7 @@ cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cu
     const int box_x = (row_bytes >= 128 ? 128 : 64) / es;
     CUtensorMap km;
     if (!encode_2d(&km, dtype == MSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   const_cast<void *>(a.k_idx), row_bytes / es, (unsigned long long)a.B * a.Hik * a.L_max, row_bytes,
+                   const_cast<void *>(a.k_idx), row_bytes / es, a.cache.rows(a.B, a.Hik, a.L_max), row_bytes,
                    box_x, ct, row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     return dtype == MSA_F32 ? launch_scan_r<float>(a, km, row_bytes, gps, s, pdl)

@@ -106,7 +106,27 @@ msa_status_t check_params(const msa_params_t *p, Mode mode) {
     if (mode == DECODE_ONLY || (mode == ANY_ROWS && p->q_len == 1)) {
         if (p->seq_lens == nullptr) return fail(MSA_ERR_INVALID_ARG, "seq_lens is NULL");
     }
+    if (p->block_table != nullptr) {
+        if ((reinterpret_cast<uintptr_t>(p->block_table) & 3u) != 0)
+            return fail(MSA_ERR_INVALID_ARG, "block_table is not 4-byte aligned");
+        if (p->n_pages < 1) return fail(MSA_ERR_INVALID_ARG, "n_pages %d < 1 with a block table", p->n_pages);
+        const int hmax = p->n_kv_heads > p->n_idx_k_heads ? p->n_kv_heads : p->n_idx_k_heads;
+        if ((long long)p->n_pages * hmax * p->block_size >= (1LL << 31))
+            return fail(MSA_ERR_UNSUPPORTED, "n_pages * heads * block_size must stay below 2^31 cache rows");
+    }
     return MSA_OK;
+}
+
+// Layout of the caches a call reads: contiguous, or pages named by the block table.
+CacheMap cache_of(const msa_params_t &p) {
+    CacheMap c{};
+    if (p.block_table != nullptr) {
+        c.table = p.block_table;
+        c.nbt = (p.max_seq_len + p.block_size - 1) / p.block_size;
+        c.n_pages = p.n_pages;
+        c.page_log2 = __builtin_ctz((unsigned)p.block_size);
+    }
+    return c;
 }
 
 msa_status_t check_ptr(const void *ptr, const char *name, bool nullable = false) {
@@ -189,7 +209,13 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
             L.blocks_per_split = (int)((nb + S - 1) / S);
             L.S = (nb + L.blocks_per_split - 1) / L.blocks_per_split;
         } else {
-            L.S = p.top_k < kSparseSplits ? p.top_k : kSparseSplits;
+            // the splits of a (sequence, group) form one cluster; as many as one wave of CTAs holds:
+            // the largest power of two <= kSparseSplits with batch * groups * S <= SMs (a second
+            // wave of clusters would double the kernel's time)
+            const long long bg = (long long)p.batch * p.n_kv_heads;
+            int S = kSparseSplits;
+            while (S > 1 && bg * S > n_sm) S >>= 1;
+            L.S = p.top_k < S ? p.top_k : S;
             L.blocks_per_split = (p.top_k + L.S - 1) / L.S;
         }
         L.counters = off;
@@ -377,6 +403,7 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
     a.block_scores = mode == MSA_SCORES_BLOCKMAX ? scores_out : nullptr;
     a.sched = reinterpret_cast<unsigned *>(ws) + kSchedWord;
     a.status = reinterpret_cast<int *>(ws);
+    a.cache = cache_of(*p);
     e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     return MSA_OK;
@@ -450,6 +477,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
     a.force = (p->flags & MSA_FORCE_SINK_LOCAL) != 0;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(wsb);
+    a.cache = cache_of(*p);
     cudaError_t e;
     if (!after_scan) {  // the scan zeroes the counters in the fused path
         e = cudaMemsetAsync(a.counters, 0, (size_t)p->batch * p->n_kv_heads * 4, s);
@@ -517,6 +545,7 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.sched = reinterpret_cast<unsigned *>(wsb) + kSchedWord;
     a.counters = reinterpret_cast<int *>(wsb + L.counters);
     a.status = reinterpret_cast<int *>(wsb);
+    a.cache = cache_of(*p);
     const bool large = p->top_k > kMaxTopKList;
     if (large) {
         // every block's score (static ranges and tails alike) into the block-score region
@@ -543,6 +572,22 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     }
     if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     return attend_decode(p, q, k_cache, v_cache, nullptr, true, L, wsb, o, ids_out, lse, s);
+}
+
+msa_status_t msa_decode_append(const msa_params_t *p, const void *k_new, const void *v_new, const void *k_idx_new,
+                               void *k_cache, void *v_cache, void *k_idx, msa_stream_t stream) {
+    MSA_TRY(check_params(p, DECODE_ONLY));
+    MSA_TRY(check_ptr(k_new, "k_new"));
+    MSA_TRY(check_ptr(v_new, "v_new"));
+    MSA_TRY(check_ptr(k_idx_new, "k_idx_new"));
+    MSA_TRY(check_ptr(k_cache, "k_cache"));
+    MSA_TRY(check_ptr(v_cache, "v_cache"));
+    MSA_TRY(check_ptr(k_idx, "k_idx"));
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    cudaError_t e = launch_append(*p, cache_of(*p), k_new, v_new, k_idx_new, k_cache, v_cache, k_idx, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    return MSA_OK;
 }
 
 msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
@@ -576,6 +621,7 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
     a.Bk = p->block_size; a.k = p->top_k; a.q_start = p->q_start; a.L_max = p->max_seq_len; a.r = r;
     a.scale_log2 = p->softmax_scale * 1.4426950408889634f;
     a.status = reinterpret_cast<int *>(ws);
+    a.cache = cache_of(*p);
     unsigned char *w = static_cast<unsigned char *>(ws);
     a.counts = reinterpret_cast<int *>(w + L.counts);
     a.offsets = reinterpret_cast<int *>(w + L.offsets);
@@ -602,6 +648,8 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->idx_dim != 64) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes idx_dim 64");
     if (p->block_size < 32) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes block_size >= 32");
+    if (p->block_table != nullptr && p->block_size < 128)
+        return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring of a paged cache takes block_size >= 128");
     MSA_TRY(check_ptr(q_idx, "q_idx"));
     MSA_TRY(check_ptr(k_idx, "k_idx"));
     MSA_TRY(check_ptr(ids_out, "ids_out"));
@@ -623,6 +671,7 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     a.part_s = reinterpret_cast<float *>(w + L.part_s);
     a.part_i = reinterpret_cast<int *>(w + L.part_i);
     a.status = reinterpret_cast<int *>(ws);
+    a.cache = cache_of(*p);
     const char *why = "clearing the prefill index piece counters";
     cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)L.n_mt * p->batch * p->n_kv_heads * 4, (cudaStream_t)stream);
     if (e == cudaSuccess) e = launch_prefill_index(a, q_idx, k_idx, L.grid, (cudaStream_t)stream, &why);

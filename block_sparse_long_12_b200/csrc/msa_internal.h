@@ -52,6 +52,7 @@ struct AttnArgs {
     int cluster;               // > 1: the S splits of a (b, g) form one cluster and merge in shared memory
     int force;                 // MSA_FORCE_SINK_LOCAL: the selection keeps block 0 and the last block
     int *status;
+    CacheMap cache;            // K/V cache layout (contiguous or paged)
 };
 
 struct PoolTopkArgs {
@@ -85,6 +86,7 @@ struct PrefillIdxArgs {
     float *part_s;             // [units][n_seg][Kt][256] per-segment row lists of split units
     int *part_i;
     int *status;
+    CacheMap cache;            // index-key cache layout (paged: pages of a multiple of 128 tokens)
 };
 
 // Key tiles (128 keys) of the i-th prefill index unit in processing order:
@@ -125,6 +127,7 @@ struct PrefillAttnArgs {
     int B, T, Hq, G, D, Bk, k, q_start, L_max, r;
     float scale_log2;
     int *status;
+    CacheMap cache;            // K/V cache layout (contiguous or paged)
     // one pass over query rows [t0, t0 + Tn)
     int t0, Tn;
     int nbv;                   // blocks visible to the pass's last row: buckets per (b, g)
@@ -132,7 +135,7 @@ struct PrefillAttnArgs {
     int *counts;               // [B*G*nbv] pairs per bucket (zeroed before the pass)
     int *offsets;              // [B*G*nbv] first member of each bucket
     int *rank;                 // [B*Tn*G*k] rank of each pair in its bucket (-1: not attended)
-    int *members;              // [pairs] member tt * k + slot, grouped by bucket
+    int *members;              // [pairs] member (tt << 5) | slot, grouped by bucket (k <= 32)
     int4 *tiles;               // [max_tiles] (bucket, first member, member count, 0)
     int *n_tiles;
     int *block_sums;           // [2 * scan blocks] pairs and tiles of each scan block's buckets
@@ -172,6 +175,8 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
                                  cudaStream_t s, const char **why);
 cudaError_t launch_set_wait_limit(int *ws, unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_append(const msa_params_t &p, const CacheMap &cache, const void *k_new, const void *v_new,
+                          const void *ki_new, void *k, void *v, void *ki, cudaStream_t s);
 cudaError_t launch_wait_never(int *ws, cudaStream_t s);
 
 int num_sms();

@@ -61,7 +61,7 @@ constexpr int kRun = 8;         // consecutive tiles of the list a CTA takes at 
 struct TileInfo {
     int bkt, start, cnt, last;  // last: the CTA's next tile is another bucket (or none)
     int b, g, n, pad;
-    int mem[kPtRows];           // member i: row tt * k + slot
+    int mem[kPtRows];           // member i: (row tt << 5) | slot
 };
 
 struct PtBars {
@@ -121,6 +121,22 @@ __device__ inline void tmem_st<32>(uint32_t taddr, const uint32_t (&r)[32]) {
         : "memory");
 }
 __device__ inline void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 2^x for x <= 0 on the FMA pipe, so that part of the softmax's exponentials leave the MUFU
+// unit: x is clamped at -125 (2^-125 stands for anything smaller, also for -inf), rounded to the
+// nearest integer n by adding 1.5 * 2^23 (n then sits in the low mantissa bits, and n << 23 equals
+// those bits shifted by 23), 2^(x - n) with x - n in [-1/2, 1/2] comes from a cubic fitted to 2^f
+// by least squares in relative error at Chebyshev nodes (max relative error 7.5e-5, against the
+// 2^-9 of the bf16 that P is stored in), and 2^n is added to its exponent field.
+__device__ __forceinline__ float exp2_poly(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float f = x - (t - 12582912.f);
+    float p = fmaf(f, 0.0551716648f, 0.242611125f);
+    p = fmaf(p, f, 0.693260968f);
+    p = fmaf(p, f, 0.999928057f);
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
 
 // 2^x with the hardware approximation (2^-inf = +0).
 __device__ __forceinline__ float exp2_approx(float x) {
@@ -275,7 +291,7 @@ __global__ void pa_scatter_kernel(const PrefillAttnArgs a) {
         const int tt = (int)(rest % a.Tn);
         const int b = (int)(rest / a.Tn);
         const int id = a.ids[(((size_t)b * a.T + a.t0 + tt) * a.G + g) * a.k + j];
-        a.members[a.offsets[((size_t)b * a.G + g) * a.nbv + id] + rk] = tt * a.k + j;
+        a.members[a.offsets[((size_t)b * a.G + g) * a.nbv + id] + rk] = (tt << 5) | j;  // k <= 32
     }
 }
 
@@ -391,7 +407,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             if (!__shfl_sync(FULL, ok, 0)) break;
             if (lane == 0) {
                 mbar_arrive_expect_tx(&S.kv_full[ks], 2 * NH * KVH);
-                const int row = (b * a.G + g) * a.L_max + n * BK;
+                const int row = a.cache.row(b, g, a.G, a.L_max, n * BK);
                 unsigned char *dst = smKV + ks * KV_STAGE;
                 for (int h = 0; h < NH; ++h) tc::tma_load_2d(dst + h * KVH, &kmap, h * 64, row, &S.kv_full[ks]);
                 for (int h = 0; h < NH; ++h)
@@ -419,7 +435,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             for (int q = 0; q < kPtRows / 32; ++q) {
                 const int m = lane + 32 * q;
                 if (m < cnt) {
-                    const int qrow = ((b * a.T + a.t0 + mem[q] / a.k) * a.Hq) + g * r;
+                    const int qrow = ((b * a.T + a.t0 + (mem[q] >> 5)) * a.Hq) + g * r;
                     for (int h = 0; h < NH; ++h)
                         tc::tma_load_2d(smQ + qs * Q_STAGE + h * kHalf + m * r * 128, &qmap, h * 64, qrow,
                                         &S.q_full[qs]);
@@ -509,7 +525,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
                 const TileInfo &I = S.info[il % kInfoSlots];
                 n = I.n;
                 valid = m_i < I.cnt;
-                if (valid) pos = a.q_start + a.t0 + I.mem[m_i] / a.k;
+                if (valid) pos = a.q_start + a.t0 + (I.mem[m_i] >> 5);
                 info_release(il);
             }
             const bool any = __any_sync(FULL, valid);
@@ -549,18 +565,26 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             float ls = 0.f;
             if (any) {
                 const float off = valid ? -m2 : 0.f;
-                uint32_t pk[CW / 2];
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                // 32 keys at a time: 16 packed pairs go to TMEM before the next 32 are exponentiated
 #pragma unroll
-                for (int e = 0; e < CW / 2; ++e) {
-                    const float p0 = exp2_approx(fmaf(__uint_as_float(zr[2 * e]), c, off));
-                    const float p1 = exp2_approx(fmaf(__uint_as_float(zr[2 * e + 1]), c, off));
-                    acc[e & 3] += p0 + p1;
-                    const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                    pk[e] = *reinterpret_cast<const uint32_t *>(&pb);
+                for (int h2 = 0; h2 < CW / 32; ++h2) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e2 = 0; e2 < 16; ++e2) {
+                        const int e = h2 * 16 + e2;
+                        // one pair in four on the FMA pipe, the rest on MUFU
+                        const float x0 = fmaf(__uint_as_float(zr[2 * e]), c, off);
+                        const float x1 = fmaf(__uint_as_float(zr[2 * e + 1]), c, off);
+                        const float p0 = (e & 3) == 3 ? exp2_poly(x0) : exp2_approx(x0);
+                        const float p1 = (e & 3) == 3 ? exp2_poly(x1) : exp2_approx(x1);
+                        acc[e & 3] += p0 + p1;
+                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                        pk[e2] = *reinterpret_cast<const uint32_t *>(&pb);
+                    }
+                    tmem_st<16>(tmem + lane_addr + sb * BK + hf * (CW / 2) + h2 * 16, pk);
                 }
                 ls = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                tmem_st<CW / 2>(tmem + lane_addr + sb * BK + hf * (CW / 2), pk);
                 tmem_st_wait();
             }
             if (hf == 0) S.ml_m[sb][row] = m2;
@@ -590,7 +614,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
                 valid = m_i < I.cnt;
                 if (valid) {
                     const int mem = I.mem[m_i];
-                    pl = ((I.b * a.Tn + mem / a.k) * a.G + I.g) * a.k + mem % a.k;  // the pair's index in this pass
+                    pl = ((I.b * a.Tn + (mem >> 5)) * a.G + I.g) * a.k + (mem & 31);  // the pair's index in this pass
                 }
                 info_release(il);
             }
@@ -795,7 +819,7 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
                    (unsigned long long)a.B * a.T * a.Hq, (unsigned long long)a.D * 2, 64, a.r,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    const unsigned long long rows = (unsigned long long)a.B * a.G * a.L_max;
+    const unsigned long long rows = a.cache.rows(a.B, a.G, a.L_max);
     if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(k_cache), a.D, rows,
                    (unsigned long long)a.D * 2, 64, a.Bk, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&vm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(v_cache), a.D, rows,

@@ -179,7 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int acc = 0; acc < kAccs; ++acc)
                     tc::tma_load_3d(smA + acc * kABytes, &qmap, 0, g, b * a.T + m0 + acc * kRows, &S.a_full);
                 const int hik = g % a.Hik;
-                const int row0 = (b * a.Hik + hik) * a.L_max;
                 bool ok = true;
                 for (int n = w.n0; n < w.n1; ++n, ++it) {
                     const int st = it % kStages;
@@ -188,7 +187,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&S.full[st], kTileBytes);
-                    tc::tma_load_2d(smB + st * kTileBytes, &kmap, 0, row0 + n * kKeys, &S.full[st]);
+                    // a 128-key tile lies inside one page (paged caches have pages of a multiple of 128 keys)
+                    tc::tma_load_2d(smB + st * kTileBytes, &kmap, 0, a.cache.row(b, hik, a.Hik, a.L_max, n * kKeys),
+                                    &S.full[st]);
                 }
                 if (!ok) break;
             }
@@ -419,7 +420,7 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
     }
     // k_idx [B*Hik*Lmax, 64] bf16: box of 64 dims x 128 keys
     if (!encode_2d(&km, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void *>(k_idx), 64,
-                   (unsigned long long)a.B * a.Hik * a.L_max, 128, 64, kKeys, CU_TENSOR_MAP_SWIZZLE_128B)) {
+                   a.cache.rows(a.B, a.Hik, a.L_max), 128, 64, kKeys, CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "encoding the index-key tensor map failed";
         return cudaErrorInvalidValue;
     }

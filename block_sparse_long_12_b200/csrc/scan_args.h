@@ -17,6 +17,28 @@ constexpr int kTailPools = 4;          // interleaved pools (counters) of the sc
 // between the CTAs.
 __host__ __device__ inline int scan_tail_blocks(int nb) { return nb / 4; }
 
+// Where token `tok` of head h of sequence b sits in a cache of H heads (rows of head_dim or idx_dim
+// elements): contiguous [B, H, L_max, row], or paged [n_pages, H, page, row] where a block table of
+// nbt entries per sequence names the page of each block of page (= block_size) tokens.  Page ids
+// outside [0, n_pages) are out of contract; they are clamped so that nothing is read outside the
+// pool.
+struct CacheMap {
+    const int *table;  // nullptr: contiguous
+    int nbt;           // table entries per sequence
+    int n_pages;
+    int page_log2;     // log2 of the tokens per page
+    __host__ __device__ inline int row(int b, int h, int H, int L_max, int tok) const {
+        if (table == nullptr) return (b * H + h) * L_max + tok;
+        int pg = table[b * nbt + (tok >> page_log2)];
+        pg = pg < 0 ? 0 : (pg >= n_pages ? n_pages - 1 : pg);
+        return ((pg * H + h) << page_log2) + (tok & ((1 << page_log2) - 1));
+    }
+    // rows of the tensor a TMA map covers
+    __host__ __device__ inline unsigned long long rows(int B, int H, int L_max) const {
+        return table == nullptr ? (unsigned long long)B * H * L_max : ((unsigned long long)n_pages * H) << page_log2;
+    }
+};
+
 // ---- decode index scan (Step 1 for decode): persistent, 1 CTA per SM
 constexpr int kScanChunkBytes = 8192;   // ring stage: bytes of index keys per TMA copy
 
@@ -44,6 +66,7 @@ struct ScanArgs {
     float *block_scores;   // [B, 1, G, nb_max] (nullable)
     int *counters;         // [B, G] attention arrival counters, zeroed by CTA 0 (nullable)
     int *status;
+    CacheMap cache;        // index-key cache layout (contiguous or paged)
 };
 
 }  // namespace msa

@@ -131,7 +131,24 @@ typedef struct {
     float softmax_scale;  /* > 0; 1/sqrt(head_dim) in the usual attention      */
     int dtype;            /* msa_dtype_t; prefill entries take MSA_BF16 only   */
     int flags;            /* MSA_SCORES_* / MSA_DENSE / MSA_FORCE_SINK_LOCAL   */
+    const int32_t *block_table; /* NULL: contiguous caches; else paged, see below */
+    int n_pages;          /* pages in each pool when block_table != NULL       */
 } msa_params_t;
+/*
+ * Paged caches (block_table != NULL): the K, V and index-K caches are pools of
+ * n_pages pages of block_size tokens each, page-major and head-major inside a
+ * page:
+ *   k, v   [n_pages, n_kv_heads, block_size, head_dim]
+ *   k_idx  [n_pages, n_idx_k_heads, block_size, idx_dim]
+ * and block_table (device int32 [B, ceil(max_seq_len / block_size)]) names the
+ * page that holds block n of sequence b (tokens n*block_size ..) in all three
+ * pools.  One MSA block is one page, so a selected block is fetched from one
+ * place and a serving loop can hand out pages as sequences grow.  Entries for
+ * blocks a call can see must lie in [0, n_pages) (others are out of contract:
+ * kernels clamp them and never read outside the pools).  All entries take it
+ * except msa_prefill_index_topk with block_size < 128 (its 128-key tiles must
+ * lie inside one page), which returns MSA_ERR_UNSUPPORTED.
+ */
 
 /*
  * Step 1a (+1b): index scores.  Exactly one of MSA_SCORES_TOKEN or
@@ -230,6 +247,19 @@ MSA_API msa_status_t msa_decode_fused_noalloc(const msa_params_t *params, const 
  */
 MSA_API msa_status_t msa_noalloc_get_status(int *status, msa_stream_t stream);
 MSA_API msa_status_t msa_noalloc_clear_status(msa_stream_t stream);
+
+/*
+ * Serving step before msa_decode_fused (not part of the method): the new token
+ * of every sequence -- k_new and v_new [B, n_kv_heads, head_dim], k_idx_new
+ * [B, n_idx_k_heads, idx_dim], params.dtype, contiguous -- is written to its
+ * position seq_lens[b] - 1 of the K, V and index-K caches (contiguous or paged,
+ * as params say).  With the new token's q and q_idx it is all one decode step
+ * takes from the host, so a caller can bring them in one copy; the caches are
+ * otherwise untouched.
+ */
+MSA_API msa_status_t msa_decode_append(const msa_params_t *params, const void *k_new, const void *v_new,
+                                       const void *k_idx_new, void *k_cache, void *v_cache, void *k_idx,
+                                       msa_stream_t stream);
 
 /*
  * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,

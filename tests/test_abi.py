@@ -161,3 +161,25 @@ def test_failure_detection_calls_check_arguments(lib):
     # valid arguments reach the device, which is missing here
     assert L.msa_diag_wait_timeout(a, 256, None) == lib.MSA_ERR_CUDA
     assert L.msa_noalloc_clear_status(None) == lib.MSA_ERR_CUDA
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers: host-only argument checks")
+def test_paged_params_rejected_before_launch(lib):
+    L = lib.lib()
+    a = 0x10000
+    ws = ctypes.c_size_t(1 << 30)
+    ptrs = [a, a, a, a, a, a, None, None, a]
+    p = good_params(lib)
+    p.block_table = a
+    p.n_pages = 0
+    assert L.msa_decode_fused(ctypes.byref(p), *ptrs, ws, None) == lib.MSA_ERR_INVALID_ARG
+    p.n_pages = 64
+    p.block_table = a + 2  # not 4-byte aligned
+    assert L.msa_decode_fused(ctypes.byref(p), *ptrs, ws, None) == lib.MSA_ERR_INVALID_ARG
+    p.block_table = a
+    p.n_pages = 1 << 22  # pools of more than 2^31 rows
+    assert L.msa_decode_fused(ctypes.byref(p), *ptrs, ws, None) == lib.MSA_ERR_UNSUPPORTED
+    # the prefill index reads 128-key tiles: pages must hold at least 128 keys
+    pp = good_params(lib, q_len=100, block_size=64)
+    pp.block_table, pp.n_pages = a, 64
+    assert L.msa_prefill_index_topk(ctypes.byref(pp), a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
