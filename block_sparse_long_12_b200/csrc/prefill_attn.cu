@@ -44,17 +44,17 @@ namespace msa {
 
 namespace {
 
-constexpr int kPtThreads = 512;
 constexpr int kPtRows = 128;
 constexpr int kPtSm0 = 4;       // first softmax warp
-constexpr int kPtSmWarps = 8;
-constexpr int kPtEpi0 = 12;     // first epilogue warp
 constexpr int kPtEpiWarps = 4;
+constexpr int kMaxSpq = 4;      // softmax warps per TMEM lane quadrant: BK / 32 (32 keys each)
+// warps of the tile kernel for a block size: 4 control warps, 4 * BK / 32 softmax warps, 4 epilogue warps
+__host__ __device__ constexpr int pt_threads(int bk) { return (4 + 4 * (bk / 32) + kPtEpiWarps) * 32; }
 constexpr int kHalf = 16384;    // one 128-row x 128-byte operand tile
 constexpr int kInfoSlots = 6;   // tiles staged ahead in shared memory
 // every role but the stager releases a tile's info slot: K/V producer, MMA issuer, Q gather,
 // the softmax warps, the epilogue warps
-constexpr int kInfoConsumers = 3 + kPtSmWarps + kPtEpiWarps;
+__host__ __device__ constexpr int info_consumers(int bk) { return 3 + 4 * (bk / 32) + kPtEpiWarps; }
 constexpr int kRun = 8;         // consecutive tiles of the list a CTA takes at a time
 
 // One tile as the roles read it: its block, members, and whether the next tile changes block.
@@ -75,9 +75,9 @@ struct PtBars {
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort_flag;
-    float red_m[2][2][kPtRows];  // [buffer][column half][row] raw max of the half row
-    float ml_m[2][kPtRows];      // [buffer][row] row max, log2 domain
-    float ml_l[2][2][kPtRows];   // [buffer][column half][row] sum of the half row
+    float red_m[2][kMaxSpq][kPtRows];  // [buffer][key part][row] raw max of the part
+    float ml_m[2][kPtRows];            // [buffer][row] row max, log2 domain
+    float ml_l[2][kMaxSpq][kPtRows];   // [buffer][key part][row] sum of the part
     TileInfo info[kInfoSlots];
 };
 
@@ -145,19 +145,19 @@ __device__ __forceinline__ float exp2_approx(float x) {
     return y;
 }
 
-// Barrier over the two softmax warps of one lane quadrant (64 threads) that also ANDs a
-// per-thread flag across them, so both warps leave a loop at the same barrier when either
-// has given up a wait.
-__device__ inline bool pair_sync_and(int id, bool ok) {
+// Barrier over the softmax warps of one lane quadrant (nthreads threads) that also ANDs a
+// per-thread flag across them, so all of them leave a loop at the same barrier when any has
+// given up a wait.
+__device__ inline bool quad_sync_and(int id, int nthreads, bool ok) {
     uint32_t r;
     __syncwarp();
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, 64, p;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)ok), "r"(id)
+        : "r"((uint32_t)ok), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
 }
@@ -297,14 +297,17 @@ __global__ void pa_scatter_kernel(const PrefillAttnArgs a) {
 
 // ------------------------------------------------------------------ tiles
 template <int D, int BK>
-__global__ void __launch_bounds__(kPtThreads, 1)
+__global__ void __launch_bounds__(pt_threads(BK), 1)
     pa_tile_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap, const PrefillAttnArgs a) {
     constexpr int NH = D / 64;               // 64-dim halves of a row
     constexpr int KVH = BK * 128;            // bytes of one 64-dim half of a K or V block tile
     constexpr int KV_STAGE = 2 * NH * KVH;   // K halves, then V halves
     constexpr int Q_STAGE = NH * kHalf;
-    constexpr int CW = BK / 2;               // S columns of one softmax warp
+    constexpr int SPQ = BK / 32;             // softmax warps per lane quadrant
+    constexpr int SMW = 4 * SPQ;             // softmax warps
+    constexpr int EPI0 = kPtSm0 + SMW;       // first epilogue warp
+    constexpr int CW = 32;                   // S columns of one softmax warp
     constexpr uint32_t O_COL = 2 * BK;       // TMEM: S/P buffers [0, 2 BK), O buffers [2 BK, 2 BK + 2 D)
     constexpr uint32_t TMEM_COLS = 512;
     static_assert(2 * BK + 2 * D <= 512, "TMEM budget");
@@ -321,13 +324,13 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             mbar_init(&S.kv_full[i], 1); mbar_init(&S.kv_empty[i], 1);
             mbar_init(&S.q_full[i], 1); mbar_init(&S.q_empty[i], 1);
             mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1);
-            mbar_init(&S.p_full[i], kPtSmWarps);
+            mbar_init(&S.p_full[i], SMW);
             mbar_init(&S.o_full[i], 1); mbar_init(&S.o_empty[i], kPtEpiWarps);
-            mbar_init(&S.ml_full[i], kPtSmWarps); mbar_init(&S.ml_empty[i], kPtEpiWarps);
+            mbar_init(&S.ml_full[i], SMW); mbar_init(&S.ml_empty[i], kPtEpiWarps);
         }
         for (int i = 0; i < kInfoSlots; ++i) {
             mbar_init(&S.info_full[i], 1);
-            mbar_init(&S.info_empty[i], kInfoConsumers);
+            mbar_init(&S.info_empty[i], info_consumers(BK));
         }
         mbar_init(&S.mma_done, 1);
         S.abort_flag = 0;
@@ -503,14 +506,14 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             tc::mma_commit(&S.mma_done);
             mbar_wait(&S.mma_done, 0, a.status);
         }
-    } else if (warp >= kPtSm0 && warp < kPtSm0 + kPtSmWarps) {
+    } else if (warp >= kPtSm0 && warp < EPI0) {
         // ------------------------------------------------ softmax
-        // Warps w and w + 4 share TMEM lane quadrant w % 4 (one row per lane); half hf takes the
-        // block's keys [hf*CW, hf*CW + CW).  Every wait of a tile comes before the pair barrier,
-        // whose AND makes any failure uniform over the pair.
+        // Warps w, w + 4, ... share TMEM lane quadrant w % 4 (one row per lane); part hf takes the
+        // block's keys [hf*CW, hf*CW + CW).  Every wait of a tile comes before the quadrant
+        // barrier, whose AND makes any failure uniform over the quadrant's warps.
         const int sw = warp - kPtSm0;
         const int qd = sw & 3, hf = sw >> 2;
-        const int pair_bar = 1 + qd;
+        const int quad_bar = 1 + qd;
         const int row = qd * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
         const int m_i = row / r;
@@ -558,10 +561,13 @@ __global__ void __launch_bounds__(kPtThreads, 1)
                 mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             }
             S.red_m[sb][hf][row] = mb;
-            ok = pair_sync_and(pair_bar, ok);
+            ok = quad_sync_and(quad_bar, SPQ * 32, ok);
             if (!ok) break;
-            // every lane of both warps has read its S half: P may now overwrite the S buffer
-            const float m2 = fmaxf(mb, S.red_m[sb][hf ^ 1][row]) * c;  // row max in the log2 domain
+            // every lane of the quadrant's warps has read its S part: P may now overwrite the S buffer
+            float mr = S.red_m[sb][0][row];
+#pragma unroll
+            for (int j = 1; j < SPQ; ++j) mr = fmaxf(mr, S.red_m[sb][j][row]);
+            const float m2 = mr * c;  // row max in the log2 domain
             float ls = 0.f;
             if (any) {
                 const float off = valid ? -m2 : 0.f;
@@ -596,7 +602,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
                 mbar_arrive1(&S.ml_full[sb]);
             }
         }
-    } else if (warp >= kPtEpi0) {
+    } else if (warp >= EPI0) {
         // ------------------------------------------------ epilogue: one pair row per lane
         // A pair's r x D outputs are stored chunk-major ([D / 8 chunks][r heads][8 dims]), so the r
         // heads of a member -- r consecutive lanes -- write r * 16 contiguous bytes per store.
@@ -621,7 +627,9 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             const bool any = __any_sync(FULL, valid);
             if (!__all_sync(FULL, tc::wait_or_abort(&S.ml_full[ob], par, abort_flag, a.status))) break;
             const float m2 = S.ml_m[ob][row];
-            const float l = S.ml_l[ob][0][row] + S.ml_l[ob][1][row];
+            float l = 0.f;
+#pragma unroll
+            for (int j = 0; j < SPQ; ++j) l += S.ml_l[ob][j][row];
             __syncwarp();
             if (lane == 0) mbar_arrive1(&S.ml_empty[ob]);
             if (!__all_sync(FULL, tc::wait_or_abort(&S.o_full[ob], par, abort_flag, a.status))) break;
@@ -780,7 +788,7 @@ cudaError_t launch_tiles(const PrefillAttnArgs &a, const CUtensorMap &qm, const 
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    pa_tile_kernel<D, BK><<<grid, kPtThreads, smem, s>>>(qm, km, vm, a);
+    pa_tile_kernel<D, BK><<<grid, pt_threads(BK), smem, s>>>(qm, km, vm, a);
     return cudaGetLastError();
 }
 
