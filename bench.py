@@ -195,19 +195,21 @@ def timed_steps(fn, steps, flush, stream):
 
 
 def read_stream_gbs(dev, gib: int = 4) -> float:
-    """A read-only HBM reference measured here: torch's sum over a buffer of `gib` GiB (32 times L2),
-    best of 5 after a warm-up, CUDA events.  The driver's copy peak moves every byte twice (read and
-    write), so a kernel that only reads can exceed it; this is the read-only counterpart."""
-    x = torch.ones(gib << 28, dtype=torch.int32, device=dev)
-    torch.sum(x, dtype=torch.int64)
+    """A read-only HBM reference measured here: the faster of torch's max and sum over a float32
+    buffer of `gib` GiB (32 times L2), best of 5 each after a warm-up, CUDA events.  The driver's copy
+    peak moves every byte twice (read and write), so a kernel that only reads can exceed it; this is
+    the read-only counterpart."""
+    x = torch.ones(gib << 28, dtype=torch.float32, device=dev)
     best = float("inf")
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        torch.sum(x, dtype=torch.int64)
-        b.record()
-        b.synchronize()
-        best = min(best, a.elapsed_time(b) * 1e-3)
+    for op in (torch.amax, torch.sum):
+        op(x)
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            op(x)
+            b.record()
+            b.synchronize()
+            best = min(best, a.elapsed_time(b) * 1e-3)
     n = x.numel() * 4
     del x
     torch.cuda.empty_cache()
