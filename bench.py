@@ -6,7 +6,8 @@ the caches resident in HBM.  Metric: microseconds per decode step per layer
 (lower is better).  Also reported, each with its roofline fraction and the
 CPU oracle timed on this host:
   * every other workload: tiny fp32 decode, 16K causal prefill, ragged
-    batch-8 128K decode, batch-4 1M decode (``configs``);
+    batch-8 128K decode, batch-4 1M decode, 128K prefill with k 128 of 2,048
+    blocks (``configs``);
   * the 1M decode with one shared index-K head and the large-k regime;
   * the 1M-token chunked causal prefill (tok/s, tensor-core fraction);
   * the dense GQA decode over the same cache, and an end-to-end number with
@@ -564,6 +565,10 @@ def run_ours(args, world, rank, local):
             torch.cuda.empty_cache()
         configs["prefill_causal_16k"] = run_prefill(WORKLOADS["prefill_causal_16k"], world, rank, local, stream,
                                                     peaks, peak_kind, oracle_rows=0 if args.no_cpu_baseline else 256)
+        torch.cuda.empty_cache()
+        configs["prefill_ctx128k_large_k"] = run_prefill(WORKLOADS["prefill_ctx128k_large_k"], world, rank, local,
+                                                         stream, peaks, peak_kind,
+                                                         oracle_rows=0 if args.no_cpu_baseline else 32)
         torch.cuda.empty_cache()
 
     shared = None if args.no_shared_index else run_extra_decode("decode_ctx1m_shared_idx", args, world, rank, local,

@@ -233,7 +233,8 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
 PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm) {
     PrefillIdxPlan L{};
     L.n_mt = (p.q_len + 255) / 256;
-    L.kt = p.top_k <= 8 ? 8 : p.top_k <= 16 ? 16 : 32;
+    L.kt = p.top_k <= 8 ? 8 : p.top_k <= 16 ? 16 : p.top_k <= kMaxTopKList ? 32 : 0;
+    L.blk_stride = (p.q_start + p.q_len - 1) / p.block_size + 1;
     const long long units = (long long)L.n_mt * p.batch * p.n_kv_heads;
     const int max_tiles = prefill_unit_tiles(0, L.n_mt, p.q_len, p.q_start, p.block_size);
     const int gran = p.block_size > 128 ? p.block_size / 128 : 1;
@@ -261,6 +262,8 @@ PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm) {
     off += round256(part);
     L.part_i = off;
     off += round256(part);
+    L.blk_scores = off;
+    if (L.kt == 0) off += round256((size_t)p.batch * p.q_len * p.n_kv_heads * L.blk_stride * 4);
     L.total = off;
     return L;
 }
@@ -595,8 +598,6 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
                                      msa_stream_t stream) {
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_sparse_attn_prefill takes no flags");
-    if (p->top_k > kMaxTopKList)
-        return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes at most %d blocks per row", kMaxTopKList);
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->block_size != 64 && p->block_size != 128)
         return fail(MSA_ERR_UNSUPPORTED, "prefill attention takes block_size 64 or 128");
@@ -643,8 +644,6 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags & ~MSA_FORCE_SINK_LOCAL)
         return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes only MSA_FORCE_SINK_LOCAL");
-    if (p->top_k > kMaxTopKList)
-        return fail(MSA_ERR_UNSUPPORTED, "prefill index TopK keeps at most %d blocks per row", kMaxTopKList);
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
     if (p->idx_dim != 64) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes idx_dim 64");
     if (p->block_size < 32) return fail(MSA_ERR_UNSUPPORTED, "prefill index scoring takes block_size >= 32");
@@ -672,9 +671,24 @@ msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, co
     a.part_i = reinterpret_cast<int *>(w + L.part_i);
     a.status = reinterpret_cast<int *>(ws);
     a.cache = cache_of(*p);
+    if (L.kt == 0) {
+        a.blk_scores = reinterpret_cast<float *>(w + L.blk_scores);
+        a.blk_stride = L.blk_stride;
+    }
     const char *why = "clearing the prefill index piece counters";
     cudaError_t e = cudaMemsetAsync(a.counters, 0, (size_t)L.n_mt * p->batch * p->n_kv_heads * 4, (cudaStream_t)stream);
     if (e == cudaSuccess) e = launch_prefill_index(a, q_idx, k_idx, L.grid, (cudaStream_t)stream, &why);
+    if (e == cudaSuccess && L.kt == 0) {
+        // large k: the k best of each row's stored block scores
+        LargeTopkArgs la{};
+        la.scores = a.blk_scores; la.stride = L.blk_stride;
+        la.rows = p->batch * p->q_len * p->n_kv_heads; la.q_len = p->q_len; la.q_start = p->q_start;
+        la.G = p->n_kv_heads; la.Bk = p->block_size; la.k = p->top_k; la.L_max = p->max_seq_len;
+        la.prefill = 1; la.force = a.force;
+        la.ids_out = ids_out; la.top_scores_out = top_scores_out;
+        why = "prefill large-k TopK launch";
+        e = launch_large_topk(la, (cudaStream_t)stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e, why);
     return MSA_OK;
 }

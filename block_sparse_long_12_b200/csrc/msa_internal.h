@@ -87,6 +87,10 @@ struct PrefillIdxArgs {
     int *part_i;
     int *status;
     CacheMap cache;            // index-key cache layout (paged: pages of a multiple of 128 tokens)
+    // large k: every visible block's score, row (b * T + t) * G + g at blk_scores + row * blk_stride
+    // (the radix select takes the k best afterwards); null when the epilogue keeps the lists
+    float *blk_scores;
+    long long blk_stride;      // blocks visible to the call's last row
 };
 
 // Key tiles (128 keys) of the i-th prefill index unit in processing order:
@@ -109,8 +113,9 @@ __host__ __device__ inline int prefill_seg_tiles(int nt, int n_seg, int Bk) {
 
 // How a prefill index call splits its work and where its scratch lives.
 struct PrefillIdxPlan {
-    int n_mt, n_seg, grid, kt;
-    size_t counters, part_s, part_i, total;
+    int n_mt, n_seg, grid, kt;  // kt 0: large k (block scores stored, then the radix select)
+    long long blk_stride;
+    size_t counters, part_s, part_i, blk_scores, total;
 };
 PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm);
 
@@ -119,6 +124,14 @@ PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm);
 // rows' r heads against one block, giving one partial output per pair that a merge
 // combines per row by log-sum-exp.
 constexpr int kPrefillRowsPerPass = 8192;
+// Rows per pass for top_k blocks per row: kPrefillRowsPerPass up to kMaxTopKList, fewer beyond
+// so that a pass's (row, block) pairs -- and its per-pair partials -- stay within those of
+// kPrefillRowsPerPass rows of kMaxTopKList blocks.
+__host__ __device__ inline int prefill_rows_per_pass(int top_k) {
+    return top_k <= kMaxTopKList ? kPrefillRowsPerPass : kPrefillRowsPerPass * kMaxTopKList / top_k;
+}
+// A tile member is (row of the pass << kSlotBits) | slot of the row's list (slot < kMaxTopK).
+constexpr int kSlotBits = 10;
 
 struct PrefillAttnArgs {
     const int *ids;            // [B, T, G, k]
@@ -135,7 +148,7 @@ struct PrefillAttnArgs {
     int *counts;               // [B*G*nbv] pairs per bucket (zeroed before the pass)
     int *offsets;              // [B*G*nbv] first member of each bucket
     int *rank;                 // [B*Tn*G*k] rank of each pair in its bucket (-1: not attended)
-    int *members;              // [pairs] member (tt << 5) | slot, grouped by bucket (k <= 32)
+    int *members;              // [pairs] member (tt << kSlotBits) | slot, grouped by bucket
     int4 *tiles;               // [max_tiles] (bucket, first member, member count, 0)
     int *n_tiles;
     int *block_sums;           // [2 * scan blocks] pairs and tiles of each scan block's buckets

@@ -14,7 +14,7 @@
 // log-sum-exp into the row's output.  No tile computes a row that did not
 // select its block.
 //
-// Per pass over up to kPrefillRowsPerPass query rows:
+// Per pass over up to prefill_rows_per_pass(k) query rows:
 //   pa_count_kernel     pairs per bucket and each pair's rank in it;
 //   pa_tilecount_kernel pairs and tiles per scan block of 1024 buckets;
 //   pa_emit_kernel      bucket offsets and the tile list (bucket order);
@@ -37,7 +37,8 @@
 //     warps 12-15 epilogue: O / sum as bf16, stored chunk-major per pair so
 //                 that the r heads of a member (consecutive lanes) write
 //                 whole lines, and the log2 sum per pair;
-//   pa_merge_kernel     per row and group: log-sum-exp of its pairs -> o, lse.
+//   pa_merge_kernel     per row and group: log-sum-exp of its pairs -> o, lse
+//                       (pa_merge_many_kernel for lists beyond 32 blocks).
 #include "tcgen05.cuh"
 
 namespace msa {
@@ -61,7 +62,7 @@ constexpr int kRun = 8;         // consecutive tiles of the list a CTA takes at 
 struct TileInfo {
     int bkt, start, cnt, last;  // last: the CTA's next tile is another bucket (or none)
     int b, g, n, pad;
-    int mem[kPtRows];           // member i: (row tt << 5) | slot
+    int mem[kPtRows];           // member i: (row tt << kSlotBits) | slot
 };
 
 struct PtBars {
@@ -291,7 +292,7 @@ __global__ void pa_scatter_kernel(const PrefillAttnArgs a) {
         const int tt = (int)(rest % a.Tn);
         const int b = (int)(rest / a.Tn);
         const int id = a.ids[(((size_t)b * a.T + a.t0 + tt) * a.G + g) * a.k + j];
-        a.members[a.offsets[((size_t)b * a.G + g) * a.nbv + id] + rk] = (tt << 5) | j;  // k <= 32
+        a.members[a.offsets[((size_t)b * a.G + g) * a.nbv + id] + rk] = (tt << kSlotBits) | j;
     }
 }
 
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(pt_threads(BK), 1)
             for (int q = 0; q < kPtRows / 32; ++q) {
                 const int m = lane + 32 * q;
                 if (m < cnt) {
-                    const int qrow = ((b * a.T + a.t0 + (mem[q] >> 5)) * a.Hq) + g * r;
+                    const int qrow = ((b * a.T + a.t0 + (mem[q] >> kSlotBits)) * a.Hq) + g * r;
                     for (int h = 0; h < NH; ++h)
                         tc::tma_load_2d(smQ + qs * Q_STAGE + h * kHalf + m * r * 128, &qmap, h * 64, qrow,
                                         &S.q_full[qs]);
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(pt_threads(BK), 1)
                 const TileInfo &I = S.info[il % kInfoSlots];
                 n = I.n;
                 valid = m_i < I.cnt;
-                if (valid) pos = a.q_start + a.t0 + (I.mem[m_i] >> 5);
+                if (valid) pos = a.q_start + a.t0 + (I.mem[m_i] >> kSlotBits);
                 info_release(il);
             }
             const bool any = __any_sync(FULL, valid);
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(pt_threads(BK), 1)
                 valid = m_i < I.cnt;
                 if (valid) {
                     const int mem = I.mem[m_i];
-                    pl = ((I.b * a.Tn + (mem >> 5)) * a.G + I.g) * a.k + (mem & 31);  // the pair's index in this pass
+                    pl = ((I.b * a.Tn + (mem >> kSlotBits)) * a.G + I.g) * a.k + (mem & ((1 << kSlotBits) - 1));  // the pair's index in this pass
                 }
                 info_release(il);
             }
@@ -772,6 +773,124 @@ __global__ void __launch_bounds__(256, 2) pa_merge_kernel(const PrefillAttnArgs 
     }
 }
 
+// k > kMaxTopKList: the same merge over the row's slots in chunks of 32.  A first pass over the
+// chunks' log2 sums keeps each head's running maximum and rescaled sum; the second weights the
+// partials.
+template <int PER>
+__global__ void __launch_bounds__(256, 2) pa_merge_many_kernel(const PrefillAttnArgs a) {
+    __shared__ float s_lse[8][32 * 16];        // per warp: [slot of the chunk][head] log2 sums
+    __shared__ float s_m[8][16], s_inv[8][16];
+    const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long w = blockIdx.x * 8LL + wib;
+    if (w >= (long long)a.B * a.Tn * a.G) return;  // whole warps only; no block-wide barrier below
+    const int g = (int)(w % a.G);
+    const long long rest = w / a.G;
+    const int tt = (int)(rest % a.Tn);
+    const int b = (int)(rest / a.Tn);
+    const int t = a.t0 + tt;
+    const int pos = a.q_start + t;
+    const int r = a.r, k = a.k, D = a.D;
+    const int rs = __ffs(r) - 1;
+    const size_t pl0 = (((size_t)b * a.Tn + tt) * a.G + g) * k;
+    const int *row_ids = a.ids + (((size_t)b * a.T + t) * a.G + g) * k;
+    float *L = s_lse[wib];
+    // slots j0 .. j0 + 31: which are attended, and their log2 sums into L
+    auto load_chunk = [&](int j0) -> unsigned {
+        bool v = false;
+        if (j0 + lane < k) {
+            const int id = row_ids[j0 + lane];
+            v = pair_valid(id, a.Bk, pos) && id < a.nbv;
+        }
+        const unsigned vm = __ballot_sync(FULL, v);
+        __syncwarp();  // the previous chunk's readers are done with L
+        for (int e = lane; e < 32 * r; e += 32)
+            L[e] = (vm >> (e >> rs)) & 1u ? a.part_lse[(pl0 + j0) * r + e] : -INFINITY;
+        __syncwarp();
+        return vm;
+    };
+    float m = -INFINITY, sum = 0.f;  // lane < r: head `lane`
+    for (int j0 = 0; j0 < k; j0 += 32) {
+        load_chunk(j0);
+        if (lane < r) {
+            float mc = -INFINITY;
+            for (int j = 0; j < 32; ++j) mc = fmaxf(mc, L[j * r + lane]);
+            const float mn = fmaxf(m, mc);
+            if (mn > -INFINITY) {
+                sum = m > -INFINITY ? sum * exp2_approx(m - mn) : 0.f;
+                for (int j = 0; j < 32; ++j) sum += exp2_approx(L[j * r + lane] - mn);
+                m = mn;
+            }
+        }
+    }
+    if (lane < r) {
+        s_m[wib][lane] = m;
+        s_inv[wib][lane] = sum > 0.f ? 1.f / sum : 0.f;
+        if (a.lse != nullptr)
+            a.lse[((size_t)b * a.T + t) * a.Hq + g * r + lane] =
+                sum > 0.f ? (m + log2f(sum)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncwarp();
+    const int nch = r * D / 8, cph = D / 8;
+    float acc[PER][8];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+    constexpr int NBATCH = PER >= 8 ? 1 : PER >= 4 ? 2 : 4;
+    for (int j0 = 0; j0 < k; j0 += 32) {
+        unsigned mk = load_chunk(j0);
+        while (mk) {
+            int js[NBATCH];
+#pragma unroll
+            for (int q = 0; q < NBATCH; ++q) {
+                js[q] = mk ? __ffs(mk) - 1 : -1;
+                if (mk) mk &= mk - 1;
+            }
+            uint4 raw[NBATCH][PER];
+#pragma unroll
+            for (int q = 0; q < NBATCH; ++q)
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    const int c = lane + 32 * i;
+                    raw[q][i] = make_uint4(0u, 0u, 0u, 0u);
+                    if (js[q] >= 0 && c < nch)
+                        raw[q][i] = __ldcs(reinterpret_cast<const uint4 *>(a.part_o + (pl0 + j0 + js[q]) * r * D) + c);
+                }
+#pragma unroll
+            for (int q = 0; q < NBATCH; ++q) {
+                if (js[q] < 0) continue;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    const int c = lane + 32 * i;
+                    if (c >= nch) continue;
+                    const int hh = c & (r - 1);
+                    const float wt = exp2_approx(L[js[q] * r + hh] - s_m[wib][hh]) * s_inv[wib][hh];
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw[q][i]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(h[e]);
+                        acc[i][2 * e] = fmaf(wt, f.x, acc[i][2 * e]);
+                        acc[i][2 * e + 1] = fmaf(wt, f.y, acc[i][2 * e + 1]);
+                    }
+                }
+            }
+        }
+    }
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(a.o) + (((size_t)b * a.T + t) * a.Hq + g * r) * D;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int c = lane + 32 * i;
+        if (c >= nch) continue;
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const __nv_bfloat162 o2 = __floats2bfloat162_rn(acc[i][2 * e], acc[i][2 * e + 1]);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&o2);
+        }
+        reinterpret_cast<uint4 *>(o)[(c & (r - 1)) * cph + (c >> rs)] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
 template <int D, int BK>
 size_t tile_smem_bytes() {
     return 1024 + 2 * (size_t)(D / 64) * kHalf + 2 * (size_t)(2 * (D / 64) * BK * 128) + sizeof(PtBars) + 64;
@@ -798,7 +917,8 @@ PrefillAttnPlan prefill_attn_plan(const msa_params_t &p) {
     PrefillAttnPlan L{};
     const int r = p.n_q_heads / p.n_kv_heads;
     const int tt = 128 / r;
-    L.rows = p.q_len < kPrefillRowsPerPass ? p.q_len : kPrefillRowsPerPass;
+    const int per_pass = prefill_rows_per_pass(p.top_k);
+    L.rows = p.q_len < per_pass ? p.q_len : per_pass;
     L.nbv_max = (p.q_start + p.q_len - 1) / p.block_size + 1;
     const size_t pairs = (size_t)p.batch * L.rows * p.n_kv_heads * p.top_k;
     const size_t buckets = (size_t)p.batch * p.n_kv_heads * L.nbv_max;
@@ -835,9 +955,10 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
         return cudaErrorInvalidValue;
     a.tt = 128 / a.r;
     cudaError_t e = cudaSuccess;
-    for (int t0 = 0; t0 < a.T && e == cudaSuccess; t0 += kPrefillRowsPerPass) {
+    const int per_pass = prefill_rows_per_pass(a.k);
+    for (int t0 = 0; t0 < a.T && e == cudaSuccess; t0 += per_pass) {
         a.t0 = t0;
-        a.Tn = a.T - t0 < kPrefillRowsPerPass ? a.T - t0 : kPrefillRowsPerPass;
+        a.Tn = a.T - t0 < per_pass ? a.T - t0 : per_pass;
         a.nbv = (a.q_start + t0 + a.Tn - 1) / a.Bk + 1;
         const long long pairs = (long long)a.B * a.Tn * a.G * a.k;
         const int pgrid = (int)((pairs + 255) / 256 < 4LL * n_sm ? (pairs + 255) / 256 : 4LL * n_sm);
@@ -860,7 +981,12 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
         const long long warps = (long long)a.B * a.Tn * a.G;
         const int mgrid = (int)((warps + 7) / 8);
         const int per = (a.r * a.D / 8 + 31) / 32;  // 16-byte chunks per lane
-        if (per <= 1) pa_merge_kernel<1><<<mgrid, 256, 0, s>>>(a);
+        if (a.k > kMaxTopKList) {
+            if (per <= 1) pa_merge_many_kernel<1><<<mgrid, 256, 0, s>>>(a);
+            else if (per <= 2) pa_merge_many_kernel<2><<<mgrid, 256, 0, s>>>(a);
+            else if (per <= 4) pa_merge_many_kernel<4><<<mgrid, 256, 0, s>>>(a);
+            else pa_merge_many_kernel<8><<<mgrid, 256, 0, s>>>(a);
+        } else if (per <= 1) pa_merge_kernel<1><<<mgrid, 256, 0, s>>>(a);
         else if (per <= 2) pa_merge_kernel<2><<<mgrid, 256, 0, s>>>(a);
         else if (per <= 4) pa_merge_kernel<4><<<mgrid, 256, 0, s>>>(a);
         else pa_merge_kernel<8><<<mgrid, 256, 0, s>>>(a);

@@ -28,7 +28,9 @@
 //               tcgen05.ld of the scores, causal mask on diagonal tiles,
 //               3-input max per 32 columns, block max, and a sorted top-k per
 //               row in shared memory; the groups' lists are merged per row
-//               when the piece ends.
+//               when the piece ends.  For k beyond the lists (large k) the
+//               epilogue stores every visible block's score instead, and a
+//               radix select per row (large_topk.cu) keeps the k best.
 // The next tile's MMAs overlap the epilogue of the current one.
 #include "tcgen05.cuh"
 
@@ -43,7 +45,8 @@ constexpr int kKeys = 128;              // keys per tile (N)
 constexpr int kThreads = 640;           // 4 control warps + 16 epilogue warps
 constexpr int kEpiWarp0 = 4;
 constexpr int kEpiThreads = 512;
-// ring stages: the per-row lists take K x 512 x 8 bytes of shared memory
+// ring stages: the per-row lists take K x 512 x 8 bytes of shared memory (K = 0: no lists, the
+// block scores are stored for a radix select)
 template <int K> struct PiShape { static constexpr int S = K >= 32 ? 4 : 6; };
 constexpr int kMaxStages = 6;
 constexpr int kTileBytes = kKeys * 128; // 128 rows of 64 bf16
@@ -80,13 +83,19 @@ struct SmemTopK {
     int j;
     float thr_s;
     int thr_i;
+    float *store = nullptr;  // K = 0: the row's stored block scores (insert writes score n at n)
     __device__ inline void reset() {
+        if constexpr (K == 0) return;
 #pragma unroll
         for (int i = 0; i < K; ++i) { s[i * kEpiThreads + j] = -INFINITY; id[i * kEpiThreads + j] = 0x7fffffff; }
         thr_s = -INFINITY;
         thr_i = 0x7fffffff;
     }
     __device__ inline void insert(float cs, int ci) {
+        if constexpr (K == 0) {
+            if (store != nullptr) store[ci] = cs;
+            return;
+        }
         if (!better(cs, ci, thr_s, thr_i)) return;
 #pragma unroll
         for (int i = 0; i < K; ++i) {
@@ -258,9 +267,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = m0 + rl;
             const int pos = a.q_start + t;
             const int pos_min = a.q_start + m0;  // smallest position of the unit
-            // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank above every score
-            auto forced = [&](int blk) { return a.force && (blk == 0 || blk == pos / BK); };
+            // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank above every score (large
+            // k: the radix select applies it to the stored scores)
+            auto forced = [&](int blk) { return K > 0 && a.force && (blk == 0 || blk == pos / BK); };
             top.reset();
+            if constexpr (K == 0) {
+                // rows past the call's last one are never stored (their block range is outside)
+                const long long row = ((long long)b * a.T + (t < a.T ? t : a.T - 1)) * a.G + g;
+                top.store = t < a.T ? a.blk_scores + row * a.blk_stride : nullptr;
+            }
             float bm = -INFINITY;
             for (int n = w.n0; n < w.n1 && ok; ++n, ++ti) {
                 if ((two_groups ? (n & 1) : 0) != grp) continue;  // the other group's tile
@@ -314,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // After an abort every warp still runs every barrier of every piece (its waits fail fast).
             const bool whole = w.n_parts == 1;
             named_barrier(1, kEpiThreads);
-            if (grp == 0) {
+            if (K > 0 && grp == 0) {
                 // merge the two groups' lists of each row (disjoint block sets)
                 const int ja = e * 32 + lane, jb = ja + 8 * 32;
                 const size_t o = (((size_t)b * a.T + t) * a.G + g) * a.k;
@@ -426,6 +441,7 @@ cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, con
     }
     const int grid = n_sm;  // the plan's CTA count (at most one per SM)
     *why = "prefill index kernel launch";
+    if (a.blk_scores != nullptr) return launch_kb<0>(a, qm, km, grid, s);
     return a.k <= 8 ? launch_kb<8>(a, qm, km, grid, s) : a.k <= 16 ? launch_kb<16>(a, qm, km, grid, s)
                                                              : launch_kb<32>(a, qm, km, grid, s);
 }

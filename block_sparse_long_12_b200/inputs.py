@@ -63,8 +63,9 @@ class Workload:
 
 
 # The workloads: tiny fp32 decode, 16K causal prefill, ragged batched 128K
-# decode, 1M decode (batch 1 and 4), 1M chunked causal prefill, and 1M decode
-# with one index-K head shared by every group.
+# decode, 1M decode (batch 1 and 4), 1M chunked causal prefill, 1M decode
+# with one index-K head shared by every group, and the large-k regime in
+# decode (1M) and prefill (128K).
 WORKLOADS = {
     "decode_fp32_ctx4k": Workload("decode_fp32_ctx4k", "decode", 1, 4096, 4, 1, 1, 64, 32, 64, 8,
                                   "f32", seed=1001),
@@ -85,6 +86,10 @@ WORKLOADS = {
     # 1M tokens, about 6 % selected (k 1024)
     "decode_ctx1m_large_k": Workload("decode_ctx1m_large_k", "decode", 1, 1048576, 64, 8, 8, 128, 64, 64, 1024,
                                      "bf16", hot_blocks=32, seed=1007),
+    # the same density in prefill: 128K tokens in 64-token blocks (2,048 of them), k 128 (6.25 %),
+    # 8192-token chunks
+    "prefill_ctx128k_large_k": Workload("prefill_ctx128k_large_k", "prefill", 1, 131072, 64, 8, 8, 128, 64, 64, 128,
+                                        "bf16", hot_blocks=32, chunk=8192, seed=1008),
 }
 
 

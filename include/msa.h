@@ -123,7 +123,7 @@ typedef struct {
     int head_dim;         /* D: 64 or 128                                      */
     int idx_dim;          /* di: idx_dim * sizeof(elem) in {64, 128, 256} bytes */
     int block_size;       /* Bk: 16..256, power of two                         */
-    int top_k;            /* 1..1024; the prefill entries take 1..32           */
+    int top_k;            /* 1..1024                                           */
     int q_len;            /* decode entries: 1; prefill: chunk length          */
     int q_start;          /* prefill: absolute position of query row 0         */
     int max_seq_len;      /* Lmax, the caches' token stride                    */
@@ -191,7 +191,11 @@ MSA_API msa_status_t msa_sparse_attn_decode(const msa_params_t *params, const vo
 
 /*
  * Step 2 for a causal prefill chunk: query rows t = 0..q_len-1 at positions
- * q_start + t, each with its own list ids[b, t, g, :].  bf16 only.
+ * q_start + t, each with its own list ids[b, t, g, :].  bf16 only; block_size
+ * 64 or 128.  Work is by block: every (row, listed block) pair leaves a partial
+ * output in ws that a merge combines per row, in passes of 8192 rows (fewer
+ * when top_k > 32: 8192 * 32 / top_k, so that ws does not grow with top_k).
+ * Entries of ids that are -1 or name a block after the row are skipped.
  */
 MSA_API msa_status_t msa_sparse_attn_prefill(const msa_params_t *params, const void *q, const void *k_cache,
                                      const void *v_cache, const int32_t *ids, void *o, float *lse,
@@ -263,12 +267,16 @@ MSA_API msa_status_t msa_decode_append(const msa_params_t *params, const void *k
 
 /*
  * Step 1 for a causal prefill chunk, fused: index scores on tensor cores,
- * block max pool and TopK in the epilogue; scores are never stored.
+ * block max pool and TopK in the epilogue; token scores are never stored.
  * ids_out [B, q_len, G, top_k]; top_scores_out nullable.  bf16 only.
  * The work (every query row against every key it can see) is cut into equal
  * ranges, one per SM; ws holds the per-row lists of rows whose keys were
  * split between ranges until they are merged (msa_workspace_size(params,
  * MSA_ENTRY_PREFILL_INDEX_TOPK) bytes, contents need no initialisation).
+ * top_k up to 32 keeps sorted lists per row in the epilogue; above 32 the
+ * epilogue stores every visible block score of every row in ws (B * q_len *
+ * G * ((q_start + q_len - 1) / block_size + 1) floats) and a radix select
+ * per row keeps the k best, in the same order.
  */
 MSA_API msa_status_t msa_prefill_index_topk(const msa_params_t *params, const void *q_idx, const void *k_idx,
                                     int32_t *ids_out, float *top_scores_out, void *ws, size_t ws_bytes,

@@ -119,10 +119,11 @@ def test_bad_pointers_rejected_before_launch(lib):
     pp = good_params(lib, q_len=100, q_start=4000)
     rc = L.msa_prefill_index_topk(ctypes.byref(pp), a, a, a, None, a, ws, None)
     assert rc == lib.MSA_ERR_INVALID_ARG
-    # prefill entries keep warp lists: at most 32 blocks per row
+    # large k in prefill: lists of more than 32 blocks pass the checks (then fail on the fake pointers'
+    # workspace size, not on top_k)
     pk = good_params(lib, q_len=100, top_k=64)
-    assert L.msa_prefill_index_topk(ctypes.byref(pk), a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
-    assert L.msa_sparse_attn_prefill(ctypes.byref(pk), a, a, a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
+    assert L.msa_sparse_attn_prefill(ctypes.byref(pk), a, a, a, a, a, None, a, ctypes.c_size_t(64),
+                                     None) == lib.MSA_ERR_WORKSPACE
     # index scores need exactly one score granularity
     rc = L.msa_index_score(ctypes.byref(p), a, a, a, a, ws, None)
     assert rc == lib.MSA_ERR_INVALID_ARG
@@ -183,3 +184,13 @@ def test_paged_params_rejected_before_launch(lib):
     pp = good_params(lib, q_len=100, block_size=64)
     pp.block_table, pp.n_pages = a, 64
     assert L.msa_prefill_index_topk(ctypes.byref(pp), a, a, a, None, a, ws, None) == lib.MSA_ERR_UNSUPPORTED
+
+
+def test_prefill_attention_workspace_does_not_grow_with_k(lib):
+    """Passes hold 8192 * 32 / k rows beyond k = 32, so the per-pair partials keep one size."""
+    base = lib.msa_workspace_size(good_params(lib, q_len=16384, q_start=0, max_seq_len=16384, top_k=32),
+                                  lib.MSA_ENTRY_ATTN_PREFILL)
+    for k in (64, 256, 1024):
+        n = lib.msa_workspace_size(good_params(lib, q_len=16384, q_start=0, max_seq_len=16384, top_k=k),
+                                   lib.MSA_ENTRY_ATTN_PREFILL)
+        assert base * 0.99 <= n <= base * 1.01, (k, n, base)
