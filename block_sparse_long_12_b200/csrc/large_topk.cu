@@ -10,7 +10,8 @@
 // digits of 12, 12 and 8 bits over the score bits, the same over the id bits only when blocks tie
 // at the k-th score), takes the k keys at or above it and sorts them once (bitonic).  Rows of
 // up to 16,384 blocks keep their keys in registers; longer rows re-read the scores from global
-// memory in every pass (L2 keeps them).
+// memory in every pass (L2 keeps them).  Prefill rows with k up to 256 take one warp per row
+// instead (warp_topk_kernel).
 #include "msa_device.cuh"
 
 namespace msa {
@@ -210,6 +211,119 @@ __global__ void __launch_bounds__(kLargeThreads) large_topk_kernel(const LargeTo
     }
 }
 
+// Prefill rows (one list per query row: many rows, each of at most a few thousand blocks) with
+// k <= kWarpRowMaxK: one warp per row.  The k-th largest score is found exactly by a radix select
+// over the 32 order-preserving score bits (four passes of 8-bit digits, a 256-bin histogram per
+// warp in shared memory, the scores re-read from L2 in each pass); every block above that score
+// is taken, and of the blocks at it the lowest ids, scanned in id order.  The k keys are then
+// ranked by counting (keys are distinct: score bits above the complemented id).
+constexpr int kWarpRowMaxK = 256;
+constexpr int kWarpRows = 8;  // rows (warps) per CTA
+
+__global__ void __launch_bounds__(kWarpRows * 32) warp_topk_kernel(const LargeTopkArgs a) {
+    __shared__ unsigned hist[kWarpRows][256];
+    __shared__ unsigned long long cand[kWarpRows][kWarpRowMaxK];
+    const int wib = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long row = (long long)blockIdx.x * kWarpRows + wib;
+    if (row >= a.rows) return;  // whole warps only; no CTA-wide barrier below
+    const int t = (int)((row / a.G) % a.q_len);
+    int pos = a.q_start + t;
+    if (pos >= a.L_max) pos = a.L_max - 1;
+    const int nb = pos / a.Bk + 1;
+    const int kk = a.k < nb ? a.k : nb;
+    const float *src = a.scores + row * a.stride;
+    const unsigned lt = (1u << lane) - 1u;  // lanes below this one
+    auto bits_of = [&](int n) -> uint32_t {
+        // MSA_FORCE_SINK_LOCAL: block 0 and the row's own block rank above every score
+        return score_bits((a.force && (n == 0 || n == nb - 1)) ? INFINITY : src[n]);
+    };
+    unsigned *H = hist[wib];
+    uint32_t prefix = 0, mask = 0;
+    int rem = kk;  // rank of the k-th score among the scores that match the prefix so far
+    if (kk < nb) {
+#pragma unroll 1
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = lane; i < 256; i += 32) H[i] = 0;
+            __syncwarp();
+            for (int n0 = 0; n0 < nb; n0 += 32) {
+                const int n = n0 + lane;
+                const uint32_t u = n < nb ? bits_of(n) : 0u;
+                const unsigned d = (n < nb && (u & mask) == prefix) ? ((u >> shift) & 255u) : 0xffffffffu;
+                const unsigned peers = __match_any_sync(FULL, d);
+                if (d != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&H[d], (unsigned)__popc(peers));
+            }
+            __syncwarp();
+            // lane l sums bins 255 - 8 l .. 248 - 8 l (from the top); the lane whose running count
+            // reaches rem holds the digit
+            unsigned c[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = H[255 - 8 * lane - i];
+                sum += c[i];
+            }
+            unsigned incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned v = __shfl_up_sync(FULL, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int dsel = -1, rsel = 0;
+            if (incl - sum < (unsigned)rem && (unsigned)rem <= incl) {
+                unsigned above = incl - sum;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (dsel < 0 && above + c[i] >= (unsigned)rem) {
+                        dsel = 255 - 8 * lane - i;
+                        rsel = rem - (int)above;
+                    }
+                    above += c[i];
+                }
+            }
+            const int from = __ffs(__ballot_sync(FULL, dsel >= 0)) - 1;
+            dsel = __shfl_sync(FULL, dsel, from);
+            rsel = __shfl_sync(FULL, rsel, from);
+            prefix |= (uint32_t)dsel << shift;
+            mask |= 255u << shift;
+            rem = rsel;
+            __syncwarp();  // H is read before the next pass clears it
+        }
+    }
+    // kk < nb: every score above `prefix` is taken, and `rem` of the scores equal to it, lowest ids
+    // first; kk == nb: every block
+    unsigned long long *C = cand[wib];
+    int taken = 0, eq_seen = 0;
+    for (int n0 = 0; n0 < nb; n0 += 32) {
+        const int n = n0 + lane;
+        const uint32_t u = n < nb ? bits_of(n) : 0u;
+        const bool gt = n < nb && (kk == nb || u > prefix);
+        const bool eq = n < nb && kk < nb && u == prefix;
+        const unsigned be = __ballot_sync(FULL, eq);
+        const bool take = gt || (eq && eq_seen + __popc(be & lt) < rem);
+        const unsigned bt = __ballot_sync(FULL, take);
+        if (take) C[taken + __popc(bt & lt)] = ((unsigned long long)u << 32) | (uint32_t)~(uint32_t)n;
+        taken += __popc(bt);
+        eq_seen += __popc(be);
+    }
+    __syncwarp();
+    // rank of each key among the kk (distinct) keys: its slot in the list
+    for (int i = lane; i < kk; i += 32) {
+        const unsigned long long key = C[i];
+        int rank = 0;
+        for (int j = 0; j < kk; ++j) rank += C[j] > key ? 1 : 0;
+        const size_t o = (size_t)row * a.k + rank;
+        const int id = (int)~(uint32_t)key;
+        a.ids_out[o] = id;
+        if (a.ids_copy != nullptr) a.ids_copy[o] = id;
+        if (a.top_scores_out != nullptr) a.top_scores_out[o] = bits_score((uint32_t)(key >> 32));
+    }
+    for (int i = kk + lane; i < a.k; i += 32) {
+        const size_t o = (size_t)row * a.k + i;
+        a.ids_out[o] = -1;
+        if (a.ids_copy != nullptr) a.ids_copy[o] = -1;
+        if (a.top_scores_out != nullptr) a.top_scores_out[o] = -INFINITY;
+    }
+}
+
 // Block maxima of stored token scores (rows of L_max) over the visible tokens of every block,
 // one warp per (row, block), for the large-k TopK that reads block scores.
 __global__ void __launch_bounds__(256) token_block_max_kernel(const LargeTopkArgs a, const float *tok,
@@ -243,6 +357,10 @@ __global__ void __launch_bounds__(256) token_block_max_kernel(const LargeTopkArg
 
 cudaError_t launch_large_topk(const LargeTopkArgs &a, cudaStream_t s) {
     if (a.rows <= 0) return cudaSuccess;
+    if (a.prefill && a.k <= kWarpRowMaxK) {
+        warp_topk_kernel<<<(unsigned)((a.rows + kWarpRows - 1) / kWarpRows), kWarpRows * 32, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     large_topk_kernel<<<(unsigned)a.rows, kLargeThreads, 0, s>>>(a);
     return cudaGetLastError();
 }

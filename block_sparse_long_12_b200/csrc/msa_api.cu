@@ -234,7 +234,8 @@ PrefillIdxPlan prefill_index_plan(const msa_params_t &p, int n_sm) {
     PrefillIdxPlan L{};
     L.n_mt = (p.q_len + 255) / 256;
     L.kt = p.top_k <= 8 ? 8 : p.top_k <= 16 ? 16 : p.top_k <= kMaxTopKList ? 32 : 0;
-    L.blk_stride = (p.q_start + p.q_len - 1) / p.block_size + 1;
+    // a row's block scores padded to whole 32-block windows (the stage writes them 16 at a time)
+    L.blk_stride = ((p.q_start + p.q_len - 1) / p.block_size + 1 + 31) / 32 * 32;
     const long long units = (long long)L.n_mt * p.batch * p.n_kv_heads;
     const int max_tiles = prefill_unit_tiles(0, L.n_mt, p.q_len, p.q_start, p.block_size);
     const int gran = p.block_size > 128 ? p.block_size / 128 : 1;

@@ -87,14 +87,14 @@ __device__ inline void mbar_arrive1(uint64_t *bar) {
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]: A (M x 16 bf16) read from tensor memory, lane i = row i,
-// two bf16 per 32-bit column, lower k in the low half.
-__device__ inline void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                   uint32_t accumulate) {
+// two bf16 per 32-bit column, lower k in the low half; the accumulate flag fixed at compile time.
+template <bool ACC>
+__device__ inline void mma_bf16_ts_c(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "n"(ACC ? 1 : 0)
         : "memory");
 }
 
@@ -455,16 +455,19 @@ __global__ void __launch_bounds__(pt_threads(BK), 1)
         bool pend_last = false, ok = true;
         // O = P V of tile `il` (its P overwrote its S buffer); frees the S buffer and, after a
         // bucket's last tile, the K/V stage
+        // descriptor bases of the Q, K and V operands in stage 0 (the issue loops only add offsets)
+        const uint64_t qd0 = tc::sw128_kmajor_desc(smem_u32(smQ)), kd0 = tc::sw128_kmajor_desc(smem_u32(smKV));
+        const uint64_t vd0 = sw128_mnmajor_desc(smem_u32(smKV + NH * KVH), KVH);
         auto issue_pv = [&](int il, int ks, bool last) -> bool {
             const int ob = il & 1;
             if (!tc::wait_or_abort(&S.p_full[ob], (il >> 1) & 1, abort_flag, a.status)) return false;
             if (!tc::wait_or_abort(&S.o_empty[ob], ((il >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
             tc::fence_after_sync();
-            const uint32_t v_addr = smem_u32(smKV + ks * KV_STAGE + NH * KVH);
+            const uint64_t vd = tc::desc_add(vd0, (uint32_t)(ks * KV_STAGE));
+            const uint32_t od = tmem + O_COL + ob * D, pa = tmem + ob * BK;
+            mma_bf16_ts_c<false>(od, pa, vd, idesc_pv);
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-                mma_bf16_ts(tmem + O_COL + ob * D, tmem + ob * BK + kk * 8, sw128_mnmajor_desc(v_addr + kk * 2048, KVH),
-                            idesc_pv, kk > 0 ? 1u : 0u);
+            for (int kk = 1; kk < BK / 16; ++kk) mma_bf16_ts_c<true>(od, pa + kk * 8, tc::desc_add(vd, kk * 2048), idesc_pv);
             tc::mma_commit(&S.o_full[ob]);
             tc::mma_commit(&S.s_empty[ob]);
             if (last) tc::mma_commit(&S.kv_empty[ks]);
@@ -486,12 +489,14 @@ __global__ void __launch_bounds__(pt_threads(BK), 1)
                     ok = false;
                 } else {
                     tc::fence_after_sync();
-                    const uint32_t q_addr = smem_u32(smQ + sb * Q_STAGE), k_addr = smem_u32(smKV + ks * KV_STAGE);
+                    const uint64_t qd = tc::desc_add(qd0, (uint32_t)(sb * Q_STAGE));
+                    const uint64_t kd = tc::desc_add(kd0, (uint32_t)(ks * KV_STAGE));
+                    const uint32_t sd = tmem + sb * BK;
+                    tc::mma_bf16_ss_c<false>(sd, qd, kd, idesc_qk);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        tc::mma_bf16_ss(tmem + sb * BK, tc::sw128_kmajor_desc(q_addr + (kk >> 2) * kHalf + (kk & 3) * 32),
-                                        tc::sw128_kmajor_desc(k_addr + (kk >> 2) * KVH + (kk & 3) * 32), idesc_qk,
-                                        kk > 0);
+                    for (int kk = 1; kk < D / 16; ++kk)
+                        tc::mma_bf16_ss_c<true>(sd, tc::desc_add(qd, (kk >> 2) * kHalf + (kk & 3) * 32),
+                                                tc::desc_add(kd, (kk >> 2) * KVH + (kk & 3) * 32), idesc_qk);
                     tc::mma_commit(&S.q_empty[sb]);
                     tc::mma_commit(&S.s_full[sb]);
                     if (pend >= 0 && !issue_pv(pend, pend_ks, pend_last)) ok = false;

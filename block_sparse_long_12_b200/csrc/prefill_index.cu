@@ -76,6 +76,13 @@ __device__ inline void mbar_arrive(uint64_t *bar) {
 // Row-wise sorted top-K (score desc, id asc) kept in shared memory, entry i of
 // list j at [i * kEpiThreads + j] (consecutive threads, consecutive words); the
 // K-th entry is mirrored in registers so that a losing block costs one compare.
+// K = 0 (large k): block scores are staged per row in shared memory, 32 blocks per window and
+// two windows, rows padded to kStageRow floats (16-byte reads of different rows stay clear of
+// each other's banks), and written to the workspace a window at a time as whole 64-byte runs.
+constexpr int kStageRow = 36;
+constexpr int kStageFloats = kUnitRows * kStageRow;  // one window
+template <int K> constexpr size_t stage_bytes() { return K == 0 ? (size_t)2 * kStageFloats * 4 : 0; }
+
 template <int K>
 struct SmemTopK {
     float *s;
@@ -83,7 +90,7 @@ struct SmemTopK {
     int j;
     float thr_s;
     int thr_i;
-    float *store = nullptr;  // K = 0: the row's stored block scores (insert writes score n at n)
+    float *store = nullptr;  // K = 0: this row in window buffer 0 of the stage
     __device__ inline void reset() {
         if constexpr (K == 0) return;
 #pragma unroll
@@ -93,7 +100,7 @@ struct SmemTopK {
     }
     __device__ inline void insert(float cs, int ci) {
         if constexpr (K == 0) {
-            if (store != nullptr) store[ci] = cs;
+            store[((ci >> 5) & 1) * kStageFloats + (ci & 31)] = cs;
             return;
         }
         if (!better(cs, ci, thr_s, thr_i)) return;
@@ -112,6 +119,21 @@ struct SmemTopK {
         thr_i = id[(K - 1) * kEpiThreads + j];
     }
 };
+
+// Barrier over nthreads threads (named barrier id) that also ANDs a per-thread flag across them.
+__device__ inline bool epi_sync_and(int id, int nthreads, bool ok) {
+    uint32_t r;
+    __syncwarp();
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)ok), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
 
 // Max over the 32 keys j0..j0+31 of one row, counting only keys j <= pos.
 __device__ inline float chunk_max_masked(const uint32_t (&r)[32], int j0, int pos) {
@@ -133,7 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *smB = base + kAccs * kABytes;             // [kStages][128 keys][128 B]
     float *list_s = reinterpret_cast<float *>(smB + kStages * kTileBytes);  // [K][512]
     int *list_i = reinterpret_cast<int *>(list_s + K * kEpiThreads);        // [K][512]
-    Smem &S = *reinterpret_cast<Smem *>(list_i + K * kEpiThreads);
+    float *stage = reinterpret_cast<float *>(list_i + K * kEpiThreads);     // K = 0: [2][256][kStageRow]
+    Smem &S = *reinterpret_cast<Smem *>(reinterpret_cast<unsigned char *>(stage) + stage_bytes<K>());
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int BG = a.B * a.G;
@@ -207,6 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16_f32(kRows, kKeys);
+            // descriptor bases (the issue loop only adds offsets: see tc::desc_add)
+            const uint64_t ad0 = tc::sw128_kmajor_desc(smem_u32(smA)), bd0 = tc::sw128_kmajor_desc(smem_u32(smB));
             int it = 0, ti = 0, pc = 0;
             Piece w;
             for (int p = blockIdx.x; p < n_pieces && !*abort_flag; p += gridDim.x) {
@@ -223,15 +248,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc::fence_after_sync();
-                    const uint32_t b_addr = smem_u32(smB + st * kTileBytes);
+                    const uint64_t bd = tc::desc_add(bd0, (uint32_t)(st * kTileBytes));
+                    const uint32_t d0 = tmem + (uint32_t)(buf * kAccs * kKeys);
 #pragma unroll
                     for (int acc = 0; acc < kAccs; ++acc) {
-                        const uint32_t a_addr = smem_u32(smA + acc * kABytes);
-                        const uint32_t d = tmem + (uint32_t)((buf * kAccs + acc) * kKeys);
+                        const uint64_t ad = tc::desc_add(ad0, acc * kABytes);
+                        const uint32_t d = d0 + acc * kKeys;
+                        tc::mma_bf16_ss_c<false>(d, ad, bd, idesc);
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            tc::mma_bf16_ss(d, tc::sw128_kmajor_desc(a_addr + ks * 32),
-                                            tc::sw128_kmajor_desc(b_addr + ks * 32), idesc, ks > 0);
+                        for (int ks = 1; ks < 4; ++ks)
+                            tc::mma_bf16_ss_c<true>(d, tc::desc_add(ad, ks * 32), tc::desc_add(bd, ks * 32), idesc);
                     }
                     tc::mma_commit(&S.empty[st]);
                     tc::mma_commit(&S.acc_full[buf]);
@@ -271,19 +297,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             // k: the radix select applies it to the stored scores)
             auto forced = [&](int blk) { return K > 0 && a.force && (blk == 0 || blk == pos / BK); };
             top.reset();
-            if constexpr (K == 0) {
-                // rows past the call's last one are never stored (their block range is outside)
-                const long long row = ((long long)b * a.T + (t < a.T ? t : a.T - 1)) * a.G + g;
-                top.store = t < a.T ? a.blk_scores + row * a.blk_stride : nullptr;
-            }
-            float bm = -INFINITY;
-            for (int n = w.n0; n < w.n1 && ok; ++n, ++ti) {
-                if ((two_groups ? (n & 1) : 0) != grp) continue;  // the other group's tile
-                const int buf = ti & 1;
-                if (!tc::wait_or_abort(&S.acc_full[buf], (ti >> 1) & 1, abort_flag, a.status)) {
-                    ok = false;
-                    break;
+            if constexpr (K == 0) top.store = stage + rl * kStageRow;
+            // K = 0: the piece's blocks, and the stage written to the workspace after each window's
+            // last block (every epilogue thread takes part, so no thread leaves the tile loop early)
+            const int blk_lo = w.n0 * kKeys / BK, blk_hi = (w.n1 * kKeys + BK - 1) / BK - 1;
+            auto flush = [&](int win) {
+                const int te = e * 32 + lane, r = te >> 1, h = te & 1, tr = m0 + r;
+                const int c0 = win * 32 + h * 16;
+                if (tr >= a.T) return;
+                const float *src = stage + (win & 1) * kStageFloats + r * kStageRow + h * 16;
+                float *dst = a.blk_scores + (((long long)b * a.T + tr) * a.G + g) * a.blk_stride + c0;
+                if (c0 >= blk_lo && c0 + 15 <= blk_hi) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        reinterpret_cast<float4 *>(dst)[q] = reinterpret_cast<const float4 *>(src)[q];
+                } else {
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i >= blk_lo && c0 + i <= blk_hi) dst[i] = src[i];
                 }
+            };
+            float bm = -INFINITY;
+            // one tile of this group: scores from TMEM, causal mask on diagonal tiles, maxima per 32
+            // columns, block maxima into the row's list (or the stage); false when a wait gave up
+            auto do_tile = [&](int n, int ti_) -> bool {
+                const int buf = ti_ & 1;
+                if (!__all_sync(FULL, tc::wait_or_abort(&S.acc_full[buf], (ti_ >> 1) & 1, abort_flag, a.status)))
+                    return false;
                 tc::fence_after_sync();
                 const uint32_t col = tmem + lane_addr + (uint32_t)((buf * kAccs + acc) * kKeys);
                 const int kb = n * kKeys;
@@ -323,6 +362,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int c = 1; c < CPB; ++c) v = fmaxf(v, cm[q * CPB + c]);
                         const int blk = n * (kKeys / BK) + q;
                         if (!diag || blk * BK <= pos) top.insert(forced(blk) ? INFINITY : v, blk);
+                    }
+                }
+                return true;
+            };
+            if constexpr (K == 0) {
+                // every epilogue thread walks every tile of the piece (no thread leaves early), so that
+                // all of them meet at each window's end: a window ends with its 32nd block or the piece
+                for (int n = w.n0; n < w.n1; ++n, ++ti) {
+                    const int last_blk = BK >= kKeys ? ((n + 1) % (BK / kKeys) == 0 ? n / (BK / kKeys) : -1)
+                                                     : (n + 1) * (kKeys / BK) - 1;
+                    const bool win_end = last_blk >= 0 && ((last_blk & 31) == 31 || n == w.n1 - 1);
+                    if (ok && (two_groups ? (n & 1) : 0) == grp) ok = do_tile(n, ti);
+                    if (win_end) {
+                        ok = epi_sync_and(3, kEpiThreads, ok);
+                        if (ok) flush(last_blk >> 5);
+                    }
+                }
+            } else {
+                for (int n = w.n0; n < w.n1 && ok; ++n, ++ti) {
+                    if ((two_groups ? (n & 1) : 0) != grp) continue;  // the other group's tile
+                    if (!do_tile(n, ti)) {
+                        ok = false;
+                        break;
                     }
                 }
             }
@@ -396,7 +458,7 @@ template <int K, int BK>
 cudaError_t launch_k(const PrefillIdxArgs &a, const CUtensorMap &qm, const CUtensorMap &km, int grid,
                      cudaStream_t s) {
     const size_t smem = 1024 + kAccs * kABytes + PiShape<K>::S * kTileBytes + (size_t)K * kEpiThreads * 8 +
-                        sizeof(Smem) + 64;
+                        stage_bytes<K>() + sizeof(Smem) + 64;
     static bool attr = false;
     if (!attr) {
         cudaError_t e =

@@ -79,6 +79,26 @@ __device__ inline void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// The same with the accumulate flag fixed at compile time.  The issuing thread shares its
+// sub-partition's issue slots with busy epilogue or softmax warps, so the hot issue loops keep
+// to the MMA itself: descriptors advance by desc_add on a precomputed base.
+template <bool ACC>
+__device__ inline void mma_bf16_ss_c(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "n"(ACC ? 1 : 0)
+        : "memory");
+}
+// A descriptor for an operand `bytes` further on in shared memory (the start address field holds
+// address >> 4 in 14 bits and shared memory addresses stay below 2^18, so the sum cannot carry
+// out of the field).
+__device__ inline uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+    const uint32_t lo = (uint32_t)desc + (bytes >> 4), hi = (uint32_t)(desc >> 32);
+    return ((uint64_t)hi << 32) | lo;
+}
+
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
 __device__ inline void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
