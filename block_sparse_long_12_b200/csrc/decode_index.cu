@@ -101,20 +101,18 @@ struct ChunkCursor {
     }
 };
 
-// Warps per CTA and stages per warp ring: one index-K head per stream (GPS 1)
-// keeps the index query in registers and affords 12 warps; several groups
-// on one stream (GPS > 1) read it from shared memory and use 8 warps.
-template <int GPS> struct ScanShape {
-    static constexpr int W = GPS == 1 ? 12 : 8;
-};
 // several groups on one bf16 stream of 128- or 256-byte rows are scored on tensor cores
 template <typename T, int GPS, int ROWB> constexpr bool scan_mma() { return GPS > 1 && sizeof(T) == 2 && ROWB >= 128; }
+// Warps per CTA (W): one index-K head per stream (GPS 1) keeps the index query in registers and
+// affords 12 warps; several groups on one stream read it from shared memory (CUDA cores, 8 warps)
+// or hold it as mma fragments (12 warps while the batch's bookkeeping leaves the shared memory:
+// their per-chunk work is a chain of dependent instructions, so more warps hide more of its
+// latency; 8 beyond).
 
-// S: ring stages per warp (2; 3 when tensor-core scoring leaves the room and the batch allows)
-template <typename T, int GPS, int ROWB, int S>
-__global__ void __launch_bounds__(ScanShape<GPS>::W * 32, 1)
+// S: ring stages per warp (2)
+template <typename T, int GPS, int ROWB, int S, int W>
+__global__ void __launch_bounds__(W * 32, 1)
     decode_scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
-    constexpr int W = ScanShape<GPS>::W;
     constexpr int ES = (int)sizeof(T);
     constexpr int EPV = Vec16<T>::N;      // elements per 16-byte vector
     constexpr int NCH = ROWB / 16;        // 16-byte vectors per index-key row
@@ -602,10 +600,9 @@ __global__ void fill_neg_inf_kernel(const FillArgs a) {
         a.scores[i] = -INFINITY;
 }
 
-template <typename T, int GPS, int ROWB, int S>
+template <typename T, int GPS, int ROWB, int S, int W>
 size_t scan_smem_bytes(int B) {
     constexpr bool MMA = scan_mma<T, GPS, ROWB>();
-    constexpr int W = ScanShape<GPS>::W;
     constexpr int DI = ROWB / (int)sizeof(T);
     constexpr bool QREG = GPS == 1 && DI <= 64;
     return 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 + (size_t)GPS * DI * 4 +
@@ -613,13 +610,12 @@ size_t scan_smem_bytes(int B) {
            kTailPools * 4 + 4 + 64;
 }
 
-template <typename T, int GPS, int ROWB, int S>
+template <typename T, int GPS, int ROWB, int S, int W>
 cudaError_t launch_scan_s(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
-    constexpr int W = ScanShape<GPS>::W;
-    const size_t smem = scan_smem_bytes<T, GPS, ROWB, S>(a.B);
+    const size_t smem = scan_smem_bytes<T, GPS, ROWB, S, W>(a.B);
     static size_t attr_bytes = 0;  // opt-in raised on demand (smem grows with the batch)
     if (smem > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB, S>,
+        cudaError_t e = cudaFuncSetAttribute(decode_scan_kernel<T, GPS, ROWB, S, W>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr_bytes = smem;
@@ -634,15 +630,16 @@ cudaError_t launch_scan_s(const ScanArgs &a, const CUtensorMap &km, cudaStream_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, ROWB, S>, km, a);
+    return cudaLaunchKernelEx(&cfg, decode_scan_kernel<T, GPS, ROWB, S, W>, km, a);
 }
 
 template <typename T, int GPS, int ROWB>
 cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
+    if constexpr (GPS == 1) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
     if constexpr (scan_mma<T, GPS, ROWB>()) {
-        if (scan_smem_bytes<T, GPS, ROWB, 3>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 3>(a, km, s, pdl);
+        if (scan_smem_bytes<T, GPS, ROWB, 2, 12>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
     }
-    return launch_scan_s<T, GPS, ROWB, 2>(a, km, s, pdl);
+    return launch_scan_s<T, GPS, ROWB, 2, 8>(a, km, s, pdl);
 }
 
 template <typename T, int ROWB>
