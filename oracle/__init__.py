@@ -10,7 +10,10 @@ Two independent formulations live here:
   the oracle proper, wrapped below through ctypes;
 * ``numpy_twin.py``, a vectorised NumPy restatement written differently
   (rank counting instead of sorting, masks instead of gathers), used only to
-  cross-check the C code.
+  cross-check the C code;
+* ``mxfp8.py``, the MXFP8 storage of index keys (E4M3 elements, one E8M0 scale
+  per 32): its quantiser and its exact decoding to float32, after which Step 1
+  runs through the C oracle like every other workload.
 
 Method source: "MiniMax wird duenn: M3-Attention anhand eines einzigen
 Diagramms entschluesselt" (atlascloud.ai), section 1, Step 1 (index branch:
