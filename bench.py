@@ -8,7 +8,8 @@ CPU oracle timed on this host:
   * every other workload: tiny fp32 decode, 16K causal prefill, ragged
     batch-8 128K decode, batch-4 1M decode, 128K prefill with k 128 of 2,048
     blocks (``configs``);
-  * the 1M decode with one shared index-K head and the large-k regime;
+  * the 1M decode with one shared index-K head, the large-k regime, and
+    MXFP8 index keys;
   * the 1M-token chunked causal prefill (tok/s, tensor-core fraction);
   * the dense GQA decode over the same cache, and an end-to-end number with
     host<->device copies inside the timed region.
@@ -357,7 +358,9 @@ def workload_config(w, n):
 # ----------------------------------------------------------------------------- decode timing
 def decode_bytes(w, lens_host) -> tuple[int, int]:
     es = 2 if w.dtype == "bf16" else 4
-    idx = sum(lens_host) * w.n_idx_k_heads * w.idx_dim * es  # every index key read once
+    # every index key read once: idx_dim elements, or MXFP8 codes plus one scale byte per 32
+    row = w.idx_dim + w.idx_dim // 32 if w.idx_format == "mxfp8" else w.idx_dim * es
+    idx = sum(lens_host) * w.n_idx_k_heads * row
     kv = 0
     for L in lens_host:  # the selected blocks' K and V (the visible part of each)
         nb = -(-L // w.block_size)
@@ -371,7 +374,13 @@ def time_decode(w, rank, world, local, stream, flush, steps, warmup, clk=None, s
     dev = torch.device("cuda", local)
     inp = make_inputs(w, device=dev, seed=rank_seed(w, rank))
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
-    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
+    k_scale = None
+    if w.idx_format == "mxfp8":  # the index-key cache as MXFP8, quantised once before timing
+        k_idx, k_scale = api.quantize_index_k(k_idx)
+        inp["k_idx"], inp["k_idx_scale"] = k_idx, k_scale
+        torch.cuda.synchronize()
+    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens,
+                        k_idx_scale=k_scale)
     ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, dev)
     o = torch.empty_like(q)
     ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device=dev)
@@ -424,6 +433,7 @@ def decode_summary(w, r, peaks, peak_kind, cpu=None) -> dict:
          "context": (min(r["lens_host"]), max(r["lens_host"])) if min(r["lens_host"]) != max(r["lens_host"])
          else r["lens_host"][0],
          "n_idx_k_heads": w.n_idx_k_heads, "block_size": w.block_size, "top_k": w.top_k, "dtype": w.dtype,
+         "index_keys": w.idx_format,
          "algorithmic_bytes": idx_b + kv_b, "step_roofline": hbm_frac(idx_b + kv_b, r["step_us"], peaks),
          "peak_kind": peak_kind}
     if "scan_us" in r:
@@ -603,6 +613,8 @@ def run_ours(args, world, rank, local):
                                                                 stream, flush, peaks, peak_kind)
     large_k = None if args.no_large_k else run_extra_decode("decode_ctx1m_large_k", args, world, rank, local, stream,
                                                             flush, peaks, peak_kind)
+    mxfp8_idx = None if args.no_mxfp8 else run_extra_decode("decode_ctx1m_mxfp8_idx", args, world, rank, local,
+                                                            stream, flush, peaks, peak_kind)
     prefill = None
     if not args.no_prefill:
         del flush_buf
@@ -651,6 +663,7 @@ def run_ours(args, world, rank, local):
         "configs": configs,
         "shared_index_head": shared,
         "large_k": large_k,
+        "mxfp8_index_keys": mxfp8_idx,
         "prefill": prefill,
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -660,8 +673,9 @@ def run_ours(args, world, rank, local):
 
 def run_extra_decode(name, args, world, rank, local, stream, flush, peaks, peak_kind):
     """The 1M decode step with one index-K head shared by the 8 groups (the index stream is 1/8 as
-    long), or the large-k regime (64-token blocks, k 1024 of 16,384; the middle stage is then the
-    radix select, the last the attention over 268 MB of K/V).  Same timing as the main step."""
+    long), the large-k regime (64-token blocks, k 1024 of 16,384; the middle stage is then the
+    radix select, the last the attention over 268 MB of K/V), or MXFP8 index keys (66 bytes per key
+    row instead of 128).  Same timing as the main step."""
     w = WORKLOADS[name]
     r = time_decode(w, rank, world, local, stream, flush, max(3, min(args.steps, 500)), args.warmup)
     d = decode_summary(w, r, peaks, peak_kind)
@@ -767,6 +781,7 @@ def main():
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' sub-lines")
     ap.add_argument("--no-shared-index", action="store_true", help="skip the shared index-K head decode step")
     ap.add_argument("--no-large-k", action="store_true", help="skip the large-k (k 1024 of 16,384 blocks) decode step")
+    ap.add_argument("--no-mxfp8", action="store_true", help="skip the decode step with MXFP8 index keys")
     args = ap.parse_args()
     world, rank, local = dist_setup()
     try:

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA, MSA_ERR_TIMEOUT = range(6)
 MSA_F32, MSA_BF16 = 0, 1
 MSA_SCORES_TOKEN, MSA_SCORES_BLOCKMAX, MSA_DENSE, MSA_FORCE_SINK_LOCAL = 1, 2, 8, 16
+MSA_IDX_PLAIN, MSA_IDX_MXFP8 = 0, 1
 (MSA_ENTRY_INDEX_SCORE, MSA_ENTRY_MAXPOOL_TOPK, MSA_ENTRY_ATTN_DECODE, MSA_ENTRY_ATTN_PREFILL,
  MSA_ENTRY_DECODE_FUSED, MSA_ENTRY_PREFILL_INDEX_TOPK) = range(6)
 
@@ -26,7 +27,7 @@ EXPORTED = ["msa_index_score", "msa_block_maxpool_topk", "msa_sparse_attn_decode
             "msa_decode_fused", "msa_prefill_index_topk", "msa_workspace_size", "msa_last_error_string",
             "msa_status_string", "msa_get_device_status", "msa_clear_device_status", "msa_set_stage_events",
             "msa_decode_fused_noalloc", "msa_noalloc_get_status", "msa_noalloc_clear_status", "msa_set_wait_limit",
-            "msa_diag_wait_timeout", "msa_decode_append"]
+            "msa_diag_wait_timeout", "msa_decode_append", "msa_quantize_index_k"]
 
 
 class MsaError(RuntimeError):
@@ -42,6 +43,7 @@ class Params(ctypes.Structure):
         ("block_size", ctypes.c_int), ("top_k", ctypes.c_int), ("q_len", ctypes.c_int), ("q_start", ctypes.c_int),
         ("max_seq_len", ctypes.c_int), ("seq_lens", ctypes.c_void_p), ("softmax_scale", ctypes.c_float),
         ("dtype", ctypes.c_int), ("flags", ctypes.c_int), ("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int),
+        ("idx_format", ctypes.c_int), ("k_idx_scale", ctypes.c_void_p),
     ]
 
 
@@ -73,6 +75,7 @@ def lib() -> ctypes.CDLL:
             "msa_set_wait_limit": [vp, ctypes.c_uint64, st],
             "msa_diag_wait_timeout": [vp, sz, st],
             "msa_decode_append": [P, vp, vp, vp, vp, vp, vp, st],
+            "msa_quantize_index_k": [P, vp, ctypes.c_longlong, vp, vp, st],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -196,3 +199,8 @@ def msa_diag_wait_timeout(ws, stream=None):
 def msa_decode_append(params, k_new, v_new, k_idx_new, k_cache, v_cache, k_idx, stream=None):
     _check(lib().msa_decode_append(ctypes.byref(params), _ptr(k_new), _ptr(v_new), _ptr(k_idx_new), _ptr(k_cache),
                                    _ptr(v_cache), _ptr(k_idx), _stream(stream)))
+
+
+def msa_quantize_index_k(params, src, rows, codes, scales, stream=None):
+    _check(lib().msa_quantize_index_k(ctypes.byref(params), _ptr(src), int(rows), _ptr(codes), _ptr(scales),
+                                      _stream(stream)))

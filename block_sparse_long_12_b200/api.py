@@ -26,23 +26,39 @@ def dtype_code(t: torch.Tensor) -> int:
 
 def make_params(*, batch, n_q_heads, n_kv_heads, n_idx_k_heads, head_dim, idx_dim, block_size, top_k,
                 max_seq_len, dtype, q_len=1, q_start=0, seq_lens=None, softmax_scale=None, flags=0,
-                block_table=None, n_pages=0) -> Params:
-    """block_table (int32 [B, ceil(max_seq_len / block_size)], device) selects paged caches of n_pages pages."""
+                block_table=None, n_pages=0, k_idx_scale=None) -> Params:
+    """block_table (int32 [B, ceil(max_seq_len / block_size)], device) selects paged caches of n_pages pages;
+    k_idx_scale (uint8 E8M0 scales, one per 32 index dims) selects MXFP8 index keys."""
     return Params(batch, n_q_heads, n_kv_heads, n_idx_k_heads, head_dim, idx_dim, block_size, top_k, q_len,
                   q_start, max_seq_len, seq_lens.data_ptr() if seq_lens is not None else None,
                   float(softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(head_dim)), dtype, flags,
-                  block_table.data_ptr() if block_table is not None else None, int(n_pages))
+                  block_table.data_ptr() if block_table is not None else None, int(n_pages),
+                  _lib.MSA_IDX_MXFP8 if k_idx_scale is not None else _lib.MSA_IDX_PLAIN,
+                  k_idx_scale.data_ptr() if k_idx_scale is not None else None)
+
+
+def quantize_index_k(k_idx: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """MXFP8 copy of a bf16 index-key tensor [..., di]: (codes uint8 [..., di], scales uint8 [..., di / 32])."""
+    di = k_idx.shape[-1]
+    rows = k_idx.numel() // di
+    codes = torch.empty(k_idx.shape, dtype=torch.uint8, device=k_idx.device)
+    scales = torch.empty(k_idx.shape[:-1] + (di // 32,), dtype=torch.uint8, device=k_idx.device)
+    p = make_params(batch=1, n_q_heads=1, n_kv_heads=1, n_idx_k_heads=1, head_dim=64, idx_dim=di, block_size=16,
+                    top_k=1, max_seq_len=16, dtype=_lib.MSA_BF16)
+    _lib.msa_quantize_index_k(p, k_idx.contiguous(), rows, codes, scales, stream)
+    return codes, scales
 
 
 def params_from(q, q_idx, k, k_idx, *, block_size, top_k, seq_lens=None, q_start=0, softmax_scale=None,
-                flags=0) -> Params:
-    """Params for q [B, Tq, Hq, D], q_idx [B, Tq, G, di], k [B, G, L, D], k_idx [B, Hik, L, di]."""
+                flags=0, k_idx_scale=None) -> Params:
+    """Params for q [B, Tq, Hq, D], q_idx [B, Tq, G, di], k [B, G, L, D], k_idx [B, Hik, L, di] (bf16, or
+    MXFP8 codes with their scales k_idx_scale [B, Hik, L, di / 32])."""
     B, Tq, Hq, D = q.shape
     _, G, L, _ = k.shape
     return make_params(batch=B, n_q_heads=Hq, n_kv_heads=G, n_idx_k_heads=k_idx.shape[1], head_dim=D,
                        idx_dim=q_idx.shape[-1], block_size=block_size, top_k=top_k, max_seq_len=L,
                        dtype=dtype_code(q), q_len=Tq, q_start=q_start, seq_lens=seq_lens,
-                       softmax_scale=softmax_scale, flags=flags)
+                       softmax_scale=softmax_scale, flags=flags, k_idx_scale=k_idx_scale)
 
 
 def workspace(params, entry: int, device) -> torch.Tensor:
@@ -54,11 +70,13 @@ def workspace(params, entry: int, device) -> torch.Tensor:
 
 
 def decode(q, q_idx, k, v, k_idx, seq_lens, *, block_size, top_k, softmax_scale=None, ws=None, out=None,
-           stream=None, force_sink_local=False):
+           stream=None, force_sink_local=False, k_idx_scale=None):
     """One fused MSA decode step.  Returns (o [B,1,Hq,D], ids [B,1,G,k], lse [B,1,Hq]).
-    force_sink_local: the selection always keeps block 0 and the query's own block."""
+    force_sink_local: the selection always keeps block 0 and the query's own block.
+    k_idx_scale: k_idx holds MXFP8 codes with these scales (quantize_index_k)."""
     p = params_from(q, q_idx, k, k_idx, block_size=block_size, top_k=top_k, seq_lens=seq_lens,
-                    softmax_scale=softmax_scale, flags=MSA_FORCE_SINK_LOCAL if force_sink_local else 0)
+                    softmax_scale=softmax_scale, flags=MSA_FORCE_SINK_LOCAL if force_sink_local else 0,
+                    k_idx_scale=k_idx_scale)
     B, _, Hq, D = q.shape
     G = k.shape[1]
     if ws is None:

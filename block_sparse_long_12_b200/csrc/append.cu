@@ -55,7 +55,8 @@ cudaError_t launch_append(const msa_params_t &p, const CacheMap &cache, const vo
     a.seq_lens = p.seq_lens;
     a.B = p.batch; a.Hkv = p.n_kv_heads; a.Hik = p.n_idx_k_heads; a.L_max = p.max_seq_len;
     a.kv_vecs = p.head_dim * es / 16;
-    a.ki_vecs = p.idx_dim * es / 16;
+    // MXFP8 index keys are quantised into their cache by launch_mxfp8_append instead
+    a.ki_vecs = p.idx_format == MSA_IDX_MXFP8 ? 0 : p.idx_dim * es / 16;
     a.cache = cache;
     const long long n = (long long)p.batch * (2 * a.Hkv * a.kv_vecs + a.Hik * a.ki_vecs);
     const int grid = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);

@@ -24,6 +24,8 @@
 // warp-distributed sorted list keeps the warp's best blocks.  At the end of
 // each piece the warp lists are merged into one sorted candidate list per
 // group; decode_select_kernel merges the pieces of a segment.
+#include <type_traits>
+
 #include "tcgen05.cuh"
 
 namespace msa {
@@ -101,6 +103,9 @@ struct ChunkCursor {
     }
 };
 
+// MXFP8 keys: the E8M0 scales of a chunk's rows are copied beside its codes, at most 256 bytes
+constexpr int kScaleStage = 256;
+template <typename T> constexpr bool is_fp8() { return sizeof(T) == 1; }
 // several groups on one bf16 stream of 128- or 256-byte rows are scored on tensor cores
 template <typename T, int GPS, int ROWB> constexpr bool scan_mma() { return GPS > 1 && sizeof(T) == 2 && ROWB >= 128; }
 // Warps per CTA (W): one index-K head per stream (GPS 1) keeps the index query in registers and
@@ -122,11 +127,14 @@ __global__ void __launch_bounds__(W * 32, 1)
     // queries, padded to 16 rows, times the chunk's keys) on mma.sync tensor-core fragments
     constexpr bool MMA = scan_mma<T, GPS, ROWB>();
     constexpr int KS = DI / 16;           // k-steps of 16 index dims
+    constexpr bool FP8 = is_fp8<T>();     // MXFP8 keys: E4M3 codes, one E8M0 scale per 32 dims
+    constexpr int SPR = FP8 ? DI / 32 : 0;  // scale bytes per row
     const int CT = a.chunk_tokens;        // tokens per chunk (<= block size, 8 KB at most)
 
     extern __shared__ unsigned char smem_raw[];
     unsigned char *ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);  // [W][S][8 KB]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + (size_t)W * S * kScanChunkBytes);
+    unsigned char *sring = ring + (size_t)W * S * kScanChunkBytes;                    // FP8: [W][S][256]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sring + (FP8 ? (size_t)W * S * kScaleStage : 0));
     float *lists_s = reinterpret_cast<float *>(bars + W * S);                 // [W][GPS][32]
     int *lists_i = reinterpret_cast<int *>(lists_s + W * GPS * 32);
     float *q_s = reinterpret_cast<float *>(lists_i + W * GPS * 32);           // [GPS][DI] (QREG: unused)
@@ -198,8 +206,11 @@ __global__ void __launch_bounds__(W * 32, 1)
     // the next grid may start its prologue while this grid runs
     pdl_allow_next_grid();
 
-    const T *qg = reinterpret_cast<const T *>(a.q_idx);
+    // the index query: the keys' type, or bf16 beside MXFP8 keys
+    using QT = typename std::conditional<is_fp8<T>(), __nv_bfloat16, T>::type;
+    const QT *qg = reinterpret_cast<const QT *>(a.q_idx);
     unsigned char *my_ring = ring + (size_t)w * S * kScanChunkBytes;
+    unsigned char *my_sring = sring + (size_t)w * S * kScaleStage;
     uint64_t *my_bars = bars + w * S;
     const bool want_cand = a.cand_s != nullptr;
     const uint32_t chunk_bytes = (uint32_t)CT * ROWB;
@@ -281,7 +292,17 @@ __global__ void __launch_bounds__(W * 32, 1)
             if (lane == 0) {
                 const int slot = issued % S;
                 unsigned char *dst = my_ring + (size_t)slot * kScanChunkBytes;
-                mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
+                if constexpr (FP8) {
+                    // the chunk's scales, clipped to the scale tensor (its row count is a multiple of 16,
+                    // chunks start at multiples of 16 rows: whole 16-byte units)
+                    const long long left = a.k_scale_rows - row;
+                    const uint32_t sb = (uint32_t)((left < CT ? left : CT) * SPR);
+                    mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes + sb);
+                    bulk_g2s(my_sring + (size_t)slot * kScaleStage, a.k_scale + (size_t)row * SPR, sb, &my_bars[slot],
+                             l2_evict_first_policy());
+                } else {
+                    mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
+                }
                 tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
                 if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
             }
@@ -312,8 +333,8 @@ __global__ void __launch_bounds__(W * 32, 1)
     // one chunk of nt index-key rows of segment (b, hik) starting at token tok_base: fp32 dot
     // products with the index query (qv in registers, or qsrc in shared memory, or the qa
     // fragments on tensor cores), running max m
-    auto scan_chunk = [&](const unsigned char *base, int nt, int b, int hik, int tok_base, const float *qv_,
-                          const float *qsrc, float *m) {
+    auto scan_chunk = [&](const unsigned char *base, const unsigned char *sbase, int nt, int b, int hik, int tok_base,
+                          const float *qv_, const float *qsrc, float *m) {
         if constexpr (MMA) {
             // S = Q_idx K^T, 8 keys per tile; lane (grp, tig) holds S[grp][2 tig, 2 tig + 1] of each
             // tile.  The k-steps run over all tiles in turn, so consecutive MMAs are independent.
@@ -359,17 +380,48 @@ __global__ void __launch_bounds__(W * 32, 1)
                 float dot[GPS];
 #pragma unroll
                 for (int gl = 0; gl < GPS; ++gl) dot[gl] = 0.f;
-                if (live) {
+                // position of 16-byte vector c16 of row `tok` in the swizzled tile
+                auto vec_at = [&](int c16) -> uint4 {
+                    int o;
+                    if constexpr (ROWB == 64) {
+                        o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
+                    } else {
+                        o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
+                    }
+                    return *reinterpret_cast<const uint4 *>(base + o);
+                };
+                if (live && FP8) {
+                    // per 32 dims (two vectors): the code products, then their E8M0 scale
+#pragma unroll
+                    for (int j = 0; j < (FP8 ? SPR : 1); ++j) {
+                        const float sc = e8m0_to_float(sbase[tok * SPR + j]);
+                        float part[GPS];
+#pragma unroll
+                        for (int gl = 0; gl < GPS; ++gl) part[gl] = 0.f;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int c16 = 2 * j + h;
+                            float f[EPV];
+                            Vec16<T>::unpack(vec_at(c16), f);
+                            if constexpr (QREG) {
+#pragma unroll
+                                for (int e = 0; e < EPV; ++e) part[0] = fmaf(qv_[c16 * EPV + e], f[e], part[0]);
+                            } else {
+#pragma unroll
+                                for (int gl = 0; gl < GPS; ++gl) {
+                                    const float *qq = qsrc + gl * DI + c16 * EPV;
+#pragma unroll
+                                    for (int e = 0; e < EPV; ++e) part[gl] = fmaf(qq[e], f[e], part[gl]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int gl = 0; gl < GPS; ++gl) dot[gl] = fmaf(sc, part[gl], dot[gl]);
+                    }
+                } else if (live) {
 #pragma unroll
                     for (int c16 = 0; c16 < NCH; ++c16) {
-                        // position of 16-byte vector c16 of row `tok` in the swizzled tile
-                        int o;
-                        if constexpr (ROWB == 64) {
-                            o = tok * 64 + ((c16 ^ ((tok >> 1) & 3)) << 4);
-                        } else {
-                            o = (c16 >> 3) * (CT * 128) + tok * 128 + (((c16 & 7) ^ (tok & 7)) << 4);
-                        }
-                        const uint4 u = *reinterpret_cast<const uint4 *>(base + o);
+                        const uint4 u = vec_at(c16);
                         float f[EPV];
                         Vec16<T>::unpack(u, f);
                         if constexpr (QREG) {
@@ -445,7 +497,7 @@ __global__ void __launch_bounds__(W * 32, 1)
         if (p.b != q_b || p.hik != q_h) {
             q_b = p.b; q_h = p.hik;
             if constexpr (QREG) {
-                const T *src = qg + ((size_t)p.b * a.G + p.hik) * DI;
+                const QT *src = qg + ((size_t)p.b * a.G + p.hik) * DI;
 #pragma unroll
                 for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
             } else if constexpr (MMA) {
@@ -480,7 +532,8 @@ __global__ void __launch_bounds__(W * 32, 1)
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;
-                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, p.b, p.hik, n * Bk + c * CT, qv, q_s, m);
+                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, my_sring + (size_t)slot * kScaleStage, nt, p.b, p.hik,
+                           n * Bk + c * CT, qv, q_s, m);
                 __syncwarp();
                 ++consumed;
                 refill();
@@ -540,7 +593,7 @@ __global__ void __launch_bounds__(W * 32, 1)
                 qb = r.x;
                 qh = r.y;
                 if constexpr (QREG) {
-                    const T *src = qg + ((size_t)qb * a.G + qh) * DI;
+                    const QT *src = qg + ((size_t)qb * a.G + qh) * DI;
 #pragma unroll
                     for (int e = 0; e < DI; ++e) qv[e] = load_elem(src + e);
                 } else if constexpr (MMA) {
@@ -567,7 +620,8 @@ __global__ void __launch_bounds__(W * 32, 1)
                 }
                 int nt = bt - c * CT;
                 nt = nt < CT ? nt : CT;
-                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, nt, r.x, r.y, r.z * Bk + c * CT, qv, my_q, m);
+                scan_chunk(my_ring + (size_t)slot * kScanChunkBytes, my_sring + (size_t)slot * kScaleStage, nt, r.x, r.y,
+                           r.z * Bk + c * CT, qv, my_q, m);
                 __syncwarp();
                 ++consumed;
                 refill();
@@ -605,7 +659,8 @@ size_t scan_smem_bytes(int B) {
     constexpr bool MMA = scan_mma<T, GPS, ROWB>();
     constexpr int DI = ROWB / (int)sizeof(T);
     constexpr bool QREG = GPS == 1 && DI <= 64;
-    return 1024 + (size_t)W * S * kScanChunkBytes + W * S * 8 + (size_t)W * GPS * 32 * 8 + (size_t)GPS * DI * 4 +
+    return 1024 + (size_t)W * S * kScanChunkBytes + (is_fp8<T>() ? (size_t)W * S * kScaleStage : 0) + W * S * 8 +
+           (size_t)W * GPS * 32 * 8 + (size_t)GPS * DI * 4 +
            (size_t)W * 4 * 16 + (QREG || MMA ? 0 : (size_t)W * GPS * DI * 4) + (size_t)(B + 1) * 16 + (size_t)B * 12 +
            kTailPools * 4 + 4 + 64;
 }
@@ -635,11 +690,14 @@ cudaError_t launch_scan_s(const ScanArgs &a, const CUtensorMap &km, cudaStream_t
 
 template <typename T, int GPS, int ROWB>
 cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t s, bool pdl) {
-    if constexpr (GPS == 1) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
-    if constexpr (scan_mma<T, GPS, ROWB>()) {
-        if (scan_smem_bytes<T, GPS, ROWB, 2, 12>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
+    if constexpr (GPS == 1) {
+        return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
+    } else {
+        if constexpr (scan_mma<T, GPS, ROWB>()) {
+            if (scan_smem_bytes<T, GPS, ROWB, 2, 12>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
+        }
+        return launch_scan_s<T, GPS, ROWB, 2, 8>(a, km, s, pdl);
     }
-    return launch_scan_s<T, GPS, ROWB, 2, 8>(a, km, s, pdl);
 }
 
 template <typename T, int ROWB>
@@ -666,7 +724,9 @@ cudaError_t launch_scan_r(const ScanArgs &a, const CUtensorMap &km, int rowb, in
 }  // namespace
 
 cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cudaStream_t s, bool pdl) {
-    const int es = dtype == MSA_F32 ? 4 : 2;
+    // MXFP8 keys (a.k_scale set): one byte per index dim
+    const bool fp8 = a.k_scale != nullptr;
+    const int es = fp8 ? 1 : dtype == MSA_F32 ? 4 : 2;
     int ct = kScanChunkBytes / row_bytes;
     if (ct > a.Bk) ct = a.Bk;
     a.chunk_tokens = ct;
@@ -674,10 +734,12 @@ cudaError_t launch_decode_scan(ScanArgs a, int dtype, int row_bytes, int gps, cu
     // (64 for 64-byte rows), swizzled so that one lane per row reads without bank conflicts
     const int box_x = (row_bytes >= 128 ? 128 : 64) / es;
     CUtensorMap km;
-    if (!encode_2d(&km, dtype == MSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   const_cast<void *>(a.k_idx), row_bytes / es, a.cache.rows(a.B, a.Hik, a.L_max), row_bytes,
+    const CUtensorMapDataType ty = fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : dtype == MSA_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_2d(&km, ty, const_cast<void *>(a.k_idx), row_bytes / es, a.cache.rows(a.B, a.Hik, a.L_max), row_bytes,
                    box_x, ct, row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    if (fp8) return launch_scan_r<e4m3_t>(a, km, row_bytes, gps, s, pdl);
     return dtype == MSA_F32 ? launch_scan_r<float>(a, km, row_bytes, gps, s, pdl)
                             : launch_scan_r<__nv_bfloat16>(a, km, row_bytes, gps, s, pdl);
 }

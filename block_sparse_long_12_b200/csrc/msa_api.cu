@@ -65,6 +65,11 @@ msa_status_t check_device(int *n_sm) {
 
 enum Mode { DECODE_ONLY, PREFILL_ONLY, ANY_ROWS };
 
+// bytes of one index-key row: idx_dim elements of params.dtype, or one E4M3 byte each (MXFP8)
+int idx_row_bytes(const msa_params_t &p) {
+    return p.idx_dim * (p.idx_format == MSA_IDX_MXFP8 ? 1 : elem_size(p.dtype));
+}
+
 msa_status_t check_params(const msa_params_t *p, Mode mode) {
     if (p == nullptr) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
     if (p->dtype != MSA_F32 && p->dtype != MSA_BF16) return fail(MSA_ERR_INVALID_ARG, "dtype %d unknown", p->dtype);
@@ -82,9 +87,20 @@ msa_status_t check_params(const msa_params_t *p, Mode mode) {
     if (gps > kMaxGroupsPerSeg || !pow2(gps))
         return fail(MSA_ERR_UNSUPPORTED, "%d groups sharing one index-K head (supported: 1, 2, 4, 8)", gps);
     if (p->head_dim != 64 && p->head_dim != 128) return fail(MSA_ERR_UNSUPPORTED, "head_dim %d (64 or 128)", p->head_dim);
-    const int row = p->idx_dim * elem_size(p->dtype);
+    if (p->idx_format != MSA_IDX_PLAIN && p->idx_format != MSA_IDX_MXFP8)
+        return fail(MSA_ERR_INVALID_ARG, "idx_format %d unknown", p->idx_format);
+    const int row = idx_row_bytes(*p);
     if (p->idx_dim < 1 || (row != 64 && row != 128 && row != 256))
         return fail(MSA_ERR_UNSUPPORTED, "idx_dim %d: an index-key row must be 64, 128 or 256 bytes", p->idx_dim);
+    if (p->idx_format == MSA_IDX_MXFP8) {
+        if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "MXFP8 index keys go with bf16 tensors");
+        if (mode != DECODE_ONLY && !(mode == ANY_ROWS && p->q_len == 1))
+            return fail(MSA_ERR_UNSUPPORTED, "MXFP8 index keys are read by the decode entries only");
+        if (p->k_idx_scale == nullptr) return fail(MSA_ERR_INVALID_ARG, "k_idx_scale is NULL with MXFP8 index keys");
+        if (!aligned16(p->k_idx_scale)) return fail(MSA_ERR_INVALID_ARG, "k_idx_scale is not 16-byte aligned");
+        if (p->block_table == nullptr && p->max_seq_len % 16 != 0)
+            return fail(MSA_ERR_UNSUPPORTED, "MXFP8 index keys need max_seq_len a multiple of 16");
+    }
     if (!pow2(p->block_size) || p->block_size < 16 || p->block_size > 256)
         return fail(MSA_ERR_UNSUPPORTED, "block_size %d (a power of two in [16, 256])", p->block_size);
     if (p->top_k < 1) return fail(MSA_ERR_INVALID_ARG, "top_k %d < 1", p->top_k);
@@ -115,6 +131,13 @@ msa_status_t check_params(const msa_params_t *p, Mode mode) {
             return fail(MSA_ERR_UNSUPPORTED, "n_pages * heads * block_size must stay below 2^31 cache rows");
     }
     return MSA_OK;
+}
+
+// MXFP8 index keys: the scan reads their scales beside the codes.
+void set_scales(ScanArgs &a, const msa_params_t &p) {
+    if (p.idx_format != MSA_IDX_MXFP8) return;
+    a.k_scale = p.k_idx_scale;
+    a.k_scale_rows = (long long)a.cache.rows(p.batch, p.n_idx_k_heads, p.max_seq_len);
 }
 
 // Layout of the caches a call reads: contiguous, or pages named by the block table.
@@ -408,7 +431,8 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
     a.sched = reinterpret_cast<unsigned *>(ws) + kSchedWord;
     a.status = reinterpret_cast<int *>(ws);
     a.cache = cache_of(*p);
-    e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
+    set_scales(a, *p);
+    e = launch_decode_scan(a, p->dtype, idx_row_bytes(*p), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     return MSA_OK;
 }
@@ -558,7 +582,8 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     }
     cudaError_t e = stage_mark(0, s);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    e = launch_decode_scan(a, p->dtype, p->idx_dim * elem_size(p->dtype), p->n_kv_heads / p->n_idx_k_heads, s, false);
+    set_scales(a, *p);
+    e = launch_decode_scan(a, p->dtype, idx_row_bytes(*p), p->n_kv_heads / p->n_idx_k_heads, s, false);
     if (e != cudaSuccess) return cuda_fail(e, "index scan launch");
     if (large) {
         if ((e = stage_mark(1, s)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
@@ -590,7 +615,26 @@ msa_status_t msa_decode_append(const msa_params_t *p, const void *k_new, const v
     int n_sm = 0;
     MSA_TRY(check_device(&n_sm));
     cudaError_t e = launch_append(*p, cache_of(*p), k_new, v_new, k_idx_new, k_cache, v_cache, k_idx, (cudaStream_t)stream);
+    if (e == cudaSuccess && p->idx_format == MSA_IDX_MXFP8)
+        e = launch_mxfp8_append(*p, cache_of(*p), k_idx_new, static_cast<uint8_t *>(k_idx),
+                                const_cast<uint8_t *>(p->k_idx_scale), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    return MSA_OK;
+}
+
+msa_status_t msa_quantize_index_k(const msa_params_t *p, const void *src, long long rows, uint8_t *codes,
+                                  uint8_t *scales, msa_stream_t stream) {
+    if (p == nullptr) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->idx_dim != 64 && p->idx_dim != 128 && p->idx_dim != 256)
+        return fail(MSA_ERR_UNSUPPORTED, "idx_dim %d: MXFP8 index keys take 64, 128 or 256 dims", p->idx_dim);
+    if (rows < 0) return fail(MSA_ERR_INVALID_ARG, "rows %lld < 0", rows);
+    MSA_TRY(check_ptr(src, "src"));
+    MSA_TRY(check_ptr(codes, "codes"));
+    MSA_TRY(check_ptr(scales, "scales"));
+    int n_sm = 0;
+    MSA_TRY(check_device(&n_sm));
+    cudaError_t e = launch_mxfp8_quantize(src, rows, p->idx_dim, codes, scales, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "quantise launch");
     return MSA_OK;
 }
 

@@ -8,6 +8,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -37,6 +39,31 @@ template <> struct Vec16<__nv_bfloat16> {
         f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
     }
 };
+
+// FP8 E4M3 codes of MXFP8 index keys: unpacked without their block scale (the scan applies it)
+struct e4m3_t {
+    uint8_t v;
+};
+template <> struct Vec16<e4m3_t> {
+    static constexpr int N = 16;
+    __device__ static inline void unpack(const uint4 &u, float (&f)[16]) {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                // two codes, the lower byte first, to two halves, then to fp32 (both exact)
+                const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> (16 * h)), __NV_E4M3);
+                const float2 p = __half22float2(*reinterpret_cast<const __half2 *>(&r));
+                f[4 * i + 2 * h] = p.x;
+                f[4 * i + 2 * h + 1] = p.y;
+            }
+    }
+};
+// An E8M0 scale byte as fp32: 2^(e - 127); 0 gives the subnormal 2^-127, 255 NaN.
+__device__ inline float e8m0_to_float(uint32_t e) {
+    return e == 0 ? __uint_as_float(0x00400000u) : (e == 255 ? __uint_as_float(0x7fc00000u) : __uint_as_float(e << 23));
+}
 
 __device__ inline float load_elem(const float *p) { return *p; }
 __device__ inline float load_elem(const __nv_bfloat16 *p) { return __bfloat162float(*p); }

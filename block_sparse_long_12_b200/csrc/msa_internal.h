@@ -188,6 +188,10 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, const void *q, const void *k_
 cudaError_t launch_prefill_index(const PrefillIdxArgs &a, const void *q_idx, const void *k_idx, int n_sm,
                                  cudaStream_t s, const char **why);
 cudaError_t launch_set_wait_limit(int *ws, unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_mxfp8_quantize(const void *src, long long rows, int di, uint8_t *codes, uint8_t *scales,
+                                  cudaStream_t s);
+cudaError_t launch_mxfp8_append(const msa_params_t &p, const CacheMap &cache, const void *ki_new, uint8_t *codes,
+                                uint8_t *scales, cudaStream_t s);
 cudaError_t launch_append(const msa_params_t &p, const CacheMap &cache, const void *k_new, const void *v_new,
                           const void *ki_new, void *k, void *v, void *ki, cudaStream_t s);
 cudaError_t launch_wait_never(int *ws, cudaStream_t s);

@@ -67,6 +67,10 @@ struct ScanArgs {
     int *counters;         // [B, G] attention arrival counters, zeroed by CTA 0 (nullable)
     int *status;
     CacheMap cache;        // index-key cache layout (contiguous or paged)
+    // MXFP8 index keys: E8M0 scales [rows, di / 32] beside the E4M3 codes (nullptr: plain keys);
+    // rows = the code tensor's rows, a multiple of 16
+    const uint8_t *k_scale;
+    long long k_scale_rows;
 };
 
 }  // namespace msa

@@ -49,6 +49,7 @@ class Workload:
     min_seq_len: int = 0    # >0: decode lengths drawn uniformly in [min, max]
     chunk: int = 0          # prefill query chunk length (0 = whole sequence)
     seed: int = 0
+    idx_format: str = "plain"  # "mxfp8": the index keys are stored as MXFP8 (quantised from these draws)
 
     @property
     def softmax_scale(self) -> float:
@@ -65,7 +66,7 @@ class Workload:
 # The workloads: tiny fp32 decode, 16K causal prefill, ragged batched 128K
 # decode, 1M decode (batch 1 and 4), 1M chunked causal prefill, 1M decode
 # with one index-K head shared by every group, and the large-k regime in
-# decode (1M) and prefill (128K).
+# decode (1M) and prefill (128K), and the 1M decode with MXFP8 index keys.
 WORKLOADS = {
     "decode_fp32_ctx4k": Workload("decode_fp32_ctx4k", "decode", 1, 4096, 4, 1, 1, 64, 32, 64, 8,
                                   "f32", seed=1001),
@@ -90,6 +91,9 @@ WORKLOADS = {
     # 8192-token chunks
     "prefill_ctx128k_large_k": Workload("prefill_ctx128k_large_k", "prefill", 1, 131072, 64, 8, 8, 128, 64, 64, 128,
                                         "bf16", hot_blocks=32, chunk=8192, seed=1008),
+    # the 1M decode with the index-key cache stored as MXFP8 (66 bytes per 64-dim key instead of 128)
+    "decode_ctx1m_mxfp8_idx": Workload("decode_ctx1m_mxfp8_idx", "decode", 1, 1048576, 64, 8, 8, 128, 64, 128, 16,
+                                       "bf16", hot_blocks=32, seed=1004, idx_format="mxfp8"),
 }
 
 

@@ -84,6 +84,12 @@ typedef enum {
 
 typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype_t;
 
+/* params.idx_format: storage of the index-key cache k_idx */
+typedef enum {
+    MSA_IDX_PLAIN = 0,   /* params.dtype, like every other tensor                    */
+    MSA_IDX_MXFP8 = 1    /* MXFP8: E4M3 codes plus one E8M0 scale per 32 dims (below) */
+} msa_idx_format_t;
+
 /* params.flags */
 enum {
     MSA_SCORES_TOKEN = 1,    /* token scores s_j  [B, q_len, G, max_seq_len]  */
@@ -133,7 +139,23 @@ typedef struct {
     int flags;            /* MSA_SCORES_* / MSA_DENSE / MSA_FORCE_SINK_LOCAL   */
     const int32_t *block_table; /* NULL: contiguous caches; else paged, see below */
     int n_pages;          /* pages in each pool when block_table != NULL       */
+    int idx_format;       /* msa_idx_format_t (0: plain)                       */
+    const uint8_t *k_idx_scale; /* MSA_IDX_MXFP8: the index keys' scales, below */
 } msa_params_t;
+/*
+ * MXFP8 index keys (idx_format = MSA_IDX_MXFP8; decode entries and
+ * msa_index_score with q_len 1, dtype MSA_BF16, idx_dim 64, 128 or 256): k_idx
+ * holds one FP8 E4M3 code per index dimension (uint8, [.., idx_dim]) and
+ * k_idx_scale one E8M0 byte per 32 of them ([.., idx_dim / 32], same row
+ * order as k_idx, contiguous or paged alike); key value = 2^(scale - 127) *
+ * E4M3(code).  The index query stays bf16 and the scores accumulate in fp32.
+ * The pages name MXFP8 only as the format of the official quantised checkpoints
+ * (docs.clore.ai "MiniMax M3", deployment table and checkpoint list); reading
+ * it as the microscaling format, it is offered here as the storage of the
+ * index-key cache, the stream the decode scan reads: 66 bytes per 64-dim row
+ * instead of 128.  msa_quantize_index_k writes it; msa_decode_append quantises
+ * the new token's key when idx_format says so.
+ */
 /*
  * Paged caches (block_table != NULL): the K, V and index-K caches are pools of
  * n_pages pages of block_size tokens each, page-major and head-major inside a
@@ -253,13 +275,26 @@ MSA_API msa_status_t msa_noalloc_get_status(int *status, msa_stream_t stream);
 MSA_API msa_status_t msa_noalloc_clear_status(msa_stream_t stream);
 
 /*
+ * MXFP8 quantisation of `rows` index-key rows (src bf16 [rows, idx_dim], device):
+ * per 32 consecutive dims the shared exponent floor(log2 max|v|) - 8 clamped to
+ * [-127, 127] (an all-zero block takes -127), stored as E8M0 (exponent + 127) in
+ * scales [rows, idx_dim / 32]; each v / 2^shared rounded to the nearest E4M3
+ * value, ties to even, saturating at 448, stored in codes [rows, idx_dim].
+ * params gives idx_dim (64, 128 or 256); idx_format is not read.
+ */
+MSA_API msa_status_t msa_quantize_index_k(const msa_params_t *params, const void *src, long long rows,
+                                          uint8_t *codes, uint8_t *scales, msa_stream_t stream);
+
+/*
  * Serving step before msa_decode_fused (not part of the method): the new token
  * of every sequence -- k_new and v_new [B, n_kv_heads, head_dim], k_idx_new
  * [B, n_idx_k_heads, idx_dim], params.dtype, contiguous -- is written to its
  * position seq_lens[b] - 1 of the K, V and index-K caches (contiguous or paged,
- * as params say).  With the new token's q and q_idx it is all one decode step
- * takes from the host, so a caller can bring them in one copy; the caches are
- * otherwise untouched.
+ * as params say).  With idx_format MSA_IDX_MXFP8, k_idx_new is bf16 and is
+ * quantised as msa_quantize_index_k does into k_idx (codes) and
+ * params.k_idx_scale.  With the new token's q and q_idx it is all one decode
+ * step takes from the host, so a caller can bring them in one copy; the caches
+ * are otherwise untouched.
  */
 MSA_API msa_status_t msa_decode_append(const msa_params_t *params, const void *k_new, const void *v_new,
                                        const void *k_idx_new, void *k_cache, void *v_cache, void *k_idx,

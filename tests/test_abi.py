@@ -194,3 +194,27 @@ def test_prefill_attention_workspace_does_not_grow_with_k(lib):
         n = lib.msa_workspace_size(good_params(lib, q_len=16384, q_start=0, max_seq_len=16384, top_k=k),
                                    lib.MSA_ENTRY_ATTN_PREFILL)
         assert base * 0.99 <= n <= base * 1.01, (k, n, base)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers: host-only argument checks")
+@pytest.mark.parametrize("kw,fmt,scale,status", [
+    (dict(), 2, 0x10000, "INVALID_ARG"),                        # unknown index-key format
+    (dict(), 1, None, "INVALID_ARG"),                           # MXFP8 without scales
+    (dict(), 1, 0x10008, "INVALID_ARG"),                        # scales not 16-byte aligned
+    (dict(dtype=0), 1, 0x10000, "UNSUPPORTED"),                 # MXFP8 keys beside fp32 tensors
+    (dict(max_seq_len=4100), 1, 0x10000, "UNSUPPORTED"),        # scale rows not in whole 16-row units
+    (dict(idx_dim=32), 1, 0x10000, "UNSUPPORTED"),              # a 32-byte code row
+], ids=lambda v: str(v))
+def test_mxfp8_params_rejected_before_launch(lib, kw, fmt, scale, status):
+    p = good_params(lib, **kw)
+    p.idx_format, p.k_idx_scale = fmt, scale
+    fake = 0x10000
+    L = lib.lib()
+    rc = L.msa_decode_fused(ctypes.byref(p), fake, fake, fake, fake, fake, fake, None, None, fake,
+                            ctypes.c_size_t(1 << 30), None)
+    assert rc == getattr(lib, "MSA_ERR_" + status), (rc, L.msa_last_error_string())
+    # the prefill entries do not read MXFP8 keys
+    pp = good_params(lib, q_len=100)
+    pp.idx_format, pp.k_idx_scale = 1, 0x10000
+    assert L.msa_prefill_index_topk(ctypes.byref(pp), fake, fake, fake, None, fake, ctypes.c_size_t(1 << 30),
+                                    None) == lib.MSA_ERR_UNSUPPORTED
