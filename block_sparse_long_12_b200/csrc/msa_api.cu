@@ -9,6 +9,8 @@
 
 #include "msa_internal.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace msa {
 namespace {
 
@@ -303,6 +305,13 @@ size_t maxpool_topk_ws_bytes(const msa_params_t &p) {
 
 using namespace msa;
 
+// An NVTX range over one entry's launches, named after the entry (Nsight Systems / Compute show
+// it; without a tool attached the calls return at once).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+
 extern "C" {
 
 const char *msa_last_error_string(void) { return g_err.c_str(); }
@@ -401,6 +410,7 @@ msa_status_t msa_diag_wait_timeout(void *ws, size_t ws_bytes, msa_stream_t strea
 
 msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const void *k_idx, float *scores_out,
                              void *ws, size_t ws_bytes, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_index_score");
     MSA_TRY(check_params(p, ANY_ROWS));
     const int mode = p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX);
     if (mode != MSA_SCORES_TOKEN && mode != MSA_SCORES_BLOCKMAX)
@@ -439,6 +449,7 @@ msa_status_t msa_index_score(const msa_params_t *p, const void *q_idx, const voi
 
 msa_status_t msa_block_maxpool_topk(const msa_params_t *p, const float *scores_in, int32_t *ids_out,
                                     float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_block_maxpool_topk");
     MSA_TRY(check_params(p, ANY_ROWS));
     if (p->flags & (MSA_SCORES_TOKEN | MSA_DENSE))
         return fail(MSA_ERR_INVALID_ARG,
@@ -520,6 +531,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
 msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
                                     const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
                                     msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_sparse_attn_decode");
     MSA_TRY(check_params(p, DECODE_ONLY));
     if (p->flags & (MSA_SCORES_TOKEN | MSA_SCORES_BLOCKMAX | MSA_FORCE_SINK_LOCAL))
         return fail(MSA_ERR_INVALID_ARG, "score and selection flags do not apply to attention from given ids");
@@ -542,6 +554,7 @@ msa_status_t msa_sparse_attn_decode(const msa_params_t *p, const void *q, const 
 msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *q_idx, const void *k_cache,
                               const void *v_cache, const void *k_idx, void *o, int32_t *ids_out, float *lse, void *ws,
                               size_t ws_bytes, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_decode_fused");
     MSA_TRY(check_params(p, DECODE_ONLY));
     if (p->flags & ~MSA_FORCE_SINK_LOCAL)
         return fail(MSA_ERR_INVALID_ARG,
@@ -605,6 +618,7 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
 
 msa_status_t msa_decode_append(const msa_params_t *p, const void *k_new, const void *v_new, const void *k_idx_new,
                                void *k_cache, void *v_cache, void *k_idx, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_decode_append");
     MSA_TRY(check_params(p, DECODE_ONLY));
     MSA_TRY(check_ptr(k_new, "k_new"));
     MSA_TRY(check_ptr(v_new, "v_new"));
@@ -624,6 +638,7 @@ msa_status_t msa_decode_append(const msa_params_t *p, const void *k_new, const v
 
 msa_status_t msa_quantize_index_k(const msa_params_t *p, const void *src, long long rows, uint8_t *codes,
                                   uint8_t *scales, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_quantize_index_k");
     if (p == nullptr) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
     if (p->idx_dim != 64 && p->idx_dim != 128 && p->idx_dim != 256)
         return fail(MSA_ERR_UNSUPPORTED, "idx_dim %d: MXFP8 index keys take 64, 128 or 256 dims", p->idx_dim);
@@ -641,6 +656,7 @@ msa_status_t msa_quantize_index_k(const msa_params_t *p, const void *src, long l
 msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const void *k_cache, const void *v_cache,
                                      const int32_t *ids, void *o, float *lse, void *ws, size_t ws_bytes,
                                      msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_sparse_attn_prefill");
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags != 0) return fail(MSA_ERR_INVALID_ARG, "msa_sparse_attn_prefill takes no flags");
     if (p->dtype != MSA_BF16) return fail(MSA_ERR_UNSUPPORTED, "prefill entries take bf16 only");
@@ -686,6 +702,7 @@ msa_status_t msa_sparse_attn_prefill(const msa_params_t *p, const void *q, const
 
 msa_status_t msa_prefill_index_topk(const msa_params_t *p, const void *q_idx, const void *k_idx, int32_t *ids_out,
                                     float *top_scores_out, void *ws, size_t ws_bytes, msa_stream_t stream) {
+    NvtxRange nvtx_range("msa_prefill_index_topk");
     MSA_TRY(check_params(p, PREFILL_ONLY));
     if (p->flags & ~MSA_FORCE_SINK_LOCAL)
         return fail(MSA_ERR_INVALID_ARG, "msa_prefill_index_topk takes only MSA_FORCE_SINK_LOCAL");

@@ -6,6 +6,7 @@
   python profile_run.py prefill_chunks --context 1048576 --chunks 16,64,127 --steps 1
   python profile_run.py scan_shared --context 1048576 --steps 3
   python profile_run.py large_k --context 262144 --steps 3
+  python profile_run.py decode_mxfp8 --context 262144 --steps 3
 
 Inputs are the seeded synthetic workloads of ``inputs`` at the requested
 size (1M-token shapes: 64 query heads, 8 KV groups, head dim 128, index dim
@@ -26,7 +27,11 @@ def run_decode(args, name="decode_ctx1m"):
     w = WORKLOADS[name].scaled(max_seq_len=args.context, batch=args.batch)
     inp = make_inputs(w, device="cuda")
     q, q_idx, k, v, k_idx, lens = (inp[n] for n in ("q", "q_idx", "k", "v", "k_idx", "seq_lens"))
-    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens)
+    scale = None
+    if w.idx_format == "mxfp8":
+        k_idx, scale = api.quantize_index_k(k_idx)
+    p = api.params_from(q, q_idx, k, k_idx, block_size=w.block_size, top_k=w.top_k, seq_lens=lens,
+                        k_idx_scale=scale)
     ws = api.workspace(p, _lib.MSA_ENTRY_DECODE_FUSED, "cuda")
     o = torch.empty_like(q)
     ids = torch.empty(w.batch, 1, w.n_kv_heads, w.top_k, dtype=torch.int32, device="cuda")
@@ -121,7 +126,7 @@ def run_scan_shared(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("what", choices=["decode", "prefill_index", "prefill_attn", "prefill_chunks", "scan_shared",
-                                     "large_k"])
+                                     "large_k", "decode_mxfp8"])
     ap.add_argument("--context", type=int, default=262144)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--chunk", type=int, default=8192)
@@ -131,7 +136,8 @@ def main():
     {"decode": run_decode, "prefill_index": run_prefill_index, "prefill_attn": run_prefill_attn,
      "prefill_chunks": run_prefill_chunks,
      "scan_shared": run_scan_shared,
-     "large_k": lambda a: run_decode(a, "decode_ctx1m_large_k")}[args.what](args)
+     "large_k": lambda a: run_decode(a, "decode_ctx1m_large_k"),
+     "decode_mxfp8": lambda a: run_decode(a, "decode_ctx1m_mxfp8_idx")}[args.what](args)
 
 
 if __name__ == "__main__":

@@ -91,6 +91,37 @@ def test_index_scores_mxfp8():
                 assert err.max() <= 1e-5, (flags, b, g, err.max())
 
 
+def test_index_scores_mxfp8_wide_magnitudes():
+    """Index keys whose rows span 2^-30 .. 2^30 (block scales from tiny to large, many subnormal
+    E4M3 codes beside each block's maximum): token scores against the oracle on the decoded keys."""
+    _lib, api = _api()
+    w = small(batch=2, max_seq_len=2048, min_seq_len=2048)
+    inp = make_inputs(w, device="cuda")
+    g = torch.Generator(device="cpu").manual_seed(9)
+    mag = torch.pow(2.0, torch.randint(-30, 31, (w.batch, w.n_idx_k_heads, w.max_seq_len, 1), generator=g).float())
+    spread = torch.pow(2.0, torch.randint(-12, 1, (w.batch, w.n_idx_k_heads, w.max_seq_len, w.idx_dim), generator=g).float())
+    k_idx = (inp["k_idx"].float().cpu() * mag * spread).to(torch.bfloat16).cuda()
+    codes, scales = api.quantize_index_k(k_idx)
+    inp = dict(inp, k_idx=k_idx)
+    x = f32_inputs(inp, codes, scales)
+    p_or = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
+    p = api.params_from(inp["q"], inp["q_idx"], inp["k"], codes, block_size=w.block_size, top_k=w.top_k,
+                        seq_lens=inp["seq_lens"], flags=_lib.MSA_SCORES_TOKEN, k_idx_scale=scales)
+    out = torch.empty(w.batch, 1, w.n_kv_heads, w.max_seq_len, dtype=torch.float32, device="cuda")
+    _lib.msa_index_score(p, inp["q_idx"], codes, out, api.workspace(p, _lib.MSA_ENTRY_INDEX_SCORE, "cuda"))
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    assert (mxfp8.E4M3_TABLE[codes.cpu().numpy() & 0x7F] < 2.0 ** -6).mean() > 0.01, "few subnormal codes"
+    for b in range(w.batch):
+        pos = int(x["seq_lens"][b]) - 1
+        for gg in range(w.n_kv_heads):
+            ref = oracle.token_scores(p_or, x["q_idx"], x["k_idx"], b, 0, gg, pos)
+            # relative to the row's key magnitude: fp32 sums of products spanning 2^24
+            scale = np.abs(x["k_idx"][b, gg % w.n_idx_k_heads, :pos + 1]).max(axis=-1) * 8.0
+            err = np.abs(got[b, 0, gg, :pos + 1] - ref) / np.maximum(scale, 1e-30)
+            assert err.max() <= 1e-5, (b, gg, err.max())
+
+
 @pytest.mark.parametrize("case", [
     dict(),                                                             # ragged batch, per-group index heads
     dict(n_idx_k_heads=1, hot_blocks=0),                                # one index head shared by 4 groups
