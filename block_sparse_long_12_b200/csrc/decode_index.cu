@@ -123,8 +123,8 @@ __global__ void __launch_bounds__(W * 32, 1)
     constexpr int NCH = ROWB / 16;        // 16-byte vectors per index-key row
     constexpr int DI = ROWB / ES;         // index dim
     constexpr bool QREG = GPS == 1 && DI <= 64;
-    // several groups on one bf16 stream: the scores of a chunk are a small GEMM (the groups' index
-    // queries, padded to 16 rows, times the chunk's keys) on mma.sync tensor-core fragments
+    // several groups on one bf16 stream: the scores of a chunk are a small GEMM (the chunk's keys
+    // times the groups' index queries, padded to 8 columns) on mma.sync tensor-core fragments
     constexpr bool MMA = scan_mma<T, GPS, ROWB>();
     constexpr int KS = DI / 16;           // k-steps of 16 index dims
     constexpr bool FP8 = is_fp8<T>();     // MXFP8 keys: E4M3 codes, one E8M0 scale per 32 dims
@@ -311,9 +311,9 @@ __global__ void __launch_bounds__(W * 32, 1)
     };
     refill();
 
-    // A fragments of the groups' index queries (rows = the GPS groups of the stream, zero rows up to
-    // 16; columns = index dims), loaded when the warp moves to another stream
-    uint32_t qa[MMA ? KS : 1][4];
+    // B fragments of the groups' index queries (columns = the GPS groups of the stream, zero columns
+    // up to 8; rows = index dims), loaded when the warp moves to another stream
+    uint32_t qb[MMA ? KS : 1][2];
     auto load_qa = [&](int b, int hik) {
         if constexpr (MMA) {
             const int grp = lane >> 2, tig = lane & 3;
@@ -322,10 +322,8 @@ __global__ void __launch_bounds__(W * 32, 1)
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
                 const int c0 = ks * 16 + tig * 2;
-                qa[ks][0] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0) : 0u;
-                qa[ks][1] = 0u;
-                qa[ks][2] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0 + 8) : 0u;
-                qa[ks][3] = 0u;
+                qb[ks][0] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0) : 0u;
+                qb[ks][1] = grp < GPS ? *reinterpret_cast<const uint32_t *>(src + c0 + 8) : 0u;
             }
         }
     };
@@ -336,43 +334,52 @@ __global__ void __launch_bounds__(W * 32, 1)
     auto scan_chunk = [&](const unsigned char *base, const unsigned char *sbase, int nt, int b, int hik, int tok_base,
                           const float *qv_, const float *qsrc, float *m) {
         if constexpr (MMA) {
-            // S = Q_idx K^T, 8 keys per tile; lane (grp, tig) holds S[grp][2 tig, 2 tig + 1] of each
-            // tile.  The k-steps run over all tiles in turn, so consecutive MMAs are independent.
-            constexpr int NTL = kScanChunkBytes / ROWB / 8;  // key tiles of a full chunk
+            // S^T = K Q_idx^T, 16 keys (rows) by the 8 group columns per tile, so no MMA row is
+            // padding; lane (grp, tig) holds the scores of keys grp and grp + 8 of each tile for
+            // groups 2 tig and 2 tig + 1, and keeps their running maxima in m[0], m[1] (reduced
+            // over the lanes at the block end).  Every tile's A fragments are loaded before its
+            // MMAs; the tiles' accumulators are independent.
+            constexpr int NKT = kScanChunkBytes / ROWB / 16;  // key tiles of a full chunk
             const uint32_t tile = smem_u32(base);
-            const int grp = lane >> 2, tig = lane & 3, mi = lane >> 3;
-            float sv[NTL][4];
+            const int grp = lane >> 2, tig = lane & 3;
+            const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, ahalf = lane >> 4;
+            float sv[NKT][4];
 #pragma unroll
-            for (int kn = 0; kn < NTL; ++kn) sv[kn][0] = sv[kn][1] = sv[kn][2] = sv[kn][3] = 0.f;
+            for (int kt = 0; kt < NKT; ++kt) {
+                sv[kt][0] = sv[kt][1] = sv[kt][2] = sv[kt][3] = 0.f;
+                if (kt * 16 < nt) {
+                    uint32_t af[KS][4];
 #pragma unroll
-            for (int ks = 0; ks < KS; ks += 2) {
-                const int d0 = (ks + (mi >> 1)) * 16 + (mi & 1) * 8;
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const int d0 = ks * 16 + ahalf * 8;
+                        ldsm_x4(tile + (d0 >> 6) * (CT * 128) + sw128(kt * 16 + arow, (d0 & 63) >> 3), af[ks][0], af[ks][1],
+                                af[ks][2], af[ks][3]);
+                    }
 #pragma unroll
-                for (int kn = 0; kn < NTL; ++kn) {
-                    if (kn * 8 < nt) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4(tile + (d0 >> 6) * (CT * 128) + sw128(kn * 8 + (lane & 7), (d0 & 63) >> 3), b0, b1, b2, b3);
-                        mma_16816(sv[kn], qa[ks], b0, b1);
-                        mma_16816(sv[kn], qa[ks + 1], b2, b3);
+                    for (int ks = 0; ks < KS; ++ks) mma_16816_pure(sv[kt], af[ks], qb[ks][0], qb[ks][1]);
+                }
+            }
+            float c0 = m[0], c1 = m[1];
+#pragma unroll
+            for (int kt = 0; kt < NKT; ++kt) {
+                const int k0 = kt * 16 + grp, k1 = k0 + 8;
+                const bool v0 = k0 < nt && !failed, v1 = k1 < nt && !failed;
+                c0 = tc::fmax3(c0, v0 ? sv[kt][0] : -INFINITY, v1 ? sv[kt][2] : -INFINITY);
+                c1 = tc::fmax3(c1, v0 ? sv[kt][1] : -INFINITY, v1 ? sv[kt][3] : -INFINITY);
+                if (a.token_scores != nullptr && !failed) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int gl = 2 * tig + h;
+                        if (gl < GPS) {
+                            float *ts = a.token_scores + ((size_t)b * a.G + hik + Hik * gl) * a.L_max + tok_base;
+                            if (v0) ts[k0] = sv[kt][h];
+                            if (v1) ts[k1] = sv[kt][2 + h];
+                        }
                     }
                 }
             }
-            float cmax = -INFINITY;
-#pragma unroll
-            for (int kn = 0; kn < NTL; ++kn) {
-                const int k0 = kn * 8 + tig * 2;
-                const float s0 = (k0 < nt && !failed) ? sv[kn][0] : -INFINITY;
-                const float s1 = (k0 + 1 < nt && !failed) ? sv[kn][1] : -INFINITY;
-                cmax = tc::fmax3(cmax, s0, s1);
-                if (a.token_scores != nullptr && grp < GPS && !failed) {
-                    float *ts = a.token_scores + ((size_t)b * a.G + hik + Hik * grp) * a.L_max + tok_base;
-                    if (k0 < nt) ts[k0] = s0;
-                    if (k0 + 1 < nt) ts[k0 + 1] = s1;
-                }
-            }
-            // the 4 lanes of a group reduce at the block end
-#pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) m[gl] = fmaxf(m[gl], gl == grp ? cmax : -INFINITY);
+            m[0] = c0;
+            m[1] = c1;
         } else {
             for (int t0 = 0; t0 < nt; t0 += 32) {
                 const int tok = t0 + lane;  // one index-key row per lane
@@ -451,17 +458,18 @@ __global__ void __launch_bounds__(W * 32, 1)
     };
 
     // every lane ends with the block's max of each group: a butterfly over the lanes, or, with
-    // tensor-core scores (lanes 4 g .. 4 g + 3 hold group g), a reduction over those 4 lanes
-    // and one broadcast per group
+    // tensor-core scores (the 8 lanes of one tig hold groups 2 tig and 2 tig + 1), a reduction
+    // over those 8 lanes and one broadcast per group
     auto block_max = [&](float *m) {
         if constexpr (MMA) {
-            float mine = -INFINITY;
+            float c0 = m[0], c1 = m[1];
 #pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) mine = gl == (lane >> 2) ? m[gl] : mine;
-            mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 1));
-            mine = fmaxf(mine, __shfl_xor_sync(FULL, mine, 2));
+            for (int o = 4; o < 32; o <<= 1) {
+                c0 = fmaxf(c0, __shfl_xor_sync(FULL, c0, o));
+                c1 = fmaxf(c1, __shfl_xor_sync(FULL, c1, o));
+            }
 #pragma unroll
-            for (int gl = 0; gl < GPS; ++gl) m[gl] = __shfl_sync(FULL, mine, gl * 4);
+            for (int gl = 0; gl < GPS; ++gl) m[gl] = __shfl_sync(FULL, (gl & 1) ? c1 : c0, gl >> 1);
         } else {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)

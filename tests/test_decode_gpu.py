@@ -109,12 +109,14 @@ def test_decode_exact_lengths_edges():
     assert idn[0, 0, :, 0].tolist() == [0] * 4 and (idn[0, 0, :, 1:] == -1).all()
 
 
-@pytest.mark.parametrize("hik", [4, 1], ids=["hik4", "hik1"])
-def test_index_scores_and_pool_topk(hik):
-    """Stored token / block scores, then the stand-alone pool + TopK entry (hik 1: the four groups
-    share one index-K stream and are scored together on tensor cores)."""
+@pytest.mark.parametrize("hik,di,gk", [(4, 64, 4), (1, 64, 4), (1, 128, 4), (1, 64, 8), (1, 64, 2)],
+                         ids=["hik4", "hik1", "hik1_di128", "hik1_g8", "hik1_g2"])
+def test_index_scores_and_pool_topk(hik, di, gk):
+    """Stored token / block scores, then the stand-alone pool + TopK entry (hik < groups: the
+    groups that share one index-K stream, 2, 4 or 8 of them, are scored together on tensor cores,
+    64- and 128-dim index keys)."""
     api = _api()
-    w = small(dtype="bf16", hot_blocks=4, n_idx_k_heads=hik)
+    w = small(dtype="bf16", hot_blocks=4, n_idx_k_heads=hik, idx_dim=di, n_kv_heads=gk, n_q_heads=4 * gk)
     inp = make_inputs(w, device="cuda")
     x = to_np(inp)
     p = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
