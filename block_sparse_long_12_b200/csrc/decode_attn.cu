@@ -395,10 +395,148 @@ __device__ void select_group_topk(const AttnArgs &a, int b, int g, const SegInfo
     __syncthreads();
 }
 
-// Scratch bytes select_group_topk needs (lists of n_cta pieces of k entries).
+// Descending bitonic sort of 32 keys held one per lane.
+__device__ inline unsigned long long warp_sort32_desc(unsigned long long v, int lane) {
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(FULL, v, stride);
+            const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+            v = keep_max ? (v > o ? v : o) : (v < o ? v : o);
+        }
+    return v;
+}
+
+// Final TopK of group g of sequence b from the block scores of every block of
+// its stream.  Groups that share one index-K stream take this way: the scan
+// keeps no per-piece lists for them (every CTA of the scan would hold a piece
+// of the one stream) and leaves every block's score.  Every thread's best
+// block of its share (blocks tid, tid + nthr, ...) is one of the candidates,
+// so the k-th best of the threads' bests is a floor that the final k all
+// reach; a second pass gathers the blocks at or above it and one warp (or the
+// CTA) sorts them.  If more than kSortCap reach the floor, every warp keeps
+// the k best of its share that do and one warp merges the warps' lists.
+// Leaves the list in sel_s / sel_i[0..32), padded with (-inf, -1).  Called by
+// every thread of the CTA.
+__device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int k = a.k;
+    int L = a.seq_lens[b];
+    L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
+    const int nb = (L + a.Bk - 1) / a.Bk;
+    const float *tsc = a.tail_scores + ((size_t)b * a.G + g) * ((a.L_max + a.Bk - 1) / a.Bk);
+    // scratch: survivors [kSortCap] | the warps' sorted bests [nwarps][32] | floor | count
+    unsigned long long *keys = reinterpret_cast<unsigned long long *>(scratch);
+    unsigned long long *wl = keys + kSortCap;
+    unsigned long long *floor_key = wl + nwarps * 32;
+    int *cnt = reinterpret_cast<int *>(floor_key + 1);
+    if (tid == 0) *cnt = 0;
+    if (tid < 32) {
+        sel_s[tid] = -INFINITY;
+        sel_i[tid] = -1;
+    }
+    constexpr int kBatch = 16;  // loads in flight per thread
+    unsigned long long best = 0ull;  // below every real key
+    for (int base = 0; base < nb; base += nthr * kBatch) {
+        float v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = base + u * nthr + tid;
+            v[u] = n < nb ? tsc[n] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = base + u * nthr + tid;
+            const unsigned long long key = n < nb ? sel_key(v[u], n) : 0ull;
+            best = key > best ? key : best;
+        }
+    }
+    wl[warp * 32 + lane] = warp_sort32_desc(best, lane);
+    __syncthreads();
+    if (warp == 0) {
+        unsigned long long t = wl[lane];
+        for (int w2 = 1; w2 < nwarps; ++w2) t = warp_merge_top32(t, wl[w2 * 32 + lane], lane);
+        // 0 when fewer than k threads hold a block (nb < k): every block survives
+        const unsigned long long fk = __shfl_sync(FULL, t, k - 1);
+        if (lane == 0) *floor_key = fk;
+    }
+    __syncthreads();
+    const unsigned long long fk = *floor_key;
+    for (int base = 0; base < nb; base += nthr * kBatch) {
+        float v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = base + u * nthr + tid;
+            v[u] = n < nb ? tsc[n] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int n = base + u * nthr + tid;
+            const unsigned long long key = n < nb ? sel_key(v[u], n) : 0ull;
+            const bool keep = n < nb && key >= fk;
+            const unsigned msk = __ballot_sync(FULL, keep);
+            if (msk != 0u) {
+                int at = 0;
+                if (lane == 0) at = atomicAdd(cnt, __popc(msk));
+                at = __shfl_sync(FULL, at, 0) + __popc(msk & ((1u << lane) - 1u));
+                if (keep && at < kSortCap) keys[at] = key;
+            }
+        }
+    }
+    __syncthreads();
+    const int m = *cnt;
+    if (m <= 64) {
+        if (warp == 0) {
+            unsigned long long v[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) v[j] = lane + 32 * j < m ? keys[lane + 32 * j] : 0ull;
+            warp_sort64_desc(v, lane);
+            if (lane < k && lane < m) sel_unkey(v[0], sel_s[lane], sel_i[lane]);
+        }
+        __syncthreads();
+        return;
+    }
+    if (m <= kSortCap) {
+        int P = 128;
+        while (P < m) P <<= 1;
+        for (int i = m + tid; i < P; i += nthr) keys[i] = 0ull;
+        __syncthreads();
+        block_sort_desc(keys, P);
+        if (tid < k) sel_unkey(keys[tid], sel_s[tid], sel_i[tid]);
+        __syncthreads();
+        return;
+    }
+    // many blocks at the floor: the k best of each warp's share that reach it, then one merge
+    WarpTopK t;
+    t.reset();
+    for (int base = warp * 32; base < nb; base += nwarps * 32) {
+        const int n = base + lane;
+        const float v = n < nb ? tsc[n] : -INFINITY;
+        unsigned msk = __ballot_sync(FULL, n < nb && sel_key(v, n) >= fk && better(v, n, t.thr_s, t.thr_i));
+        while (msk) {
+            const int l = __ffs(msk) - 1;
+            msk &= msk - 1;
+            t.insert(__shfl_sync(FULL, v, l), base + l, k, lane);
+        }
+    }
+    __syncthreads();  // every thread is done with the survivors' keys
+    float *tl_s = reinterpret_cast<float *>(keys);  // [nwarps][32]
+    int *tl_i = reinterpret_cast<int *>(tl_s + nwarps * 32);
+    tl_s[warp * 32 + lane] = t.s;
+    tl_i[warp * 32 + lane] = t.id;
+    __syncthreads();
+    if (warp == 0) warp_merge_sorted_lists<1>(tl_s, tl_i, nwarps, k, 32, k, sel_s, sel_i, lane);
+    __syncthreads();
+}
+
+// Scratch bytes the selection needs: select_group_topk's lists of n_cta pieces of k entries and
+// its survivors, or select_from_scores' survivors and per-warp lists.
 __host__ __device__ inline size_t select_scratch_bytes(int n_cta, int k) {
     const size_t cap = (size_t)n_cta * k;
-    return cap * 8 + 32 * 4 + (cap > (size_t)kSortCap ? cap : (size_t)kSortCap) * 8;
+    const size_t lists = cap * 8 + 32 * 4 + (cap > (size_t)kSortCap ? cap : (size_t)kSortCap) * 8;
+    const size_t scores = (size_t)kSortCap * 8 + (32 * 32 + 1) * 8 + 16;
+    return lists > scores ? lists : scores;
 }
 
 // The last split CTA of (b, g) merges the normalised partial outputs of all
@@ -516,11 +654,17 @@ __device__ inline void force_sink_local(const AttnArgs &a, int b, float *sel_s, 
     __syncthreads();
 }
 
+// SO: the stream's groups share one index-K head (a.scores_only): the selection reads every
+// block's score instead of the scan's per-piece lists
+template <bool SO>
 __device__ inline void group_list(const AttnArgs &a, int b, int g, const SegInfo info, unsigned char *scratch,
                                   float *sel_s, int *sel_i) {
     if (a.dense) return;
     if (a.cand_s != nullptr) {
-        select_group_topk(a, b, g, info, scratch, sel_s, sel_i);
+        if constexpr (SO)
+            select_from_scores(a, b, g, scratch, sel_s, sel_i);
+        else
+            select_group_topk(a, b, g, info, scratch, sel_s, sel_i);
         if (a.force) force_sink_local(a, b, sel_s, sel_i);
         if (blockIdx.x == 0 && threadIdx.x < a.k) {
             const size_t o = ((size_t)b * a.G + g) * a.k + threadIdx.x;
@@ -588,11 +732,14 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const int nb = (L + a.Bk - 1) / a.Bk;
 
     // where the scan leaves this group's lists is known from seq_lens alone
-    const SegInfo info = (!a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
+    const SegInfo info = (!a.dense && a.cand_s != nullptr && !a.scores_only) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
     __shared__ int last_flag;
-    group_list(a, b, g, info, ring, sel_s, sel_i);
+    if (a.scores_only)
+        group_list<true>(a, b, g, info, ring, sel_s, sel_i);
+    else
+        group_list<false>(a, b, g, info, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1)
     const int bps = a.blocks_per_split;
@@ -775,7 +922,7 @@ constexpr int kMaxStages = 4;     // K/V ring stages (mbarriers reserved)
 constexpr int kMmaRows = 16;      // query rows of the fragment (heads of the group, padded)
 constexpr int kMaxCluster = 8;    // splits of a group that form one cluster
 
-template <int D>
+template <int D, bool SO>
 __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const __grid_constant__ CUtensorMap kmap,
                                                                       const __grid_constant__ CUtensorMap vmap,
                                                                       const AttnArgs a) {
@@ -832,10 +979,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1) decode_attn_mma_kernel(const _
     const int nb = (L + a.Bk - 1) / a.Bk;
 
     // where the scan leaves this group's lists is known from seq_lens alone
-    const SegInfo info = (!a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
+    const SegInfo info = (!SO && !a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
-    group_list(a, b, g, info, ring, sel_s, sel_i);
+    group_list<SO>(a, b, g, info, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1), each cut into tiles of KT keys
     const int j0 = s * a.blocks_per_split;
@@ -1113,8 +1260,8 @@ cudaError_t launch_attn_r(const AttnArgs &a, cudaStream_t s, bool pdl) {
     return launch_attn_t<T, D, 16>(a, s, pdl);
 }
 
-template <int D>
-cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
+template <int D, bool SO>
+cudaError_t launch_mma_t(AttnArgs a, cudaStream_t s, bool pdl) {
     a.cluster = (!a.dense && a.S <= kMaxCluster) ? a.S : 1;
     const int KT = a.Bk < 128 ? a.Bk : 128;
     const size_t stage = (size_t)2 * (D / 64) * KT * 128;
@@ -1134,7 +1281,7 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
                         ((size_t)kMmaRows * D + kMaxCluster + (size_t)kMaxCluster * kMmaRows) * 4 + 64;
     static size_t attr_bytes = 0;
     if (smem > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(decode_attn_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(decode_attn_mma_kernel<D, SO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)smem);
         if (e != cudaSuccess) return e;
         attr_bytes = smem;
@@ -1167,7 +1314,12 @@ cudaError_t launch_mma(AttnArgs a, cudaStream_t s, bool pdl) {
     }
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, decode_attn_mma_kernel<D>, km, vm, a);
+    return cudaLaunchKernelEx(&cfg, decode_attn_mma_kernel<D, SO>, km, vm, a);
+}
+
+template <int D>
+cudaError_t launch_mma(const AttnArgs &a, cudaStream_t s, bool pdl) {
+    return a.scores_only ? launch_mma_t<D, true>(a, s, pdl) : launch_mma_t<D, false>(a, s, pdl);
 }
 
 
@@ -1284,8 +1436,8 @@ __global__ void __launch_bounds__(WideShape<D>::NW * 32, 1)
         if (lane == 0) {
             unsigned char *st = my_ring + (size_t)slot * STAGE;
             mbar_arrive_expect_tx(&my_bars[slot], STAGE);
-#pragma unroll
             const int row = a.cache.row(b, g, a.G, a.L_max, key0);
+#pragma unroll
             for (int h = 0; h < NH; ++h) {
                 tc::tma_load_2d(st + h * KVH, &kmap, h * 64, row, &my_bars[slot]);
                 tc::tma_load_2d(st + (NH + h) * KVH, &vmap, h * 64, row, &my_bars[slot]);

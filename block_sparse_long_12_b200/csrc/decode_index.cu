@@ -214,6 +214,9 @@ __global__ void __launch_bounds__(W * 32, 1)
     uint64_t *my_bars = bars + w * S;
     const bool want_cand = a.cand_s != nullptr;
     const uint32_t chunk_bytes = (uint32_t)CT * ROWB;
+    // the index keys are read once: evict-first in L2, so that the stream does not push out what
+    // the attention kernel reads next (the lists, block scores and counters this kernel writes)
+    const uint64_t stream_pol = l2_evict_first_policy();
 
     // The shared tail (the last quarter of every stream's blocks): every warp takes tail blocks,
     // one at a time, until the pools are empty; a tail block leaves only its scores
@@ -303,8 +306,9 @@ __global__ void __launch_bounds__(W * 32, 1)
                 } else {
                     mbar_arrive_expect_tx(&my_bars[slot], chunk_bytes);
                 }
-                tc::tma_load_2d(dst, &kmap, 0, row, &my_bars[slot]);
-                if constexpr (ROWB == 256) tc::tma_load_2d(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot]);
+                tc::tma_load_2d_hint(dst, &kmap, 0, row, &my_bars[slot], stream_pol);
+                if constexpr (ROWB == 256)
+                    tc::tma_load_2d_hint(dst + CT * 128, &kmap, 128 / ES, row, &my_bars[slot], stream_pol);
             }
             ++issued;
         }

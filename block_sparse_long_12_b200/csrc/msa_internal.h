@@ -37,6 +37,7 @@ struct AttnArgs {
     const float *cand_s;       // scan candidates [n_seg, n_cta, G/Hik, k]: select in the kernel (fused decode)
     const int *cand_i;
     const float *tail_scores;  // [B, G, nb_max] block scores of the segments' tails (fused decode)
+    int scores_only;           // groups share one index-K stream: no lists, every block's score in tail_scores
     int n_cta;
     int *ids_out;              // nullable (fused decode)
     float *top_scores_out;     // nullable (fused decode)
