@@ -411,14 +411,23 @@ __device__ inline unsigned long long warp_sort32_desc(unsigned long long v, int 
 // Final TopK of group g of sequence b from the block scores of every block of
 // its stream.  Groups that share one index-K stream take this way: the scan
 // keeps no per-piece lists for them (every CTA of the scan would hold a piece
-// of the one stream) and leaves every block's score.  Every thread's best
-// block of its share (blocks tid, tid + nthr, ...) is one of the candidates,
-// so the k-th best of the threads' bests is a floor that the final k all
-// reach; a second pass gathers the blocks at or above it and one warp (or the
-// CTA) sorts them.  If more than kSortCap reach the floor, every warp keeps
-// the k best of its share that do and one warp merges the warps' lists.
-// Leaves the list in sel_s / sel_i[0..32), padded with (-inf, -1).  Called by
-// every thread of the CTA.
+// of the one stream) and leaves every block's score.  The scores are staged
+// in shared memory by one bulk copy (chunks of what the scratch holds), so
+// that both passes read shared memory: every thread's best block of its
+// share (blocks tid, tid + nthr, ...) is one of the candidates, so the k-th
+// best of the threads' bests is a floor that the final k all reach; the
+// second pass gathers the blocks at or above it and one warp (or the CTA)
+// sorts them.  If more than kSortCap reach the floor, every warp keeps the k
+// best of its share that do and one warp merges the warps' lists.  Leaves the
+// list in sel_s / sel_i[0..32), padded with (-inf, -1).  Called by every
+// thread of the CTA.
+constexpr int kScoreStageOff = 12352;  // scratch bytes before the staged scores (16-byte aligned)
+// Every thread's shared-memory writes before the tensor copies (async proxy) that reuse the
+// scratch for K/V tiles, then a CTA barrier.
+__device__ inline void fence_scratch_for_tma() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+}
 __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned char *scratch, float *sel_s, int *sel_i) {
     const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
     const int k = a.k;
@@ -426,31 +435,55 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
     L = L < 0 ? 0 : (L > a.L_max ? a.L_max : L);
     const int nb = (L + a.Bk - 1) / a.Bk;
     const float *tsc = a.tail_scores + ((size_t)b * a.G + g) * ((a.L_max + a.Bk - 1) / a.Bk);
-    // scratch: survivors [kSortCap] | the warps' sorted bests [nwarps][32] | floor | count
+    // scratch: survivors [kSortCap] | the warps' sorted bests [nwarps][32] | floor | barrier | count | staged scores
     unsigned long long *keys = reinterpret_cast<unsigned long long *>(scratch);
     unsigned long long *wl = keys + kSortCap;
     unsigned long long *floor_key = wl + nwarps * 32;
-    int *cnt = reinterpret_cast<int *>(floor_key + 1);
-    if (tid == 0) *cnt = 0;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(floor_key + 1);
+    int *cnt = reinterpret_cast<int *>(bar + 1);
+    float *stage = reinterpret_cast<float *>(scratch + kScoreStageOff);
+    // floats per chunk (a multiple of 4, 3 spare for the alignment shift)
+    const int cap = ((a.ring_bytes - kScoreStageOff) / 4 - 3) / 4 * 4;
+    // the bulk copy starts at the first 16-byte aligned score; the h scores before it and the
+    // ragged end are loaded by the threads; score i of a chunk sits at stage[i + sh]
+    const int h = (int)(((16u - ((uint32_t)reinterpret_cast<uintptr_t>(tsc) & 15u)) & 15u) >> 2);
+    const int sh = (4 - h) & 3;
+    if (tid == 0) {
+        *cnt = 0;
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
     if (tid < 32) {
         sel_s[tid] = -INFINITY;
         sel_i[tid] = -1;
     }
-    constexpr int kBatch = 16;  // loads in flight per thread
-    unsigned long long best = 0ull;  // below every real key
-    for (int base = 0; base < nb; base += nthr * kBatch) {
-        float v[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int n = base + u * nthr + tid;
-            v[u] = n < nb ? tsc[n] : 0.f;
+    __syncthreads();
+    uint32_t phase = 0;
+    auto stage_chunk = [&](int c0, int cn) {
+        const int hh = h < cn ? h : cn;
+        const int body = (cn - hh) / 4 * 4;
+        if (tid == 0 && body > 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // earlier reads of the stage first
+            mbar_arrive_expect_tx(bar, (uint32_t)body * 4);
+            bulk_g2s(stage + hh + sh, tsc + c0 + hh, (uint32_t)body * 4, bar, l2_evict_normal_policy());
         }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int n = base + u * nthr + tid;
-            const unsigned long long key = n < nb ? sel_key(v[u], n) : 0ull;
+        for (int i = tid; i < cn; i += nthr)
+            if (i < hh || i >= hh + body) stage[i + sh] = tsc[c0 + i];
+        if (body > 0) {
+            mbar_wait(bar, phase, a.status);
+            phase ^= 1u;
+        }
+        __syncthreads();
+    };
+    unsigned long long best = 0ull;  // below every real key
+    for (int c0 = 0; c0 < nb; c0 += cap) {
+        const int cn = nb - c0 < cap ? nb - c0 : cap;
+        stage_chunk(c0, cn);
+        for (int i = tid; i < cn; i += nthr) {
+            const unsigned long long key = sel_key(stage[i + sh], c0 + i);
             best = key > best ? key : best;
         }
+        if (c0 + cap < nb) __syncthreads();  // the next chunk overwrites the stage
     }
     wl[warp * 32 + lane] = warp_sort32_desc(best, lane);
     __syncthreads();
@@ -463,18 +496,13 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
     }
     __syncthreads();
     const unsigned long long fk = *floor_key;
-    for (int base = 0; base < nb; base += nthr * kBatch) {
-        float v[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int n = base + u * nthr + tid;
-            v[u] = n < nb ? tsc[n] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int n = base + u * nthr + tid;
-            const unsigned long long key = n < nb ? sel_key(v[u], n) : 0ull;
-            const bool keep = n < nb && key >= fk;
+    for (int c0 = 0; c0 < nb; c0 += cap) {
+        const int cn = nb - c0 < cap ? nb - c0 : cap;
+        if (nb > cap) stage_chunk(c0, cn);  // one chunk: its scores are still staged
+        for (int i0 = 0; i0 < cn; i0 += nthr) {
+            const int i = i0 + tid;
+            const unsigned long long key = i < cn ? sel_key(stage[i + sh], c0 + i) : 0ull;
+            const bool keep = i < cn && key >= fk;
             const unsigned msk = __ballot_sync(FULL, keep);
             if (msk != 0u) {
                 int at = 0;
@@ -483,8 +511,9 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
                 if (keep && at < kSortCap) keys[at] = key;
             }
         }
+        __syncthreads();
     }
-    __syncthreads();
+    if (tid == 0) asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
     const int m = *cnt;
     if (m <= 64) {
         if (warp == 0) {
@@ -494,7 +523,7 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
             warp_sort64_desc(v, lane);
             if (lane < k && lane < m) sel_unkey(v[0], sel_s[lane], sel_i[lane]);
         }
-        __syncthreads();
+        fence_scratch_for_tma();
         return;
     }
     if (m <= kSortCap) {
@@ -504,7 +533,7 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
         __syncthreads();
         block_sort_desc(keys, P);
         if (tid < k) sel_unkey(keys[tid], sel_s[tid], sel_i[tid]);
-        __syncthreads();
+        fence_scratch_for_tma();
         return;
     }
     // many blocks at the floor: the k best of each warp's share that reach it, then one merge
@@ -527,7 +556,7 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
     tl_i[warp * 32 + lane] = t.id;
     __syncthreads();
     if (warp == 0) warp_merge_sorted_lists<1>(tl_s, tl_i, nwarps, k, 32, k, sel_s, sel_i, lane);
-    __syncthreads();
+    fence_scratch_for_tma();
 }
 
 // Scratch bytes the selection needs: select_group_topk's lists of n_cta pieces of k entries and
@@ -535,7 +564,7 @@ __device__ void select_from_scores(const AttnArgs &a, int b, int g, unsigned cha
 __host__ __device__ inline size_t select_scratch_bytes(int n_cta, int k) {
     const size_t cap = (size_t)n_cta * k;
     const size_t lists = cap * 8 + 32 * 4 + (cap > (size_t)kSortCap ? cap : (size_t)kSortCap) * 8;
-    const size_t scores = (size_t)kSortCap * 8 + (32 * 32 + 1) * 8 + 16;
+    const size_t scores = (size_t)kScoreStageOff + 16384;  // chunks of 4,096 scores at least
     return lists > scores ? lists : scores;
 }
 

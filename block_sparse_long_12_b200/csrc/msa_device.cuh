@@ -135,6 +135,12 @@ __device__ inline uint64_t l2_evict_first_policy() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+// L2 policy for data read again soon by other CTAs.
+__device__ inline uint64_t l2_evict_normal_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 // TMA bulk copy global -> shared (contiguous bytes, 16-byte aligned, size a
 // multiple of 16), completion counted on `bar`.
 __device__ inline void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar,

@@ -77,6 +77,40 @@ def test_decode_fused_variants(case):
     compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
 
 
+def test_shared_stream_selection_in_chunks():
+    """Groups on one index-K stream select from every block's score, staged in shared memory in
+    chunks when the stream has more blocks than one chunk holds (16-token blocks: 6,250 blocks)."""
+    w = small(block_size=16, top_k=32, max_seq_len=100000, min_seq_len=90000, batch=2, n_idx_k_heads=1, hot_blocks=12)
+    inp = make_inputs(w, device="cuda")
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+
+
+def test_shared_stream_selection_many_at_floor():
+    """Block scores that repeat with a period of 128 blocks (the index keys of block n equal those
+    of block n mod 128): the k-th best of the selecting threads' bests is then a floor that many
+    blocks reach (k times the number of periods, 768), beyond what is sorted at once; ids and
+    outputs against the oracle, and equal scores taken by lower id."""
+    w = small(block_size=64, top_k=32, max_seq_len=196608, min_seq_len=196608, batch=1, n_idx_k_heads=1,
+              hot_blocks=0)
+    inp = make_inputs(w, device="cuda")
+    period = 128 * w.block_size
+    ki = inp["k_idx"]
+    for t0 in range(period, w.max_seq_len, period):
+        ki[:, :, t0:t0 + period] = ki[:, :, :period]
+    o, ids, lse = run_fused(inp, w)
+    x = to_np(inp)
+    compare_decode(x, oracle_params(x, block_size=w.block_size, top_k=w.top_k), o, ids, lse)
+    # every selected block is the lowest-id copy's class mate: within a class the lower ids come first
+    idn = ids.cpu().numpy()[0, 0]
+    for g in range(w.n_kv_heads):
+        sel = idn[g][idn[g] >= 0]
+        for c in np.unique(sel % 128):
+            mates = np.sort(sel[sel % 128 == c])
+            assert mates.tolist() == list(range(c, c + 128 * len(mates), 128)), (g, c, mates)
+
+
 @pytest.mark.parametrize("case", [
     dict(),                                                           # ragged, partial last blocks
     dict(n_idx_k_heads=1, hot_blocks=0),                               # groups on one shared stream (tensor cores)
