@@ -761,14 +761,11 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnArg
     const int nb = (L + a.Bk - 1) / a.Bk;
 
     // where the scan leaves this group's lists is known from seq_lens alone
-    const SegInfo info = (!a.dense && a.cand_s != nullptr && !a.scores_only) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
+    const SegInfo info = (!a.dense && a.cand_s != nullptr) ? seg_pieces(a, b, g % a.Hik) : SegInfo{-1, 0};
     pdl_wait_prior_grid();  // the scan's candidates are complete from here on
     pdl_allow_next_grid();
     __shared__ int last_flag;
-    if (a.scores_only)
-        group_list<true>(a, b, g, info, ring, sel_s, sel_i);
-    else
-        group_list<false>(a, b, g, info, ring, sel_s, sel_i);
+    group_list<false>(a, b, g, info, ring, sel_s, sel_i);
 
     // this split's blocks: list positions [j0, j1)
     const int bps = a.blocks_per_split;

@@ -196,6 +196,12 @@ msa_status_t decode_fused_scratch_bytes(const msa_params_t *p, size_t *bytes) {
     return MSA_OK;
 }
 
+// Groups that share one index-K stream, bf16 K/V (the tensor-core attention kernel): the scan
+// keeps no per-piece lists and the attention kernel selects from every block's score.
+static bool shared_stream_scores(const msa_params_t &p) {
+    return p.n_kv_heads > p.n_idx_k_heads && p.dtype == MSA_BF16 && !(p.flags & MSA_DENSE);
+}
+
 DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_sm) {
     DecodeWs L{};
     L.n_cta = n_sm < 256 ? n_sm : 256;
@@ -210,7 +216,7 @@ DecodeWs decode_ws_layout(const msa_params_t &p, bool scan, bool attend, int n_s
         // large k: no per-piece lists; the scan leaves every block's score and a radix select
         // writes the ids.  Groups that share one index-K stream: no lists either; the attention
         // kernel selects from every block's score
-        const size_t cand = (large || gps > 1) ? 0 : (size_t)n_seg * L.n_cta * gps * p.top_k * 4;
+        const size_t cand = (large || shared_stream_scores(p)) ? 0 : (size_t)n_seg * L.n_cta * gps * p.top_k * 4;
         L.cand_s = off;
         off += round256(cand);
         L.cand_i = off;
@@ -505,7 +511,7 @@ static msa_status_t attend_decode(const msa_params_t *p, const void *q, const vo
         a.cand_i = reinterpret_cast<const int *>(wsb + L.cand_i);
         a.tail_scores = reinterpret_cast<const float *>(wsb + L.tail_scores);
         a.ids_out = ids_out;
-        a.scores_only = p->n_kv_heads > p->n_idx_k_heads;
+        a.scores_only = shared_stream_scores(*p);
     }
     a.n_cta = L.n_cta;
     a.part_o = reinterpret_cast<float *>(wsb + L.part_o);
@@ -590,7 +596,7 @@ msa_status_t msa_decode_fused(const msa_params_t *p, const void *q, const void *
     a.status = reinterpret_cast<int *>(wsb);
     a.cache = cache_of(*p);
     const bool large = p->top_k > kMaxTopKList;
-    if (large || p->n_kv_heads > p->n_idx_k_heads) {
+    if (large || shared_stream_scores(*p)) {
         // every block's score (static ranges and tails alike) into the block-score region: for
         // the radix select (large k), or for the attention kernel's selection when groups share
         // one index-K stream (every scan CTA would hold a piece of it: too many lists to merge)

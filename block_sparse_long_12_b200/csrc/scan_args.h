@@ -71,6 +71,9 @@ struct ScanArgs {
     // rows = the code tensor's rows, a multiple of 16
     const uint8_t *k_scale;
     long long k_scale_rows;
+    // the stream's TMA loads evict-first in L2 (set by the launcher for streams of at most
+    // kEvictFirstMaxBytes; evict-normal beyond)
+    int stream_evict_first;
 };
 
 }  // namespace msa
