@@ -122,6 +122,37 @@ def test_index_scores_mxfp8_wide_magnitudes():
             assert err.max() <= 1e-5, (b, gg, err.max())
 
 
+def test_index_scores_mxfp8_exact_products():
+    """The scan's products of bf16 query elements and E4M3 codes are exact in fp32 (8 + 4
+    significant bits) and its sums run in a fixed order, so the index query times 2^20 (beyond f16's
+    range) gives exactly 2^20 times the scores, bit for bit; the scores against the oracle on the
+    decoded keys."""
+    _lib, api = _api()
+    w = small(batch=2, max_seq_len=3008, min_seq_len=3008)
+    inp = make_inputs(w, device="cuda")
+    q = inp["q_idx"]
+    q = torch.where(q.abs() < 2.0 ** -14, torch.zeros_like(q), q)  # no tiny elements: no underflow
+    codes, scales = api.quantize_index_k(inp["k_idx"])
+    outs = []
+    for qq in (q, q * 2.0 ** 20):
+        p = api.params_from(inp["q"], qq, inp["k"], codes, block_size=w.block_size, top_k=w.top_k,
+                            seq_lens=inp["seq_lens"], flags=_lib.MSA_SCORES_TOKEN, k_idx_scale=scales)
+        out = torch.empty(w.batch, 1, w.n_kv_heads, w.max_seq_len, dtype=torch.float32, device="cuda")
+        _lib.msa_index_score(p, qq, codes, out, api.workspace(p, _lib.MSA_ENTRY_INDEX_SCORE, "cuda"))
+        outs.append(out)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[1], outs[0] * 2.0 ** 20)
+    x = f32_inputs(dict(inp, q_idx=q), codes, scales)
+    p_or = oracle_params(x, block_size=w.block_size, top_k=w.top_k)
+    got = outs[0].cpu().numpy()
+    for b in range(w.batch):
+        pos = int(x["seq_lens"][b]) - 1
+        for g in range(w.n_kv_heads):
+            ref = oracle.token_scores(p_or, x["q_idx"], x["k_idx"], b, 0, g, pos)
+            err = np.abs(got[b, 0, g, :pos + 1] - ref) / np.maximum(np.abs(ref), 1.0)
+            assert err.max() <= 1e-5, (b, g, err.max())
+
+
 @pytest.mark.parametrize("case", [
     dict(),                                                             # ragged batch, per-group index heads
     dict(n_idx_k_heads=1, hot_blocks=0),                                # one index head shared by 4 groups
