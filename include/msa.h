@@ -229,9 +229,13 @@ MSA_API msa_status_t msa_sparse_attn_prefill(const msa_params_t *params, const v
  * One decode step, Steps 1 and 2 fused into back-to-back kernels on `stream`
  * (the block list never leaves the device).  ids_out and lse are nullable.
  * top_k up to 32: the scan keeps per-range candidate lists and the attention
- * kernel finishes the TopK; larger top_k: the scan stores every block's score
- * in ws, a radix select per (sequence, group) writes the list, and the
- * attention splits each group's blocks over about two CTAs per SM.
+ * kernel finishes the TopK (bf16 caches whose groups share one index-K head,
+ * n_idx_k_heads < n_kv_heads: no lists, the scan stores every block's score in
+ * ws and the attention kernel selects from those); larger top_k: the scan
+ * stores every block's score in ws, a radix select per (sequence, group)
+ * writes the list, and the attention splits each group's blocks over about
+ * two CTAs per SM.  The index-key loads are marked evict-first in L2 when the
+ * index-key cache is at most 2 GiB.
  */
 MSA_API msa_status_t msa_decode_fused(const msa_params_t *params, const void *q, const void *q_idx,
                               const void *k_cache, const void *v_cache, const void *k_idx, void *o,
