@@ -110,9 +110,9 @@ template <typename T> constexpr bool is_fp8() { return sizeof(T) == 1; }
 template <typename T, int GPS, int ROWB> constexpr bool scan_mma() { return GPS > 1 && sizeof(T) == 2 && ROWB >= 128; }
 // Warps per CTA (W): one index-K head per stream (GPS 1) keeps the index query in registers and
 // affords 12 warps; several groups on one stream read it from shared memory (CUDA cores, 8 warps)
-// or hold it as mma fragments (12 warps while the batch's bookkeeping leaves the shared memory:
-// their per-chunk work is a chain of dependent instructions, so more warps hide more of its
-// latency; 8 beyond).
+// or hold it as mma fragments (8 warps with three ring stages each while the batch's bookkeeping
+// leaves the shared memory, two beyond: measured at 1M with one shared head, 57.0 us per step
+// against 58.3 with 12 warps of two stages, the same bytes in flight).
 
 // S: ring stages per warp (2)
 template <typename T, int GPS, int ROWB, int S, int W>
@@ -707,7 +707,7 @@ cudaError_t launch_scan_t(const ScanArgs &a, const CUtensorMap &km, cudaStream_t
         return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
     } else {
         if constexpr (scan_mma<T, GPS, ROWB>()) {
-            if (scan_smem_bytes<T, GPS, ROWB, 2, 12>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 2, 12>(a, km, s, pdl);
+            if (scan_smem_bytes<T, GPS, ROWB, 3, 8>(a.B) <= 232448) return launch_scan_s<T, GPS, ROWB, 3, 8>(a, km, s, pdl);
         }
         return launch_scan_s<T, GPS, ROWB, 2, 8>(a, km, s, pdl);
     }
